@@ -1,0 +1,306 @@
+/*
+ * wkv_oracle.c -- plain, slow, fp64 CPU reference for the WKV recurrences.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing on the product path links, loads or calls
+ * this file: it exists so that the tests, the smoke check and the bench's CPU
+ * baseline can compare the CUDA kernels against an obviously correct
+ * evaluation. It shares no code, header or constant with the CUDA sources.
+ *
+ * What it computes (every function below cites the definition it follows):
+ *
+ *  RWKV-4 WKV (the operator that RWKV_TimeMix.forward calls as
+ *  RUN_CUDA(B, T, C, time_decay, time_first, k, v) on the RWKV-LM v4 code
+ *  walkthrough page "代码连连看——RWKV", section RWKV_TimeMix), per channel c with
+ *  decay rate w = exp(time_decay) > 0 and bonus u = time_first:
+ *
+ *      a_t = sum_{i<t} e^{-(t-1-i) w + k_i} v_i        b_t = sum_{i<t} e^{-(t-1-i) w + k_i}
+ *      y_t = (a_t + e^{u+k_t} v_t) / (b_t + e^{u+k_t})
+ *
+ *  evaluated by the plain linear recurrence a <- e^{-w} a + e^{k} v,
+ *  b <- e^{-w} b + e^{k}. To stay inside fp64 range every lane first subtracts
+ *  its largest key K* = max_t k_t from all keys: numerator and denominator are
+ *  both multiplied by e^{-K*}, so y is unchanged (an exact identity). This
+ *  oracle does NOT use the running-max (aa, bb, pp) form.
+ *
+ *  RWKV-4 WKV backward: the chain rule of the definition above, written out
+ *  with stored per-step a_t, b_t, D_t = b_t + e^{u+k_t}, y_t.
+ *
+ *  RWKV-6 head-state WKV (the RWKV6_OP operator of the rwkv-ops package page,
+ *  section "rwkv6op 使用方法", call and argument tables), per head with key
+ *  index i and value index j:
+ *
+ *      o_t[j]    = sum_i r_t[i] * ( S_{t-1}[i][j] + u[i] k_t[i] v_t[j] )
+ *      S_t[i][j] = w_t[i] * S_{t-1}[i][j] + k_t[i] v_t[j]
+ *
+ *  with S_{-1} = 0 or a caller-given initial state.
+ *
+ * Layouts: activations [B][T][C] row-major, C fastest. All inputs are fp64
+ * (the Python wrapper widens float32 / bf16 inputs exactly).
+ * Parallelism: OpenMP over independent lanes / heads only; every lane's
+ * arithmetic is sequential in t and identical to the single-thread order.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <stdio.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+static int all_finite(const double *x, int64_t n) {
+    for (int64_t i = 0; i < n; ++i)
+        if (!isfinite(x[i])) return 0;
+    return 1;
+}
+
+/* ------------------------------------------------------------------------ */
+/* RWKV-4 forward                                                            */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * y[B][T][C] from w[C], u[C], k[B][T][C], v[B][T][C].
+ * Optional outputs (pass NULL to skip), each [B][C]:
+ *   a_end, b_end : a_T and b_T multiplied by e^{-K*}  (the state after the
+ *                  last token, in the shifted scale)
+ *   kmax         : K* = max_t k_t of the lane
+ * Returns 0 on success, 1 if any produced value is not finite.
+ */
+int oracle_wkv4_forward(int64_t B, int64_t T, int64_t C,
+                        const double *w, const double *u,
+                        const double *k, const double *v, double *y,
+                        double *a_end, double *b_end, double *kmax)
+{
+    int bad = 0;
+    #pragma omp parallel for collapse(2) schedule(static) reduction(|:bad)
+    for (int64_t bi = 0; bi < B; ++bi) {
+        for (int64_t c = 0; c < C; ++c) {
+            const int64_t base = bi * T * C + c;
+            double K = -INFINITY;
+            for (int64_t t = 0; t < T; ++t) {
+                double kt = k[base + t * C];
+                if (kt > K) K = kt;
+            }
+            if (T == 0) K = 0.0;
+            const double decay = exp(-w[c]);          /* e^{-w} */
+            double a = 0.0, b = 0.0;                   /* a_0 = b_0 = 0 */
+            for (int64_t t = 0; t < T; ++t) {
+                const int64_t idx = base + t * C;
+                const double ek = exp(k[idx] - K);           /* e^{k_t}   (shifted) */
+                const double eu = exp(u[c] + k[idx] - K);    /* e^{u+k_t} (shifted) */
+                const double yt = (a + eu * v[idx]) / (b + eu);
+                if (!isfinite(yt)) bad = 1;
+                y[idx] = yt;
+                a = decay * a + ek * v[idx];                 /* a_{t+1} */
+                b = decay * b + ek;                          /* b_{t+1} */
+            }
+            if (a_end) a_end[bi * C + c] = a;
+            if (b_end) b_end[bi * C + c] = b;
+            if (kmax) kmax[bi * C + c] = K;
+        }
+    }
+    return bad;
+}
+
+/* ------------------------------------------------------------------------ */
+/* RWKV-4 backward                                                           */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Gradients of L = sum_t gy_t . y_t with respect to k, v (per element) and
+ * w, u (per channel, summed over the batch and time).
+ *
+ * Derivation (D_t = b_t + e^{u+k_t}, y_t as in the forward):
+ *   direct terms of token t    rho_t = e^{u+k_t} / D_t
+ *                              dy_t/dv_t = rho_t,  dy_t/dk_t = rho_t (v_t - y_t),
+ *                              dy_t/du   = rho_t (v_t - y_t)
+ *   through the past sums      dy_t/da_t = 1/D_t,  dy_t/db_t = -y_t/D_t
+ *   alpha_t = gy_t / D_t,  beta_t = gy_t y_t / D_t
+ *   A_i = sum_{t>i} alpha_t e^{-(t-1-i) w},  B_i likewise with beta
+ *     gv_i += e^{k_i} A_i,   gk_i += e^{k_i} (v_i A_i - B_i)
+ *   w enters only through a_t, b_t:  da_{t+1}/dw = e^{-w} (da_t/dw - a_t)
+ *     gw = sum_t alpha_t da_t/dw - beta_t db_t/dw          (forward form)
+ *   and, independently, with A'_i = sum_{t>i} (t-1-i) alpha_t e^{-(t-1-i) w}
+ *     gw = -sum_i e^{k_i} (v_i A'_i - B'_i)                 (reverse form)
+ *
+ * gk, gv: [B][T][C]. gw, gu: [C]. gw_rev (nullable): [C], the reverse-form gw,
+ * returned only so the two derivations can be checked against each other.
+ * Per-lane sums are added over the batch in increasing b.
+ */
+int oracle_wkv4_backward(int64_t B, int64_t T, int64_t C,
+                         const double *w, const double *u,
+                         const double *k, const double *v, const double *gy,
+                         double *gk, double *gv, double *gw, double *gu,
+                         double *gw_rev)
+{
+    int bad = 0;
+    double *lane_gw = (double *)calloc((size_t)(B * C) + 1, sizeof(double));
+    double *lane_gu = (double *)calloc((size_t)(B * C) + 1, sizeof(double));
+    double *lane_gwr = (double *)calloc((size_t)(B * C) + 1, sizeof(double));
+    if (!lane_gw || !lane_gu || !lane_gwr) {
+        free(lane_gw); free(lane_gu); free(lane_gwr);
+        return 2;
+    }
+
+    #pragma omp parallel reduction(|:bad)
+    {
+        double *D = (double *)malloc(sizeof(double) * (size_t)(T + 1));
+        double *Y = (double *)malloc(sizeof(double) * (size_t)(T + 1));
+        if (!D || !Y) bad = 2;
+        #pragma omp for collapse(2) schedule(static)
+        for (int64_t bi = 0; bi < B; ++bi) {
+            for (int64_t c = 0; c < C; ++c) {
+                if (!D || !Y) continue;
+                const int64_t base = bi * T * C + c;
+                double K = -INFINITY;
+                for (int64_t t = 0; t < T; ++t)
+                    if (k[base + t * C] > K) K = k[base + t * C];
+                if (T == 0) K = 0.0;
+                const double decay = exp(-w[c]);
+                double a = 0.0, b = 0.0, da = 0.0, db = 0.0;
+                double s_gw = 0.0, s_gu = 0.0;
+                /* forward sweep: outputs, direct gradient terms, gw forward form */
+                for (int64_t t = 0; t < T; ++t) {
+                    const int64_t idx = base + t * C;
+                    const double ek = exp(k[idx] - K);
+                    const double eu = exp(u[c] + k[idx] - K);
+                    const double Dt = b + eu;
+                    const double yt = (a + eu * v[idx]) / Dt;
+                    D[t] = Dt;
+                    Y[t] = yt;
+                    const double rho = eu / Dt;
+                    gv[idx] = gy[idx] * rho;
+                    gk[idx] = gy[idx] * rho * (v[idx] - yt);
+                    s_gu += gy[idx] * rho * (v[idx] - yt);
+                    const double alpha = gy[idx] / Dt;
+                    const double beta = gy[idx] * yt / Dt;
+                    s_gw += alpha * da - beta * db;
+                    const double da_next = decay * (da - a);
+                    const double db_next = decay * (db - b);
+                    a = decay * a + ek * v[idx];
+                    b = decay * b + ek;
+                    da = da_next;
+                    db = db_next;
+                }
+                /* reverse sweep: contributions through the future sums */
+                double A = 0.0, Bs = 0.0, Ap = 0.0, Bp = 0.0, s_gwr = 0.0;
+                for (int64_t i = T - 1; i >= 0; --i) {
+                    const int64_t idx = base + i * C;
+                    const double ek = exp(k[idx] - K);
+                    /* A, Bs hold A_i, B_i; Ap, Bp hold A'_i, B'_i */
+                    gv[idx] += ek * A;
+                    gk[idx] += ek * (v[idx] * A - Bs);
+                    s_gwr -= ek * (v[idx] * Ap - Bp);
+                    const double alpha = gy[idx] / D[i];
+                    const double beta = gy[idx] * Y[i] / D[i];
+                    const double Ap_next = decay * (Ap + A);
+                    const double Bp_next = decay * (Bp + Bs);
+                    A = alpha + decay * A;
+                    Bs = beta + decay * Bs;
+                    Ap = Ap_next;
+                    Bp = Bp_next;
+                }
+                lane_gw[bi * C + c] = s_gw;
+                lane_gu[bi * C + c] = s_gu;
+                lane_gwr[bi * C + c] = s_gwr;
+            }
+        }
+        free(D);
+        free(Y);
+    }
+    if (bad) {
+        free(lane_gw); free(lane_gu); free(lane_gwr);
+        return bad;
+    }
+    for (int64_t c = 0; c < C; ++c) {
+        double sw = 0.0, su = 0.0, swr = 0.0;
+        for (int64_t bi = 0; bi < B; ++bi) {
+            sw += lane_gw[bi * C + c];
+            su += lane_gu[bi * C + c];
+            swr += lane_gwr[bi * C + c];
+        }
+        gw[c] = sw;
+        gu[c] = su;
+        if (gw_rev) gw_rev[c] = swr;
+    }
+    free(lane_gw); free(lane_gu); free(lane_gwr);
+    if (!all_finite(gk, B * T * C) || !all_finite(gv, B * T * C) ||
+        !all_finite(gw, C) || !all_finite(gu, C))
+        return 1;
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* RWKV-6 head-state forward                                                 */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * r, k, v, w: [B][T][H*K] (w is the per-step decay in (0, 1]); u: [H*K].
+ * init_state (nullable): [n_state][H][K][K], indexed [.][h][i][j] with i the
+ *   key index and j the value index. Sample b starts from
+ *   init_state[state_map[b]] when state_map is given, else from
+ *   init_state[0] when n_state == 1, else from init_state[b] (n_state == B).
+ *   Without init_state every sample starts from S = 0.
+ * o: [B][T][H*K].  final_state (nullable): [B][H][K][K], S after the last token.
+ * The value dimension equals the key dimension (K), as in the package's
+ * (num_heads, head_size, head_size) state shape.
+ * Returns 0 on success, 1 on a non-finite output, 3 on a bad state index.
+ */
+int oracle_wkv6_forward(int64_t B, int64_t T, int64_t H, int64_t K,
+                        const double *r, const double *k, const double *v,
+                        const double *w, const double *u,
+                        const double *init_state, const int32_t *state_map,
+                        int64_t n_state, double *o, double *final_state)
+{
+    const int64_t HK = H * K;
+    int bad = 0;
+    #pragma omp parallel reduction(|:bad)
+    {
+        double *S = (double *)malloc(sizeof(double) * (size_t)(K * K));
+        if (!S) bad = 2;
+        #pragma omp for collapse(2) schedule(static)
+        for (int64_t bi = 0; bi < B; ++bi) {
+            for (int64_t h = 0; h < H; ++h) {
+                if (!S) continue;
+                if (init_state) {
+                    int64_t sidx;
+                    if (state_map) sidx = state_map[bi];
+                    else sidx = (n_state == 1) ? 0 : bi;
+                    if (sidx < 0 || sidx >= n_state) { bad |= 3; continue; }
+                    memcpy(S, init_state + (sidx * H + h) * K * K,
+                           sizeof(double) * (size_t)(K * K));
+                } else {
+                    memset(S, 0, sizeof(double) * (size_t)(K * K));
+                }
+                for (int64_t t = 0; t < T; ++t) {
+                    const int64_t row = (bi * T + t) * HK + h * K;
+                    /* output uses S_{t-1} plus the bonus of the current token */
+                    for (int64_t j = 0; j < K; ++j) {
+                        double acc = 0.0;
+                        for (int64_t i = 0; i < K; ++i)
+                            acc += r[row + i] * (S[i * K + j] + u[h * K + i] * k[row + i] * v[row + j]);
+                        o[row + j] = acc;
+                        if (!isfinite(acc)) bad |= 1;
+                    }
+                    /* then the state absorbs the current token */
+                    for (int64_t i = 0; i < K; ++i)
+                        for (int64_t j = 0; j < K; ++j)
+                            S[i * K + j] = w[row + i] * S[i * K + j] + k[row + i] * v[row + j];
+                }
+                if (final_state)
+                    memcpy(final_state + (bi * H + h) * K * K, S,
+                           sizeof(double) * (size_t)(K * K));
+            }
+        }
+        free(S);
+    }
+    return bad;
+}

@@ -1,0 +1,81 @@
+"""Plant plausible mistakes in a copy of the oracle source and check that the
+pins catch each one (CPU only; the committed oracle itself is untouched).
+"""
+
+import numpy as np
+import pytest
+
+from _pins import rel_err, wkv4_direct_sum, wkv4_fd_grads, wkv6_direct_sum
+
+MUTATIONS = {
+    # RWKV-4 forward: the bonus u dropped from the current token's weight
+    "wkv4_drop_bonus": ("const double eu = exp(u[c] + k[idx] - K);    /* e^{u+k_t} (shifted) */",
+                        "const double eu = exp(k[idx] - K);"),
+    # RWKV-4 forward: the newest token decayed once too often
+    "wkv4_extra_decay": ("a = decay * a + ek * v[idx];                 /* a_{t+1} */",
+                         "a = decay * (a + ek * v[idx]);"),
+    # RWKV-4 backward: wrong sign on the beta adjoint in gk
+    "wkv4_gk_sign": ("gk[idx] += ek * (v[idx] * A - Bs);", "gk[idx] += ek * (v[idx] * A + Bs);"),
+    # RWKV-4 backward: dropped term in the d/dw recurrence
+    "wkv4_gw_term": ("const double da_next = decay * (da - a);", "const double da_next = decay * da;"),
+    # RWKV-4 backward: local gu term with v and y swapped
+    "wkv4_gu_swap": ("s_gu += gy[idx] * rho * (v[idx] - yt);", "s_gu += gy[idx] * rho * (yt - v[idx]);"),
+    # RWKV-6: transposed outer product in the state update
+    "wkv6_transpose": ("S[i * K + j] = w[row + i] * S[i * K + j] + k[row + i] * v[row + j];",
+                       "S[i * K + j] = w[row + i] * S[i * K + j] + k[row + j] * v[row + i];"),
+    # RWKV-6: bonus indexed by the value dimension
+    "wkv6_u_index": ("u[h * K + i] * k[row + i] * v[row + j]", "u[h * K + j] * k[row + i] * v[row + j]"),
+    # RWKV-6: decay indexed by the value dimension
+    "wkv6_w_index": ("S[i * K + j] = w[row + i] * S[i * K + j]", "S[i * K + j] = w[row + j] * S[i * K + j]"),
+}
+
+
+@pytest.fixture(scope="module")
+def variants(tmp_path_factory, oracle):
+    src = oracle.source_text()
+    out = {}
+    for name, (old, new) in MUTATIONS.items():
+        assert src.count(old) == 1, f"mutation {name} does not match the oracle source"
+        d = tmp_path_factory.mktemp(name)
+        out[name] = oracle.build_variant(src.replace(old, new), str(d))
+    return out
+
+
+def _wkv4_pins_fail(var):
+    rng = np.random.default_rng(31)
+    C, T = 3, 10
+    w = np.exp(rng.uniform(-3, 1, size=C))
+    u = rng.uniform(-1, 1, size=C)
+    k = rng.normal(size=(1, T, C))
+    v = rng.normal(size=(1, T, C))
+    gy = rng.normal(size=k.shape)
+    if rel_err(var.wkv4_forward(w, u, k, v), wkv4_direct_sum(w, u, k, v)) > 1e-9:
+        return True
+    got = var.wkv4_backward(w, u, k, v, gy)
+    num = wkv4_fd_grads(var.wkv4_forward, w, u, k, v, gy)
+    return any(rel_err(g, n) > 1e-6 for g, n in zip(got, num))
+
+
+def _wkv6_pins_fail(var):
+    rng = np.random.default_rng(32)
+    B, T, H, K = 1, 8, 2, 4
+    r, k, v = (rng.normal(size=(B, T, H * K)) for _ in range(3))
+    w = rng.uniform(0.3, 1.0, size=(B, T, H * K))
+    u = rng.uniform(-1, 1, size=(H, K))
+    o, _ = var.wkv6_forward(r, k, v, w, u)
+    return rel_err(o, wkv6_direct_sum(r, k, v, w, u, K)) > 1e-9
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_mutation_is_caught(variants, name):
+    check = _wkv4_pins_fail if name.startswith("wkv4") else _wkv6_pins_fail
+    assert check(variants[name]), f"planted mistake {name} passed every pin"
+
+
+def test_unmutated_source_passes(oracle):
+    class _Orig:
+        wkv4_forward = staticmethod(oracle.wkv4_forward)
+        wkv4_backward = staticmethod(oracle.wkv4_backward)
+        wkv6_forward = staticmethod(oracle.wkv6_forward)
+    assert not _wkv4_pins_fail(_Orig)
+    assert not _wkv6_pins_fail(_Orig)
