@@ -1,0 +1,207 @@
+/*
+ * wkv.h -- C ABI of the B200 (sm_100a) WKV kernel library libwkv_b200.so.
+ *
+ * The library evaluates RWKV's WKV time-mixing recurrence on one GPU:
+ *   - RWKV-4 WKV forward and backward (the operator RWKV_TimeMix.forward calls
+ *     as RUN_CUDA(B, T, C, time_decay, time_first, k, v); RWKV-LM v4 code
+ *     walkthrough page "代码连连看——RWKV", section RWKV_TimeMix),
+ *   - the same RWKV-4 recurrence as a state-carrying step over batched,
+ *     variable-length inference slots (web-rwkv crate page, section
+ *     "批量推理" / batched inference: slots, token_chunk_size, empty slots
+ *     skipped, state persisting across run() calls),
+ *   - the RWKV-6 head-state recurrence forward (rwkv-ops package page,
+ *     section "rwkv6op 使用方法": RWKV6_OP call and argument tables).
+ *
+ * RWKV-4 definition, per lane (b, c), with decay rate w_c > 0 (the model's
+ * exp(time_decay_c)) and bonus u_c (time_first_c):
+ *
+ *   y_t = ( sum_{i<t} e^{-(t-1-i) w + k_i} v_i + e^{u + k_t} v_t )
+ *       / ( sum_{i<t} e^{-(t-1-i) w + k_i}     + e^{u + k_t} )
+ *
+ * evaluated with the overflow-safe running-max state (aa, bb, pp): the past
+ * sums are a = aa * 2^pp and b = bb * 2^pp. NOTE: pp is kept as a base-2
+ * exponent everywhere it is stored (checkpoints, slot state), so that a state
+ * written by one call is read back bit for bit by the next.
+ *
+ * RWKV-6 definition, per (batch b, head h), key index i, value index j:
+ *
+ *   o_t[j]    = sum_i r_t[i] * ( S_{t-1}[i][j] + u[i] k_t[i] v_t[j] )
+ *   S_t[i][j] = w_t[i] * S_{t-1}[i][j] + k_t[i] v_t[j]
+ *
+ * Conventions shared by every entry point
+ *   Memory      All pointers are DEVICE pointers unless stated otherwise. The
+ *               caller owns every buffer; the library allocates nothing on
+ *               these paths and keeps no per-call state.
+ *   Layout      Activations are dense row-major [B][T][C] (C fastest), with no
+ *               padding. Per-channel parameters are dense [C] float32.
+ *   Alignment   Every device pointer must be 16-byte aligned.
+ *   Sizes       64-bit. A zero B, T or C (S, N) is a valid no-op (WKV_OK).
+ *   dtype       WKV_F32 or WKV_BF16 selects the storage type of the
+ *               activations (k, v, y, gy, gk, gv, r, w, o); arithmetic and
+ *               recurrent state are float32 in both cases. bf16 outputs are
+ *               rounded to nearest even.
+ *   C granularity  C must be a multiple of 4 for WKV_F32 and of 8 for
+ *               WKV_BF16 (rows must be whole 16-byte units).
+ *   Streams     `stream` is a cudaStream_t (NULL = legacy default stream).
+ *               Every call is asynchronous on that stream and never
+ *               synchronises the device.
+ *   Errors      Argument errors are detected on the host, before anything is
+ *               launched, and returned as WKV_ERR_INVALID_ARG or
+ *               WKV_ERR_UNSUPPORTED; a launch failure returns WKV_ERR_CUDA.
+ *               wkv_last_error() gives a one-line message for the calling
+ *               thread's most recent failure. No C++ exception crosses this
+ *               interface. Kernels never trap: a bounded wait that gives up
+ *               records a code that wkv_device_error() returns.
+ *   Threads     The library is thread-safe; calls on different streams may
+ *               run concurrently.
+ */
+#ifndef WKV_B200_H
+#define WKV_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define WKV_ABI_VERSION 1
+
+/* Steps between two RWKV-4 forward state checkpoints (see wkv4_forward). */
+#define WKV4_CKPT_LEN 32
+
+typedef enum {
+    WKV_OK = 0,
+    WKV_ERR_INVALID_ARG = 1, /* null/misaligned pointer, negative size, bad dtype */
+    WKV_ERR_UNSUPPORTED = 2, /* well-formed request outside what the kernels cover */
+    WKV_ERR_CUDA = 3,        /* a CUDA runtime call or kernel launch failed       */
+    WKV_ERR_DEVICE = 4       /* a kernel recorded a device-side error code        */
+} wkv_status;
+
+typedef enum { WKV_F32 = 0, WKV_BF16 = 1 } wkv_dtype;
+
+/* Device-side error codes reported by wkv_device_error (bit flags). */
+#define WKV_DEVERR_WAIT_TIMEOUT 0x1u /* a bounded wait on a copy gave up      */
+#define WKV_DEVERR_BAD_SLOT     0x2u /* a slot's token range was out of bounds */
+#define WKV_DEVERR_BAD_STATE    0x4u /* a state_map entry was out of range    */
+
+/* ABI version of the loaded library (WKV_ABI_VERSION). */
+int wkv_abi_version(void);
+
+/* Static, human-readable name of a wkv_status value. */
+const char *wkv_status_string(int status);
+
+/* Message of the calling thread's last failing call ("" if none). */
+const char *wkv_last_error(void);
+
+/*
+ * Read (and, if reset != 0, clear) the device-side error word of the current
+ * device. SYNCHRONOUS: waits for all work on the current device. *code gets
+ * an OR of WKV_DEVERR_* bits (0 = no error).
+ */
+wkv_status wkv_device_error(uint32_t *code, int reset);
+
+/* ------------------------------------------------------------------------ */
+/* RWKV-4                                                                    */
+/* ------------------------------------------------------------------------ */
+
+/* Number of floats of the checkpoint buffer: B * ceil(T / WKV4_CKPT_LEN) * 3 * C. */
+size_t wkv4_ckpt_floats(int64_t B, int64_t T, int64_t C);
+
+/*
+ * RWKV-4 WKV forward.
+ *   w, u   [C] float32. w is the per-step decay RATE (> 0): the state is
+ *          multiplied by e^{-w} per token. u is the current-token bonus.
+ *   k, v   [B][T][C] of `dtype`.
+ *   y      [B][T][C] of `dtype`, written. May be NULL to only produce ckpt.
+ *   ckpt   NULL, or [B][ceil(T/WKV4_CKPT_LEN)][3][C] float32, written: entry
+ *          [b][n] holds (aa, bb, pp) of every channel *before* token
+ *          n * WKV4_CKPT_LEN of sample b (pp base 2). wkv4_backward reads it.
+ * The state starts from the empty past (aa = bb = 0, pp = -1e38).
+ */
+wkv_status wkv4_forward(int64_t B, int64_t T, int64_t C, int dtype,
+                        const float *w, const float *u,
+                        const void *k, const void *v, void *y,
+                        float *ckpt, void *stream);
+
+/* Bytes of device workspace wkv4_backward needs (has_ckpt: ckpt != NULL). */
+size_t wkv4_backward_workspace_bytes(int64_t B, int64_t T, int64_t C, int has_ckpt);
+
+/*
+ * RWKV-4 WKV backward: gradients of L = sum(gy * y) for y = wkv4_forward(...).
+ *   gy          [B][T][C] of `dtype`.
+ *   ckpt        the checkpoints wkv4_forward wrote for the same inputs, or
+ *               NULL (then they are regenerated inside `workspace`).
+ *   gk, gv      [B][T][C] of `dtype`, written (not accumulated).
+ *   gw, gu      [C] float32, written: dL/dw and dL/du summed over batch and
+ *               time. (dL/dtime_decay = gw * w.) The batch sum is taken in a
+ *               fixed order, so results are run-to-run deterministic.
+ *   workspace   device scratch of at least
+ *               wkv4_backward_workspace_bytes(B, T, C, ckpt != NULL) bytes,
+ *               16-byte aligned; its contents on entry are ignored.
+ */
+wkv_status wkv4_backward(int64_t B, int64_t T, int64_t C, int dtype,
+                         const float *w, const float *u,
+                         const void *k, const void *v, const void *gy,
+                         const float *ckpt,
+                         void *gk, void *gv, float *gw, float *gu,
+                         void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Set S slot states [S][3][C] float32 to the empty past
+ * (aa = bb = 0, pp = -1e38).
+ */
+wkv_status wkv4_state_init(int64_t S, int64_t C, float *state, void *stream);
+
+/*
+ * One batched inference call over S slots (web-rwkv's batched inference).
+ *   k, v, y     [n_tokens][C] of `dtype`: the tokens of all slots packed back
+ *               to back, slot 0 first; y is written for every consumed token.
+ *   cu_tokens   DEVICE int32 [S+1], cu_tokens[0] = 0, nondecreasing: slot s
+ *               consumes tokens cu_tokens[s] .. cu_tokens[s+1]-1 in order. A
+ *               slot with no tokens is skipped and its state left untouched.
+ *               A slot whose range is decreasing or exceeds n_tokens is
+ *               skipped too and WKV_DEVERR_BAD_SLOT is recorded.
+ *   state       [S][3][C] float32 (aa, bb, pp per channel, pp base 2), read
+ *               and written in place: it carries each slot across calls.
+ * Feeding a sequence in several calls gives bit-identical y and state to
+ * feeding it in one call, and bit-identical y to wkv4_forward on the same
+ * tokens (all three run the same float32 step in the same order).
+ */
+wkv_status wkv4_chunk_step(int64_t S, int64_t C, int dtype,
+                           const float *w, const float *u,
+                           const void *k, const void *v, void *y, int64_t n_tokens,
+                           const int32_t *cu_tokens, float *state, void *stream);
+
+/* ------------------------------------------------------------------------ */
+/* RWKV-6                                                                    */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * RWKV-6 head-state WKV forward (RWKV6_OP(head_size=K)(r, k, v, w, u,
+ * with_state, init_state, state_map) on the rwkv-ops package page).
+ *   K            head size; 64 is the supported value (else UNSUPPORTED).
+ *   dtype        WKV_BF16 (else UNSUPPORTED).
+ *   r, k, v, w   [B][T][H*K] bf16; w is the per-step decay, in (0, 1].
+ *   u            [H*K] float32 (the (num_heads, head_size) bonus, flattened).
+ *   init_state   NULL (every sample starts from S = 0) or
+ *                [n_state][H][K][K] float32, indexed [.][h][i][j] with i the
+ *                key index and j the value index.
+ *   state_map    NULL or DEVICE int32 [B]: sample b starts from
+ *                init_state[state_map[b]]. Without it, n_state must be 1
+ *                (shared) or B (one per sample). An out-of-range entry makes
+ *                that sample start from zero and records WKV_DEVERR_BAD_STATE.
+ *   final_state  NULL or [B][H][K][K] float32, written: S after the last token.
+ *   o            [B][T][H*K] bf16, written.
+ */
+wkv_status wkv6_forward(int64_t B, int64_t T, int64_t H, int64_t K, int dtype,
+                        const void *r, const void *k, const void *v, const void *w,
+                        const float *u,
+                        const float *init_state, const int32_t *state_map, int64_t n_state,
+                        float *final_state, void *o, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WKV_B200_H */

@@ -1,0 +1,169 @@
+// wkv_device.cuh -- device-side building blocks shared by the WKV kernels:
+// storage-type traits, hardware exp2 / reciprocal, mbarrier and TMA wrappers
+// (sm_100a inline PTX), bounded waits, and the RWKV-4 running-max step.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "wkv.h"
+#include "wkv_internal.h"
+
+namespace wkv {
+
+// log2(e): the RWKV-4 kernels run the recurrence in base 2, so every
+// exponential is a single ex2 instruction.
+constexpr float kLog2e = 1.4426950408889634f;
+// pp of the empty past: a finite "minus infinity" (no inf - inf under ftz).
+constexpr float kEmptyPP = -1.0e38f;
+// Give up a wait on a copy after this many nanoseconds (then record an error).
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// ----------------------------------------------------------------------------
+// storage types
+// ----------------------------------------------------------------------------
+template <class E> struct Elem;
+template <> struct Elem<float> {
+  static __device__ __forceinline__ float to_f32(float x) { return x; }
+  static __device__ __forceinline__ float from_f32(float x) { return x; }
+  static constexpr CUtensorMapDataType tma_type = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+};
+template <> struct Elem<__nv_bfloat16> {
+  static __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+  static __device__ __forceinline__ __nv_bfloat16 from_f32(float x) { return __float2bfloat16_rn(x); }
+  static constexpr CUtensorMapDataType tma_type = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+};
+
+// ----------------------------------------------------------------------------
+// hardware transcendental instructions (PTX ex2.approx / rcp.approx)
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float rcp(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void record_error(unsigned* err, unsigned code) {
+  if (err) atomicOr(err, code);
+}
+
+// ----------------------------------------------------------------------------
+// mbarrier (shared::cta) and TMA
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+// Make barrier initialisation visible to the async (TMA) proxy.
+__device__ __forceinline__ void mbar_init_fence() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for phase `parity` of `bar` to complete, for at most kWaitLimitNs.
+// Returns false (and records WKV_DEVERR_WAIT_TIMEOUT) if it never does.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, unsigned* err) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      record_error(err, WKV_DEVERR_WAIT_TIMEOUT);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// 3-D tiled bulk tensor load global -> shared (no multicast), completion
+// signalled on `bar` as transaction bytes. x is the innermost coordinate.
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y,
+                                            int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
+      "[%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+
+// ----------------------------------------------------------------------------
+// RWKV-4 step, running-max form in base 2.
+//
+// State of one lane: the past sums a = aa * 2^pp, b = bb * 2^pp. Inputs are
+// pre-scaled by log2(e): k2 = k*log2e, u2 = u*log2e, w2 = w*log2e.
+// Output of token t:  q = max(pp, u2+k2); y = (2^{pp-q} aa + 2^{u2+k2-q} v)
+//                                          / (2^{pp-q} bb + 2^{u2+k2-q})
+// Absorb token t:     q' = max(pp-w2, k2); aa <- 2^{pp-w2-q'} aa + 2^{k2-q'} v,
+//                     bb <- 2^{pp-w2-q'} bb + 2^{k2-q'}, pp <- q'.
+// In each pair one exponent is 0, so a pair costs one ex2 and a select.
+// All roundings are explicit (_rn intrinsics) so that every kernel that runs
+// this step produces bit-identical results from the same state and inputs.
+// ----------------------------------------------------------------------------
+struct Wkv4State {
+  float aa, bb, pp;
+};
+
+__device__ __forceinline__ Wkv4State wkv4_empty_state() { return {0.f, 0.f, kEmptyPP}; }
+
+__device__ __forceinline__ float wkv4_output(const Wkv4State& s, float k2, float v, float u2) {
+  const float cur = __fadd_rn(u2, k2);
+  const float d = __fsub_rn(s.pp, cur);
+  const float e = ex2(-fabsf(d));
+  const bool past_max = d >= 0.f;
+  const float e1 = past_max ? 1.f : e;
+  const float e2 = past_max ? e : 1.f;
+  const float num = __fmaf_rn(e1, s.aa, __fmul_rn(e2, v));
+  const float den = __fmaf_rn(e1, s.bb, e2);
+  return __fmul_rn(num, rcp(den));
+}
+
+__device__ __forceinline__ void wkv4_absorb(Wkv4State& s, float k2, float v, float w2) {
+  const float past = __fsub_rn(s.pp, w2);
+  const float d = __fsub_rn(past, k2);
+  const float e = ex2(-fabsf(d));
+  const bool past_max = d >= 0.f;
+  const float e1 = past_max ? 1.f : e;
+  const float e2 = past_max ? e : 1.f;
+  s.aa = __fmaf_rn(e1, s.aa, __fmul_rn(e2, v));
+  s.bb = __fmaf_rn(e1, s.bb, e2);
+  s.pp = past_max ? past : k2;
+}
+
+}  // namespace wkv

@@ -1,0 +1,121 @@
+"""Host-side checks of the C ABI that need no GPU.
+
+The library must load on a machine without a GPU, export every function that
+include/wkv.h declares, and reject malformed arguments before it touches the
+CUDA runtime.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "wkv.h")
+
+
+@pytest.fixture(scope="module")
+def W():
+    from rwkv_wkv_linear_mix_b200 import build
+    build.build()
+    from rwkv_wkv_linear_mix_b200 import wkv
+    return wkv
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*([A-Za-z_][A-Za-z0-9_]*)\s*\(",
+                       src, flags=re.M)
+    return sorted(set(n for n in names if n.startswith("wkv")))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("wkv4_forward", "wkv4_backward", "wkv4_chunk_step", "wkv4_state_init", "wkv6_forward",
+              "wkv4_backward_workspace_bytes", "wkv4_ckpt_floats", "wkv_status_string", "wkv_last_error",
+              "wkv_device_error", "wkv_abi_version"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(W):
+    lib = ctypes.CDLL(W.LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(lib, n), f"{n} declared in wkv.h but not exported"
+    assert set(declared_functions()) == set(W.SIGNATURES), "binding signatures out of sync with wkv.h"
+
+
+def test_version_and_strings(W):
+    L = W.lib()
+    assert L.wkv_abi_version() == 1
+    assert L.wkv_status_string(0) == b"WKV_OK"
+    assert L.wkv_status_string(2) == b"WKV_ERR_UNSUPPORTED"
+    assert L.wkv_status_string(99) == b"WKV_ERR_UNKNOWN"
+
+
+def test_size_helpers(W):
+    L = W.lib()
+    assert L.wkv4_ckpt_floats(2, 64, 128) == 2 * 2 * 3 * 128
+    assert L.wkv4_ckpt_floats(1, 33, 8) == 1 * 2 * 3 * 8
+    assert L.wkv4_ckpt_floats(0, 10, 8) == 0
+    ws = L.wkv4_backward_workspace_bytes(2, 64, 128, 1)
+    assert ws >= 2 * 2 * 128 * 4
+    assert L.wkv4_backward_workspace_bytes(2, 64, 128, 0) >= ws + 2 * 2 * 3 * 128 * 4
+
+
+FAKE = 1 << 20  # 16-byte aligned, never dereferenced: every call below fails validation first
+
+
+def _fwd(L, B, T, C, dt, w=FAKE, u=FAKE, k=FAKE, v=FAKE, y=FAKE, ck=None):
+    return L.wkv4_forward(B, T, C, dt, w, u, k, v, y, ck, None)
+
+
+def test_forward_argument_errors(W):
+    L = W.lib()
+    assert _fwd(L, -1, 4, 8, 0) == W.WKV_ERR_INVALID_ARG
+    assert _fwd(L, 1, 4, 8, 7) == W.WKV_ERR_INVALID_ARG          # unknown dtype
+    assert _fwd(L, 1, 4, 6, 0) == W.WKV_ERR_UNSUPPORTED          # C % 4
+    assert _fwd(L, 1, 4, 12, 1) == W.WKV_ERR_UNSUPPORTED         # C % 8 for bf16
+    assert _fwd(L, 1, 4, 8, 0, k=None) == W.WKV_ERR_INVALID_ARG
+    assert b"k is NULL" in L.wkv_last_error()
+    assert _fwd(L, 1, 4, 8, 0, v=FAKE + 4) == W.WKV_ERR_INVALID_ARG
+    assert b"aligned" in L.wkv_last_error()
+    assert _fwd(L, 1, 4, 8, 0, y=None, ck=None) == W.WKV_ERR_INVALID_ARG
+    assert _fwd(L, 1, 1 << 31, 8, 0) == W.WKV_ERR_UNSUPPORTED
+    # empty problems are valid no-ops and launch nothing
+    assert _fwd(L, 0, 4, 8, 0) == W.WKV_OK
+    assert _fwd(L, 3, 0, 8, 0) == W.WKV_OK
+
+
+def test_backward_argument_errors(W):
+    L = W.lib()
+    args = [FAKE] * 11
+    # workspace too small
+    rc = L.wkv4_backward(2, 8, 8, 0, *args[:10], FAKE, 0, None)
+    assert rc == W.WKV_ERR_INVALID_ARG and b"workspace" in L.wkv_last_error()
+    rc = L.wkv4_backward(2, 8, 8, 0, FAKE, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None)
+    assert rc == W.WKV_ERR_INVALID_ARG and b"gy" in L.wkv_last_error()
+    assert L.wkv4_backward(2, 8, 10, 0, *args[:10], FAKE, 1 << 30, None) == W.WKV_ERR_UNSUPPORTED
+
+
+def test_chunk_and_wkv6_argument_errors(W):
+    L = W.lib()
+    assert L.wkv4_chunk_step(4, 8, 0, FAKE, FAKE, FAKE, FAKE, FAKE, -1, FAKE, FAKE, None) == W.WKV_ERR_INVALID_ARG
+    assert L.wkv4_chunk_step(4, 8, 0, FAKE, FAKE, FAKE, FAKE, FAKE, 10, None, FAKE, None) == W.WKV_ERR_INVALID_ARG
+    assert L.wkv4_chunk_step(0, 8, 0, FAKE, FAKE, FAKE, FAKE, FAKE, 0, FAKE, FAKE, None) == W.WKV_OK
+    wk6 = lambda B=1, T=4, H=2, K=64, dt=1, init=None, smap=None, ns=0: L.wkv6_forward(
+        B, T, H, K, dt, FAKE, FAKE, FAKE, FAKE, FAKE, init, smap, ns, None, FAKE, None)
+    assert wk6(K=32) == W.WKV_ERR_UNSUPPORTED
+    assert wk6(dt=0) == W.WKV_ERR_UNSUPPORTED
+    assert wk6(B=-1) == W.WKV_ERR_INVALID_ARG
+    assert wk6(B=3, init=FAKE, ns=2) == W.WKV_ERR_INVALID_ARG     # n_state neither 1 nor B
+    assert wk6(B=3, init=FAKE, ns=0) == W.WKV_ERR_INVALID_ARG
+    assert wk6(B=0) == W.WKV_OK
+
+
+def test_binding_refuses_cpu_tensors(W):
+    import torch
+    k = torch.zeros(1, 4, 8)
+    with pytest.raises(ValueError):
+        W.wkv4_forward(torch.zeros(8), torch.zeros(8), k, k)

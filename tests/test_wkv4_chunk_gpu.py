@@ -1,0 +1,102 @@
+"""GPU checks of wkv4_chunk_step: web-rwkv-style batched inference slots
+(web-rwkv crate page, section "批量推理" / batched inference)."""
+
+import numpy as np
+import pytest
+import torch
+
+from _dev import TOL, dev, host64, need_gpu, rel_err
+from rwkv_wkv_linear_mix_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def W():
+    need_gpu()
+    from rwkv_wkv_linear_mix_b200 import wkv
+    wkv.device_error(reset=True)
+    return wkv
+
+
+def feed(W, inp, chunk, w, u, k, v):
+    """Feed every slot's prompt in calls of at most `chunk` tokens; return
+    y in the original packed order and the final state."""
+    lengths, offs = inp["lengths"], inp["offsets"]
+    S, C = len(lengths), k.shape[1]
+    state = W.wkv4_state_init(S, C, k.device)
+    y = torch.empty_like(k)
+    done = np.zeros(S, np.int64)
+    for take in synth.feed_schedule(lengths, chunk):
+        idx = np.concatenate([np.arange(offs[s] + done[s], offs[s] + done[s] + take[s]) for s in range(S)])
+        idx_t = torch.from_numpy(idx).cuda()
+        cu = torch.from_numpy(np.concatenate([[0], np.cumsum(take)]).astype(np.int32)).cuda()
+        yc = W.wkv4_chunk_step(w, u, k[idx_t].contiguous(), v[idx_t].contiguous(), cu, state)
+        y[idx_t] = yc
+        done += take
+    return y, state
+
+
+@pytest.fixture(scope="module")
+def slots():
+    return synth.wkv4_slot_inputs(S=32, C=4096, len_lo=1, len_hi=512, dtype="bf16", seed=0)
+
+
+def test_chunked_equals_whole_bitwise(W, slots):
+    w, u, k, v = dev(slots["w"]), dev(slots["u"]), dev(slots["k"]), dev(slots["v"])
+    y32, s32 = feed(W, slots, 32, w, u, k, v)
+    yall, sall = feed(W, slots, 1 << 30, w, u, k, v)
+    y7, s7 = feed(W, slots, 7, w, u, k, v)
+    assert torch.equal(y32, yall) and torch.equal(s32, sall)
+    assert torch.equal(y7, yall) and torch.equal(s7, sall)
+    assert W.device_error(reset=True) == 0
+
+
+def test_equals_forward_bitwise_and_oracle(W, oracle, slots):
+    w, u, k, v = dev(slots["w"]), dev(slots["u"]), dev(slots["k"]), dev(slots["v"])
+    y, state = feed(W, slots, 32, w, u, k, v)
+    offs = slots["offsets"]
+    for s in range(len(slots["lengths"])):
+        a, b = int(offs[s]), int(offs[s + 1])
+        yf = W.wkv4_forward(w, u, k[a:b][None].contiguous(), v[a:b][None].contiguous())
+        assert torch.equal(yf[0], y[a:b]), f"slot {s}"
+    for s in (0, 5, 17, 31):
+        a, b = int(offs[s]), int(offs[s + 1])
+        ref, st = oracle.wkv4_forward(slots["w"], slots["u"], slots["k32"][None, a:b], slots["v32"][None, a:b],
+                                      return_state=True)
+        assert rel_err(host64(y[a:b]), ref[0]) < TOL["bf16"]
+        aa, bb, pp = (host64(state[s, i]) for i in range(3))
+        np.testing.assert_allclose(np.log(bb) + pp * np.log(2.0), np.log(st["b_end"][0]) + st["kmax"][0],
+                                   rtol=0, atol=1e-3)
+        assert rel_err(aa / bb, st["a_end"][0] / st["b_end"][0]) < 1e-3
+
+
+def test_empty_slots_untouched_and_bad_ranges(W):
+    S, C = 6, 64
+    rng = np.random.default_rng(3)
+    w = dev(np.exp(rng.uniform(-6, 1, C)).astype(np.float32))
+    u = dev(rng.uniform(-1, 1, C).astype(np.float32))
+    take = np.array([3, 0, 5, 0, 1, 2])
+    n = int(take.sum())
+    k = dev(rng.normal(size=(n, C)).astype(np.float32))
+    v = dev(rng.normal(size=(n, C)).astype(np.float32))
+    state = W.wkv4_state_init(S, C, k.device)
+    state.normal_()
+    before = state.clone()
+    cu = torch.from_numpy(np.concatenate([[0], np.cumsum(take)]).astype(np.int32)).cuda()
+    W.wkv4_chunk_step(w, u, k, v, cu, state)
+    for s in range(S):
+        assert torch.equal(state[s], before[s]) == (take[s] == 0)
+    assert W.device_error(reset=True) == 0
+    # decreasing or out-of-range slots are skipped and reported
+    bad = torch.tensor([0, 3, 2, 100, 100, 101, n], dtype=torch.int32, device="cuda")
+    before = state.clone()
+    W.wkv4_chunk_step(w, u, k, v, bad, state)
+    assert W.device_error(reset=True) & W.WKV_DEVERR_BAD_SLOT
+    for s in (1, 2, 4):
+        assert torch.equal(state[s], before[s])
+
+
+def test_state_init_values(W):
+    st = W.wkv4_state_init(3, 16, "cuda")
+    assert torch.all(st[:, 0] == 0) and torch.all(st[:, 1] == 0) and torch.all(st[:, 2] == -1e38)

@@ -1,0 +1,71 @@
+"""GPU parity of wkv6_forward against the fp64 oracle (RWKV6_OP of the
+rwkv-ops package page, section "rwkv6op 使用方法")."""
+
+import numpy as np
+import pytest
+import torch
+
+from _dev import TOL, dev, host64, need_gpu, rel_err
+from rwkv_wkv_linear_mix_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def W():
+    need_gpu()
+    from rwkv_wkv_linear_mix_b200 import wkv
+    wkv.device_error(reset=True)
+    return wkv
+
+
+def run(W, inp, **kw):
+    return W.wkv6_forward(dev(inp["r"]), dev(inp["k"]), dev(inp["v"]), dev(inp["w"]), dev(inp["u"]), **kw)
+
+
+def ref(oracle, inp, H, **kw):
+    return oracle.wkv6_forward(inp["r32"], inp["k32"], inp["v32"], inp["w32"], inp["u"].reshape(H, 64), **kw)
+
+
+@pytest.mark.parametrize("B,T,H", [(1, 64, 1), (2, 100, 2), (1, 1, 3), (2, 257, 2), (1, 130, 1)])
+def test_matches_oracle(W, oracle, B, T, H):
+    inp = synth.wkv6_inputs(synth.Wkv6Recipe("t", B, T, H), seed=B + T + H)
+    o, fs = run(W, inp)
+    ro, rfs = ref(oracle, inp, H)
+    assert rel_err(host64(o), ro) < TOL["bf16"]
+    assert rel_err(host64(fs), rfs) < TOL["bf16"]
+    assert W.device_error(reset=True) == 0
+
+
+def test_init_state_and_map(W, oracle):
+    B, T, H = 3, 70, 2
+    inp = synth.wkv6_inputs(synth.Wkv6Recipe("t", B, T, H), seed=11)
+    rng = np.random.default_rng(2)
+    init = rng.normal(size=(2, H, 64, 64)).astype(np.float32)
+    smap = np.array([1, 0, 1], np.int32)
+    o, fs = run(W, inp, init_state=dev(init), state_map=dev(smap))
+    ro, rfs = ref(oracle, inp, H, init_state=init, state_map=smap)
+    assert rel_err(host64(o), ro) < TOL["bf16"]
+    assert rel_err(host64(fs), rfs) < TOL["bf16"]
+    o1, _ = run(W, inp, init_state=dev(init[:1]))
+    ro1, _ = ref(oracle, inp, H, init_state=init[:1])
+    assert rel_err(host64(o1), ro1) < TOL["bf16"]
+    # out-of-range map entry: that sample starts from zero, error recorded
+    bad = np.array([0, 5, 1], np.int32)
+    ob, _ = run(W, inp, init_state=dev(init), state_map=dev(bad))
+    assert W.device_error(reset=True) & W.WKV_DEVERR_BAD_STATE
+    rz, _ = ref(oracle, {n: x[1:2] if n != "u" else x for n, x in inp.items()}, H)
+    assert rel_err(host64(ob[1:2]), rz) < TOL["bf16"]
+
+
+def test_c2048_config_sampled_heads(W, oracle):
+    rec = synth.WKV6_RECIPES["wkv6_fwd_bf16_c2048"]
+    inp = synth.wkv6_inputs(rec, seed=0)
+    o, fs = run(W, inp)
+    for (b, h) in [(0, 0), (3, 17), (7, 31)]:
+        sl = slice(h * 64, (h + 1) * 64)
+        sub = {n: inp[n + "32"][b:b + 1, :, sl] for n in ("r", "k", "v", "w")}
+        ro, rfs = oracle.wkv6_forward(sub["r"], sub["k"], sub["v"], sub["w"], inp["u"][sl].reshape(1, 64))
+        assert rel_err(host64(o[b:b + 1, :, sl]), ro) < TOL["bf16"], (b, h)
+        assert rel_err(host64(fs[b, h]), rfs[0, 0]) < TOL["bf16"], (b, h)
+    assert W.device_error(reset=True) == 0
