@@ -18,10 +18,12 @@
  *   y_t = ( sum_{i<t} e^{-(t-1-i) w + k_i} v_i + e^{u + k_t} v_t )
  *       / ( sum_{i<t} e^{-(t-1-i) w + k_i}     + e^{u + k_t} )
  *
- * evaluated with the overflow-safe running-max state (aa, bb, pp): the past
- * sums are a = aa * 2^pp and b = bb * 2^pp. NOTE: pp is kept as a base-2
- * exponent everywhere it is stored (checkpoints, slot state), so that a state
- * written by one call is read back bit for bit by the next.
+ * evaluated with the overflow-safe running-max state: the past sums are
+ * a = aa * 2^(P + ref) and b = bb * 2^(P + ref) with P = base - n * w * log2(e).
+ * ref = fl(k_first * log2(e)) is a per-lane reference fixed by the first key
+ * the lane absorbs (k_first = k[b][0][c] for wkv4_forward), so exponents have
+ * the size of the key range, not of the keys; n counts the decay steps since
+ * the exponent was last set, so the decay never accumulates rounding error.
  *
  * RWKV-6 definition, per (batch b, head h), key index i, value index j:
  *
@@ -115,9 +117,10 @@ size_t wkv4_ckpt_floats(int64_t B, int64_t T, int64_t C);
  *   k, v   [B][T][C] of `dtype`.
  *   y      [B][T][C] of `dtype`, written. May be NULL to only produce ckpt.
  *   ckpt   NULL, or [B][ceil(T/WKV4_CKPT_LEN)][3][C] float32, written: entry
- *          [b][n] holds (aa, bb, pp) of every channel *before* token
- *          n * WKV4_CKPT_LEN of sample b (pp base 2). wkv4_backward reads it.
- * The state starts from the empty past (aa = bb = 0, pp = -1e38).
+ *          [b][m] holds (aa, bb, P) of every channel *before* token
+ *          m * WKV4_CKPT_LEN of sample b (P relative to the lane's ref).
+ *          wkv4_backward reads it.
+ * The state starts from the empty past (aa = bb = 0, exponent -1e38).
  */
 wkv_status wkv4_forward(int64_t B, int64_t T, int64_t C, int dtype,
                         const float *w, const float *u,
@@ -148,8 +151,8 @@ wkv_status wkv4_backward(int64_t B, int64_t T, int64_t C, int dtype,
                          void *workspace, size_t workspace_bytes, void *stream);
 
 /*
- * Set S slot states [S][3][C] float32 to the empty past
- * (aa = bb = 0, pp = -1e38).
+ * Set S slot states [S][5][C] float32 to the empty past:
+ * aa = bb = 0, base = -1e38, n = 0, ref = 0 (ref is set by the first token).
  */
 wkv_status wkv4_state_init(int64_t S, int64_t C, float *state, void *stream);
 
@@ -162,8 +165,10 @@ wkv_status wkv4_state_init(int64_t S, int64_t C, float *state, void *stream);
  *               slot with no tokens is skipped and its state left untouched.
  *               A slot whose range is decreasing or exceeds n_tokens is
  *               skipped too and WKV_DEVERR_BAD_SLOT is recorded.
- *   state       [S][3][C] float32 (aa, bb, pp per channel, pp base 2), read
- *               and written in place: it carries each slot across calls.
+ *   state       [S][5][C] float32 (aa, bb, base, n, ref per channel), read
+ *               and written in place: it carries each slot across calls. A
+ *               slot whose base is still -1e38 (empty) takes ref from the
+ *               first token it absorbs.
  * Feeding a sequence in several calls gives bit-identical y and state to
  * feeding it in one call, and bit-identical y to wkv4_forward on the same
  * tokens (all three run the same float32 step in the same order).

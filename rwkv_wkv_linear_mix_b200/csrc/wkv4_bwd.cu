@@ -13,9 +13,10 @@
 //                    gw -= e^{k_i} (v_i A'_i - B'_i)
 // A, B, A', B' follow the reverse recurrences A_{i-1} = alpha_i + e^{-w} A_i,
 // A'_{i-1} = e^{-w} (A'_i + A_i). They are carried as mantissas under one
-// shared base-2 exponent r (A = Am * 2^r) that is a running max of the term
-// exponents -q_t - (t-1-i) w, exactly like the forward's pp; then the factor
-// e^{k_i} * 2^r has exponent <= 0 because q_t >= pp_t >= k_i - (t-1-i) w.
+// shared base-2 exponent R (A = Am * 2^R) that is a running max of the term
+// exponents -q_t - (t-1-i) w, kept like the forward's exponent as a base and
+// an exact step count; then the factor e^{k_i} * 2^R has exponent <= 0
+// because q_t >= P_t >= k_i - (t-1-i) w.
 //
 // Kernel shape. One thread per lane, one warp = 32 channels of one sample.
 // Time is walked in reverse, one checkpoint interval (WKV4_CKPT_LEN = 32
@@ -45,6 +46,7 @@ __global__ void __launch_bounds__(32) wkv4_bwd_kernel(const __grid_constant__ CU
                                                       const __grid_constant__ CUtensorMap tg, int T, int C,
                                                       int ncb, const float* __restrict__ w,
                                                       const float* __restrict__ u,
+                                                      const E* __restrict__ kraw,
                                                       const float* __restrict__ ckpt, E* __restrict__ gk,
                                                       E* __restrict__ gv, float* __restrict__ part_gw,
                                                       float* __restrict__ part_gu, unsigned* err) {
@@ -79,17 +81,20 @@ __global__ void __launch_bounds__(32) wkv4_bwd_kernel(const __grid_constant__ CU
   const float w2 = valid ? __fmul_rn(w[c], kLog2e) : 0.f;
   const float u2 = valid ? __fmul_rn(u[c], kLog2e) : 0.f;
   const int64_t lane_off = (int64_t)b * T * C + c;
+  // lane reference exponent: the same value the forward derived from token 0
+  const float ref = valid ? wkv4_ref(Elem<E>::to_f32(kraw[lane_off])) : 0.f;
   const float* ckl = ckpt + (int64_t)b * nck * 3 * C + c;
 
-  // reverse carry: A = Am 2^r etc.; r starts at the "empty" exponent
-  float r2 = kEmptyPP, Am = 0.f, Bm = 0.f, Apm = 0.f, Bpm = 0.f;
+  // reverse carry: A = Am 2^R etc. with R = rbase - rn * w2 (counted decay,
+  // as in the forward); R starts at the "empty" exponent
+  float rbase = kEmptyPP, rn = 0.f, Am = 0.f, Bm = 0.f, Apm = 0.f, Bpm = 0.f;
   float gw_acc = 0.f, gu_acc = 0.f;
 
   // checkpoint of the interval processed next (prefetched one interval ahead)
-  Wkv4State nxt = {0.f, 0.f, 0.f};
+  Wkv4State nxt = {0.f, 0.f, 0.f, 0.f};
   if (valid && nck > 0) {
     const float* p = ckl + (int64_t)(nck - 1) * 3 * C;
-    nxt = {p[0], p[C], p[2 * (int64_t)C]};
+    nxt = {p[0], p[C], p[2 * (int64_t)C], 0.f};
   }
 
   int it = 0;
@@ -101,7 +106,7 @@ __global__ void __launch_bounds__(32) wkv4_bwd_kernel(const __grid_constant__ CU
     Wkv4State st = nxt;
     if (valid && j > 0) {
       const float* p = ckl + (int64_t)(j - 1) * 3 * C;
-      nxt = {p[0], p[C], p[2 * (int64_t)C]};
+      nxt = {p[0], p[C], p[2 * (int64_t)C], 0.f};
     }
     const bool ok = mbar_wait_bounded(&sm.full[s], (it / STAGES) & 1, err);
     if (!__all_sync(0xffffffffu, ok)) break;
@@ -114,8 +119,8 @@ __global__ void __launch_bounds__(32) wkv4_bwd_kernel(const __grid_constant__ CU
         if (jj < n) {
           saa[jj] = st.aa;
           sbb[jj] = st.bb;
-          spp[jj] = st.pp;
-          const float k2 = __fmul_rn(Elem<E>::to_f32(sm.k[s][jj][lane]), kLog2e);
+          spp[jj] = wkv4_exponent(st, w2);
+          const float k2 = wkv4_key(Elem<E>::to_f32(sm.k[s][jj][lane]), ref);
           const float vv = Elem<E>::to_f32(sm.v[s][jj][lane]);
           wkv4_absorb(st, k2, vv, w2);
         }
@@ -126,7 +131,7 @@ __global__ void __launch_bounds__(32) wkv4_bwd_kernel(const __grid_constant__ CU
 #pragma unroll
       for (int jj = kBwdL - 1; jj >= 0; --jj) {
         if (jj < n) {
-          const float k2 = __fmul_rn(Elem<E>::to_f32(sm.k[s][jj][lane]), kLog2e);
+          const float k2 = wkv4_key(Elem<E>::to_f32(sm.k[s][jj][lane]), ref);
           const float vv = Elem<E>::to_f32(sm.v[s][jj][lane]);
           const float g = Elem<E>::to_f32(sm.gy[s][jj][lane]);
           // output of token jj: D = 2^q * den
@@ -148,15 +153,15 @@ __global__ void __launch_bounds__(32) wkv4_bwd_kernel(const __grid_constant__ CU
           float gkv = __fmul_rn(gloc, __fsub_rn(vv, yv));
           gu_acc = __fadd_rn(gu_acc, gkv);
           // tokens after jj, through the carried sums
-          const float f = ex2(__fadd_rn(k2, r2));
+          const float f = ex2(__fadd_rn(k2, __fmaf_rn(-rn, w2, rbase)));
           gvv = __fmaf_rn(f, Am, gvv);
           gkv = __fmaf_rn(f, __fmaf_rn(vv, Am, -Bm), gkv);
           gw_acc = __fmaf_rn(-f, __fmaf_rn(vv, Apm, -Bpm), gw_acc);
           gkl[(int64_t)jj * C] = Elem<E>::from_f32(gkv);
           gvl[(int64_t)jj * C] = Elem<E>::from_f32(gvv);
-          // fold token jj into the carry (new exponent max(r - w, -q))
-          const float older = __fsub_rn(r2, w2);
-          const float dd = __fadd_rn(older, q);  // older - (-q)
+          // fold token jj into the carry (new exponent max(R - w, -q))
+          const float rn1 = __fadd_rn(rn, 1.f);
+          const float dd = __fmaf_rn(-rn1, w2, __fadd_rn(rbase, q));  // (R - w) - (-q)
           const float ef = ex2(-fabsf(dd));
           const bool keep = dd >= 0.f;
           const float fo = keep ? 1.f : ef;
@@ -165,7 +170,8 @@ __global__ void __launch_bounds__(32) wkv4_bwd_kernel(const __grid_constant__ CU
           Bpm = __fmul_rn(fo, __fadd_rn(Bpm, Bm));
           Am = __fmaf_rn(fo, Am, __fmul_rn(fn, alpha));
           Bm = __fmaf_rn(fo, Bm, __fmul_rn(fn, beta));
-          r2 = keep ? older : -q;
+          rbase = keep ? rbase : -q;
+          rn = keep ? rn1 : 0.f;
         }
       }
     }
@@ -210,7 +216,8 @@ static wkv_status run_bwd(const Wkv4BwdArgs& a, cudaStream_t stream, unsigned* e
   float* part_gw = a.part;
   float* part_gu = a.part + a.B * a.C;
   wkv4_bwd_kernel<E, STAGES><<<(unsigned)(ncb * a.B), 32, 0, stream>>>(
-      tk, tv, tg, (int)a.T, (int)a.C, ncb, a.w, a.u, a.ckpt, static_cast<E*>(a.gk), static_cast<E*>(a.gv),
+      tk, tv, tg, (int)a.T, (int)a.C, ncb, a.w, a.u, static_cast<const E*>(a.k), a.ckpt,
+      static_cast<E*>(a.gk), static_cast<E*>(a.gv),
       part_gw, part_gu, err);
   wkv4_reduce_kernel<<<(unsigned)ceil_div(a.C, 256), 256, 0, stream>>>(part_gw, part_gu, (int)a.B, (int)a.C,
                                                                        a.gw, a.gu);

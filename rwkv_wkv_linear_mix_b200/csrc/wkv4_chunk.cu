@@ -3,9 +3,9 @@
 // batched inference: num_batch slots, at most token_chunk_size tokens per
 // run() call, empty slots skipped, state persisting between calls).
 //
-// One warp serves 32 channels of one slot: it loads the slot's (aa, bb, pp)
-// from the persistent state, runs the same float32 step as wkv4_forward over
-// the slot's tokens of this call, writes y and stores the state back. A call
+// One warp serves 32 channels of one slot: it loads the slot's
+// (aa, bb, base, n, ref) from the persistent state, runs the same float32
+// step as wkv4_forward over the slot's tokens of this call, writes y and stores the state back. A call
 // moves at most a few tens of MB, so the kernel is latency bound: each warp
 // issues the loads of a whole group of tokens before it starts computing.
 #include "wkv_device.cuh"
@@ -34,8 +34,10 @@ __global__ void __launch_bounds__(32) wkv4_chunk_kernel(int C, int ncb, const fl
   }
   if (c >= C) return;
 
-  float* sp = state + (int64_t)s * 3 * C + c;
-  Wkv4State st = {sp[0], sp[C], sp[2 * (int64_t)C]};
+  float* sp = state + (int64_t)s * 5 * C + c;
+  Wkv4State st = {sp[0], sp[C], sp[2 * (int64_t)C], sp[3 * (int64_t)C]};
+  // a slot that has absorbed nothing yet takes its reference from this call's first token
+  const float ref = st.base == kEmptyPP ? wkv4_ref(Elem<E>::to_f32(k[beg * C + c])) : sp[4 * (int64_t)C];
   const float w2 = __fmul_rn(w[c], kLog2e);
   const float u2 = __fmul_rn(u[c], kLog2e);
   const E* kp = k + beg * C + c;
@@ -54,27 +56,28 @@ __global__ void __launch_bounds__(32) wkv4_chunk_kernel(int C, int ncb, const fl
 #pragma unroll
     for (int j = 0; j < kChunkGroup; ++j) {
       if (t0 + j < n) {
-        const float k2 = __fmul_rn(kk[j], kLog2e);
-        const float yv = wkv4_output(st, k2, vv[j], u2);
-        wkv4_absorb(st, k2, vv[j], w2);
+        const float k2 = wkv4_key(kk[j], ref);
+        const float yv = wkv4_token(st, k2, vv[j], u2, w2);
         yp[(t0 + j) * C] = Elem<E>::from_f32(yv);
       }
     }
   }
   sp[0] = st.aa;
   sp[C] = st.bb;
-  sp[2 * (int64_t)C] = st.pp;
+  sp[2 * (int64_t)C] = st.base;
+  sp[3 * (int64_t)C] = st.n;
+  sp[4 * (int64_t)C] = ref;
 }
 
 __global__ void wkv4_state_init_kernel(int64_t total, int C, float* __restrict__ state) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= total) return;
-  const int64_t comp = (i / C) % 3;  // 0: aa, 1: bb, 2: pp
+  const int64_t comp = (i / C) % 5;  // 0: aa, 1: bb, 2: base, 3: n, 4: ref
   state[i] = comp == 2 ? kEmptyPP : 0.f;
 }
 
 wkv_status launch_wkv4_state_init(int64_t S, int64_t C, float* state, cudaStream_t stream, const char** why) {
-  const int64_t total = S * 3 * C;
+  const int64_t total = S * 5 * C;
   wkv4_state_init_kernel<<<(unsigned)ceil_div(total, 256), 256, 0, stream>>>(total, (int)C, state);
   if (cudaGetLastError() != cudaSuccess) {
     *why = "wkv4_state_init kernel launch failed";

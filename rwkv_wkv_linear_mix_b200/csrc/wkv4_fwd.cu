@@ -5,7 +5,7 @@
 // running-max recurrence of wkv_device.cuh.
 //
 // Design. The recurrence is sequential in t and independent per lane (b, c),
-// so one thread owns one lane and keeps (aa, bb, pp) in registers for the
+// so one thread owns one lane and keeps its state in registers for the
 // whole sequence. A CTA is one warp = 32 consecutive channels of one sample.
 // The warp streams its [T x 32] slices of k and v through a ring of STAGES
 // shared-memory tiles of LT time steps, filled by 3-D TMA loads (box
@@ -14,7 +14,8 @@
 // has consumed it, so STAGES-1 tiles are always in flight per warp. y is
 // written straight from registers (one 64/128-byte row segment per warp and
 // step). Every WKV4_CKPT_LEN steps the state is written to the checkpoint
-// buffer that the backward pass restarts from.
+// buffer that the backward pass restarts from; its exponent P is relative to the
+// lane reference fl(k[b][0][c] * log2e), which the backward recomputes.
 #include "wkv_device.cuh"
 #include "wkv_internal.h"
 
@@ -61,6 +62,7 @@ __global__ void __launch_bounds__(32) wkv4_fwd_kernel(const __grid_constant__ CU
   const float w2 = valid ? __fmul_rn(w[c], kLog2e) : 0.f;
   const float u2 = valid ? __fmul_rn(u[c], kLog2e) : 0.f;
   Wkv4State st = wkv4_empty_state();
+  float ref = 0.f;  // set from the lane's first key once the first tile lands
   E* yl = y ? y + (int64_t)b * T * C + c : nullptr;
   const int64_t nck = (T + WKV4_CKPT_LEN - 1) / WKV4_CKPT_LEN;
   float* ckl = ckpt ? ckpt + (int64_t)b * nck * 3 * C + c : nullptr;
@@ -73,28 +75,27 @@ __global__ void __launch_bounds__(32) wkv4_fwd_kernel(const __grid_constant__ CU
       float* p = ckl + (int64_t)(t0 / WKV4_CKPT_LEN) * 3 * C;
       p[0] = st.aa;
       p[C] = st.bb;
-      p[2 * (int64_t)C] = st.pp;
+      p[2 * (int64_t)C] = wkv4_exponent(st, w2);
     }
     const bool ok = mbar_wait_bounded(&sm.full[s], (i / STAGES) & 1, err);
     if (!__all_sync(0xffffffffu, ok)) break;
+    if (i == 0) ref = wkv4_ref(Elem<E>::to_f32(sm.k[0][0][lane]));
     const int n = min(LT, T - t0);
     if (valid) {
       E* yt = yl ? yl + (int64_t)t0 * C : nullptr;
       if (n == LT) {
 #pragma unroll 8
         for (int j = 0; j < LT; ++j) {
-          const float k2 = __fmul_rn(Elem<E>::to_f32(sm.k[s][j][lane]), kLog2e);
+          const float k2 = wkv4_key(Elem<E>::to_f32(sm.k[s][j][lane]), ref);
           const float vv = Elem<E>::to_f32(sm.v[s][j][lane]);
-          const float yv = wkv4_output(st, k2, vv, u2);
-          wkv4_absorb(st, k2, vv, w2);
+          const float yv = wkv4_token(st, k2, vv, u2, w2);
           if (yt) yt[(int64_t)j * C] = Elem<E>::from_f32(yv);
         }
       } else {
         for (int j = 0; j < n; ++j) {
-          const float k2 = __fmul_rn(Elem<E>::to_f32(sm.k[s][j][lane]), kLog2e);
+          const float k2 = wkv4_key(Elem<E>::to_f32(sm.k[s][j][lane]), ref);
           const float vv = Elem<E>::to_f32(sm.v[s][j][lane]);
-          const float yv = wkv4_output(st, k2, vv, u2);
-          wkv4_absorb(st, k2, vv, w2);
+          const float yv = wkv4_token(st, k2, vv, u2, w2);
           if (yt) yt[(int64_t)j * C] = Elem<E>::from_f32(yv);
         }
       }

@@ -126,44 +126,82 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
 // ----------------------------------------------------------------------------
 // RWKV-4 step, running-max form in base 2.
 //
-// State of one lane: the past sums a = aa * 2^pp, b = bb * 2^pp. Inputs are
-// pre-scaled by log2(e): k2 = k*log2e, u2 = u*log2e, w2 = w*log2e.
-// Output of token t:  q = max(pp, u2+k2); y = (2^{pp-q} aa + 2^{u2+k2-q} v)
-//                                          / (2^{pp-q} bb + 2^{u2+k2-q})
-// Absorb token t:     q' = max(pp-w2, k2); aa <- 2^{pp-w2-q'} aa + 2^{k2-q'} v,
-//                     bb <- 2^{pp-w2-q'} bb + 2^{k2-q'}, pp <- q'.
-// In each pair one exponent is 0, so a pair costs one ex2 and a select.
+// State of one lane: the past sums a = aa * 2^(P + ref), b = bb * 2^(P + ref)
+// with P = base - n * w2. Three choices keep every exponent accurate to one
+// rounding, however long the sequence and however large the keys:
+//  * ref = fl(k_first * log2e) is a per-lane reference fixed by the first key
+//    the lane absorbs; a key enters as kk = fl(k * log2e - ref) (one fused
+//    multiply-add), so exponents have the size of the key range.
+//  * the decay is counted, not accumulated: while the past keeps the maximum
+//    only the step count n grows, and P is formed with one fused
+//    multiply-add whenever it is needed (repeated P -= w2 would drift by up to
+//    half an ulp per step, always in the same direction).
+//  * each max-pair costs one ex2 and a select (one of its exponents is 0).
+// u2 = u * log2e, w2 = w * log2e. For token t with kk:
+//   output  zo = (u2 + kk) - P;   y = (2^{min(-zo,0)} aa + 2^{min(zo,0)} v)
+//                                   / (2^{min(-zo,0)} bb + 2^{min(zo,0)})
+//   absorb  z1 = kk - (P - w2);   aa <- 2^{min(-z1,0)} aa + 2^{min(z1,0)} v,
+//                                 bb likewise, and (base, n) <- (base, n + 1)
+//                                 if z1 <= 0 else (kk, 0).
 // All roundings are explicit (_rn intrinsics) so that every kernel that runs
 // this step produces bit-identical results from the same state and inputs.
 // ----------------------------------------------------------------------------
 struct Wkv4State {
-  float aa, bb, pp;
+  float aa, bb, base, n;
 };
 
-__device__ __forceinline__ Wkv4State wkv4_empty_state() { return {0.f, 0.f, kEmptyPP}; }
+__device__ __forceinline__ Wkv4State wkv4_empty_state() { return {0.f, 0.f, kEmptyPP, 0.f}; }
 
-__device__ __forceinline__ float wkv4_output(const Wkv4State& s, float k2, float v, float u2) {
-  const float cur = __fadd_rn(u2, k2);
-  const float d = __fsub_rn(s.pp, cur);
-  const float e = ex2(-fabsf(d));
-  const bool past_max = d >= 0.f;
-  const float e1 = past_max ? 1.f : e;
-  const float e2 = past_max ? e : 1.f;
-  const float num = __fmaf_rn(e1, s.aa, __fmul_rn(e2, v));
-  const float den = __fmaf_rn(e1, s.bb, e2);
-  return __fmul_rn(num, rcp(den));
+// Reference exponent of a lane whose first absorbed key is k_first.
+__device__ __forceinline__ float wkv4_ref(float k_first) { return __fmul_rn(k_first, kLog2e); }
+
+// Key in base-2 units relative to the lane reference.
+__device__ __forceinline__ float wkv4_key(float k, float ref) { return __fmaf_rn(k, kLog2e, -ref); }
+
+// Exponent P of the past sums (one rounding).
+__device__ __forceinline__ float wkv4_exponent(const Wkv4State& s, float w2) {
+  return __fmaf_rn(-s.n, w2, s.base);
 }
 
-__device__ __forceinline__ void wkv4_absorb(Wkv4State& s, float k2, float v, float w2) {
-  const float past = __fsub_rn(s.pp, w2);
-  const float d = __fsub_rn(past, k2);
-  const float e = ex2(-fabsf(d));
-  const bool past_max = d >= 0.f;
-  const float e1 = past_max ? 1.f : e;
-  const float e2 = past_max ? e : 1.f;
-  s.aa = __fmaf_rn(e1, s.aa, __fmul_rn(e2, v));
-  s.bb = __fmaf_rn(e1, s.bb, e2);
-  s.pp = past_max ? past : k2;
+// Output of the token, then absorb it. Returns y.
+__device__ __forceinline__ float wkv4_token(Wkv4State& s, float kk, float v, float u2, float w2) {
+  const float y0 = __fsub_rn(kk, s.base);
+  // output pair: current token (u2 + kk) against the past P
+  const float zo = __fmaf_rn(s.n, w2, __fadd_rn(y0, u2));
+  const float eo = ex2(-fabsf(zo));
+  const bool po = zo <= 0.f;  // past holds the maximum
+  const float e1 = po ? 1.f : eo;
+  const float e2 = po ? eo : 1.f;
+  const float num = __fmaf_rn(e1, s.aa, __fmul_rn(e2, v));
+  const float den = __fmaf_rn(e1, s.bb, e2);
+  const float y = __fmul_rn(num, rcp(den));
+  // absorb pair: token kk against the decayed past P - w2
+  const float n1 = __fadd_rn(s.n, 1.f);
+  const float z1 = __fmaf_rn(n1, w2, y0);
+  const float ea = ex2(-fabsf(z1));
+  const bool pa = z1 <= 0.f;
+  const float f1 = pa ? 1.f : ea;
+  const float f2 = pa ? ea : 1.f;
+  s.aa = __fmaf_rn(f1, s.aa, __fmul_rn(f2, v));
+  s.bb = __fmaf_rn(f1, s.bb, f2);
+  s.base = pa ? s.base : kk;
+  s.n = pa ? n1 : 0.f;
+  return y;
+}
+
+// Absorb only (no output).
+__device__ __forceinline__ void wkv4_absorb(Wkv4State& s, float kk, float v, float w2) {
+  const float y0 = __fsub_rn(kk, s.base);
+  const float n1 = __fadd_rn(s.n, 1.f);
+  const float z1 = __fmaf_rn(n1, w2, y0);
+  const float ea = ex2(-fabsf(z1));
+  const bool pa = z1 <= 0.f;
+  const float f1 = pa ? 1.f : ea;
+  const float f2 = pa ? ea : 1.f;
+  s.aa = __fmaf_rn(f1, s.aa, __fmul_rn(f2, v));
+  s.bb = __fmaf_rn(f1, s.bb, f2);
+  s.base = pa ? s.base : kk;
+  s.n = pa ? n1 : 0.f;
 }
 
 }  // namespace wkv

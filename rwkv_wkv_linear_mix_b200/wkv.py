@@ -180,18 +180,21 @@ def wkv4_backward(w, u, k, v, gy, ckpt: Optional[torch.Tensor] = None, *, gk=Non
     return gk, gv, gw, gu
 
 
+STATE_ROWS = 5  # aa, bb, base, n, ref
+
+
 def wkv4_state_init(S: int, C: int, device, state: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """Slot states [S, 3, C] float32 set to the empty past (pp base 2)."""
+    """Slot states [S, 5, C] float32 (aa, bb, base, n, ref) set to the empty past."""
     if state is None:
-        state = torch.empty((S, 3, C), dtype=torch.float32, device=device)
-    _want(state, "state", dtype=torch.float32, shape=(S, 3, C))
+        state = torch.empty((S, STATE_ROWS, C), dtype=torch.float32, device=device)
+    _want(state, "state", dtype=torch.float32, shape=(S, STATE_ROWS, C))
     _check(_lib.wkv4_state_init(S, C, _ptr(state), _stream(state)), "wkv4_state_init")
     return state
 
 
 def wkv4_chunk_step(w, u, k, v, cu_tokens: torch.Tensor, state: torch.Tensor, *, y=None) -> torch.Tensor:
     """One batched inference call. k, v: [N, C] packed tokens of all slots;
-    cu_tokens: int32 [S+1] on the device; state: [S, 3, C] float32 (in/out)."""
+    cu_tokens: int32 [S+1] on the device; state: [S, 5, C] float32 (in/out)."""
     N, C = k.shape
     S = state.shape[0]
     dev = k.device
@@ -200,7 +203,7 @@ def wkv4_chunk_step(w, u, k, v, cu_tokens: torch.Tensor, state: torch.Tensor, *,
     _want(w, "w", dtype=torch.float32, shape=(C,), device=dev)
     _want(u, "u", dtype=torch.float32, shape=(C,), device=dev)
     _want(cu_tokens, "cu_tokens", dtype=torch.int32, shape=(S + 1,), device=dev)
-    _want(state, "state", dtype=torch.float32, shape=(S, 3, C), device=dev)
+    _want(state, "state", dtype=torch.float32, shape=(S, STATE_ROWS, C), device=dev)
     y = torch.empty_like(k) if y is None else y
     _want(y, "y", dtype=k.dtype, shape=k.shape, device=dev)
     _check(_lib.wkv4_chunk_step(S, C, _dtype_code(k), _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(y), N,

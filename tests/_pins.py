@@ -9,17 +9,18 @@ mismatch here.
 import numpy as np
 
 
-def rel_err(x, ref):
-    """max_i |x_i - ref_i| / max(|ref_i|, rms(ref)).
+def rel_err(x, ref, floor=0.0):
+    """max_i |x_i - ref_i| / max(|ref_i|, rms(ref), floor).
 
     The denominator is floored at the RMS of the reference tensor so that
-    entries near zero (cancelling sums) do not dominate.
+    entries near zero (cancelling sums) do not dominate, and at `floor` for
+    references that are zero up to round-off.
     """
     x = np.asarray(x, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     if ref.size == 0:
         return 0.0
-    floor = float(np.sqrt(np.mean(ref ** 2)))
+    floor = max(float(np.sqrt(np.mean(ref ** 2))), floor)
     den = np.maximum(np.abs(ref), floor)
     den = np.where(den == 0, 1.0, den)
     return float(np.max(np.abs(x - ref) / den))

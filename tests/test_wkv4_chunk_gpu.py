@@ -65,8 +65,9 @@ def test_equals_forward_bitwise_and_oracle(W, oracle, slots):
         ref, st = oracle.wkv4_forward(slots["w"], slots["u"], slots["k32"][None, a:b], slots["v32"][None, a:b],
                                       return_state=True)
         assert rel_err(host64(y[a:b]), ref[0]) < TOL["bf16"]
-        aa, bb, pp = (host64(state[s, i]) for i in range(3))
-        np.testing.assert_allclose(np.log(bb) + pp * np.log(2.0), np.log(st["b_end"][0]) + st["kmax"][0],
+        aa, bb, base, n, ref = (host64(state[s, i]) for i in range(5))
+        P = base - n * slots["w"].astype(np.float64) * np.log2(np.e)
+        np.testing.assert_allclose(np.log(bb) + (P + ref) * np.log(2.0), np.log(st["b_end"][0]) + st["kmax"][0],
                                    rtol=0, atol=1e-3)
         assert rel_err(aa / bb, st["a_end"][0] / st["b_end"][0]) < 1e-3
 
@@ -100,3 +101,17 @@ def test_empty_slots_untouched_and_bad_ranges(W):
 def test_state_init_values(W):
     st = W.wkv4_state_init(3, 16, "cuda")
     assert torch.all(st[:, 0] == 0) and torch.all(st[:, 1] == 0) and torch.all(st[:, 2] == -1e38)
+    assert torch.all(st[:, 3] == 0) and torch.all(st[:, 4] == 0)
+
+
+def test_large_keys_keep_precision(W, oracle):
+    # keys shifted by 1000: the per-slot reference keeps the exponents small
+    S, C = 3, 64
+    inp = synth.wkv4_slot_inputs(S=S, C=C, len_lo=40, len_hi=90, dtype="f32", seed=4)
+    k = (inp["k32"] + np.float32(1000.0)).astype(np.float32)
+    y, _ = feed(W, inp, 16, dev(inp["w"]), dev(inp["u"]), dev(k), dev(inp["v32"]))
+    offs = inp["offsets"]
+    for s in range(S):
+        a, b = int(offs[s]), int(offs[s + 1])
+        ref = oracle.wkv4_forward(inp["w"], inp["u"], k[None, a:b], inp["v32"][None, a:b])
+        assert rel_err(host64(y[a:b]), ref[0]) < TOL["f32"]

@@ -130,11 +130,13 @@ def test_checkpoint_state_matches_oracle(W, oracle):
     inp = synth.wkv4_inputs(rec, seed=9)
     _, ck = run_fwd(W, inp, want_ckpt=True)
     ck = host64(ck)
+    # lane reference: fl(k[b, 0, c] * log2 e) in float32
+    ref_exp = (inp["k32"][:, 0, :] * np.float32(1.4426950408889634)).astype(np.float32).astype(np.float64)
     for n in (1, 2):
         t = 32 * n
         _, st = oracle.wkv4_forward(inp["w"], inp["u"], inp["k32"][:, :t], inp["v32"][:, :t], return_state=True)
         log_b = np.log(st["b_end"]) + st["kmax"]
         ratio = st["a_end"] / st["b_end"]
         aa, bb, pp = ck[:, n, 0], ck[:, n, 1], ck[:, n, 2]
-        np.testing.assert_allclose(np.log(bb) + pp * np.log(2.0), log_b, rtol=0, atol=1e-4)
+        np.testing.assert_allclose(np.log(bb) + (pp + ref_exp) * np.log(2.0), log_b, rtol=0, atol=1e-4)
         assert rel_err(aa / bb, ratio) < 1e-4
