@@ -149,8 +149,11 @@ __global__ void __launch_bounds__(32) wkv4_bwd_kernel(const __grid_constant__ CU
           const float alpha = __fmul_rn(g, rd);   // alpha_t * 2^q
           const float beta = __fmul_rn(alpha, yv);  // beta_t * 2^q
           const float gloc = __fmul_rn(alpha, e2);  // gy_t rho_t
+          // v - y = e1 (bb v - aa) / den: no cancellation against v when the
+          // current token dominates (y within rounding of v)
+          const float vmy = __fmul_rn(__fmul_rn(e1, __fmaf_rn(sbb[jj], vv, -saa[jj])), rd);
           float gvv = gloc;
-          float gkv = __fmul_rn(gloc, __fsub_rn(vv, yv));
+          float gkv = __fmul_rn(gloc, vmy);
           gu_acc = __fadd_rn(gu_acc, gkv);
           // tokens after jj, through the carried sums
           const float f = ex2(__fadd_rn(k2, __fmaf_rn(-rn, w2, rbase)));
