@@ -178,6 +178,32 @@ wkv_status wkv4_chunk_step(int64_t S, int64_t C, int dtype,
                            const void *k, const void *v, void *y, int64_t n_tokens,
                            const int32_t *cu_tokens, float *state, void *stream);
 
+/*
+ * wkv4_backward without a workspace argument, for callers that cannot
+ * allocate device memory per call (code behind a plain C interface that only
+ * receives the tensors it reads and writes, or latency-critical loops that
+ * must not call cudaMalloc/cudaFree). The paper (the pages this library
+ * follows) has no counterpart: this is a deployment convenience of the
+ * library, not part of the method.
+ *   Arguments and results are those of wkv4_backward; the workspace is a
+ *   file-scope device array of 4 MiB that every GPU loading the library
+ *   keeps until the process exits.
+ *   Problems needing more than that (2*B*C floats of partial sums, plus the
+ *   checkpoints when ckpt is NULL) return WKV_ERR_UNSUPPORTED: pass ckpt, or
+ *   call wkv4_backward.
+ *   The first call on a device looks up the array's device address (with that
+ *   device current); make that first call before any stream capture.
+ *   All calls share the array: calls whose kernels overlap on the GPU race on
+ *   it and must be serialised by the caller. Nothing in it needs clearing:
+ *   every scratch element a call reads was written earlier in that call.
+ *   Allocates nothing (no cudaMalloc, cudaFree or allocating library call).
+ */
+wkv_status wkv4_backward_noalloc(int64_t B, int64_t T, int64_t C, int dtype,
+                                 const float *w, const float *u,
+                                 const void *k, const void *v, const void *gy,
+                                 const float *ckpt,
+                                 void *gk, void *gv, float *gw, float *gu, void *stream);
+
 /* ------------------------------------------------------------------------ */
 /* RWKV-6                                                                    */
 /* ------------------------------------------------------------------------ */

@@ -90,6 +90,8 @@ wkv_status check_act(int64_t B, int64_t T, int64_t C, int dtype) {
 
 }  // namespace
 
+void set_last_error(const char* why) { t_last_error = why ? why : ""; }
+
 bool encode_tmap_3d(CUtensorMap* map, const void* base, CUtensorMapDataType type, size_t elem_bytes, uint64_t d0,
                     uint64_t d1, uint64_t d2, uint32_t b0, uint32_t b1, uint32_t b2, const char** why) {
   auto fn = encode_fn();

@@ -75,6 +75,9 @@ struct Wkv6FwdArgs {
   void* o;
 };
 
+// Record `why` as the calling thread's wkv_last_error() message.
+void set_last_error(const char* why);
+
 // Each launcher enqueues its kernels on `stream` and returns WKV_OK or an
 // error status with a static message in *why. `err` is the device error word.
 wkv_status launch_wkv4_forward(const Wkv4FwdArgs& a, cudaStream_t stream, unsigned* err, const char** why);

@@ -37,6 +37,7 @@ SIGNATURES = {
     "wkv4_state_init": (_int, [_i64, _i64, _vp, _vp]),
     "wkv4_chunk_step": (_int, [_i64, _i64, _int, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp]),
     "wkv6_forward": (_int, [_i64, _i64, _i64, _i64, _int] + [_vp] * 7 + [_i64, _vp, _vp, _vp]),
+    "wkv4_backward_noalloc": (_int, [_i64, _i64, _i64, _int] + [_vp] * 11),
 }
 
 
@@ -177,6 +178,29 @@ def wkv4_backward(w, u, k, v, gy, ckpt: Optional[torch.Tensor] = None, *, gk=Non
     _check(_lib.wkv4_backward(B, T, C, _dtype_code(k), _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(gy), _ptr(ckpt),
                               _ptr(gk), _ptr(gv), _ptr(gw), _ptr(gu), _ptr(workspace),
                               workspace.numel() * workspace.element_size(), _stream(k)), "wkv4_backward")
+    return gk, gv, gw, gu
+
+
+def wkv4_backward_noalloc(w, u, k, v, gy, ckpt: Optional[torch.Tensor] = None, *, gk=None, gv=None, gw=None,
+                          gu=None):
+    """wkv4_backward with the library's static device scratch instead of a
+    workspace (for callers that cannot allocate per call; see wkv.h).
+    Outputs may be passed in preallocated. Returns (gk, gv, gw, gu)."""
+    B, T, C = k.shape
+    dev = k.device
+    for name, t in (("k", k), ("v", v), ("gy", gy)):
+        _want(t, name, dtype=k.dtype, shape=k.shape, device=dev)
+    _want(w, "w", dtype=torch.float32, shape=(C,), device=dev)
+    _want(u, "u", dtype=torch.float32, shape=(C,), device=dev)
+    if ckpt is not None:
+        _want(ckpt, "ckpt", dtype=torch.float32, shape=ckpt_shape(B, T, C), device=dev)
+    gk = torch.empty_like(k) if gk is None else gk
+    gv = torch.empty_like(k) if gv is None else gv
+    gw = torch.empty(C, dtype=torch.float32, device=dev) if gw is None else gw
+    gu = torch.empty(C, dtype=torch.float32, device=dev) if gu is None else gu
+    _check(_lib.wkv4_backward_noalloc(B, T, C, _dtype_code(k), _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(gy),
+                                      _ptr(ckpt), _ptr(gk), _ptr(gv), _ptr(gw), _ptr(gu), _stream(k)),
+           "wkv4_backward_noalloc")
     return gk, gv, gw, gu
 
 
