@@ -52,16 +52,22 @@ def _stale(target: str, deps) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    """Compile and link the library if any source changed; return its path."""
-    if not force and not _stale(LIB, _deps()):
-        return LIB
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose_ptxas: bool = False, out: str = None, defines=()) -> str:
+    """Compile and link the library if any source changed; return its path.
+
+    `out` and `defines` (e.g. ["WKV4_FWD_STAGES_F32=5"]) build a variant of
+    the launch-shape constants into another file, for tuning."""
+    lib = out or LIB
+    if not force and not _stale(lib, _deps()):
+        return lib
+    bdir = BUILD if out is None else os.path.splitext(out)[0] + "_build"
+    os.makedirs(bdir, exist_ok=True)
     cc = nvcc()
     extra = ["-Xptxas", "-v"] if verbose_ptxas else []
+    extra += [f"-D{d}" for d in defines]
 
     def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+        obj = os.path.join(bdir, os.path.basename(src) + ".o")
         cmd = [cc] + ARCH + NVCC_FLAGS + extra + ["-c", src, "-o", obj]
         res = subprocess.run(cmd, capture_output=True, text=True)
         if res.returncode != 0:
@@ -74,13 +80,13 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
         for _, log in results:
             sys.stderr.write(log)
     objs = [o for o, _ in results]
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [cc] + ARCH + ["-shared", "-o", tmp] + objs
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError(f"link failed:\n{res.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":

@@ -175,7 +175,8 @@ WKV_EXPORT wkv_status wkv4_forward(int64_t B, int64_t T, int64_t C, int dtype, c
 
 WKV_EXPORT size_t wkv4_backward_workspace_bytes(int64_t B, int64_t T, int64_t C, int has_ckpt) {
   if (B <= 0 || T <= 0 || C <= 0) return 0;
-  size_t bytes = 2u * (size_t)B * (size_t)C * sizeof(float);
+  // gw/gu partial sums per (sample, sequence segment, channel)
+  size_t bytes = 2u * (size_t)B * (size_t)wkv4_bwd_segments(B, T, C) * (size_t)C * sizeof(float);
   bytes = (bytes + 255) & ~(size_t)255;
   if (!has_ckpt) bytes += wkv4_ckpt_floats(B, T, C) * sizeof(float);
   return bytes;
@@ -214,7 +215,7 @@ WKV_EXPORT wkv_status wkv4_backward(int64_t B, int64_t T, int64_t C, int dtype, 
   float* part = static_cast<float*>(workspace);
   const float* ck = ckpt;
   if (!ck) {
-    size_t off = (2u * (size_t)B * (size_t)C * sizeof(float) + 255) & ~(size_t)255;
+    size_t off = (2u * (size_t)B * (size_t)wkv4_bwd_segments(B, T, C) * (size_t)C * sizeof(float) + 255) & ~(size_t)255;
     float* regen = reinterpret_cast<float*>(static_cast<char*>(workspace) + off);
     Wkv4FwdArgs fa{B, T, C, dtype, w, u, k, v, nullptr, regen};
     if (wkv_status s = launch_wkv4_forward(fa, st, err, &why)) return fail(s, why);

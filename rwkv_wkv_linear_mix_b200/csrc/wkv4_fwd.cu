@@ -4,118 +4,178 @@
 // time_first, k, v) ("代码连连看——RWKV", section RWKV_TimeMix), evaluated as the
 // running-max recurrence of wkv_device.cuh.
 //
-// Design. The recurrence is sequential in t and independent per lane (b, c),
-// so one thread owns one lane and keeps its state in registers for the
-// whole sequence. A CTA is one warp = 32 consecutive channels of one sample.
-// The warp streams its [T x 32] slices of k and v through a ring of STAGES
-// shared-memory tiles of LT time steps, filled by 3-D TMA loads (box
-// {32 ch, LT steps, 1 sample}; rows past T are zero-filled and ignored) that
-// complete on per-stage mbarriers. Lane 0 refills a stage as soon as the warp
-// has consumed it, so STAGES-1 tiles are always in flight per warp. y is
-// written straight from registers (one 64/128-byte row segment per warp and
-// step). Every WKV4_CKPT_LEN steps the state is written to the checkpoint
-// buffer that the backward pass restarts from; its exponent P is relative to the
-// lane reference fl(k[b][0][c] * log2e), which the backward recomputes.
+// Design. The recurrence is sequential in t and independent per lane (b, c).
+// A warp owns 32 consecutive channels of one sample and keeps their states in
+// registers. When there are too few lanes to fill the GPU, each lane's
+// sequence is split into NSEG segments of whole checkpoint intervals, one
+// one-warp CTA per segment, the NSEG CTAs forming a thread-block cluster:
+//   1. every CTA runs its segment from the empty past (absorb only) and leaves
+//      the segment's own state in shared memory;
+//   2. after a cluster barrier, CTA r reads the states of CTAs 0..r-1 through
+//      distributed shared memory and folds them, each decayed across the
+//      segments after it, into its exact incoming state;
+//   3. every CTA reruns its segment from that state, writing y and the
+//      checkpoints (the second read of k, v mostly hits L2).
+// With NSEG = 1 phases 1-2 vanish and the kernel is the plain sequential scan.
+// k and v stream through a ring of STAGES shared-memory tiles of LT steps,
+// filled by 3-D TMA loads (box {32 ch, LT steps, 1 sample}; rows past the
+// segment are ignored) that complete on per-stage mbarriers; lane 0 refills a
+// stage as soon as the warp has consumed it. y is written straight from
+// registers. Every WKV4_CKPT_LEN steps the state (aa, bb, P) goes to the
+// checkpoint buffer the backward restarts from; P is relative to the lane
+// reference fl(k[b][0][c] * log2e), which the backward recomputes.
 #include "wkv_device.cuh"
 #include "wkv_internal.h"
 
 namespace wkv {
 
 template <class E, int LT, int STAGES>
-struct Wkv4FwdSmem {
+struct alignas(128) Wkv4FwdSmem {
   E k[STAGES][LT][32];
   E v[STAGES][LT][32];
   uint64_t full[STAGES];
+  float seg_aa[32], seg_bb[32], seg_P[32];  // this segment's own state (phase 1)
 };
 
-template <class E, int LT, int STAGES>
-__global__ void __launch_bounds__(32) wkv4_fwd_kernel(const __grid_constant__ CUtensorMap tk,
-                                                      const __grid_constant__ CUtensorMap tv, int T, int C,
-                                                      int ncb, const float* __restrict__ w,
-                                                      const float* __restrict__ u, E* __restrict__ y,
-                                                      float* __restrict__ ckpt, unsigned* err) {
+template <class E, int LT, int STAGES, int NSEG, int NW>
+__global__ void __launch_bounds__(32 * NW) wkv4_fwd_kernel(const __grid_constant__ CUtensorMap tk,
+                                                           const __grid_constant__ CUtensorMap tv,
+                                                           const E* __restrict__ kraw, int T, int C, int ncb,
+                                                           int ngroups, const float* __restrict__ w,
+                                                           const float* __restrict__ u, E* __restrict__ y,
+                                                           float* __restrict__ ckpt, unsigned* err) {
   static_assert(WKV4_CKPT_LEN % LT == 0, "checkpoint interval must be a whole number of tiles");
-  __shared__ __align__(128) Wkv4FwdSmem<E, LT, STAGES> sm;
+  extern __shared__ __align__(128) unsigned char wkv4_fwd_dsmem[];
+  // each warp is an independent lane group with its own ring and barriers
+  Wkv4FwdSmem<E, LT, STAGES>& sm = reinterpret_cast<Wkv4FwdSmem<E, LT, STAGES>*>(wkv4_fwd_dsmem)[threadIdx.x / 32];
   constexpr uint32_t kStageBytes = 2u * LT * 32u * sizeof(E);
+  constexpr int kPasses = NSEG > 1 ? 2 : 1;
 
-  const int lane = threadIdx.x;
-  const int cb = blockIdx.x % ncb;
-  const int b = blockIdx.x / ncb;
+  const int lane = threadIdx.x % 32;
+  const int seg = NSEG > 1 ? (int)(blockIdx.x % NSEG) : 0;  // == cluster rank (1-D clusters)
+  const int group = (blockIdx.x / NSEG) * NW + threadIdx.x / 32;
+  const bool active = group < ngroups;  // a warp past the last group only joins the cluster barriers
+  const int cb = group % ncb;
+  const int b = group / ncb;
   const int c0 = cb * 32;
   const int c = c0 + lane;
-  const bool valid = c < C;
-  const int nchunk = (T + LT - 1) / LT;
+  const bool valid = active && c < C;
+  const int nck = (T + WKV4_CKPT_LEN - 1) / WKV4_CKPT_LEN;
+  const int t_beg = wkv4_seg_begin(seg, NSEG, nck) * WKV4_CKPT_LEN;
+  const int t_end = min(T, wkv4_seg_begin(seg + 1, NSEG, nck) * WKV4_CKPT_LEN);
+  const int ntile = (active && t_end > t_beg) ? (t_end - t_beg + LT - 1) / LT : 0;
+  const int total = kPasses * ntile;  // tiles streamed through the ring
 
+  auto issue = [&](int q) {
+    const int s = q % STAGES;
+    const int t = t_beg + (q % ntile) * LT;
+    mbar_arrive_expect_tx(&sm.full[s], kStageBytes);
+    tma_load_3d(&sm.k[s][0][0], &tk, &sm.full[s], c0, t, b);
+    tma_load_3d(&sm.v[s][0][0], &tv, &sm.full[s], c0, t, b);
+  };
   if (lane == 0) {
     tma_prefetch_desc(&tk);
     tma_prefetch_desc(&tv);
     for (int s = 0; s < STAGES; ++s) mbar_init(&sm.full[s], 1);
     mbar_init_fence();
-    for (int s = 0; s < STAGES && s < nchunk; ++s) {
-      mbar_arrive_expect_tx(&sm.full[s], kStageBytes);
-      tma_load_3d(&sm.k[s][0][0], &tk, &sm.full[s], c0, s * LT, b);
-      tma_load_3d(&sm.v[s][0][0], &tv, &sm.full[s], c0, s * LT, b);
-    }
+    for (int q = 0; q < STAGES && q < total; ++q) issue(q);
   }
   __syncwarp();
 
+  const int64_t lane_off = valid ? (int64_t)b * T * C + c : 0;
   const float w2 = valid ? __fmul_rn(w[c], kLog2e) : 0.f;
   const float u2 = valid ? __fmul_rn(u[c], kLog2e) : 0.f;
-  Wkv4State st = wkv4_empty_state();
-  float ref = 0.f;  // set from the lane's first key once the first tile lands
-  E* yl = y ? y + (int64_t)b * T * C + c : nullptr;
-  const int64_t nck = (T + WKV4_CKPT_LEN - 1) / WKV4_CKPT_LEN;
+  const float ref = valid ? wkv4_ref(Elem<E>::to_f32(kraw[lane_off])) : 0.f;
   float* ckl = ckpt ? ckpt + (int64_t)b * nck * 3 * C + c : nullptr;
 
-  int i = 0;
-  for (; i < nchunk; ++i) {
-    const int s = i % STAGES;
-    const int t0 = i * LT;
+  int q = 0;          // next tile to consume
+  bool ok = true;     // every wait so far completed
+  auto acquire = [&](int qq) {
+    const bool got = mbar_wait_bounded(&sm.full[qq % STAGES], (qq / STAGES) & 1, err);
+    ok = __all_sync(0xffffffffu, got);
+    return ok;
+  };
+  auto release = [&](int qq) {
+    __syncwarp();
+    if (lane == 0 && qq + STAGES < total) issue(qq + STAGES);
+  };
+
+  Wkv4State st = wkv4_empty_state();
+  if constexpr (NSEG > 1) {
+    // ---- phase 1: this segment from the empty past ----
+    for (; ok && q < ntile; ++q) {
+      if (!acquire(q)) break;
+      const int s = q % STAGES;
+      const int n = min(LT, t_end - (t_beg + q * LT));
+      if (valid) {
+#pragma unroll 4
+        for (int j = 0; j < n; ++j)
+          wkv4_absorb(st, wkv4_key(Elem<E>::to_f32(sm.k[s][j][lane]), ref), Elem<E>::to_f32(sm.v[s][j][lane]), w2);
+      }
+      release(q);
+    }
+    sm.seg_aa[lane] = st.aa;
+    sm.seg_bb[lane] = st.bb;
+    sm.seg_P[lane] = wkv4_exponent(st, w2);
+    cluster_arrive_release();
+    cluster_wait_acquire();
+    // ---- phase 2: fold the segments before this one into the incoming state ----
+    Wkv4Sum in = {0.f, 0.f, kEmptyPP};
+    for (int r = 0; r < seg; ++r) {
+      const int len = min(T, wkv4_seg_begin(r + 1, NSEG, nck) * WKV4_CKPT_LEN) -
+                      wkv4_seg_begin(r, NSEG, nck) * WKV4_CKPT_LEN;
+      const Wkv4Sum own = {ld_shared_cluster(map_shared_rank(&sm.seg_aa[lane], r)),
+                           ld_shared_cluster(map_shared_rank(&sm.seg_bb[lane], r)),
+                           ld_shared_cluster(map_shared_rank(&sm.seg_P[lane], r))};
+      in.P = __fmaf_rn(-(float)len, w2, in.P);  // decay the earlier part across segment r
+      in = wkv4_merge(in, own);
+    }
+    cluster_arrive_release();  // done reading peers; waited for before exit
+    st = {in.aa, in.bb, in.P, 0.f};
+  }
+
+  // ---- last pass: outputs and checkpoints ----
+  E* yl = y ? y + lane_off : nullptr;
+  for (; ok && q < total; ++q) {
+    const int t0 = t_beg + (q % ntile) * LT;
     if (ckl && valid && (t0 % WKV4_CKPT_LEN) == 0) {
       float* p = ckl + (int64_t)(t0 / WKV4_CKPT_LEN) * 3 * C;
       p[0] = st.aa;
       p[C] = st.bb;
       p[2 * (int64_t)C] = wkv4_exponent(st, w2);
     }
-    const bool ok = mbar_wait_bounded(&sm.full[s], (i / STAGES) & 1, err);
-    if (!__all_sync(0xffffffffu, ok)) break;
-    if (i == 0) ref = wkv4_ref(Elem<E>::to_f32(sm.k[0][0][lane]));
-    const int n = min(LT, T - t0);
+    if (!acquire(q)) break;
+    const int s = q % STAGES;
+    const int n = min(LT, t_end - t0);
     if (valid) {
       E* yt = yl ? yl + (int64_t)t0 * C : nullptr;
       if (n == LT) {
 #pragma unroll 8
         for (int j = 0; j < LT; ++j) {
-          const float k2 = wkv4_key(Elem<E>::to_f32(sm.k[s][j][lane]), ref);
-          const float vv = Elem<E>::to_f32(sm.v[s][j][lane]);
-          const float yv = wkv4_token(st, k2, vv, u2, w2);
+          const float yv = wkv4_token(st, wkv4_key(Elem<E>::to_f32(sm.k[s][j][lane]), ref),
+                                      Elem<E>::to_f32(sm.v[s][j][lane]), u2, w2);
           if (yt) yt[(int64_t)j * C] = Elem<E>::from_f32(yv);
         }
       } else {
         for (int j = 0; j < n; ++j) {
-          const float k2 = wkv4_key(Elem<E>::to_f32(sm.k[s][j][lane]), ref);
-          const float vv = Elem<E>::to_f32(sm.v[s][j][lane]);
-          const float yv = wkv4_token(st, k2, vv, u2, w2);
+          const float yv = wkv4_token(st, wkv4_key(Elem<E>::to_f32(sm.k[s][j][lane]), ref),
+                                      Elem<E>::to_f32(sm.v[s][j][lane]), u2, w2);
           if (yt) yt[(int64_t)j * C] = Elem<E>::from_f32(yv);
         }
       }
     }
-    __syncwarp();
-    if (lane == 0 && i + STAGES < nchunk) {
-      const int tn = (i + STAGES) * LT;
-      mbar_arrive_expect_tx(&sm.full[s], kStageBytes);
-      tma_load_3d(&sm.k[s][0][0], &tk, &sm.full[s], c0, tn, b);
-      tma_load_3d(&sm.v[s][0][0], &tv, &sm.full[s], c0, tn, b);
-    }
+    release(q);
   }
-  if (i < nchunk && lane == 0) {
+  if (!ok && lane == 0) {
     // A wait gave up: let the copies still in flight land before the CTA's
     // shared memory is released (each wait is itself bounded).
-    for (int j = i; j < nchunk && j < i + STAGES; ++j) mbar_wait_bounded(&sm.full[j % STAGES], (j / STAGES) & 1, err);
+    for (int qq = q; qq < total && qq < q + STAGES; ++qq)
+      mbar_wait_bounded(&sm.full[qq % STAGES], (qq / STAGES) & 1, err);
   }
+  if constexpr (NSEG > 1) cluster_wait_acquire();  // peers may still read this CTA's segment state
 }
 
-template <class E, int LT, int STAGES>
+template <class E, int LT, int STAGES, int NSEG, int NW>
 static wkv_status run_fwd(const Wkv4FwdArgs& a, cudaStream_t stream, unsigned* err, const char** why) {
   CUtensorMap tk, tv;
   const CUtensorMapDataType ty = Elem<E>::tma_type;
@@ -123,19 +183,68 @@ static wkv_status run_fwd(const Wkv4FwdArgs& a, cudaStream_t stream, unsigned* e
       !encode_tmap_3d(&tv, a.v, ty, sizeof(E), a.C, a.T, a.B, 32, LT, 1, why))
     return WKV_ERR_INVALID_ARG;
   const int ncb = (int)ceil_div(a.C, 32);
-  const dim3 grid((unsigned)(ncb * a.B));
-  wkv4_fwd_kernel<E, LT, STAGES><<<grid, 32, 0, stream>>>(tk, tv, (int)a.T, (int)a.C, ncb, a.w, a.u,
-                                                          static_cast<E*>(a.y), a.ckpt, err);
-  if (cudaGetLastError() != cudaSuccess) {
+  const int ngroups = (int)(ncb * a.B);
+  auto kern = wkv4_fwd_kernel<E, LT, STAGES, NSEG, NW>;
+  const size_t smem = NW * sizeof(Wkv4FwdSmem<E, LT, STAGES>);
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
+    *why = "wkv4_forward: shared memory configuration failed";
+    return WKV_ERR_CUDA;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(ceil_div(ngroups, NW) * NSEG));
+  cfg.blockDim = dim3(32 * NW);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  if (NSEG > 1) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = NSEG;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tk, tv, static_cast<const E*>(a.k), (int)a.T, (int)a.C, ncb,
+                                           ngroups, a.w, a.u, static_cast<E*>(a.y), a.ckpt, err);
+  if (e != cudaSuccess) {
     *why = "wkv4_forward kernel launch failed";
     return WKV_ERR_CUDA;
   }
   return WKV_OK;
 }
 
+template <class E, int LT, int STAGES, int NSEG>
+static wkv_status run_fwd_nw(const Wkv4FwdArgs& a, cudaStream_t stream, unsigned* err, const char** why) {
+  switch (wkv4_warps_per_cta(a.B, a.C, NSEG)) {
+    case 4: return run_fwd<E, LT, STAGES, NSEG, 4>(a, stream, err, why);
+    case 2: return run_fwd<E, LT, STAGES, NSEG, 2>(a, stream, err, why);
+    default: return run_fwd<E, LT, STAGES, NSEG, 1>(a, stream, err, why);
+  }
+}
+
+template <class E, int LT, int STAGES>
+static wkv_status run_fwd_nseg(const Wkv4FwdArgs& a, cudaStream_t stream, unsigned* err, const char** why) {
+  switch (wkv4_fwd_segments(a.B, a.T, a.C)) {
+    case 8: return run_fwd_nw<E, LT, STAGES, 8>(a, stream, err, why);
+    case 4: return run_fwd_nw<E, LT, STAGES, 4>(a, stream, err, why);
+    case 2: return run_fwd_nw<E, LT, STAGES, 2>(a, stream, err, why);
+    default: return run_fwd<E, LT, STAGES, 1, 1>(a, stream, err, why);
+  }
+}
+
+// Ring depth: each warp consumes its stream quickly relative to the ~1 us
+// load latency, so several tiles must be in flight per warp.
+#ifndef WKV4_FWD_STAGES_F32
+#define WKV4_FWD_STAGES_F32 3
+#endif
+#ifndef WKV4_FWD_STAGES_BF16
+#define WKV4_FWD_STAGES_BF16 3
+#endif
+
 wkv_status launch_wkv4_forward(const Wkv4FwdArgs& a, cudaStream_t stream, unsigned* err, const char** why) {
-  if (a.dtype == WKV_BF16) return run_fwd<__nv_bfloat16, 32, 3>(a, stream, err, why);
-  return run_fwd<float, 16, 3>(a, stream, err, why);
+  if (a.dtype == WKV_BF16) return run_fwd_nseg<__nv_bfloat16, 32, WKV4_FWD_STAGES_BF16>(a, stream, err, why);
+  return run_fwd_nseg<float, 16, WKV4_FWD_STAGES_F32>(a, stream, err, why);
 }
 
 }  // namespace wkv

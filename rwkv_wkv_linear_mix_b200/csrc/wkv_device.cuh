@@ -124,6 +124,34 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
 }
 
 // ----------------------------------------------------------------------------
+// thread-block clusters and distributed shared memory
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// All threads of every CTA of the cluster arrive (release: this CTA's shared
+// memory writes become visible to the cluster) / wait (acquire).
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait_acquire() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Address of the same shared-memory object in the CTA of cluster rank `rank`.
+__device__ __forceinline__ uint32_t map_shared_rank(const void* p, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+  return a;
+}
+__device__ __forceinline__ float ld_shared_cluster(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+// ----------------------------------------------------------------------------
 // RWKV-4 step, running-max form in base 2.
 //
 // State of one lane: the past sums a = aa * 2^(P + ref), b = bb * 2^(P + ref)
@@ -187,6 +215,20 @@ __device__ __forceinline__ float wkv4_token(Wkv4State& s, float kk, float v, flo
   s.base = pa ? s.base : kk;
   s.n = pa ? n1 : 0.f;
   return y;
+}
+
+// Merge two states of the same lane given in the same reference: the result
+// represents the sum of both (max-combine of their exponents P1, P2).
+struct Wkv4Sum {
+  float aa, bb, P;
+};
+__device__ __forceinline__ Wkv4Sum wkv4_merge(const Wkv4Sum& x, const Wkv4Sum& y) {
+  const float d = __fsub_rn(x.P, y.P);
+  const float e = ex2(-fabsf(d));
+  const bool xm = d >= 0.f;
+  const float fx = xm ? 1.f : e;
+  const float fy = xm ? e : 1.f;
+  return {__fmaf_rn(fx, x.aa, __fmul_rn(fy, y.aa)), __fmaf_rn(fx, x.bb, __fmul_rn(fy, y.bb)), xm ? x.P : y.P};
 }
 
 // Absorb only (no output).

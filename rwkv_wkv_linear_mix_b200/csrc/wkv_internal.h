@@ -13,6 +13,54 @@ namespace wkv {
 
 __host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// Launch-shape constants of the RWKV-4 kernels (build-time tunables).
+#ifndef WKV4_TARGET_WARPS
+#define WKV4_TARGET_WARPS (148 * 8)  // warps wanted in flight: 8 per SM of a B200
+#endif
+#ifndef WKV4_FWD_MAX_SEGMENTS
+#define WKV4_FWD_MAX_SEGMENTS 8
+#endif
+#ifndef WKV4_BWD_MAX_SEGMENTS
+#define WKV4_BWD_MAX_SEGMENTS 8
+#endif
+
+// Number of sequence segments each RWKV-4 lane is split into (the cluster
+// size of a kernel): doubled while the launch has fewer warps than
+// WKV4_TARGET_WARPS and every segment keeps at least two checkpoint
+// intervals; at most max_seg (<= 8, the portable cluster size).
+inline int wkv4_segments_capped(int64_t B, int64_t T, int64_t C, int max_seg) {
+  const int64_t groups = B * ceil_div(C, 32);
+  const int64_t nck = ceil_div(T, WKV4_CKPT_LEN);
+  int nseg = 1;
+  while (nseg < max_seg && groups * nseg < (int64_t)(WKV4_TARGET_WARPS) && nck >= 4 * nseg) nseg *= 2;
+  return nseg;
+}
+// Warps (independent 32-channel lane groups) per CTA of a split launch: the
+// GPU keeps only ~140 clusters resident at once, so a split launch packs
+// several lane groups into each CTA to stay within one wave of clusters.
+#ifndef WKV4_MAX_CLUSTERS
+#define WKV4_MAX_CLUSTERS 128
+#endif
+inline int wkv4_warps_per_cta(int64_t B, int64_t C, int nseg) {
+  if (nseg == 1) return 1;
+  const int64_t groups = B * ceil_div(C, 32);
+  int nw = 1;
+  while (nw < 4 && ceil_div(groups, nw) > WKV4_MAX_CLUSTERS) nw *= 2;
+  return nw;
+}
+
+inline int wkv4_fwd_segments(int64_t B, int64_t T, int64_t C) {
+  return wkv4_segments_capped(B, T, C, WKV4_FWD_MAX_SEGMENTS);
+}
+inline int wkv4_bwd_segments(int64_t B, int64_t T, int64_t C) {
+  return wkv4_segments_capped(B, T, C, WKV4_BWD_MAX_SEGMENTS);
+}
+
+// Segment s of nseg covers checkpoint intervals [seg_begin(s), seg_begin(s+1)).
+__host__ __device__ __forceinline__ int wkv4_seg_begin(int s, int nseg, int nck) {
+  return (int)(((int64_t)s * nck) / nseg);
+}
+
 // Encode a 3-D tiled TMA descriptor over a dense row-major tensor with
 // dims {d0 (innermost), d1, d2} of `elem_bytes`-byte elements, box
 // {b0, b1, b2}, no swizzle, out-of-bounds elements filled with zero.
@@ -45,7 +93,7 @@ struct Wkv4BwdArgs {
   void* gv;
   float* gw;
   float* gu;
-  float* part;  // [2][B][C] scratch
+  float* part;  // [2][B * wkv4_bwd_segments(B, T, C)][C] scratch
 };
 
 struct Wkv4ChunkArgs {

@@ -39,7 +39,9 @@ def check(grads, ref, dtype, tol_param=None):
     assert rel_err(gu, rgu) < tp, "gu"
 
 
-SHAPES = [(2, 64, 128), (3, 100, 72), (1, 1, 8), (2, 33, 40), (1, 257, 264), (2, 500, 32)]
+SHAPES = [(2, 64, 128), (3, 100, 72), (1, 1, 8), (2, 33, 40), (1, 257, 264), (2, 500, 32),
+          # 257 lane groups split 4 ways: 4 warps per CTA, the last CTA with one active warp
+          (1, 300, 8200)]
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])

@@ -52,14 +52,32 @@ def test_chunked_equals_whole_bitwise(W, slots):
     assert W.device_error(reset=True) == 0
 
 
-def test_equals_forward_bitwise_and_oracle(W, oracle, slots):
+def test_equals_forward_and_oracle(W, oracle, slots):
     w, u, k, v = dev(slots["w"]), dev(slots["u"]), dev(slots["k"]), dev(slots["v"])
     y, state = feed(W, slots, 32, w, u, k, v)
     offs = slots["offsets"]
+    n_exact = 0
     for s in range(len(slots["lengths"])):
         a, b = int(offs[s]), int(offs[s + 1])
         yf = W.wkv4_forward(w, u, k[a:b][None].contiguous(), v[a:b][None].contiguous())
-        assert torch.equal(yf[0], y[a:b]), f"slot {s}"
+        if b - a <= 64:
+            # wkv4_forward runs one segment here (sequential schedule): the same
+            # float32 steps in the same order, so y is bit-identical
+            assert torch.equal(yf[0], y[a:b]), f"slot {s}"
+            n_exact += 1
+        else:
+            # the forward splits the sequence across a cluster; merging the
+            # segments reorders rounding, so compare within the tolerance
+            assert rel_err(host64(yf[0]), host64(y[a:b])) < TOL["bf16"], f"slot {s}"
+    short = {"w": slots["w"], "u": slots["u"], "lengths": np.array([1, 17, 33, 64])}
+    short["offsets"] = np.concatenate([[0], np.cumsum(short["lengths"])])
+    ks = k[: int(short["offsets"][-1])].contiguous()
+    vs = v[: int(short["offsets"][-1])].contiguous()
+    ys, _ = feed(W, short, 32, w, u, ks, vs)
+    for s in range(4):
+        a, b = int(short["offsets"][s]), int(short["offsets"][s + 1])
+        yf = W.wkv4_forward(w, u, ks[a:b][None].contiguous(), vs[a:b][None].contiguous())
+        assert torch.equal(yf[0], ys[a:b]), f"short slot {s}"
     for s in (0, 5, 17, 31):
         a, b = int(offs[s]), int(offs[s + 1])
         ref, st = oracle.wkv4_forward(slots["w"], slots["u"], slots["k32"][None, a:b], slots["v32"][None, a:b],

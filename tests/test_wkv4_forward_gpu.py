@@ -28,6 +28,8 @@ def run_fwd(W, inp, **kw):
 SHAPES = [
     # (B, T, C): several tiles, ragged T and C tails, one-token and one-warp cases
     (2, 64, 128), (3, 100, 72), (1, 1, 8), (2, 33, 40), (1, 257, 264), (4, 31, 96), (1, 1000, 32),
+    # 257 lane groups split 4 ways: 4 warps per CTA, the last CTA with one active warp
+    (1, 300, 8200),
 ]
 
 
