@@ -16,7 +16,11 @@ Printed (rank 0, one JSON line): G tok*ch/s = B*T*C*N / step time, the
 end-to-end figure through the C ABI with pinned host buffers, the roofline of
 the dominant kernel (the backward) against the measured HBM bandwidth, the
 fp64 CPU oracle timed on a bounded sample, SM clocks sampled during the timed
-region, and the number of library kernels launched.
+region, and the number of library kernels launched. Under "workloads" the
+same line carries secondary single-kernel measurements (rank 0, N=1): the
+RWKV-4 fwd/bwd at the 3B width and at C=4096 (f32 and bf16) against the HBM
+peak, the 32-slot chunk step (eager and as one CUDA-graph replay), and the
+RWKV-6 head-state forward.
 
 --impl reference times the fp64 CPU oracle (the only reference this project
 has) on the same workload and metric.
@@ -52,6 +56,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the secondary workloads (larger shapes, chunk step, RWKV-6)")
     return ap.parse_args()
 
 
@@ -163,7 +169,7 @@ def cpu_baseline(inp, budget_s=12.0):
     t_total = 0.0
     c0 = 0
     slices = 0
-    while t_total < budget_s and slices < 64:
+    while t_total < budget_s and slices < 4096:
         cs = slice(c0, min(C, c0 + width))
         args = (inp["w"][cs], inp["u"][cs], inp["k32"][:, :, cs], inp["v32"][:, :, cs])
         t = time.perf_counter()
@@ -218,6 +224,131 @@ def run_reference(args):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+# ----------------------------------------------------------------------------
+# secondary workloads (same JSON line, under "workloads")
+# ----------------------------------------------------------------------------
+
+def _events_ms(fn, reps, flush, stream):
+    """Median CUDA-event time of fn() over `reps` runs, L2 flushed before each."""
+    import torch
+    out = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        out.append(a.elapsed_time(b))
+    out.sort()
+    return out[len(out) // 2]
+
+
+def secondary(dev, flush, peak):
+    """fwd/bwd of the larger RWKV-4 shapes, the slot chunk step and the RWKV-6
+    forward, each timed alone (median of a few L2-flushed launches). Inputs are
+    drawn on the device from a seeded generator with the same distributions as
+    synth's recipes (timing only; these sizes are parity-checked in tests/)."""
+    import torch
+    from rwkv_wkv_linear_mix_b200 import synth, wkv
+    stream = torch.cuda.current_stream(dev)
+    g = torch.Generator(device=dev)
+    res = {}
+    for name in ("wkv4_fb_bf16_3b", "wkv4_fb_f32_c4096", "wkv4_fb_bf16_c4096"):
+        rec = synth.WKV4_RECIPES[name]
+        g.manual_seed(0)
+        B, T, C = rec.B, rec.T, rec.C
+        dt = torch.float32 if rec.dtype == "f32" else torch.bfloat16
+        w = torch.exp(torch.rand(C, device=dev, generator=g) * (rec.td_hi - rec.td_lo) + rec.td_lo)
+        u = torch.rand(C, device=dev, generator=g) * (rec.u_hi - rec.u_lo) + rec.u_lo
+        k = (torch.randn(B, T, C, device=dev, generator=g) * rec.k_std).to(dt)
+        v = torch.randn(B, T, C, device=dev, generator=g).to(dt)
+        gy = torch.randn(B, T, C, device=dev, generator=g).to(dt)
+        y, gk, gv = torch.empty_like(k), torch.empty_like(k), torch.empty_like(k)
+        gw, gu = torch.empty(C, device=dev), torch.empty(C, device=dev)
+        ck = torch.empty(wkv.ckpt_shape(B, T, C), device=dev)
+        ws = torch.empty(max(16, wkv.wkv4_backward_workspace_bytes(B, T, C, True)), dtype=torch.uint8, device=dev)
+        fwd = lambda: wkv.wkv4_forward(w, u, k, v, y=y, ckpt=ck)
+        bwd = lambda: wkv.wkv4_backward(w, u, k, v, gy, ck, gk=gk, gv=gv, gw=gw, gu=gu, workspace=ws)
+        fwd(); bwd()
+        tf = _events_ms(fwd, 5, flush, stream)
+        tb = _events_ms(bwd, 5, flush, stream)
+        n = B * T * C
+        es = 4 if rec.dtype == "f32" else 2
+        gf, gb = 3 * es * n / (tf * 1e-3) / 1e9, 5 * es * n / (tb * 1e-3) / 1e9
+        res[name] = {"B": B, "T": T, "C": C, "dtype": rec.dtype, "fwd_ms": tf, "bwd_ms": tb,
+                     "fwd_GBps": gf, "bwd_GBps": gb, "fwd_frac": gf / peak, "bwd_frac": gb / peak,
+                     "fwd_bwd_Gtokch_per_s": n / ((tf + tb) * 1e-3) / 1e9}
+        del k, v, gy, y, gk, gv, ck, ws
+        torch.cuda.empty_cache()
+
+    # batched inference slots: 32 slots, prompts ~U{1..512}, <= 32 tokens per call
+    S, C = 32, 4096
+    inp = synth.wkv4_slot_inputs(S=S, C=C, dtype="bf16", seed=0)
+    to_bf16 = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+    w, u = torch.from_numpy(inp["w"]).to(dev), torch.from_numpy(inp["u"]).to(dev)
+    kall, vall = to_bf16(inp["k"]), to_bf16(inp["v"])
+    calls = []
+    done = np.zeros(S, np.int64)
+    for take in synth.feed_schedule(inp["lengths"], 32):
+        idx = np.concatenate([np.arange(inp["offsets"][s] + done[s], inp["offsets"][s] + done[s] + take[s])
+                              for s in range(S)])
+        it = torch.from_numpy(idx).to(dev)
+        cu = torch.from_numpy(np.concatenate([[0], np.cumsum(take)]).astype(np.int32)).to(dev)
+        calls.append((kall[it].contiguous(), vall[it].contiguous(), torch.empty(len(idx), C, dtype=torch.bfloat16,
+                                                                               device=dev), cu))
+        done += take
+    state = wkv.wkv4_state_init(S, C, dev)
+
+    def run_calls():
+        wkv.wkv4_state_init(S, C, dev, state=state)
+        for kc, vc, yc, cu in calls:
+            wkv.wkv4_chunk_step(w, u, kc, vc, cu, state, y=yc)
+
+    run_calls()
+    t_eager = _events_ms(run_calls, 5, flush, stream)
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        run_calls()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph, stream=side):
+            run_calls()
+    torch.cuda.synchronize()
+    t_graph = _events_ms(graph.replay, 5, flush, stream)
+    ntok = int(inp["lengths"].sum())
+    res["wkv4_chunk_step_bf16_slots32"] = {
+        "S": S, "C": C, "tokens": ntok, "calls": len(calls),
+        "eager_ms": t_eager, "graph_ms": t_graph, "per_call_us_graph": 1e3 * t_graph / len(calls),
+        "Gtokch_per_s_graph": ntok * C / (t_graph * 1e-3) / 1e9,
+        "GBps_graph": (6 * ntok * C + 40 * S * C * len(calls)) / (t_graph * 1e-3) / 1e9}
+    del graph
+    torch.cuda.empty_cache()
+
+    # RWKV-6 head-state forward
+    rec = synth.WKV6_RECIPES["wkv6_fwd_bf16_c2048"]
+    B, T, H = rec.B, rec.T, rec.H
+    g.manual_seed(0)
+    HK = H * 64
+    d = torch.randn(B, T, HK, device=dev, generator=g) * rec.d_std + rec.d_mean
+    w6 = torch.exp(-torch.exp(d)).to(torch.bfloat16)
+    del d
+    r6, k6, v6 = (torch.randn(B, T, HK, device=dev, generator=g).to(torch.bfloat16) for _ in range(3))
+    u6 = torch.rand(HK, device=dev, generator=g) * 2 - 1
+    o6 = torch.empty_like(r6)
+    fs6 = torch.empty(B, H, 64, 64, device=dev)
+    f6 = lambda: wkv.wkv6_forward(r6, k6, v6, w6, u6, o=o6, final_state=fs6)
+    f6()
+    t6 = _events_ms(f6, 3, flush, stream)
+    n6 = B * T * HK
+    res["wkv6_fwd_bf16_c2048"] = {"B": B, "T": T, "H": H, "K": 64, "fwd_ms": t6,
+                                  "GBps": 10 * n6 / (t6 * 1e-3) / 1e9, "frac": 10 * n6 / (t6 * 1e-3) / 1e9 / peak,
+                                  "Gtokch_per_s": n6 / (t6 * 1e-3) / 1e9}
+    assert wkv.device_error(reset=True) == 0, "a kernel recorded a device-side error"
+    return res
 
 
 # ----------------------------------------------------------------------------
@@ -357,6 +488,8 @@ def run_ours(args):
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
+    if rank == 0 and world == 1 and not args.no_secondary:
+        line["workloads"] = secondary(dev, flush, peak)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(inp)
     if rank == 0:
