@@ -93,7 +93,8 @@ wkv_status check_act(int64_t B, int64_t T, int64_t C, int dtype) {
 void set_last_error(const char* why) { t_last_error = why ? why : ""; }
 
 bool encode_tmap_3d(CUtensorMap* map, const void* base, CUtensorMapDataType type, size_t elem_bytes, uint64_t d0,
-                    uint64_t d1, uint64_t d2, uint32_t b0, uint32_t b1, uint32_t b2, const char** why) {
+                    uint64_t d1, uint64_t d2, uint32_t b0, uint32_t b1, uint32_t b2, const char** why,
+                    bool swizzle128) {
   auto fn = encode_fn();
   if (!fn) {
     *why = "cuTensorMapEncodeTiled is not available from the driver";
@@ -104,7 +105,9 @@ bool encode_tmap_3d(CUtensorMap* map, const void* base, CUtensorMapDataType type
   const cuuint32_t box[3] = {b0, b1, b2};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = fn(map, type, 3, const_cast<void*>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     *why = "cuTensorMapEncodeTiled rejected the tensor";

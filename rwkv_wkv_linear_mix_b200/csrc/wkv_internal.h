@@ -63,11 +63,13 @@ __host__ __device__ __forceinline__ int wkv4_seg_begin(int s, int nseg, int nck)
 
 // Encode a 3-D tiled TMA descriptor over a dense row-major tensor with
 // dims {d0 (innermost), d1, d2} of `elem_bytes`-byte elements, box
-// {b0, b1, b2}, no swizzle, out-of-bounds elements filled with zero.
+// {b0, b1, b2}, out-of-bounds elements filled with zero. swizzle128: write
+// the tile in the 128-byte-swizzled shared-memory layout (b0 * elem_bytes
+// must then be 128 and the destination 1024-byte aligned); else unswizzled.
 // Returns false (with a message in *why) if the driver rejects it.
 bool encode_tmap_3d(CUtensorMap* map, const void* base, CUtensorMapDataType type, size_t elem_bytes,
                     uint64_t d0, uint64_t d1, uint64_t d2, uint32_t b0, uint32_t b1, uint32_t b2,
-                    const char** why);
+                    const char** why, bool swizzle128 = false);
 
 struct Wkv4FwdArgs {
   int64_t B, T, C;

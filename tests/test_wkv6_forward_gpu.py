@@ -37,6 +37,34 @@ def test_matches_oracle(W, oracle, B, T, H):
     assert W.device_error(reset=True) == 0
 
 
+@pytest.mark.parametrize("d_mean,d_std,seed", [(1.0, 1.5, 5), (3.0, 1.0, 6), (-0.5, 2.0, 7)])
+def test_strong_decay_subchunks(W, oracle, d_mean, d_std, seed):
+    """Decays strong enough that a 64-token chunk's cumulative decay falls
+    below 2^-96 (and some w round to 0 in bf16): those chunks are processed as
+    16-, 4- and 1-token sub-chunks, which must agree with the plain loop."""
+    B, T, H = 2, 300, 2
+    rec = synth.Wkv6Recipe("t", B, T, H, d_mean=d_mean, d_std=d_std)
+    inp = synth.wkv6_inputs(rec, seed=seed)
+    rng = np.random.default_rng(seed)
+    init = rng.normal(size=(B, H, 64, 64)).astype(np.float32)
+    o, fs = run(W, inp, init_state=dev(init))
+    ro, rfs = ref(oracle, inp, H, init_state=init)
+    assert rel_err(host64(o), ro) < TOL["bf16"]
+    assert rel_err(host64(fs), rfs) < TOL["bf16"]
+    assert W.device_error(reset=True) == 0
+
+
+def test_no_decay_is_linear_attention(W, oracle):
+    """w = 1 (d = -30): the state only accumulates k^T v."""
+    B, T, H = 1, 192, 1
+    inp = synth.wkv6_inputs(synth.Wkv6Recipe("t", B, T, H, d_mean=-30.0, d_std=0.1), seed=9)
+    assert np.all(inp["w32"] == 1.0)
+    o, fs = run(W, inp)
+    ro, rfs = ref(oracle, inp, H)
+    assert rel_err(host64(o), ro) < TOL["bf16"]
+    assert rel_err(host64(fs), rfs) < TOL["bf16"]
+
+
 def test_init_state_and_map(W, oracle):
     B, T, H = 3, 70, 2
     inp = synth.wkv6_inputs(synth.Wkv6Recipe("t", B, T, H), seed=11)
