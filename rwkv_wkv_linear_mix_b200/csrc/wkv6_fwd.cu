@@ -14,75 +14,79 @@
 //        + sum_{s<j} [ (r_j * E_{j-1}) . (k_s / E_s) ] v_s
 //        + [ r_j . (u * k_j) ] v_j                                (intra)
 //   S_out = diag(E_{L-1}) S_in + sum_s (k_s * E_{L-1} / E_s)^T v_s
-// The 64x64x64 products run on the tensor cores (bf16 operands, fp32
-// accumulators in tensor memory). A bf16 operand keeps 8 significant bits;
-// where that is not enough for the 2e-2 bound the operand x is split into
-// hi = bf16(x) and lo = bf16(x - hi) and the product taken in two or three
-// passes (x y ~ xh yh + xl yh + xh yl), which keeps ~16 bits:
-//   MMA1  A  = R^ K~^T        R^ = r * E_{j-1}, K~ = k / E_s   (3 passes)
-//   MMA2  O  = R^ S_in        S_in split hi/lo                 (2 passes)
-//   MMA4  dS = K^^T V         K^ = k * E_{L-1} / E_s (<= |k|)  (1 pass)
-//   MMA3  O += mask(A) V      mask keeps s < j and puts the bonus on s = j,
-//                             split hi/lo                      (2 passes)
-// The fp32 state itself stays in registers. E is a running product of the
-// decays (no logarithms, no exponentials): R^ and K^ never exceed |r|, |k|.
-// K~ = k / E_s grows as the chunk decays, so a chunk whose total decay falls
-// below 2^-96 in some channel is processed as sub-chunks of 16, then 4, then
-// 1 token(s) (the same code with the tokens outside the sub-chunk masked:
-// r = k = 0, w = 1). A single token needs no K~, so every w in (0, 1] is
-// handled.
+// The 64x64x64 products run on the tensor cores with fp32 accumulators in
+// tensor memory:
+//   MMA1  A  = R^ K~^T      tf32: R^ = r * E_{j-1}, K~ = k / E_s
+//   MMA2  O  = R^ S_in      tf32 (the fp32 state, kept in registers)
+//   MMA4  dS = K^^T V       bf16: K^ = k * E_{L-1} / E_s (<= |k|)
+//   MMA3  O += mask(A) V    bf16, mask(A) split hi = bf16(x), lo = bf16(x - hi)
+//                           (two passes: bf16 alone would lose the 2e-2 bound)
+// mask keeps s < j and puts the bonus r_j . (u * k_j) on s = j. E is a
+// running product of the decays (no logarithms, no exponentials): R^ and K^
+// never exceed |r|, |k|. K~ = k / E_s grows as the chunk decays, so a chunk
+// whose total decay falls below 2^-96 in some channel is processed as
+// sub-chunks of 16, then 4, then 1 token(s) (the same code with the tokens
+// outside the sub-chunk masked: r = k = 0, w = 1). A single token needs no
+// K~, so every w in (0, 1] is handled.
 //
-// Kernel shape: one CTA of 256 threads per (b, h), walking its chunks in
-// order; two CTAs share an SM. TMA brings the r, k, w tiles (64 tokens x 64
-// channels, 128-byte swizzled) of the next (sub)chunk as soon as the current
-// one's are consumed, and the v tile of chunk c + 1 (double-buffered) while
-// chunk c is processed. Warp g prepares the operands of tokens 8g .. 8g + 7
-// (lane = two channels) and writes the lo halves of R^ and K~ over the r and
-// k tiles it has just read; one thread issues the MMAs; accumulators are read
-// back by warps 0-3 (columns 0-31) and 4-7 (columns 32-63), whose lanes 0-15
-// also keep the fp32 state (32 values each). Waits are bounded (2 s): a wait
-// that gives up records WKV_DEVERR_WAIT_TIMEOUT, the CTA drains its copies
-// and MMAs in flight, frees its tensor memory and exits.
+// Kernel shape: one CTA of 256 threads per (b, h), walking its chunks (and
+// sub-chunks: "units") in order; two CTAs share an SM. Per unit n:
+//   B. pass 1: product of w over each warp's 8 tokens, totals, split check
+//   C. bonus; pass 2: R^, K~ (fp32), K^ (bf16) into their tiles
+//   D. TMA starts the r, k, w tiles of unit n + 1; MMA1, MMA2, MMA4 issued
+//   E. epilogue of unit n - 1 (its O buffer) while those MMAs run
+//   F. mask(A) -> am tiles; S = diag(E) S + dS -> registers and the tf32 tile
+//   G. MMA3 issued into unit n's O buffer (two buffers alternate)
+// Warp g prepares tokens 8g .. 8g + 7 (lane = two channels); one thread
+// issues the MMAs; accumulators are read back by warps 0-3 (columns 0-31)
+// and 4-7 (columns 32-63), whose lanes 0-15 also keep the fp32 state (32
+// values each). Waits are bounded (2 s): a wait that gives up records
+// WKV_DEVERR_WAIT_TIMEOUT, the CTA drains its copies and MMAs in flight,
+// frees its tensor memory and exits.
 #include "wkv_device.cuh"
 #include "wkv_internal.h"
 
 namespace wkv {
 
+
 constexpr int kHead6 = 64;                         // head size K = V
 constexpr int kChunk6 = 64;                        // tokens per chunk
 constexpr int kThreads6 = 256;                     // 8 warps
-constexpr uint32_t kTile6 = 64u * 64u * 2u;        // one 64 x 64 bf16 tile
-constexpr uint32_t kTmemCols6 = 256;               // A: 0-63, O: 64-127, dS: 128-191
+constexpr uint32_t kTile6 = 8192;                  // 64 x 64 bf16, or one 64 x 32 fp32 panel
+constexpr uint32_t kTmemCols6 = 256;               // tensor-memory columns allocated
+constexpr uint32_t kColA = 0, kColS = 64, kColO = 128;  // A, dS, O accumulators
 constexpr float kMinChunkDecay6 = 1.2621774e-29f;  // 2^-96
 
 struct alignas(1024) Wkv6Smem {
-  uint8_t r[kTile6];     // r of the (sub)chunk; then lo(R^)   [j][i]
-  uint8_t k[kTile6];     // k of the (sub)chunk; then lo(K~)   [s][i]
-  uint8_t w[kTile6];     // w of the (sub)chunk
-  uint8_t v[2][kTile6];  // v of chunks c, c + 1               [s][jv]
-  uint8_t rh[kTile6];    // hi(R^)                             [j][i]
-  uint8_t kb[kTile6];    // hi(K~); then hi(mask(A))           [s][i] / [j][s]
-  uint8_t kh[kTile6];    // K^; then lo(mask(A))               [s][i] / [j][s]
-  uint8_t sh[kTile6];    // hi(S_in)                           [i][jv]
-  uint8_t sl[kTile6];    // lo(S_in)                           [i][jv]
+  uint8_t r[kTile6];      // bf16 r   [j][i]   of the current chunk
+  uint8_t k[kTile6];      // bf16 k   [s][i]
+  uint8_t w[kTile6];      // bf16 w   [j][i]
+  uint8_t v[2][kTile6];   // bf16 v   [s][jv]  of chunk c in v[c & 1]
+  uint8_t rf[2][kTile6];  // R^ fp32, panels [i / 32][j][i % 32]   (A of MMA1, MMA2)
+  uint8_t kf[2][kTile6];  // K~ fp32, panels [i / 32][s][i % 32]   (B of MMA1);
+                          // then hi / lo of mask(A), bf16 [j][s]  (A of MMA3)
+  uint8_t sf[2][kTile6];  // S_in fp32, panels [jv / 32][i][jv % 32] (B of MMA2; 32-byte swizzle)
+  uint8_t kh[kTile6];     // K^ bf16 [s][i] (A of MMA4); in pass 1 the w products
   float u[kHead6];
-  float wq[8][kHead6];  // product of w over each warp's 8 tokens
-  float dec[kHead6];    // E_{L-1}: decay of the state across the (sub)chunk
-  float bonus[kHead6];  // r_j . (u * k_j)
-  uint64_t rkw_bar;     // r, k, w tiles landed
-  uint64_t v_bar[2];    // v tiles landed
-  uint64_t mma_bar;     // tensor-core completion barrier
+  float dec[kHead6];      // E_{L-1}: decay of the state across the unit
+  float bonus[kHead6];    // r_j . (u * k_j)
+  uint64_t w_bar, rk_bar, v_bar[2], mma_bar;
   uint32_t tmem_base;
 };
 
-// bf16 pair (channels 2 * lane, 2 * lane + 1) of row j of a swizzled tile.
+// bf16 pair (channels 2 * lane, 2 * lane + 1) of row j of a swizzled bf16 tile.
 __device__ __forceinline__ uint32_t tile_ld2(const uint8_t* tile, int j, int lane) {
   return *reinterpret_cast<const uint32_t*>(tile + j * 128 + ((((lane >> 2) ^ (j & 7)) & 7) << 4) + 4 * (lane & 3));
 }
 __device__ __forceinline__ void tile_st2(uint8_t* tile, int j, int lane, uint32_t v) {
   *reinterpret_cast<uint32_t*>(tile + j * 128 + ((((lane >> 2) ^ (j & 7)) & 7) << 4) + 4 * (lane & 3)) = v;
 }
-// Columns 16 q .. 16 q + 15 (q in 0..3) of row `row`: 8 packed bf16 pairs.
+// Byte offset of the fp32 pair (columns 2 * lane, 2 * lane + 1) of row j of a
+// two-panel swizzled fp32 tile.
+__device__ __forceinline__ int f32_pair_off(int j, int lane) {
+  return (lane >> 4) * (int)kTile6 + j * 128 + (((((lane & 15) >> 1) ^ (j & 7)) & 7) << 4) + (lane & 1) * 8;
+}
+// Columns 16 q .. 16 q + 15 (q in 0..3) of row `row` of a bf16 tile.
 __device__ __forceinline__ void tile_st_row16(uint8_t* tile, int row, int q, const uint32_t (&p)[8]) {
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
@@ -94,6 +98,43 @@ __device__ __forceinline__ void tile_st_row16(uint8_t* tile, int row, int q, con
 __device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uint32_t& lo) {
   hi = pack_bf16x2(a, b);
   lo = pack_bf16x2(a - bf16lo(hi), b - bf16hi(hi));
+}
+
+// Pass 2 for the tokens 8g .. 8g + 7 of warp g: R^ and K~ (fp32) forwards
+// from the prefix product `pre`, K^ (bf16) backwards from the suffix product
+// `post`. FULL: the unit is the whole 64-token chunk (no masking).
+template <bool FULL>
+__device__ __forceinline__ void wkv6_prepare(Wkv6Smem& sm, int g, int lane, int off, int len, const float (&w0)[8],
+                                             const float (&w1)[8], float pre0, float pre1, float post0, float post1) {
+  const bool need_kb = FULL || len > 1;  // one token has no s < j pair
+  float e0 = pre0, e1 = pre1;
+#pragma unroll
+  for (int jj = 0; jj < 8; ++jj) {
+    const int j = 8 * g + jj;
+    const bool in = FULL || (j >= off && j < off + len);
+    const uint32_t rx = tile_ld2(sm.r, j, lane), kx = tile_ld2(sm.k, j, lane);
+    float2 rh = make_float2(bf16lo(rx) * e0, bf16hi(rx) * e1);
+    e0 *= w0[jj];
+    e1 *= w1[jj];
+    float2 kb = make_float2(bf16lo(kx) * rcp(e0), bf16hi(kx) * rcp(e1));
+    if (!FULL) {
+      if (!in) rh = make_float2(0.f, 0.f);
+      if (!(in && need_kb)) kb = make_float2(0.f, 0.f);
+    }
+    const int fo = f32_pair_off(j, lane);
+    *reinterpret_cast<float2*>(sm.rf[0] + fo) = rh;
+    *reinterpret_cast<float2*>(sm.kf[0] + fo) = kb;
+  }
+  float g0 = post0, g1 = post1;
+#pragma unroll
+  for (int jj = 7; jj >= 0; --jj) {
+    const int j = 8 * g + jj;
+    const bool in = FULL || (j >= off && j < off + len);
+    const uint32_t kx = tile_ld2(sm.k, j, lane);
+    tile_st2(sm.kh, j, lane, in ? pack_bf16x2(bf16lo(kx) * g0, bf16hi(kx) * g1) : 0u);
+    g0 *= w0[jj];
+    g1 *= w1[jj];
+  }
 }
 
 __global__ void __launch_bounds__(kThreads6, 2)
@@ -121,7 +162,8 @@ __global__ void __launch_bounds__(kThreads6, 2)
       tma_prefetch_desc(&tv);
       tma_prefetch_desc(&tw);
     }
-    mbar_init(&sm.rkw_bar, 1);
+    mbar_init(&sm.w_bar, 1);
+    mbar_init(&sm.rk_bar, 1);
     mbar_init(&sm.v_bar[0], 1);
     mbar_init(&sm.v_bar[1], 1);
     mbar_init(&sm.mma_bar, 1);
@@ -130,8 +172,19 @@ __global__ void __launch_bounds__(kThreads6, 2)
   if (warp == 0) tmem_alloc(&sm.tmem_base, kTmemCols6);
   if (tid < kHead6) sm.u[tid] = u[h * kHead6 + tid];
 
-  // fp32 state S[row][32 ch .. 32 ch + 31] in registers; hi/lo copy in sh, sl
+  // fp32 state S[row][32 ch .. 32 ch + 31] in registers; the tf32 operand
+  // copy in sf: panel ch, row `row`, 32-byte chunks XORed with row % 4
   float S[32];
+  auto store_state = [&]() {
+    if (!holder) return;
+    uint8_t* base = sm.sf[ch] + row * 128;
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      uint8_t* p = base + (((m ^ (row & 3)) & 3) << 5);
+      *reinterpret_cast<float4*>(p) = make_float4(S[8 * m], S[8 * m + 1], S[8 * m + 2], S[8 * m + 3]);
+      *reinterpret_cast<float4*>(p + 16) = make_float4(S[8 * m + 4], S[8 * m + 5], S[8 * m + 6], S[8 * m + 7]);
+    }
+  };
   {
     const float* s0 = nullptr;
     if (init_state) {
@@ -151,16 +204,7 @@ __global__ void __launch_bounds__(kThreads6, 2)
       S[e + 2] = x.z;
       S[e + 3] = x.w;
     }
-    if (holder) {
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        uint32_t ph[8], pl[8];
-#pragma unroll
-        for (int e = 0; e < 16; e += 2) split_bf16x2(S[16 * q + e], S[16 * q + e + 1], ph[e / 2], pl[e / 2]);
-        tile_st_row16(sm.sh, row, 2 * ch + q, ph);
-        tile_st_row16(sm.sl, row, 2 * ch + q, pl);
-      }
-    }
+    store_state();
   }
   fence_proxy_async_smem();
   tc_fence_before_sync();
@@ -169,14 +213,18 @@ __global__ void __launch_bounds__(kThreads6, 2)
   const uint32_t tm = sm.tmem_base;
   const uint32_t tl = tm + ((uint32_t)(32 * sp) << 16);  // this warp's TMEM lanes
 
-  // copies in flight, as seen by thread 0 (the only thread that issues them)
-  int rkw_issued = 0, rkw_done = 0, v_issued = 0, v_done = 0;
-  auto load_rkw = [&](int cc) {
-    mbar_arrive_expect_tx(&sm.rkw_bar, 3 * kTile6);
-    tma_load_3d(sm.r, &tr, &sm.rkw_bar, h * kHead6, cc * kChunk6, b);
-    tma_load_3d(sm.k, &tk, &sm.rkw_bar, h * kHead6, cc * kChunk6, b);
-    tma_load_3d(sm.w, &tw, &sm.rkw_bar, h * kHead6, cc * kChunk6, b);
-    ++rkw_issued;
+  // copies and MMA commits in flight, as seen by thread 0 (which issues them)
+  int w_issued = 0, w_done = 0, rk_issued = 0, rk_done = 0, v_issued = 0, v_done = 0, mma_issued = 0, mma_done = 0;
+  auto load_w = [&](int cc) {
+    mbar_arrive_expect_tx(&sm.w_bar, kTile6);
+    tma_load_3d(sm.w, &tw, &sm.w_bar, h * kHead6, cc * kChunk6, b);
+    ++w_issued;
+  };
+  auto load_rk = [&](int cc) {
+    mbar_arrive_expect_tx(&sm.rk_bar, 2 * kTile6);
+    tma_load_3d(sm.r, &tr, &sm.rk_bar, h * kHead6, cc * kChunk6, b);
+    tma_load_3d(sm.k, &tk, &sm.rk_bar, h * kHead6, cc * kChunk6, b);
+    ++rk_issued;
   };
   auto load_v = [&](int cc) {
     mbar_arrive_expect_tx(&sm.v_bar[cc & 1], kTile6);
@@ -184,80 +232,125 @@ __global__ void __launch_bounds__(kThreads6, 2)
     ++v_issued;
   };
   if (tid == 0 && nch > 0) {
-    load_rkw(0);
+    load_w(0);
+    load_rk(0);
     load_v(0);
   }
+  bool ok = true;
+  uint32_t mma_phase = 0;
+  // every thread waits (bounded) for a barrier phase; thread 0 books it
+  auto wait_bar = [&](uint64_t* bar, uint32_t parity, int* done, int upto) {
+    const bool got = mbar_wait_bounded(bar, parity, err);
+    if (tid == 0 && got) *done = upto;
+    ok = ok && got;
+  };
+  auto wait_mma = [&]() {
+    wait_bar(&sm.mma_bar, mma_phase, &mma_done, mma_issued);
+    mma_phase ^= 1u;
+    tc_fence_after_sync();
+  };
 
-  constexpr uint32_t id_kk = umma_idesc_bf16(64, 64, 0, 0);  // A K-major, B K-major
-  constexpr uint32_t id_km = umma_idesc_bf16(64, 64, 0, 1);  // A K-major, B MN-major
-  constexpr uint32_t id_mm = umma_idesc_bf16(64, 64, 1, 1);  // A MN-major, B MN-major
-  uint32_t rkw_phase = 0, mma_phase = 0;
-  bool mma_pending = false;  // (thread 0) an MMA commit not yet confirmed complete
-  bool ok = true, failed = false;
-  bool wait_rkw = true;  // the next (sub)chunk's r, k, w tiles are still loading
+  constexpr uint32_t idt_kk = umma_idesc_tf32(64, 64, 0, 0);  // tf32, A K-major, B K-major
+  constexpr uint32_t idt_km = umma_idesc_tf32(64, 64, 0, 1);  // tf32, A K-major, B MN-major
+  constexpr uint32_t idb_km = umma_idesc_bf16(64, 64, 0, 1);  // bf16, A K-major, B MN-major
+  constexpr uint32_t idb_mm = umma_idesc_bf16(64, 64, 1, 1);  // bf16, A MN-major, B MN-major
+
+  // the previous unit, whose O is still to be written out
+  bool prev = false;
+  int prev_t0 = 0, prev_off = 0, prev_len = 0;
+  auto epilogue = [&]() {
+    // MMA3 of the previous unit has completed (waited for by the caller)
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      float ov[16];
+      tmem_ld16(tl + kColO + 32 * ch + 16 * q, ov);
+      tmem_wait_ld();
+      if (ok && holder && row >= prev_off && row < prev_off + prev_len) {
+        uint32_t p[8];
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) p[e / 2] = pack_bf16x2(ov[e], ov[e + 1]);
+        uint4* dst = reinterpret_cast<uint4*>(o + ((int64_t)b * T + prev_t0 + row) * HK + h * kHead6 + 32 * ch + 16 * q);
+        dst[0] = make_uint4(p[0], p[1], p[2], p[3]);
+        dst[1] = make_uint4(p[4], p[5], p[6], p[7]);
+      }
+    }
+    tc_fence_before_sync();
+  };
+
+  bool failed = false;
   for (int c = 0; c < nch && !failed; ++c) {
     const int t0 = c * kChunk6;
     const int valid = min(kChunk6, T - t0);
     const uint32_t vt = smem_u32(sm.v[c & 1]);
-    if (tid == 0 && c + 1 < nch) load_v(c + 1);
-    bool v_ready = false;
     int off = 0, size = kChunk6;
+    bool first_unit = true;
+    wait_bar(&sm.w_bar, (uint32_t)c & 1u, &w_done, c + 1);
     while (off < valid) {
-      if (wait_rkw) {
-        const bool got = mbar_wait_bounded(&sm.rkw_bar, rkw_phase, err);
-        if (tid == 0 && got) rkw_done = rkw_issued;
-        ok = got && ok;
-        rkw_phase ^= 1u;
-        wait_rkw = false;
-      }
       const int len = min(size, valid - off);
-      // ---- pass 1: product of w over this warp's 8 tokens (w = 1 outside) ----
+      const bool full = len == kChunk6;
+      // ---- B. pass 1: product of w over this warp's 8 tokens (w = 1 outside) ----
       float w0[8], w1[8];
-      float p0 = 1.f, p1 = 1.f;
+      {
+        float p0 = 1.f, p1 = 1.f;
 #pragma unroll
-      for (int jj = 0; jj < 8; ++jj) {
-        const int j = 8 * warp + jj;
-        const bool in = j >= off && j < off + len;
-        const uint32_t x = tile_ld2(sm.w, j, lane);
-        w0[jj] = in ? bf16lo(x) : 1.f;
-        w1[jj] = in ? bf16hi(x) : 1.f;
-        p0 *= w0[jj];
-        p1 *= w1[jj];
+        for (int jj = 0; jj < 8; ++jj) {
+          const int j = 8 * warp + jj;
+          const bool in = full || (j >= off && j < off + len);
+          const uint32_t x = tile_ld2(sm.w, j, lane);
+          w0[jj] = in ? bf16lo(x) : 1.f;
+          w1[jj] = in ? bf16hi(x) : 1.f;
+          p0 *= w0[jj];
+          p1 *= w1[jj];
+        }
+        float* wq = reinterpret_cast<float*>(sm.kh);  // [8][64]
+        *reinterpret_cast<float2*>(wq + warp * kHead6 + 2 * lane) = make_float2(p0, p1);
       }
-      sm.wq[warp][2 * lane] = p0;
-      sm.wq[warp][2 * lane + 1] = p1;
       if (__syncthreads_or(!ok)) {
         failed = true;
         break;
       }
       float pre0 = 1.f, pre1 = 1.f, post0 = 1.f, post1 = 1.f, tot0 = 1.f, tot1 = 1.f;
+      {
+        const float* wq = reinterpret_cast<const float*>(sm.kh);
 #pragma unroll
-      for (int g = 0; g < 8; ++g) {
-        const float2 q = *reinterpret_cast<const float2*>(&sm.wq[g][2 * lane]);
-        if (g < warp) {
-          pre0 *= q.x;
-          pre1 *= q.y;
+        for (int g = 0; g < 8; ++g) {
+          const float2 q = *reinterpret_cast<const float2*>(wq + g * kHead6 + 2 * lane);
+          if (g < warp) {
+            pre0 *= q.x;
+            pre1 *= q.y;
+          }
+          if (g > warp) {
+            post0 *= q.x;
+            post1 *= q.y;
+          }
+          tot0 *= q.x;
+          tot1 *= q.y;
         }
-        if (g > warp) {
-          post0 *= q.x;
-          post1 *= q.y;
-        }
-        tot0 *= q.x;
-        tot1 *= q.y;
       }
-      // a chunk that decays below 2^-96 is split (K~ = k / E could overflow);
-      // nothing has been written yet, so the tiles are still intact
+      // a unit that decays below 2^-96 is split (K~ = k / E could overflow);
+      // nothing has been written yet, so it simply starts again smaller
       const bool deep = !(tot0 >= kMinChunkDecay6 && tot1 >= kMinChunkDecay6);
       if (__syncthreads_or(deep) && size > 1) {
         size >>= 2;
         continue;
       }
-      if (warp == 0) {
-        sm.dec[2 * lane] = tot0;
-        sm.dec[2 * lane + 1] = tot1;
+      const bool last_unit = off + len == valid;
+      // the w tile is consumed: bring the next chunk's
+      if (tid == 0 && last_unit && c + 1 < nch) load_w(c + 1);
+      if (warp == 0) *reinterpret_cast<float2*>(&sm.dec[2 * lane]) = make_float2(tot0, tot1);
+      // ---- E. write out the previous unit (its MMA3 overlapped pass 1) ----
+      if (prev) {
+        wait_mma();
+        epilogue();
       }
-      // ---- bonus r_j . (u * k_j): the four lanes 4m .. 4m + 3 of warp g take
-      // token 8g + m, 16 channels each (rows this warp owns) ----
+      // the v buffer of chunk c - 1 is free now: bring chunk c + 1's
+      if (tid == 0 && first_unit && c + 1 < nch) load_v(c + 1);
+      if (first_unit) {
+        wait_bar(&sm.rk_bar, (uint32_t)c & 1u, &rk_done, c + 1);
+        wait_bar(&sm.v_bar[c & 1], (uint32_t)(c >> 1) & 1u, &v_done, c + 1);
+      }
+      // ---- C. bonus r_j . (u * k_j): lanes 4m .. 4m + 3 of warp g take
+      // token 8g + m, 16 channels each ----
       {
         const int j = tid >> 2, part = tid & 3;
         float acc = 0.f;
@@ -279,89 +372,46 @@ __global__ void __launch_bounds__(kThreads6, 2)
         acc += __shfl_xor_sync(0xffffffffu, acc, 2);
         if (part == 0) sm.bonus[j] = (j >= off && j < off + len) ? acc : 0.f;
       }
-      __syncwarp();
-      // ---- pass 2: K^ (suffix products, backwards); then R^ and K~ with
-      // their lo halves written over the r and k rows just read ----
-      {
-        float g0 = post0, g1 = post1;
-#pragma unroll
-        for (int jj = 7; jj >= 0; --jj) {
-          const int j = 8 * warp + jj;
-          const bool in = j >= off && j < off + len;
-          const uint32_t kx = tile_ld2(sm.k, j, lane);
-          tile_st2(sm.kh, j, lane, in ? pack_bf16x2(bf16lo(kx) * g0, bf16hi(kx) * g1) : 0u);
-          g0 *= w0[jj];
-          g1 *= w1[jj];
-        }
-        float e0 = pre0, e1 = pre1;
-        const bool need_kb = len > 1;  // one token has no s < j pair
-#pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-          const int j = 8 * warp + jj;
-          const bool in = j >= off && j < off + len;
-          const uint32_t rx = tile_ld2(sm.r, j, lane), kx = tile_ld2(sm.k, j, lane);
-          uint32_t rh, rl, kbh, kbl;
-          split_bf16x2(bf16lo(rx) * e0, bf16hi(rx) * e1, rh, rl);
-          e0 *= w0[jj];
-          e1 *= w1[jj];
-          split_bf16x2(bf16lo(kx) * rcp(e0), bf16hi(kx) * rcp(e1), kbh, kbl);
-          const bool kin = in && need_kb;
-          tile_st2(sm.rh, j, lane, in ? rh : 0u);
-          tile_st2(sm.r, j, lane, in ? rl : 0u);
-          tile_st2(sm.kb, j, lane, kin ? kbh : 0u);
-          tile_st2(sm.k, j, lane, kin ? kbl : 0u);
-        }
-      }
-      if (!v_ready) {
-        ok = mbar_wait_bounded(&sm.v_bar[c & 1], (c >> 1) & 1, err) && ok;
-        if (tid == 0 && ok) v_done = c + 1;
-        v_ready = true;
-      }
+      // ---- C. pass 2 ----
+      if (full)
+        wkv6_prepare<true>(sm, warp, lane, off, len, w0, w1, pre0, pre1, post0, post1);
+      else
+        wkv6_prepare<false>(sm, warp, lane, off, len, w0, w1, pre0, pre1, post0, post1);
       fence_proxy_async_smem();
       if (__syncthreads_or(!ok)) {
         failed = true;
         break;
       }
-      // ---- MMA1 A = R^ K~^T, MMA2 O = R^ S_in, MMA4 dS = K^^T V ----
+      // ---- D. next chunk's r, k; MMA1 A = R^ K~^T, MMA2 O = R^ S_in, MMA4 dS = K^^T V ----
       if (tid == 0) {
+        if (last_unit && c + 1 < nch) load_rk(c + 1);
         tc_fence_after_sync();
-        const uint32_t rh = smem_u32(sm.rh), rl = smem_u32(sm.r), kbh = smem_u32(sm.kb), kbl = smem_u32(sm.k);
-        const uint32_t kh = smem_u32(sm.kh), sh = smem_u32(sm.sh), sl = smem_u32(sm.sl);
+        const uint32_t rf = smem_u32(sm.rf[0]), kf = smem_u32(sm.kf[0]), sf = smem_u32(sm.sf[0]);
+        const uint32_t kh = smem_u32(sm.kh);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) umma_bf16(tm + 0, umma_kmajor(rh, kk), umma_kmajor(kbh, kk), id_kk, kk > 0);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t po = (uint32_t)(kk >> 2) * kTile6 + (uint32_t)(kk & 3) * 32u;
+          umma_tf32(tm + kColA, umma_desc_sw128(rf + po, 16, 1024), umma_desc_sw128(kf + po, 16, 1024), idt_kk, kk > 0);
+        }
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) umma_bf16(tm + 0, umma_kmajor(rl, kk), umma_kmajor(kbh, kk), id_kk, true);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t po = (uint32_t)(kk >> 2) * kTile6 + (uint32_t)(kk & 3) * 32u;
+          umma_tf32(tm + kColO, umma_desc_sw128(rf + po, 16, 1024), umma_desc_sw128_32b(sf + 1024u * kk, kTile6, 512),
+                    idt_km, kk > 0);
+        }
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) umma_bf16(tm + 0, umma_kmajor(rh, kk), umma_kmajor(kbl, kk), id_kk, true);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) umma_bf16(tm + 64, umma_kmajor(rh, kk), umma_mnmajor(sh, kk), id_km, kk > 0);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) umma_bf16(tm + 64, umma_kmajor(rh, kk), umma_mnmajor(sl, kk), id_km, true);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) umma_bf16(tm + 128, umma_mnmajor(kh, kk), umma_mnmajor(vt, kk), id_mm, kk > 0);
+        for (int kk = 0; kk < 4; ++kk) umma_bf16(tm + kColS, umma_mnmajor(kh, kk), umma_mnmajor(vt, kk), idb_mm, kk > 0);
         umma_commit(&sm.mma_bar);
-        mma_pending = true;
+        ++mma_issued;
       }
-      {
-        const bool got = mbar_wait_bounded(&sm.mma_bar, mma_phase, err);
-        if (tid == 0 && got) mma_pending = false;
-        ok = got && ok;
-        mma_phase ^= 1u;
-      }
-      tc_fence_after_sync();
-      // r, k, w tiles are free: bring those of the next (sub)chunk
-      if (tid == 0 && ok) {
-        const int next = off + len < valid ? c : c + 1;
-        if (next < nch) load_rkw(next);
-      }
-      wait_rkw = true;
-      // ---- mask(A) split hi/lo into kb, kh; S = diag(E) S + dS into sh, sl ----
+      // ---- F. mask(A) -> hi / lo tiles over K~; S = diag(E) S + dS ----
+      wait_mma();
       {
         const float bj = holder ? sm.bonus[row] : 0.f;
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           float a[16];
-          tmem_ld16(tl + 0 + 32 * ch + 16 * q, a);
+          tmem_ld16(tl + kColA + 32 * ch + 16 * q, a);
           tmem_wait_ld();
           if (holder) {
             uint32_t ph[8], pl[8];
@@ -372,30 +422,20 @@ __global__ void __launch_bounds__(kThreads6, 2)
               const float a1 = s + 1 < row ? a[e + 1] : (s + 1 == row ? bj : 0.f);
               split_bf16x2(a0, a1, ph[e / 2], pl[e / 2]);
             }
-            tile_st_row16(sm.kb, row, 2 * ch + q, ph);
-            tile_st_row16(sm.kh, row, 2 * ch + q, pl);
+            tile_st_row16(sm.kf[0], row, 2 * ch + q, ph);
+            tile_st_row16(sm.kf[1], row, 2 * ch + q, pl);
           }
         }
         const float dj = holder ? sm.dec[row] : 0.f;
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           float d[16];
-          tmem_ld16(tl + 128 + 32 * ch + 16 * q, d);
+          tmem_ld16(tl + kColS + 32 * ch + 16 * q, d);
           tmem_wait_ld();
-          if (holder) {
-            uint32_t ph[8], pl[8];
 #pragma unroll
-            for (int e = 0; e < 16; e += 2) {
-              float& s0 = S[16 * q + e];
-              float& s1 = S[16 * q + e + 1];
-              s0 = fmaf(dj, s0, d[e]);
-              s1 = fmaf(dj, s1, d[e + 1]);
-              split_bf16x2(s0, s1, ph[e / 2], pl[e / 2]);
-            }
-            tile_st_row16(sm.sh, row, 2 * ch + q, ph);
-            tile_st_row16(sm.sl, row, 2 * ch + q, pl);
-          }
+          for (int e = 0; e < 16; ++e) S[16 * q + e] = fmaf(dj, S[16 * q + e], d[e]);
         }
+        store_state();
       }
       fence_proxy_async_smem();
       tc_fence_before_sync();
@@ -403,51 +443,38 @@ __global__ void __launch_bounds__(kThreads6, 2)
         failed = true;
         break;
       }
-      // ---- MMA3 O += mask(A) V ----
+      // ---- G. MMA3 O += mask(A) V (hi and lo passes); written out next unit ----
       if (tid == 0) {
         tc_fence_after_sync();
-        const uint32_t amh = smem_u32(sm.kb), aml = smem_u32(sm.kh);
+        const uint32_t amh = smem_u32(sm.kf[0]), aml = smem_u32(sm.kf[1]);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) umma_bf16(tm + 64, umma_kmajor(amh, kk), umma_mnmajor(vt, kk), id_km, true);
+        for (int kk = 0; kk < 4; ++kk) umma_bf16(tm + kColO, umma_kmajor(amh, kk), umma_mnmajor(vt, kk), idb_km, true);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) umma_bf16(tm + 64, umma_kmajor(aml, kk), umma_mnmajor(vt, kk), id_km, true);
+        for (int kk = 0; kk < 4; ++kk) umma_bf16(tm + kColO, umma_kmajor(aml, kk), umma_mnmajor(vt, kk), idb_km, true);
         umma_commit(&sm.mma_bar);
-        mma_pending = true;
+        ++mma_issued;
       }
-      {
-        const bool got = mbar_wait_bounded(&sm.mma_bar, mma_phase, err);
-        if (tid == 0 && got) mma_pending = false;
-        ok = got && ok;
-        mma_phase ^= 1u;
-      }
-      tc_fence_after_sync();
-      // ---- epilogue: this (sub)chunk's rows of o ----
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        float ov[16];
-        tmem_ld16(tl + 64 + 32 * ch + 16 * q, ov);
-        tmem_wait_ld();
-        if (ok && holder && row >= off && row < off + len) {
-          uint32_t p[8];
-#pragma unroll
-          for (int e = 0; e < 16; e += 2) p[e / 2] = pack_bf16x2(ov[e], ov[e + 1]);
-          uint4* dst = reinterpret_cast<uint4*>(o + ((int64_t)b * T + t0 + row) * HK + h * kHead6 + 32 * ch + 16 * q);
-          dst[0] = make_uint4(p[0], p[1], p[2], p[3]);
-          dst[1] = make_uint4(p[4], p[5], p[6], p[7]);
-        }
-      }
-      tc_fence_before_sync();
+      prev = true;
+      prev_t0 = t0;
+      prev_off = off;
+      prev_len = len;
+      first_unit = false;
       off += len;
     }
+  }
+  if (!failed && prev) {
+    wait_mma();
+    epilogue();
   }
   if (!failed && __syncthreads_or(!ok)) failed = true;
   if (failed) {
     // let every copy and MMA still in flight land before the shared and
     // tensor memory are released (each wait is itself bounded)
     if (tid == 0) {
-      if (rkw_done < rkw_issued) mbar_wait_bounded(&sm.rkw_bar, (uint32_t)(rkw_issued - 1) & 1u, err);
+      if (w_done < w_issued) mbar_wait_bounded(&sm.w_bar, (uint32_t)(w_issued - 1) & 1u, err);
+      if (rk_done < rk_issued) mbar_wait_bounded(&sm.rk_bar, (uint32_t)(rk_issued - 1) & 1u, err);
       for (int cc = v_done; cc < v_issued; ++cc) mbar_wait_bounded(&sm.v_bar[cc & 1], (uint32_t)(cc >> 1) & 1u, err);
-      if (mma_pending) mbar_wait_bounded(&sm.mma_bar, mma_phase ^ 1u, err);
+      if (mma_done < mma_issued) mbar_wait_bounded(&sm.mma_bar, (uint32_t)(mma_issued - 1) & 1u, err);
     }
   } else if (final_state && holder) {
     float* fs = final_state + ((int64_t)b * H + h) * kHead6 * kHead6 + row * kHead6 + 32 * ch;

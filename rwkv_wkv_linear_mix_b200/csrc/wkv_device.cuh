@@ -154,14 +154,18 @@ __device__ __forceinline__ float ld_shared_cluster(uint32_t addr) {
 // ----------------------------------------------------------------------------
 // tcgen05 (5th-generation tensor cores, accumulators in tensor memory)
 //
-// Operand tiles are 64 x 64 bf16 matrices stored as 64 rows of 128 bytes in
-// the 128-byte-swizzled layout (the 16-byte chunk index of row r is XORed
-// with r % 8; tiles are 1024-byte aligned), which is also the layout a TMA
-// load with CU_TENSOR_MAP_SWIZZLE_128B writes. Such a tile serves as a
-//  * K-major operand when its rows are M (or N) and its columns are K:
-//    the 16-element K step kk starts 32 * kk bytes into the tile;
-//  * MN-major operand when its rows are K and its columns are M (or N):
-//    the K step kk starts 2048 * kk bytes (16 rows) into the tile.
+// Operand tiles are 64 x 64 matrices stored as rows of 128 bytes in the
+// 128-byte-swizzled layout (the 16-byte chunk index of row r is XORed with
+// r % 8; tiles are 1024-byte aligned), which is also the layout a TMA load
+// with CU_TENSOR_MAP_SWIZZLE_128B writes. A bf16 tile is 64 rows of 64
+// elements; an fp32 (tf32) tile is two 8 KB panels of 64 rows x 32 columns.
+//  * K-major (rows M or N, columns K): the K step kk (16 bf16 / 8 tf32
+//    elements = 32 bytes) starts 32 * (kk % 4) bytes into its panel.
+//  * MN-major bf16 (rows K, columns M or N): the K step kk starts 2048 * kk
+//    bytes (16 rows) into the tile.
+//  * MN-major tf32 uses another swizzle (umma_desc_sw128_32b): 32-byte
+//    chunks XORed with row % 4; the K step kk (8 rows) starts 1024 * kk
+//    bytes into the panel and the second 32-column panel is LBO away.
 // An M = 64 accumulator holds row m in TMEM lane (m % 16) + 32 * (m / 16),
 // so warp q of a warpgroup reads rows 16q .. 16q + 15 in its lanes 0 .. 15.
 // ----------------------------------------------------------------------------
@@ -173,6 +177,14 @@ __device__ __forceinline__ int sw128_offset(int row, int col_bf16) {
 __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+// Descriptor of an MN-major tf32 operand in the 32-byte-granular 128-byte
+// swizzle (layout type 1: the 32-byte chunk index of row r is XORed with
+// r % 4; 4-row K groups SBO bytes apart, 32-column MN atoms LBO bytes apart).
+// This is the only swizzled layout the tensor cores take for MN-major tf32.
+__device__ __forceinline__ uint64_t umma_desc_sw128_32b(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (1ull << 61);
 }
 __device__ __forceinline__ uint64_t umma_kmajor(uint32_t tile, int kk) { return umma_desc_sw128(tile + 32u * kk, 16u, 1024u); }
 __device__ __forceinline__ uint64_t umma_mnmajor(uint32_t tile, int kk) {
@@ -192,6 +204,21 @@ __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint
   asm volatile(
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u)
+      : "memory");
+}
+// Instruction descriptor of kind::tf32: tf32 A and B (fp32 storage, low 13
+// mantissa bits ignored), f32 accumulator, M x N.
+__host__ __device__ constexpr uint32_t umma_idesc_tf32(int M, int N, int a_mn, int b_mn) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+// D[tmem] (+)= A * B for one 8-deep K step of tf32 operands.
+__device__ __forceinline__ void umma_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u)
       : "memory");
 }
