@@ -16,8 +16,8 @@
 //   S_out = diag(E_{L-1}) S_in + sum_s (k_s * E_{L-1} / E_s)^T v_s
 // The 64x64x64 products run on the tensor cores with fp32 accumulators in
 // tensor memory:
-//   MMA1  A  = R^ K~^T      tf32: R^ = r * E_{j-1}, K~ = k / E_s
-//   MMA2  O  = R^ S_in      tf32 (the fp32 state, kept in registers)
+//   MMA12 [A | O] = R^ [K~ ; S_in^T]^T   tf32, one N = 128 product:
+//                  R^ = r * E_{j-1}, K~ = k / E_s, S_in the fp32 state
 //   MMA4  dS = K^^T V       bf16: K^ = k * E_{L-1} / E_s (<= |k|)
 //   MMA3  O += mask(A) V    bf16, mask(A) split hi = bf16(x), lo = bf16(x - hi)
 //                           (two passes: bf16 alone would lose the 2e-2 bound)
@@ -33,9 +33,9 @@
 // sub-chunks: "units") in order; two CTAs share an SM. Per unit n:
 //   B. pass 1: product of w over each warp's 8 tokens, totals, split check
 //   C. bonus; pass 2: R^, K~ (fp32), K^ (bf16) into their tiles
-//   D. TMA starts the r, k, w tiles of unit n + 1; MMA1, MMA2, MMA4 issued
+//   D. TMA starts the next chunk's r, k tiles; MMA12 and MMA4 issued
 //   E. epilogue of unit n - 1 (its O buffer) while those MMAs run
-//   F. mask(A) -> am tiles; S = diag(E) S + dS -> registers and the tf32 tile
+//   F. mask(A) -> am tiles; S = diag(E) S + dS -> registers and the S^T rows
 //   G. MMA3 issued into unit n's O buffer (two buffers alternate)
 // Warp g prepares tokens 8g .. 8g + 7 (lane = two channels); one thread
 // issues the MMAs; accumulators are read back by warps 0-3 (columns 0-31)
@@ -54,7 +54,7 @@ constexpr int kChunk6 = 64;                        // tokens per chunk
 constexpr int kThreads6 = 256;                     // 8 warps
 constexpr uint32_t kTile6 = 8192;                  // 64 x 64 bf16, or one 64 x 32 fp32 panel
 constexpr uint32_t kTmemCols6 = 256;               // tensor-memory columns allocated
-constexpr uint32_t kColA = 0, kColS = 64, kColO = 128;  // A, dS, O accumulators
+constexpr uint32_t kColA = 0, kColO = 64, kColS = 128;  // A, O (adjacent: one N = 128 MMA), dS
 constexpr float kMinChunkDecay6 = 1.2621774e-29f;  // 2^-96
 
 struct alignas(1024) Wkv6Smem {
@@ -62,10 +62,11 @@ struct alignas(1024) Wkv6Smem {
   uint8_t k[kTile6];      // bf16 k   [s][i]
   uint8_t w[kTile6];      // bf16 w   [j][i]
   uint8_t v[2][kTile6];   // bf16 v   [s][jv]  of chunk c in v[c & 1]
-  uint8_t rf[2][kTile6];  // R^ fp32, panels [i / 32][j][i % 32]   (A of MMA1, MMA2)
-  uint8_t kf[2][kTile6];  // K~ fp32, panels [i / 32][s][i % 32]   (B of MMA1);
-                          // then hi / lo of mask(A), bf16 [j][s]  (A of MMA3)
-  uint8_t sf[2][kTile6];  // S_in fp32, panels [jv / 32][i][jv % 32] (B of MMA2; 32-byte swizzle)
+  uint8_t rf[2][kTile6];  // R^ fp32, panels [i / 32][j][i % 32]            (A of MMA12)
+  uint8_t bt[2][2 * kTile6];  // B of MMA12, fp32, panels [i / 32][128 rows][i % 32]:
+                              // rows 0-63 K~ [s], rows 64-127 S_in^T [jv]; after
+                              // MMA12 rows 0-63 of panel 0 / 1 hold hi / lo of
+                              // mask(A), bf16 [j][s] (A of MMA3)
   uint8_t kh[kTile6];     // K^ bf16 [s][i] (A of MMA4); in pass 1 the w products
   float u[kHead6];
   float dec[kHead6];      // E_{L-1}: decay of the state across the unit
@@ -82,9 +83,9 @@ __device__ __forceinline__ void tile_st2(uint8_t* tile, int j, int lane, uint32_
   *reinterpret_cast<uint32_t*>(tile + j * 128 + ((((lane >> 2) ^ (j & 7)) & 7) << 4) + 4 * (lane & 3)) = v;
 }
 // Byte offset of the fp32 pair (columns 2 * lane, 2 * lane + 1) of row j of a
-// two-panel swizzled fp32 tile.
-__device__ __forceinline__ int f32_pair_off(int j, int lane) {
-  return (lane >> 4) * (int)kTile6 + j * 128 + (((((lane & 15) >> 1) ^ (j & 7)) & 7) << 4) + (lane & 1) * 8;
+// two-panel swizzled fp32 tile whose panels are `panel` bytes apart.
+__device__ __forceinline__ int f32_pair_off(int j, int lane, int panel) {
+  return (lane >> 4) * panel + j * 128 + (((((lane & 15) >> 1) ^ (j & 7)) & 7) << 4) + (lane & 1) * 8;
 }
 // Columns 16 q .. 16 q + 15 (q in 0..3) of row `row` of a bf16 tile.
 __device__ __forceinline__ void tile_st_row16(uint8_t* tile, int row, int q, const uint32_t (&p)[8]) {
@@ -121,9 +122,8 @@ __device__ __forceinline__ void wkv6_prepare(Wkv6Smem& sm, int g, int lane, int 
       if (!in) rh = make_float2(0.f, 0.f);
       if (!(in && need_kb)) kb = make_float2(0.f, 0.f);
     }
-    const int fo = f32_pair_off(j, lane);
-    *reinterpret_cast<float2*>(sm.rf[0] + fo) = rh;
-    *reinterpret_cast<float2*>(sm.kf[0] + fo) = kb;
+    *reinterpret_cast<float2*>(sm.rf[0] + f32_pair_off(j, lane, kTile6)) = rh;
+    *reinterpret_cast<float2*>(sm.bt[0] + f32_pair_off(j, lane, 2 * kTile6)) = kb;
   }
   float g0 = post0, g1 = post1;
 #pragma unroll
@@ -172,17 +172,17 @@ __global__ void __launch_bounds__(kThreads6, 2)
   if (warp == 0) tmem_alloc(&sm.tmem_base, kTmemCols6);
   if (tid < kHead6) sm.u[tid] = u[h * kHead6 + tid];
 
-  // fp32 state S[row][32 ch .. 32 ch + 31] in registers; the tf32 operand
-  // copy in sf: panel ch, row `row`, 32-byte chunks XORed with row % 4
+  // fp32 state S[row][32 ch .. 32 ch + 31] in registers; its tf32 operand
+  // copy is S^T in rows 64 + jv of bt (K-major: column i = row)
   float S[32];
   auto store_state = [&]() {
     if (!holder) return;
-    uint8_t* base = sm.sf[ch] + row * 128;
+    uint8_t* base = sm.bt[row >> 5] + 64 * 128 + (row & 3) * 4;
+    const int c4 = (row & 31) >> 2;
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-      uint8_t* p = base + (((m ^ (row & 3)) & 3) << 5);
-      *reinterpret_cast<float4*>(p) = make_float4(S[8 * m], S[8 * m + 1], S[8 * m + 2], S[8 * m + 3]);
-      *reinterpret_cast<float4*>(p + 16) = make_float4(S[8 * m + 4], S[8 * m + 5], S[8 * m + 6], S[8 * m + 7]);
+    for (int e = 0; e < 32; ++e) {
+      const int jv = 32 * ch + e;
+      *reinterpret_cast<float*>(base + jv * 128 + (((c4 ^ (jv & 7)) & 7) << 4)) = S[e];
     }
   };
   {
@@ -250,8 +250,7 @@ __global__ void __launch_bounds__(kThreads6, 2)
     tc_fence_after_sync();
   };
 
-  constexpr uint32_t idt_kk = umma_idesc_tf32(64, 64, 0, 0);  // tf32, A K-major, B K-major
-  constexpr uint32_t idt_km = umma_idesc_tf32(64, 64, 0, 1);  // tf32, A K-major, B MN-major
+  constexpr uint32_t idt_12 = umma_idesc_tf32(64, 128, 0, 0);  // tf32 M64 N128, both K-major
   constexpr uint32_t idb_km = umma_idesc_bf16(64, 64, 0, 1);  // bf16, A K-major, B MN-major
   constexpr uint32_t idb_mm = umma_idesc_bf16(64, 64, 1, 1);  // bf16, A MN-major, B MN-major
 
@@ -386,21 +385,17 @@ __global__ void __launch_bounds__(kThreads6, 2)
       if (tid == 0) {
         if (last_unit && c + 1 < nch) load_rk(c + 1);
         tc_fence_after_sync();
-        const uint32_t rf = smem_u32(sm.rf[0]), kf = smem_u32(sm.kf[0]), sf = smem_u32(sm.sf[0]);
-        const uint32_t kh = smem_u32(sm.kh);
+        // descriptors advance by whole 16-byte units in their low bits
+        const uint64_t da = umma_desc_sw128(smem_u32(sm.rf[0]), 16, 1024);
+        const uint64_t db = umma_desc_sw128(smem_u32(sm.bt[0]), 16, 1024);
+        const uint64_t dk = umma_desc_sw128(smem_u32(sm.kh), 8192, 1024);
+        const uint64_t dv = umma_desc_sw128(vt, 8192, 1024);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t po = (uint32_t)(kk >> 2) * kTile6 + (uint32_t)(kk & 3) * 32u;
-          umma_tf32(tm + kColA, umma_desc_sw128(rf + po, 16, 1024), umma_desc_sw128(kf + po, 16, 1024), idt_kk, kk > 0);
-        }
+        for (int kk = 0; kk < 8; ++kk)
+          umma_tf32(tm + kColA, da + ((kk >> 2) * kTile6 + (kk & 3) * 32) / 16,
+                    db + ((kk >> 2) * 2 * kTile6 + (kk & 3) * 32) / 16, idt_12, kk > 0);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t po = (uint32_t)(kk >> 2) * kTile6 + (uint32_t)(kk & 3) * 32u;
-          umma_tf32(tm + kColO, umma_desc_sw128(rf + po, 16, 1024), umma_desc_sw128_32b(sf + 1024u * kk, kTile6, 512),
-                    idt_km, kk > 0);
-        }
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) umma_bf16(tm + kColS, umma_mnmajor(kh, kk), umma_mnmajor(vt, kk), idb_mm, kk > 0);
+        for (int kk = 0; kk < 4; ++kk) umma_bf16(tm + kColS, dk + kk * 128, dv + kk * 128, idb_mm, kk > 0);
         umma_commit(&sm.mma_bar);
         ++mma_issued;
       }
@@ -422,8 +417,8 @@ __global__ void __launch_bounds__(kThreads6, 2)
               const float a1 = s + 1 < row ? a[e + 1] : (s + 1 == row ? bj : 0.f);
               split_bf16x2(a0, a1, ph[e / 2], pl[e / 2]);
             }
-            tile_st_row16(sm.kf[0], row, 2 * ch + q, ph);
-            tile_st_row16(sm.kf[1], row, 2 * ch + q, pl);
+            tile_st_row16(sm.bt[0], row, 2 * ch + q, ph);
+            tile_st_row16(sm.bt[1], row, 2 * ch + q, pl);
           }
         }
         const float dj = holder ? sm.dec[row] : 0.f;
@@ -446,11 +441,13 @@ __global__ void __launch_bounds__(kThreads6, 2)
       // ---- G. MMA3 O += mask(A) V (hi and lo passes); written out next unit ----
       if (tid == 0) {
         tc_fence_after_sync();
-        const uint32_t amh = smem_u32(sm.kf[0]), aml = smem_u32(sm.kf[1]);
+        const uint64_t dh = umma_desc_sw128(smem_u32(sm.bt[0]), 16, 1024);
+        const uint64_t dl = umma_desc_sw128(smem_u32(sm.bt[1]), 16, 1024);
+        const uint64_t dv = umma_desc_sw128(vt, 8192, 1024);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) umma_bf16(tm + kColO, umma_kmajor(amh, kk), umma_mnmajor(vt, kk), idb_km, true);
+        for (int kk = 0; kk < 4; ++kk) umma_bf16(tm + kColO, dh + kk * 2, dv + kk * 128, idb_km, true);
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) umma_bf16(tm + kColO, umma_kmajor(aml, kk), umma_mnmajor(vt, kk), idb_km, true);
+        for (int kk = 0; kk < 4; ++kk) umma_bf16(tm + kColO, dl + kk * 2, dv + kk * 128, idb_km, true);
         umma_commit(&sm.mma_bar);
         ++mma_issued;
       }
