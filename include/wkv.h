@@ -70,7 +70,7 @@ extern "C" {
 #define WKV_ABI_VERSION 1
 
 /* Steps between two RWKV-4 forward state checkpoints (see wkv4_forward). */
-#define WKV4_CKPT_LEN 32
+#define WKV4_CKPT_LEN 16
 
 typedef enum {
     WKV_OK = 0,

@@ -12,14 +12,23 @@
 //   decay gradient   A'_i = sum_{t>i} (t-1-i) alpha_t e^{-(t-1-i) w},
 //                    gw -= e^{k_i} (v_i A'_i - B'_i)
 // A, B, A', B' follow the reverse recurrences A_{i-1} = alpha_i + e^{-w} A_i,
-// A'_{i-1} = e^{-w} (A'_i + A_i). They are carried as mantissas under one
-// shared base-2 exponent R (A = Am * 2^R) that is a running max of the term
-// exponents -q_t - (t-1-i) w, kept like the forward's exponent as a base and
-// an exact step count; then the factor e^{k_i} * 2^R has exponent <= 0
-// because q_t >= P_t >= k_i - (t-1-i) w.
+// A'_{i-1} = e^{-w} (A'_i + A_i). They are carried normalised by the
+// forward's own exponent after token i: A~_i = A_i 2^{P_{i+1}} (P the
+// base-2 exponent of the running-max state, P_{i+1} = max(P_i - w, k_i)).
+// Then every coefficient of the reverse scan is a factor the forward step
+// already forms, all <= 1 (base 2, w and k pre-scaled by log2 e):
+//   absorb of token i   f1_i = 2^{P_i - w - P_{i+1}}, f2_i = 2^{k_i - P_{i+1}}
+//   output of token i   e1_i = 2^{P_i - q_i},  e2_i = 2^{u + k_i - q_i},
+//                       den_i = e1 bb + e2,  D_i = 2^{q_i} den_i
+// (one of f1/f2 and one of e1/e2 is exactly 1), and walking i downwards
+//   gv_i += f2_i A~_i,   gk_i += f2_i (v_i A~_i - B~_i),
+//   gw   -= f2_i (v_i A~'_i - B~'_i),
+//   A~'_{i-1} = f1_i (A~'_i + A~_i),  A~_{i-1} = f1_i A~_i + gy_i e1_i / den_i
+// (B~ the same with gy_i y_i). The carries stay bounded by sum |gy| and need
+// no exponent of their own; the loop-carried dependence is one multiply-add.
 //
 // Kernel shape. One warp = 32 channels of one sample; time is walked in
-// reverse one checkpoint interval (WKV4_CKPT_LEN = 32 steps) at a time: the
+// reverse one checkpoint interval (WKV4_CKPT_LEN = 16 steps) at a time: the
 // warp restarts the forward recurrence from the interval's checkpoint, keeps
 // the 32 states in registers, then runs the 32 reverse steps. k, v, gy of an
 // interval arrive as one TMA stage of a ring. When lanes are few, each lane's
@@ -37,47 +46,37 @@ namespace wkv {
 
 constexpr int kBwdL = WKV4_CKPT_LEN;
 
+template <bool V>
+struct BoolTag {
+  static constexpr bool value = V;
+};
+
 template <class E, int STAGES>
 struct alignas(128) Wkv4BwdSmem {
   E k[STAGES][kBwdL][32];
   E v[STAGES][kBwdL][32];
   E gy[STAGES][kBwdL][32];
   uint64_t full[STAGES];
-  float carry[5][32];  // this segment's local carry: Am, Bm, Apm, Bpm, R
+  float carry[5][32];  // this segment's local carry A, B, A', B' and its product of f1
 };
 
-// Carried future sums of one lane: mantissas under the exponent R.
+// Carried future sums of one lane, normalised by 2^{P} of the forward state
+// at the point they refer to (see above).
 struct Wkv4Carry {
-  float Am, Bm, Apm, Bpm, R;
+  float A, B, Ap, Bp;
 };
-
-// Move a carry `m` steps further back in time: A' gains m A, the exponent
-// loses m w2 (A'_{i-m} = e^{-m w} (A'_i + m A_i)).
-__device__ __forceinline__ Wkv4Carry wkv4_carry_shift(Wkv4Carry c, float m, float w2) {
-  c.Apm = __fmaf_rn(m, c.Am, c.Apm);
-  c.Bpm = __fmaf_rn(m, c.Bm, c.Bpm);
-  c.R = __fmaf_rn(-m, w2, c.R);
-  return c;
-}
-
-__device__ __forceinline__ Wkv4Carry wkv4_carry_merge(const Wkv4Carry& x, const Wkv4Carry& y) {
-  const float d = __fsub_rn(x.R, y.R);
-  const float e = ex2(-fabsf(d));
-  const bool xm = d >= 0.f;
-  const float fx = xm ? 1.f : e;
-  const float fy = xm ? e : 1.f;
-  return {__fmaf_rn(fx, x.Am, __fmul_rn(fy, y.Am)), __fmaf_rn(fx, x.Bm, __fmul_rn(fy, y.Bm)),
-          __fmaf_rn(fx, x.Apm, __fmul_rn(fy, y.Apm)), __fmaf_rn(fx, x.Bpm, __fmul_rn(fy, y.Bpm)),
-          xm ? x.R : y.R};
-}
 
 // One checkpoint interval in reverse. FULL: also produce gk, gv, gw, gu;
 // otherwise only fold the interval into the carry.
+// fprod (fold-only pass) accumulates the product of the f1 factors. The
+// steps stay predicated on j < n even for whole intervals: without the
+// per-step branches the compiler interleaves all steps and runs out of
+// registers.
 template <bool FULL, class E>
 __device__ __forceinline__ void wkv4_bwd_interval(const E (*ks)[32], const E (*vs)[32], const E (*gs)[32], int lane,
-                                                  int n, Wkv4State st, float ref, float u2, float w2, float& rbase,
-                                                  float& rn, float& Am, float& Bm, float& Apm, float& Bpm,
-                                                  float& gw_acc, float& gu_acc, E* gkl, E* gvl, int C) {
+                                                  int n, Wkv4State st, float ref, float u2, float w2, Wkv4Carry& cr,
+                                                  float& fprod, float& gw_acc, float& gu_acc, E* gkl, E* gvl,
+                                                  int C) {
   // forward recompute over the interval: state before each token
   float saa[kBwdL], sbb[kBwdL], spp[kBwdL];
 #pragma unroll
@@ -89,61 +88,55 @@ __device__ __forceinline__ void wkv4_bwd_interval(const E (*ks)[32], const E (*v
       wkv4_absorb(st, wkv4_key(Elem<E>::to_f32(ks[jj][lane]), ref), Elem<E>::to_f32(vs[jj][lane]), w2);
     }
   }
+  float A = cr.A, B = cr.B, Ap = cr.Ap, Bp = cr.Bp;
 #pragma unroll
   for (int jj = kBwdL - 1; jj >= 0; --jj) {
     if (jj < n) {
       const float k2 = wkv4_key(Elem<E>::to_f32(ks[jj][lane]), ref);
       const float vv = Elem<E>::to_f32(vs[jj][lane]);
       const float g = Elem<E>::to_f32(gs[jj][lane]);
-      // output of token jj: D = 2^q * den
-      const float cur = __fadd_rn(u2, k2);
-      const float d = __fsub_rn(spp[jj], cur);
+      const float P = spp[jj];
+      // output pair of token jj: q = max(P, u + k)
+      const float d = __fsub_rn(P, __fadd_rn(u2, k2));
       const float e = ex2(-fabsf(d));
       const bool past_max = d >= 0.f;
       const float e1 = past_max ? 1.f : e;
       const float e2 = past_max ? e : 1.f;
-      const float q = past_max ? spp[jj] : cur;
-      const float num = __fmaf_rn(e1, saa[jj], __fmul_rn(e2, vv));
-      const float den = __fmaf_rn(e1, sbb[jj], e2);
-      const float rd = rcp(den);
-      const float yv = __fmul_rn(num, rd);
-      const float alpha = __fmul_rn(g, rd);     // alpha_t * 2^q
-      const float beta = __fmul_rn(alpha, yv);  // beta_t * 2^q
+      const float rd = rcp(__fmaf_rn(e1, sbb[jj], e2));
+      const float yv = __fmul_rn(__fmaf_rn(e1, saa[jj], __fmul_rn(e2, vv)), rd);
+      // absorb pair of token jj: P' = max(P - w, k)
+      const float z = __fsub_rn(k2, __fsub_rn(P, w2));
+      const float ea = ex2(-fabsf(z));
+      const bool keep = z <= 0.f;
+      const float f1 = keep ? 1.f : ea;
+      const float f2 = keep ? ea : 1.f;
+      const float gr = __fmul_rn(g, rd);
+      const float ag = __fmul_rn(gr, e1);  // gy e1 / den
       if constexpr (FULL) {
-        const float gloc = __fmul_rn(alpha, e2);  // gy_t rho_t
+        const float rg = __fmul_rn(gr, e2);  // gy rho
         // v - y = e1 (bb v - aa) / den: no cancellation against v when the
         // current token dominates (y within rounding of v)
         const float vmy = __fmul_rn(__fmul_rn(e1, __fmaf_rn(sbb[jj], vv, -saa[jj])), rd);
-        float gvv = gloc;
-        float gkv = __fmul_rn(gloc, vmy);
-        gu_acc = __fadd_rn(gu_acc, gkv);
-        // tokens after jj, through the carried sums
-        const float f = ex2(__fadd_rn(k2, __fmaf_rn(-rn, w2, rbase)));
-        gvv = __fmaf_rn(f, Am, gvv);
-        gkv = __fmaf_rn(f, __fmaf_rn(vv, Am, -Bm), gkv);
-        gw_acc = __fmaf_rn(-f, __fmaf_rn(vv, Apm, -Bpm), gw_acc);
+        const float gvv = __fmaf_rn(f2, A, rg);
+        const float gkv = __fmaf_rn(rg, vmy, __fmul_rn(f2, __fmaf_rn(vv, A, -B)));
+        gu_acc = __fmaf_rn(rg, vmy, gu_acc);
+        gw_acc = __fmaf_rn(-f2, __fmaf_rn(vv, Ap, -Bp), gw_acc);
         gkl[(int64_t)jj * C] = Elem<E>::from_f32(gkv);
         gvl[(int64_t)jj * C] = Elem<E>::from_f32(gvv);
       }
-      // fold token jj into the carry (new exponent max(R - w, -q))
-      const float rn1 = __fadd_rn(rn, 1.f);
-      const float dd = __fmaf_rn(-rn1, w2, __fadd_rn(rbase, q));  // (R - w) - (-q)
-      const float ef = ex2(-fabsf(dd));
-      const bool keep = dd >= 0.f;
-      const float fo = keep ? 1.f : ef;
-      const float fn = keep ? ef : 1.f;
-      Apm = __fmul_rn(fo, __fadd_rn(Apm, Am));
-      Bpm = __fmul_rn(fo, __fadd_rn(Bpm, Bm));
-      Am = __fmaf_rn(fo, Am, __fmul_rn(fn, alpha));
-      Bm = __fmaf_rn(fo, Bm, __fmul_rn(fn, beta));
-      rbase = keep ? rbase : -q;
-      rn = keep ? rn1 : 0.f;
+      if constexpr (!FULL) fprod = __fmul_rn(fprod, f1);
+      // carries for token jj - 1
+      Ap = __fmul_rn(f1, __fadd_rn(Ap, A));
+      Bp = __fmul_rn(f1, __fadd_rn(Bp, B));
+      A = __fmaf_rn(f1, A, ag);
+      B = __fmaf_rn(f1, B, __fmul_rn(ag, yv));
     }
   }
+  cr = {A, B, Ap, Bp};
 }
 
 template <class E, int STAGES, int NSEG, int NW>
-__global__ void __launch_bounds__(32 * NW) wkv4_bwd_kernel(const __grid_constant__ CUtensorMap tk,
+__global__ void __launch_bounds__(32 * NW, NSEG == 1 ? 16 : 1) wkv4_bwd_kernel(const __grid_constant__ CUtensorMap tk,
                                                            const __grid_constant__ CUtensorMap tv,
                                                            const __grid_constant__ CUtensorMap tg, int T, int C,
                                                            int ncb, int ngroups, const float* __restrict__ w,
@@ -215,66 +208,67 @@ __global__ void __launch_bounds__(32 * NW) wkv4_bwd_kernel(const __grid_constant
     if (lane == 0 && x + STAGES < total) issue(x + STAGES);
   };
 
-  // reverse carry: A = Am 2^R etc. with R = rbase - rn * w2 (counted decay,
-  // as in the forward); R starts at the "empty" exponent
-  float rbase = kEmptyPP, rn = 0.f, Am = 0.f, Bm = 0.f, Apm = 0.f, Bpm = 0.f;
+  // reverse carries (normalised by the forward exponent, see above)
+  Wkv4Carry cr = {0.f, 0.f, 0.f, 0.f};
   float gw_acc = 0.f, gu_acc = 0.f;
+  auto run_interval = [&](auto full_tag, int s, int i, const Wkv4State& st, float& fprod) {
+    constexpr bool kFull = decltype(full_tag)::value;
+    const int n = min(kBwdL, T - i * kBwdL);
+    const int64_t off = lane_off + (int64_t)i * kBwdL * C;
+    E* gkp = kFull ? gk + off : nullptr;
+    E* gvp = kFull ? gv + off : nullptr;
+    wkv4_bwd_interval<kFull, E>(sm.k[s], sm.v[s], sm.gy[s], lane, n, st, ref, u2, w2, cr, fprod, gw_acc, gu_acc,
+                                gkp, gvp, C);
+  };
 
   if constexpr (NSEG > 1) {
     // ---- phase 1: this segment's own carry, from an empty future ----
+    float fprod = 1.f;
     Wkv4State nxt = nloc > 0 ? load_ckpt(interval(0)) : Wkv4State{0.f, 0.f, 0.f, 0.f};
     for (; ok && qq < nloc; ++qq) {
       const int i = interval(qq);
       const Wkv4State st = nxt;
       if (qq + 1 < nloc) nxt = load_ckpt(interval(qq + 1));
       if (!acquire(qq)) break;
-      const int s = qq % STAGES;
-      if (valid)
-        wkv4_bwd_interval<false, E>(sm.k[s], sm.v[s], sm.gy[s], lane, min(kBwdL, T - i * kBwdL), st, ref, u2, w2,
-                                    rbase, rn, Am, Bm, Apm, Bpm, gw_acc, gu_acc, nullptr, nullptr, C);
+      if (valid) run_interval(BoolTag<false>{}, qq % STAGES, i, st, fprod);
       release(qq);
     }
-    sm.carry[0][lane] = Am;
-    sm.carry[1][lane] = Bm;
-    sm.carry[2][lane] = Apm;
-    sm.carry[3][lane] = Bpm;
-    sm.carry[4][lane] = __fmaf_rn(-rn, w2, rbase);
+    sm.carry[0][lane] = cr.A;
+    sm.carry[1][lane] = cr.B;
+    sm.carry[2][lane] = cr.Ap;
+    sm.carry[3][lane] = cr.Bp;
+    sm.carry[4][lane] = fprod;
     cluster_arrive_release();
     cluster_wait_acquire();
     // ---- phase 2: the exact carry entering this segment from the later ones ----
-    Wkv4Carry in = {0.f, 0.f, 0.f, 0.f, kEmptyPP};
+    Wkv4Carry in = {0.f, 0.f, 0.f, 0.f};
     for (int r = NSEG - 1; r > seg; --r) {
       const int len = min(T, wkv4_seg_begin(r + 1, NSEG, nck) * kBwdL) - wkv4_seg_begin(r, NSEG, nck) * kBwdL;
-      const Wkv4Carry own = {ld_shared_cluster(map_shared_rank(&sm.carry[0][lane], r)),
-                             ld_shared_cluster(map_shared_rank(&sm.carry[1][lane], r)),
-                             ld_shared_cluster(map_shared_rank(&sm.carry[2][lane], r)),
-                             ld_shared_cluster(map_shared_rank(&sm.carry[3][lane], r)),
-                             ld_shared_cluster(map_shared_rank(&sm.carry[4][lane], r))};
-      in = wkv4_carry_merge(own, wkv4_carry_shift(in, (float)len, w2));
+      const float f = ld_shared_cluster(map_shared_rank(&sm.carry[4][lane], r));
+      const float m = (float)len;
+      in = {__fmaf_rn(f, in.A, ld_shared_cluster(map_shared_rank(&sm.carry[0][lane], r))),
+            __fmaf_rn(f, in.B, ld_shared_cluster(map_shared_rank(&sm.carry[1][lane], r))),
+            __fmaf_rn(f, __fmaf_rn(m, in.A, in.Ap), ld_shared_cluster(map_shared_rank(&sm.carry[2][lane], r))),
+            __fmaf_rn(f, __fmaf_rn(m, in.B, in.Bp), ld_shared_cluster(map_shared_rank(&sm.carry[3][lane], r)))};
     }
     cluster_arrive_release();  // done reading peers; waited for before exit
-    Am = in.Am;
-    Bm = in.Bm;
-    Apm = in.Apm;
-    Bpm = in.Bpm;
-    rbase = in.R;
-    rn = 0.f;
+    cr = in;
+    gw_acc = 0.f;
+    gu_acc = 0.f;
   }
 
   // ---- last pass: gradients ----
-  Wkv4State nxt = nloc > 0 ? load_ckpt(interval(0)) : Wkv4State{0.f, 0.f, 0.f, 0.f};
-  for (; ok && qq < total; ++qq) {
-    const int i = interval(qq);
-    const Wkv4State st = nxt;
-    if (qq + 1 < total) nxt = load_ckpt(interval(qq + 1));
-    if (!acquire(qq)) break;
-    const int s = qq % STAGES;
-    if (valid) {
-      const int64_t off = lane_off + (int64_t)i * kBwdL * C;
-      wkv4_bwd_interval<true, E>(sm.k[s], sm.v[s], sm.gy[s], lane, min(kBwdL, T - i * kBwdL), st, ref, u2, w2, rbase,
-                                 rn, Am, Bm, Apm, Bpm, gw_acc, gu_acc, gk + off, gv + off, C);
+  {
+    float unused = 1.f;
+    Wkv4State nxt = nloc > 0 ? load_ckpt(interval(0)) : Wkv4State{0.f, 0.f, 0.f, 0.f};
+    for (; ok && qq < total; ++qq) {
+      const int i = interval(qq);
+      const Wkv4State st = nxt;
+      if (qq + 1 < total) nxt = load_ckpt(interval(qq + 1));
+      if (!acquire(qq)) break;
+      if (valid) run_interval(BoolTag<true>{}, qq % STAGES, i, st, unused);
+      release(qq);
     }
-    release(qq);
   }
   if (!ok) {
     if (lane == 0)
@@ -350,9 +344,9 @@ static wkv_status run_bwd(const Wkv4BwdArgs& a, cudaStream_t stream, unsigned* e
   return WKV_OK;
 }
 
-// Stages of the k/v/gy ring: two for bf16 (12 KB each); for float32 (24 KB
-// a stage) one when the sequence is split, so that the ~10 one-warp CTAs an
-// SM then holds still fit in shared memory.
+// Stages of the k/v/gy ring (one checkpoint interval each): four for bf16
+// (3 KB a stage), two for float32 (6 KB), so that the 14-16 one-warp CTAs an
+// SM holds still fit in shared memory.
 template <class E, int STAGES, int NSEG>
 static wkv_status run_bwd_nw(const Wkv4BwdArgs& a, cudaStream_t stream, unsigned* err, const char** why) {
   switch (wkv4_warps_per_cta(a.B, a.C, NSEG)) {
@@ -362,17 +356,14 @@ static wkv_status run_bwd_nw(const Wkv4BwdArgs& a, cudaStream_t stream, unsigned
   }
 }
 
-#ifndef WKV4_BWD_SPLIT_STAGES_F32
-#define WKV4_BWD_SPLIT_STAGES_F32 1
-#endif
 template <class E>
 static wkv_status run_bwd_nseg(const Wkv4BwdArgs& a, cudaStream_t stream, unsigned* err, const char** why) {
-  constexpr int kSplitStages = sizeof(E) == 2 ? 2 : WKV4_BWD_SPLIT_STAGES_F32;
+  constexpr int kStages = sizeof(E) == 2 ? 4 : 2;
   switch (wkv4_bwd_segments(a.B, a.T, a.C)) {
-    case 8: return run_bwd_nw<E, kSplitStages, 8>(a, stream, err, why);
-    case 4: return run_bwd_nw<E, kSplitStages, 4>(a, stream, err, why);
-    case 2: return run_bwd_nw<E, kSplitStages, 2>(a, stream, err, why);
-    default: return run_bwd<E, 2, 1, 1>(a, stream, err, why);
+    case 8: return run_bwd_nw<E, kStages, 8>(a, stream, err, why);
+    case 4: return run_bwd_nw<E, kStages, 4>(a, stream, err, why);
+    case 2: return run_bwd_nw<E, kStages, 2>(a, stream, err, why);
+    default: return run_bwd<E, kStages, 1, 1>(a, stream, err, why);
   }
 }
 

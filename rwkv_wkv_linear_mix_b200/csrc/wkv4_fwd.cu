@@ -44,7 +44,7 @@ __global__ void __launch_bounds__(32 * NW) wkv4_fwd_kernel(const __grid_constant
                                                            int ngroups, const float* __restrict__ w,
                                                            const float* __restrict__ u, E* __restrict__ y,
                                                            float* __restrict__ ckpt, unsigned* err) {
-  static_assert(WKV4_CKPT_LEN % LT == 0, "checkpoint interval must be a whole number of tiles");
+  static_assert(LT % WKV4_CKPT_LEN == 0, "a tile must hold whole checkpoint intervals");
   extern __shared__ __align__(128) unsigned char wkv4_fwd_dsmem[];
   // each warp is an independent lane group with its own ring and barriers
   Wkv4FwdSmem<E, LT, STAGES>& sm = reinterpret_cast<Wkv4FwdSmem<E, LT, STAGES>*>(wkv4_fwd_dsmem)[threadIdx.x / 32];
@@ -136,14 +136,16 @@ __global__ void __launch_bounds__(32 * NW) wkv4_fwd_kernel(const __grid_constant
 
   // ---- last pass: outputs and checkpoints ----
   E* yl = y ? y + lane_off : nullptr;
+  // state before token t (t a multiple of WKV4_CKPT_LEN) to the checkpoints
+  auto write_ckpt = [&](int t) {
+    float* p = ckl + (int64_t)(t / WKV4_CKPT_LEN) * 3 * C;
+    p[0] = st.aa;
+    p[C] = st.bb;
+    p[2 * (int64_t)C] = wkv4_exponent(st, w2);
+  };
   for (; ok && q < total; ++q) {
-    const int t0 = t_beg + (q % ntile) * LT;
-    if (ckl && valid && (t0 % WKV4_CKPT_LEN) == 0) {
-      float* p = ckl + (int64_t)(t0 / WKV4_CKPT_LEN) * 3 * C;
-      p[0] = st.aa;
-      p[C] = st.bb;
-      p[2 * (int64_t)C] = wkv4_exponent(st, w2);
-    }
+    const int t0 = t_beg + (q % ntile) * LT;  // a multiple of WKV4_CKPT_LEN
+    if (ckl && valid) write_ckpt(t0);
     if (!acquire(q)) break;
     const int s = q % STAGES;
     const int n = min(LT, t_end - t0);
@@ -152,12 +154,14 @@ __global__ void __launch_bounds__(32 * NW) wkv4_fwd_kernel(const __grid_constant
       if (n == LT) {
 #pragma unroll 8
         for (int j = 0; j < LT; ++j) {
+          if (j > 0 && j % WKV4_CKPT_LEN == 0 && ckl) write_ckpt(t0 + j);
           const float yv = wkv4_token(st, wkv4_key(Elem<E>::to_f32(sm.k[s][j][lane]), ref),
                                       Elem<E>::to_f32(sm.v[s][j][lane]), u2, w2);
           if (yt) yt[(int64_t)j * C] = Elem<E>::from_f32(yv);
         }
       } else {
         for (int j = 0; j < n; ++j) {
+          if (j > 0 && j % WKV4_CKPT_LEN == 0 && ckl) write_ckpt(t0 + j);
           const float yv = wkv4_token(st, wkv4_key(Elem<E>::to_f32(sm.k[s][j][lane]), ref),
                                       Elem<E>::to_f32(sm.v[s][j][lane]), u2, w2);
           if (yt) yt[(int64_t)j * C] = Elem<E>::from_f32(yv);

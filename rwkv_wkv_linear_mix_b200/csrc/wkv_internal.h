@@ -26,13 +26,18 @@ __host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) { ret
 
 // Number of sequence segments each RWKV-4 lane is split into (the cluster
 // size of a kernel): doubled while the launch has fewer warps than
-// WKV4_TARGET_WARPS and every segment keeps at least two checkpoint
-// intervals; at most max_seg (<= 8, the portable cluster size).
+// WKV4_TARGET_WARPS and every segment keeps at least WKV4_MIN_SEG_STEPS
+// steps (splitting reruns each segment, so short ones do not pay); at most
+// max_seg (<= 8, the portable cluster size).
+#ifndef WKV4_MIN_SEG_STEPS
+#define WKV4_MIN_SEG_STEPS 64
+#endif
 inline int wkv4_segments_capped(int64_t B, int64_t T, int64_t C, int max_seg) {
   const int64_t groups = B * ceil_div(C, 32);
-  const int64_t nck = ceil_div(T, WKV4_CKPT_LEN);
+  const int64_t steps = ceil_div(T, WKV4_CKPT_LEN) * WKV4_CKPT_LEN;
   int nseg = 1;
-  while (nseg < max_seg && groups * nseg < (int64_t)(WKV4_TARGET_WARPS) && nck >= 4 * nseg) nseg *= 2;
+  while (nseg < max_seg && groups * nseg < (int64_t)(WKV4_TARGET_WARPS) && steps >= 2 * WKV4_MIN_SEG_STEPS * nseg)
+    nseg *= 2;
   return nseg;
 }
 // Warps (independent 32-channel lane groups) per CTA of a split launch: the

@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(_PKG, "libwkv_b200.so")
 WKV_OK, WKV_ERR_INVALID_ARG, WKV_ERR_UNSUPPORTED, WKV_ERR_CUDA, WKV_ERR_DEVICE = range(5)
 WKV_F32, WKV_BF16 = 0, 1
 WKV_DEVERR_WAIT_TIMEOUT, WKV_DEVERR_BAD_SLOT, WKV_DEVERR_BAD_STATE = 1, 2, 4
-CKPT_LEN = 32  # WKV4_CKPT_LEN
+CKPT_LEN = 16  # WKV4_CKPT_LEN
 
 # Every symbol include/wkv.h declares, with its ctypes signature.
 _i64, _i32, _int, _vp, _sz = ctypes.c_int64, ctypes.c_int32, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t

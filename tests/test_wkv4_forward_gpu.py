@@ -127,15 +127,15 @@ def test_deterministic_and_ckpt_only(W):
 
 
 def test_checkpoint_state_matches_oracle(W, oracle):
-    # the state before token 32n, as exact sums a = aa 2^pp, b = bb 2^pp
+    # the state before token CKPT_LEN * n, as exact sums a = aa 2^pp, b = bb 2^pp
     rec = synth.WKV4_RECIPES["wkv4_fwd_f32_small"].with_shape(2, 96, 32)
     inp = synth.wkv4_inputs(rec, seed=9)
     _, ck = run_fwd(W, inp, want_ckpt=True)
     ck = host64(ck)
     # lane reference: fl(k[b, 0, c] * log2 e) in float32
     ref_exp = (inp["k32"][:, 0, :] * np.float32(1.4426950408889634)).astype(np.float32).astype(np.float64)
-    for n in (1, 2):
-        t = 32 * n
+    for n in (1, 2, 96 // W.CKPT_LEN - 1):
+        t = W.CKPT_LEN * n
         _, st = oracle.wkv4_forward(inp["w"], inp["u"], inp["k32"][:, :t], inp["v32"][:, :t], return_state=True)
         log_b = np.log(st["b_end"]) + st["kmax"]
         ratio = st["a_end"] / st["b_end"]
