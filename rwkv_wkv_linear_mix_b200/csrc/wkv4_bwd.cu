@@ -68,11 +68,11 @@ struct Wkv4Carry {
 
 // One checkpoint interval in reverse. FULL: also produce gk, gv, gw, gu;
 // otherwise only fold the interval into the carry.
-// fprod (fold-only pass) accumulates the product of the f1 factors. The
-// steps stay predicated on j < n even for whole intervals: without the
-// per-step branches the compiler interleaves all steps and runs out of
-// registers.
-template <bool FULL, class E>
+// fprod (fold-only pass) accumulates the product of the f1 factors. WHOLE
+// (n == kBwdL): the reverse steps are not predicated, so the compiler can
+// overlap the independent parts of consecutive steps; the recompute loop
+// always is (unpredicated, both loops together need too many registers).
+template <bool FULL, bool WHOLE, class E>
 __device__ __forceinline__ void wkv4_bwd_interval(const E (*ks)[32], const E (*vs)[32], const E (*gs)[32], int lane,
                                                   int n, Wkv4State st, float ref, float u2, float w2, Wkv4Carry& cr,
                                                   float& fprod, float& gw_acc, float& gu_acc, E* gkl, E* gvl,
@@ -91,7 +91,7 @@ __device__ __forceinline__ void wkv4_bwd_interval(const E (*ks)[32], const E (*v
   float A = cr.A, B = cr.B, Ap = cr.Ap, Bp = cr.Bp;
 #pragma unroll
   for (int jj = kBwdL - 1; jj >= 0; --jj) {
-    if (jj < n) {
+    if (WHOLE || jj < n) {
       const float k2 = wkv4_key(Elem<E>::to_f32(ks[jj][lane]), ref);
       const float vv = Elem<E>::to_f32(vs[jj][lane]);
       const float g = Elem<E>::to_f32(gs[jj][lane]);
@@ -217,8 +217,13 @@ __global__ void __launch_bounds__(32 * NW, NSEG == 1 ? 16 : 1) wkv4_bwd_kernel(c
     const int64_t off = lane_off + (int64_t)i * kBwdL * C;
     E* gkp = kFull ? gk + off : nullptr;
     E* gvp = kFull ? gv + off : nullptr;
-    wkv4_bwd_interval<kFull, E>(sm.k[s], sm.v[s], sm.gy[s], lane, n, st, ref, u2, w2, cr, fprod, gw_acc, gu_acc,
-                                gkp, gvp, C);
+    // unpredicated steps for whole bf16 intervals (float32 would spill)
+    if (sizeof(E) == 2 && n == kBwdL)
+      wkv4_bwd_interval<kFull, sizeof(E) == 2, E>(sm.k[s], sm.v[s], sm.gy[s], lane, n, st, ref, u2, w2, cr, fprod, gw_acc,
+                                        gu_acc, gkp, gvp, C);
+    else
+      wkv4_bwd_interval<kFull, false, E>(sm.k[s], sm.v[s], sm.gy[s], lane, n, st, ref, u2, w2, cr, fprod, gw_acc,
+                                         gu_acc, gkp, gvp, C);
   };
 
   if constexpr (NSEG > 1) {

@@ -152,12 +152,16 @@ __global__ void __launch_bounds__(32 * NW) wkv4_fwd_kernel(const __grid_constant
     if (valid) {
       E* yt = yl ? yl + (int64_t)t0 * C : nullptr;
       if (n == LT) {
+#pragma unroll
+        for (int jc = 0; jc < LT; jc += WKV4_CKPT_LEN) {
+          if (jc > 0 && ckl) write_ckpt(t0 + jc);
 #pragma unroll 8
-        for (int j = 0; j < LT; ++j) {
-          if (j > 0 && j % WKV4_CKPT_LEN == 0 && ckl) write_ckpt(t0 + j);
-          const float yv = wkv4_token(st, wkv4_key(Elem<E>::to_f32(sm.k[s][j][lane]), ref),
-                                      Elem<E>::to_f32(sm.v[s][j][lane]), u2, w2);
-          if (yt) yt[(int64_t)j * C] = Elem<E>::from_f32(yv);
+          for (int j2 = 0; j2 < WKV4_CKPT_LEN; ++j2) {
+            const int j = jc + j2;
+            const float yv = wkv4_token(st, wkv4_key(Elem<E>::to_f32(sm.k[s][j][lane]), ref),
+                                        Elem<E>::to_f32(sm.v[s][j][lane]), u2, w2);
+            if (yt) yt[(int64_t)j * C] = Elem<E>::from_f32(yv);
+          }
         }
       } else {
         for (int j = 0; j < n; ++j) {
