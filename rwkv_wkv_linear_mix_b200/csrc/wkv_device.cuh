@@ -302,8 +302,10 @@ __device__ __forceinline__ float bf16hi(uint32_t p) { return __uint_as_float(p &
 //    half an ulp per step, always in the same direction).
 //  * each max-pair costs one ex2 and a select (one of its exponents is 0).
 // u2 = u * log2e, w2 = w * log2e. For token t with kk:
-//   output  zo = (u2 + kk) - P;   y = (2^{min(-zo,0)} aa + 2^{min(zo,0)} v)
-//                                   / (2^{min(-zo,0)} bb + 2^{min(zo,0)})
+//   output  zo = (u2 + kk) - P;   y = (aa + 2^{min(zo,64)} v) / (bb + 2^{min(zo,64)})
+//           (bb >= 1 once a token is absorbed and bb <= number of tokens, so
+//           beyond 2^64 the past is far below float32 resolution of the sum;
+//           the empty past, aa = bb = 0, gives y = v exactly)
 //   absorb  z1 = kk - (P - w2);   aa <- 2^{min(-z1,0)} aa + 2^{min(z1,0)} v,
 //                                 bb likewise, and (base, n) <- (base, n + 1)
 //                                 if z1 <= 0 else (kk, 0).
@@ -330,15 +332,10 @@ __device__ __forceinline__ float wkv4_exponent(const Wkv4State& s, float w2) {
 // Output of the token, then absorb it. Returns y.
 __device__ __forceinline__ float wkv4_token(Wkv4State& s, float kk, float v, float u2, float w2) {
   const float y0 = __fsub_rn(kk, s.base);
-  // output pair: current token (u2 + kk) against the past P
+  // output: weight of the current token (u2 + kk) relative to the past P
   const float zo = __fmaf_rn(s.n, w2, __fadd_rn(y0, u2));
-  const float eo = ex2(-fabsf(zo));
-  const bool po = zo <= 0.f;  // past holds the maximum
-  const float e1 = po ? 1.f : eo;
-  const float e2 = po ? eo : 1.f;
-  const float num = __fmaf_rn(e1, s.aa, __fmul_rn(e2, v));
-  const float den = __fmaf_rn(e1, s.bb, e2);
-  const float y = __fmul_rn(num, rcp(den));
+  const float e = ex2(fminf(zo, 64.f));
+  const float y = __fmul_rn(__fmaf_rn(e, v, s.aa), rcp(__fadd_rn(s.bb, e)));
   // absorb pair: token kk against the decayed past P - w2
   const float n1 = __fadd_rn(s.n, 1.f);
   const float z1 = __fmaf_rn(n1, w2, y0);
