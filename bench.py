@@ -47,6 +47,9 @@ WORKLOAD = "wkv4_fb_f32_169m"
 METRIC = "WKV fwd+bwd throughput (G tok·ch/s)"
 UNIT = "G tok*ch/s"
 L2_FLUSH_BYTES = 320 << 20
+# sources that determine the backward kernel's code and launch shape
+BWD_SOURCES = ["rwkv_wkv_linear_mix_b200/csrc/wkv4_bwd.cu", "rwkv_wkv_linear_mix_b200/csrc/wkv_device.cuh",
+               "rwkv_wkv_linear_mix_b200/csrc/wkv_internal.h", "include/wkv.h"]
 
 
 def parse():
@@ -90,17 +93,19 @@ def kernel_source_hash(files):
 
 
 def recorded_traffic(kernel, workload, src_hash):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current source of the kernel; else None."""
-    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    """DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum)
+    from the committed ncu summary profiles/dram_traffic.txt, if it was taken
+    on the current source of the kernel; else None. Each line of that file
+    reads: kernel workload source_hash bytes_per_launch."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(p):
         return None
     with open(p) as f:
-        d = json.load(f)
-    e = d.get(f"{kernel}:{workload}")
-    if not e or e.get("source_hash") != src_hash:
-        return None
-    return e.get("bytes_per_launch")
+        for line in f:
+            parts = line.split()
+            if len(parts) == 4 and not line.startswith("#") and parts[:3] == [kernel, workload, src_hash]:
+                return float(parts[3])
+    return None
 
 
 class ClockSampler:
@@ -427,31 +432,66 @@ def run_ours(args):
     value = tok_ch * world / (step_ms_max * 1e-3) / 1e9
 
     # ---- end to end through the C ABI with pinned host buffers ----
-    hk, hv, hgy = (torch.from_numpy(np.ascontiguousarray(inp[n])).pin_memory() for n in ("k", "v", "gy"))
-    hw, hu = (torch.from_numpy(np.ascontiguousarray(inp[n])).pin_memory() for n in ("w", "u"))
+    # Every step copies its inputs host -> device, runs forward + backward and
+    # copies its results device -> host. Consecutive steps alternate between
+    # two device buffer sets on separate copy-in / compute / copy-out streams,
+    # so one step's results travel back while the next step's inputs arrive
+    # (PCIe moves both directions at once); events order each buffer's reuse.
+    H = {n: torch.from_numpy(np.ascontiguousarray(inp[n])).pin_memory() for n in ("k", "v", "gy", "w", "u")}
     hy, hgk, hgv = (torch.empty(k.shape, dtype=k.dtype).pin_memory() for _ in range(3))
     hgw, hgu = (torch.empty(C, dtype=torch.float32).pin_memory() for _ in range(2))
-    h2d = sum(t.numel() * t.element_size() for t in (hk, hv, hgy, hw, hu))
+    h2d = sum(t.numel() * t.element_size() for t in H.values())
     d2h = sum(t.numel() * t.element_size() for t in (hy, hgk, hgv, hgw, hgu))
+    sets = [dict(k=k, v=v, gy=gy, w=w, u=u, y=y, gk=gk, gv=gv, gw=gw, gu=gu, ck=ckpt, ws=ws)]
+    sets.append({n: torch.empty_like(t) for n, t in sets[0].items()})
+    s_in, s_comp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
+    last_comp, last_out = [None, None], [None, None]
 
-    def e2e_step():
-        for d, h in ((k, hk), (v, hv), (gy, hgy), (w, hw), (u, hu)):
-            d.copy_(h, non_blocking=True)
-        step()
-        for h, d in ((hy, y), (hgk, gk), (hgv, gv), (hgw, gw), (hgu, gu)):
-            h.copy_(d, non_blocking=True)
+    def e2e_step(i):
+        X = sets[i % 2]
+        with torch.cuda.stream(s_in):
+            if last_comp[i % 2] is not None:  # step i - 2 has finished reading X's inputs
+                s_in.wait_event(last_comp[i % 2])
+            for n in ("k", "v", "gy", "w", "u"):
+                X[n].copy_(H[n], non_blocking=True)
+            ev_in = torch.cuda.Event()
+            ev_in.record(s_in)
+        with torch.cuda.stream(s_comp):
+            s_comp.wait_event(ev_in)
+            if last_out[i % 2] is not None:  # step i - 2's results have left X's outputs
+                s_comp.wait_event(last_out[i % 2])
+            wkv.wkv4_forward(X["w"], X["u"], X["k"], X["v"], y=X["y"], ckpt=X["ck"])
+            ev_y = torch.cuda.Event()
+            ev_y.record(s_comp)
+            wkv.wkv4_backward(X["w"], X["u"], X["k"], X["v"], X["gy"], X["ck"], gk=X["gk"], gv=X["gv"], gw=X["gw"],
+                              gu=X["gu"], workspace=X["ws"])
+            ev_c = torch.cuda.Event()
+            ev_c.record(s_comp)
+        last_comp[i % 2] = ev_c
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_y)
+            hy.copy_(X["y"], non_blocking=True)
+            s_out.wait_event(ev_c)
+            for h, n in ((hgk, "gk"), (hgv, "gv"), (hgw, "gw"), (hgu, "gu")):
+                h.copy_(X[n], non_blocking=True)
+            ev_o = torch.cuda.Event()
+            ev_o.record(s_out)
+        last_out[i % 2] = ev_o
 
-    for _ in range(max(3, args.warmup)):
-        e2e_step()
+    for i in range(max(3, args.warmup)):
+        e2e_step(i)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     e_s, e_e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e2e_steps = max(5, min(args.steps, 20))
-    e_s.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e_e.record(stream)
+    last_comp, last_out = [None, None], [None, None]
+    e_s.record(s_in)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    s_out.wait_stream(s_in)
+    s_out.wait_stream(s_comp)
+    e_e.record(s_out)
     torch.cuda.synchronize()
     e2e_ms = torch.tensor([e_s.elapsed_time(e_e) / e2e_steps], dtype=torch.float64, device=dev)
     if world > 1:
@@ -467,8 +507,7 @@ def run_ours(args):
     bwd_bytes = 20 * tok_ch   # k, v, gy read; gk, gv written (float32)
     fwd_bytes = 12 * tok_ch   # k, v read; y written
     achieved = bwd_bytes / (bwd_ms * 1e-3) / 1e9
-    src_hash = kernel_source_hash(["rwkv_wkv_linear_mix_b200/csrc/wkv4_bwd.cu",
-                                   "rwkv_wkv_linear_mix_b200/csrc/wkv_device.cuh"])
+    src_hash = kernel_source_hash(BWD_SOURCES)
     roof = {"bound": "hbm", "kernel": "wkv4_bwd_kernel<float>", "achieved": achieved, "peak": peak,
             "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
             "traffic": recorded_traffic("wkv4_bwd_kernel", WORKLOAD, src_hash),
@@ -483,7 +522,8 @@ def run_ours(args):
         "config": {"workload": WORKLOAD, "B": B, "T": T, "C": C, "global_batch": B * world, "seq_len": T,
                    "parallelism": f"replicas{world}", "l2": "flushed (320 MB write) before every timed step",
                    "ckpt_len": wkv.CKPT_LEN},
-        "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "pipeline": "2 device buffer sets; copy-in, compute, copy-out on separate streams"},
         "roofline": roof,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,

@@ -286,18 +286,38 @@ __global__ void __launch_bounds__(32 * NW, NSEG == 1 ? 16 : 1) wkv4_bwd_kernel(c
   if constexpr (NSEG > 1) cluster_wait_acquire();  // peers may still read this CTA's carry
 }
 
-// gw[c] = sum over (b, segment) of the partials, in ascending order; same for gu.
-__global__ void wkv4_reduce_kernel(const float* __restrict__ part_gw, const float* __restrict__ part_gu, int rows,
-                                   int C, float* __restrict__ gw, float* __restrict__ gu) {
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= C) return;
-  float sw = 0.f, su = 0.f;
-  for (int r = 0; r < rows; ++r) {
-    sw += part_gw[(int64_t)r * C + c];
-    su += part_gu[(int64_t)r * C + c];
+// gw[c] = sum over (b, segment) of the partials; same for gu. A block of
+// 8 warps takes 32 channels: warp q adds rows q, q + 8, q + 16, ... in
+// ascending order, then warp 0 adds the 8 warp sums in order 0..7, so the
+// result does not depend on timing.
+constexpr int kReduceWarps = 8;
+__global__ void __launch_bounds__(32 * kReduceWarps) wkv4_reduce_kernel(const float* __restrict__ part_gw,
+                                                                       const float* __restrict__ part_gu, int rows,
+                                                                       int C, float* __restrict__ gw,
+                                                                       float* __restrict__ gu) {
+  __shared__ float sw[kReduceWarps][32], su[kReduceWarps][32];
+  const int lane = threadIdx.x % 32, q = threadIdx.x / 32;
+  const int c = blockIdx.x * 32 + lane;
+  float aw = 0.f, au = 0.f;
+  if (c < C) {
+    for (int r = q; r < rows; r += kReduceWarps) {
+      aw += part_gw[(int64_t)r * C + c];
+      au += part_gu[(int64_t)r * C + c];
+    }
   }
-  gw[c] = sw;
-  gu[c] = su;
+  sw[q][lane] = aw;
+  su[q][lane] = au;
+  __syncthreads();
+  if (q == 0 && c < C) {
+    float tw = 0.f, tu = 0.f;
+#pragma unroll
+    for (int i = 0; i < kReduceWarps; ++i) {
+      tw += sw[i][lane];
+      tu += su[i][lane];
+    }
+    gw[c] = tw;
+    gu[c] = tu;
+  }
 }
 
 template <class E, int STAGES, int NSEG, int NW>
@@ -338,8 +358,8 @@ static wkv_status run_bwd(const Wkv4BwdArgs& a, cudaStream_t stream, unsigned* e
                                      static_cast<const E*>(a.k), a.ckpt, static_cast<E*>(a.gk), static_cast<E*>(a.gv),
                                      part_gw, part_gu, err);
   if (e == cudaSuccess) {
-    wkv4_reduce_kernel<<<(unsigned)ceil_div(a.C, 256), 256, 0, stream>>>(part_gw, part_gu, (int)rows, (int)a.C,
-                                                                         a.gw, a.gu);
+    wkv4_reduce_kernel<<<(unsigned)ceil_div(a.C, 32), 32 * kReduceWarps, 0, stream>>>(part_gw, part_gu, (int)rows,
+                                                                                     (int)a.C, a.gw, a.gu);
     e = cudaGetLastError();
   }
   if (e != cudaSuccess) {
