@@ -18,12 +18,12 @@
 // Then every coefficient of the reverse scan is a factor the forward step
 // already forms, all <= 1 (base 2, w and k pre-scaled by log2 e):
 //   absorb of token i   f1_i = 2^{P_i - w - P_{i+1}}, f2_i = 2^{k_i - P_{i+1}}
-//   output of token i   e1_i = 2^{P_i - q_i},  e2_i = 2^{u + k_i - q_i},
-//                       den_i = e1 bb + e2,  D_i = 2^{q_i} den_i
-// (one of f1/f2 and one of e1/e2 is exactly 1), and walking i downwards
+//   output of token i   e_i = 2^{u + k_i - P_i} (capped at 2^64 as in the
+//                       forward), D_i = 2^{P_i} (bb_i + e_i)
+// (one of f1/f2 is exactly 1), and walking i downwards
 //   gv_i += f2_i A~_i,   gk_i += f2_i (v_i A~_i - B~_i),
 //   gw   -= f2_i (v_i A~'_i - B~'_i),
-//   A~'_{i-1} = f1_i (A~'_i + A~_i),  A~_{i-1} = f1_i A~_i + gy_i e1_i / den_i
+//   A~'_{i-1} = f1_i (A~'_i + A~_i),  A~_{i-1} = f1_i A~_i + gy_i / (bb_i + e_i)
 // (B~ the same with gy_i y_i). The carries stay bounded by sum |gy| and need
 // no exponent of their own; the loop-carried dependence is one multiply-add.
 //
@@ -96,27 +96,24 @@ __device__ __forceinline__ void wkv4_bwd_interval(const E (*ks)[32], const E (*v
       const float vv = Elem<E>::to_f32(vs[jj][lane]);
       const float g = Elem<E>::to_f32(gs[jj][lane]);
       const float P = spp[jj];
-      // output pair of token jj: q = max(P, u + k)
-      const float d = __fsub_rn(P, __fadd_rn(u2, k2));
-      const float e = ex2(-fabsf(d));
-      const bool past_max = d >= 0.f;
-      const float e1 = past_max ? 1.f : e;
-      const float e2 = past_max ? e : 1.f;
-      const float rd = rcp(__fmaf_rn(e1, sbb[jj], e2));
-      const float yv = __fmul_rn(__fmaf_rn(e1, saa[jj], __fmul_rn(e2, vv)), rd);
+      // output of token jj, in units of the past's exponent P: weight
+      // e = 2^{u + k - P} of the current token (capped as in the forward),
+      // D = 2^P (bb + e), y = (aa + e v) / (bb + e)
+      const float e = ex2(fminf(__fsub_rn(__fadd_rn(u2, k2), P), 64.f));
+      const float rd = rcp(__fadd_rn(sbb[jj], e));
+      const float yv = __fmul_rn(__fmaf_rn(e, vv, saa[jj]), rd);
       // absorb pair of token jj: P' = max(P - w, k)
       const float z = __fsub_rn(k2, __fsub_rn(P, w2));
       const float ea = ex2(-fabsf(z));
       const bool keep = z <= 0.f;
       const float f1 = keep ? 1.f : ea;
       const float f2 = keep ? ea : 1.f;
-      const float gr = __fmul_rn(g, rd);
-      const float ag = __fmul_rn(gr, e1);  // gy e1 / den
+      const float ag = __fmul_rn(g, rd);  // gy 2^P / D
       if constexpr (FULL) {
-        const float rg = __fmul_rn(gr, e2);  // gy rho
-        // v - y = e1 (bb v - aa) / den: no cancellation against v when the
+        const float rg = __fmul_rn(ag, e);  // gy rho, rho = e^{u+k} / D
+        // v - y = (bb v - aa) / (bb + e): no cancellation against v when the
         // current token dominates (y within rounding of v)
-        const float vmy = __fmul_rn(__fmul_rn(e1, __fmaf_rn(sbb[jj], vv, -saa[jj])), rd);
+        const float vmy = __fmul_rn(__fmaf_rn(sbb[jj], vv, -saa[jj]), rd);
         const float gvv = __fmaf_rn(f2, A, rg);
         const float gkv = __fmaf_rn(rg, vmy, __fmul_rn(f2, __fmaf_rn(vv, A, -B)));
         gu_acc = __fmaf_rn(rg, vmy, gu_acc);
@@ -347,6 +344,11 @@ static wkv_status run_bwd(const Wkv4BwdArgs& a, cudaStream_t stream, unsigned* e
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   if (NSEG > 1) {
+    // clusters above 8 CTAs are a non-portable size that must be opted into
+    if (NSEG > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+      *why = "non-portable cluster size refused";
+      return WKV_ERR_CUDA;
+    }
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = NSEG;
     attr[0].val.clusterDim.y = 1;
@@ -385,6 +387,9 @@ template <class E>
 static wkv_status run_bwd_nseg(const Wkv4BwdArgs& a, cudaStream_t stream, unsigned* err, const char** why) {
   constexpr int kStages = sizeof(E) == 2 ? 4 : 2;
   switch (wkv4_bwd_segments(a.B, a.T, a.C)) {
+#if WKV4_MAX_SEGMENTS_ANY > 8
+    case 16: return run_bwd_nw<E, kStages, 16>(a, stream, err, why);
+#endif
     case 8: return run_bwd_nw<E, kStages, 8>(a, stream, err, why);
     case 4: return run_bwd_nw<E, kStages, 4>(a, stream, err, why);
     case 2: return run_bwd_nw<E, kStages, 2>(a, stream, err, why);

@@ -206,6 +206,11 @@ static wkv_status run_fwd(const Wkv4FwdArgs& a, cudaStream_t stream, unsigned* e
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   if (NSEG > 1) {
+    // clusters above 8 CTAs are a non-portable size that must be opted into
+    if (NSEG > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+      *why = "non-portable cluster size refused";
+      return WKV_ERR_CUDA;
+    }
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = NSEG;
     attr[0].val.clusterDim.y = 1;
@@ -234,6 +239,9 @@ static wkv_status run_fwd_nw(const Wkv4FwdArgs& a, cudaStream_t stream, unsigned
 template <class E, int LT, int STAGES>
 static wkv_status run_fwd_nseg(const Wkv4FwdArgs& a, cudaStream_t stream, unsigned* err, const char** why) {
   switch (wkv4_fwd_segments(a.B, a.T, a.C)) {
+#if WKV4_MAX_SEGMENTS_ANY > 8
+    case 16: return run_fwd_nw<E, LT, STAGES, 16>(a, stream, err, why);
+#endif
     case 8: return run_fwd_nw<E, LT, STAGES, 8>(a, stream, err, why);
     case 4: return run_fwd_nw<E, LT, STAGES, 4>(a, stream, err, why);
     case 2: return run_fwd_nw<E, LT, STAGES, 2>(a, stream, err, why);

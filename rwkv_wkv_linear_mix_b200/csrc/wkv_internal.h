@@ -23,12 +23,15 @@ __host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) { ret
 #ifndef WKV4_BWD_MAX_SEGMENTS
 #define WKV4_BWD_MAX_SEGMENTS 8
 #endif
+// 16 segments (a non-portable cluster size) are compiled in only when one of
+// the caps above allows them.
+#define WKV4_MAX_SEGMENTS_ANY (WKV4_FWD_MAX_SEGMENTS > WKV4_BWD_MAX_SEGMENTS ? WKV4_FWD_MAX_SEGMENTS : WKV4_BWD_MAX_SEGMENTS)
 
 // Number of sequence segments each RWKV-4 lane is split into (the cluster
 // size of a kernel): doubled while the launch has fewer warps than
 // WKV4_TARGET_WARPS and every segment keeps at least WKV4_MIN_SEG_STEPS
 // steps (splitting reruns each segment, so short ones do not pay); at most
-// max_seg (<= 8, the portable cluster size).
+// max_seg (<= 16; above 8 a non-portable cluster size).
 #ifndef WKV4_MIN_SEG_STEPS
 #define WKV4_MIN_SEG_STEPS 64
 #endif
