@@ -37,10 +37,11 @@
 //   E. epilogue of unit n - 1 (its O buffer) while those MMAs run
 //   F. mask(A) -> am tiles; S = diag(E) S + dS -> registers and the S^T rows
 //   G. MMA3 issued into unit n's O buffer (two buffers alternate)
-// Warp g prepares tokens 8g .. 8g + 7 (lane = two channels); one thread
-// issues the MMAs; accumulators are read back by warps 0-3 (columns 0-31)
-// and 4-7 (columns 32-63), whose lanes 0-15 also keep the fp32 state (32
-// values each). Waits are bounded (2 s): a wait that gives up records
+// Warp g prepares tokens 8g .. 8g + 7 (lane = two channels, the bonus summed
+// over the warp by shuffles); one thread issues the MMAs; accumulators are
+// read back by warps 0-3 (columns 0-31) and 4-7 (columns 32-63) of the TMEM
+// sub-partition warp % 4, all 32 lanes busy (16x256b loads), and the same
+// threads keep the fp32 state, 16 values each. Waits are bounded (2 s): a wait that gives up records
 // WKV_DEVERR_WAIT_TIMEOUT, the CTA drains its copies and MMAs in flight,
 // frees its tensor memory and exits.
 #include "wkv_device.cuh"
@@ -87,6 +88,10 @@ __device__ __forceinline__ void tile_st2(uint8_t* tile, int j, int lane, uint32_
 __device__ __forceinline__ int f32_pair_off(int j, int lane, int panel) {
   return (lane >> 4) * panel + j * 128 + (((((lane & 15) >> 1) ^ (j & 7)) & 7) << 4) + (lane & 1) * 8;
 }
+// bf16 pair (columns col, col + 1; col even) of row `row` of a swizzled bf16 tile.
+__device__ __forceinline__ void tile_st_pair(uint8_t* tile, int row, int col, uint32_t v) {
+  *reinterpret_cast<uint32_t*>(tile + row * 128 + ((((col >> 3) ^ (row & 7)) & 7) << 4) + (col & 7) * 2) = v;
+}
 // Columns 16 q .. 16 q + 15 (q in 0..3) of row `row` of a bf16 tile.
 __device__ __forceinline__ void tile_st_row16(uint8_t* tile, int row, int q, const uint32_t (&p)[8]) {
 #pragma unroll
@@ -103,17 +108,22 @@ __device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uin
 
 // Pass 2 for the tokens 8g .. 8g + 7 of warp g: R^ and K~ (fp32) forwards
 // from the prefix product `pre`, K^ (bf16) backwards from the suffix product
-// `post`. FULL: the unit is the whole 64-token chunk (no masking).
+// `post`, and the bonus r_j . (u * k_j) of each token (this lane's two
+// channels, then summed over the warp). FULL: the unit is the whole 64-token
+// chunk (no masking).
 template <bool FULL>
 __device__ __forceinline__ void wkv6_prepare(Wkv6Smem& sm, int g, int lane, int off, int len, const float (&w0)[8],
-                                             const float (&w1)[8], float pre0, float pre1, float post0, float post1) {
+                                             const float (&w1)[8], float pre0, float pre1, float post0, float post1,
+                                             float u0, float u1) {
   const bool need_kb = FULL || len > 1;  // one token has no s < j pair
   float e0 = pre0, e1 = pre1;
+  float pb[8];  // this lane's part of each token's bonus
 #pragma unroll
   for (int jj = 0; jj < 8; ++jj) {
     const int j = 8 * g + jj;
     const bool in = FULL || (j >= off && j < off + len);
     const uint32_t rx = tile_ld2(sm.r, j, lane), kx = tile_ld2(sm.k, j, lane);
+    pb[jj] = in ? fmaf(bf16lo(rx) * u0, bf16lo(kx), bf16hi(rx) * u1 * bf16hi(kx)) : 0.f;
     float2 rh = make_float2(bf16lo(rx) * e0, bf16hi(rx) * e1);
     e0 *= w0[jj];
     e1 *= w1[jj];
@@ -124,6 +134,26 @@ __device__ __forceinline__ void wkv6_prepare(Wkv6Smem& sm, int g, int lane, int 
     }
     *reinterpret_cast<float2*>(sm.rf[0] + f32_pair_off(j, lane, kTile6)) = rh;
     *reinterpret_cast<float2*>(sm.bt[0] + f32_pair_off(j, lane, 2 * kTile6)) = kb;
+  }
+  // sum the 8 bonus parts over the warp's 32 lanes at once: each exchange
+  // halves the tokens a lane keeps, so lane l ends with token (l / 4) % 8
+  {
+    float q4[4], q2[2];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) {
+      const bool hi = lane & 16;
+      q4[m] = (hi ? pb[m + 4] : pb[m]) + __shfl_xor_sync(0xffffffffu, hi ? pb[m] : pb[m + 4], 16);
+    }
+#pragma unroll
+    for (int m = 0; m < 2; ++m) {
+      const bool hi = lane & 8;
+      q2[m] = (hi ? q4[m + 2] : q4[m]) + __shfl_xor_sync(0xffffffffu, hi ? q4[m] : q4[m + 2], 8);
+    }
+    const bool hi = lane & 4;
+    float q1 = (hi ? q2[1] : q2[0]) + __shfl_xor_sync(0xffffffffu, hi ? q2[0] : q2[1], 4);
+    q1 += __shfl_xor_sync(0xffffffffu, q1, 2);
+    q1 += __shfl_xor_sync(0xffffffffu, q1, 1);
+    if ((lane & 3) == 0) sm.bonus[8 * g + ((lane >> 2) & 7)] = q1;
   }
   float g0 = post0, g1 = post1;
 #pragma unroll
@@ -149,11 +179,16 @@ __global__ void __launch_bounds__(kThreads6, 2)
   const int h = blockIdx.x % H, b = blockIdx.x / H;
   const int64_t HK = (int64_t)H * kHead6;
   const int nch = (T + kChunk6 - 1) / kChunk6;
-  // accumulator read-back: TMEM sub-partition sp, column half ch; lanes 0-15
-  // hold row 16 sp + lane (a token j of A and O, a key i of dS and S)
+  // accumulator read-back: TMEM sub-partition sp, column half ch. With the
+  // 32x32b shape lanes 0-15 hold row 16 sp + lane (the epilogue); with the
+  // 16x256b shape every thread holds rows r0 = 16 sp + lane / 4 and r0 + 8,
+  // columns 32 ch + 8 q + 2 (lane % 4) + {0, 1}, q = 0..3 (mask and state)
   const int sp = warp & 3, ch = warp >> 2;
   const int row = 16 * sp + lane;
   const bool holder = lane < 16;
+  const int r0 = 16 * sp + (lane >> 2), r1 = r0 + 8;
+  const int cq = 32 * ch + 2 * (lane & 3);  // + 8 q
+  const float u0 = u[h * kHead6 + 2 * lane], u1 = u[h * kHead6 + 2 * lane + 1];
 
   if (tid == 0) {
     if (nch > 0) {
@@ -172,18 +207,20 @@ __global__ void __launch_bounds__(kThreads6, 2)
   if (warp == 0) tmem_alloc(&sm.tmem_base, kTmemCols6);
   if (tid < kHead6) sm.u[tid] = u[h * kHead6 + tid];
 
-  // fp32 state S[row][32 ch .. 32 ch + 31] in registers; its tf32 operand
-  // copy is S^T in rows 64 + jv of bt (K-major: column i = row)
-  float S[32];
+  // fp32 state in registers, 16 values per thread in the 16x256b layout:
+  // S[4q + e] = S[r0][cq + 8q + e], S[4q + 2 + e] = S[r1][cq + 8q + e]; its
+  // tf32 operand copy is S^T in rows 64 + jv of bt (K-major: column i)
+  float S[16];
   auto store_state = [&]() {
-    if (!holder) return;
-    uint8_t* base = sm.bt[row >> 5] + 64 * 128 + (row & 3) * 4;
-    const int c4 = (row & 31) >> 2;
 #pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const int jv = 32 * ch + e;
-      *reinterpret_cast<float*>(base + jv * 128 + (((c4 ^ (jv & 7)) & 7) << 4)) = S[e];
-    }
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = (e < 2) ? r0 : r1;
+        const int jv = cq + 8 * q + (e & 1);
+        *reinterpret_cast<float*>(sm.bt[i >> 5] + (64 + jv) * 128 + (((((i & 31) >> 2) ^ (jv & 7)) & 7) << 4) +
+                                  (i & 3) * 4) = S[4 * q + e];
+      }
   };
   {
     const float* s0 = nullptr;
@@ -196,13 +233,16 @@ __global__ void __launch_bounds__(kThreads6, 2)
       }
     }
 #pragma unroll
-    for (int e = 0; e < 32; e += 4) {
-      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (s0 && holder) x = *reinterpret_cast<const float4*>(s0 + row * kHead6 + 32 * ch + e);
-      S[e] = x.x;
-      S[e + 1] = x.y;
-      S[e + 2] = x.z;
-      S[e + 3] = x.w;
+    for (int q = 0; q < 4; ++q) {
+      float2 x0 = make_float2(0.f, 0.f), x1 = make_float2(0.f, 0.f);
+      if (s0) {
+        x0 = *reinterpret_cast<const float2*>(s0 + r0 * kHead6 + cq + 8 * q);
+        x1 = *reinterpret_cast<const float2*>(s0 + r1 * kHead6 + cq + 8 * q);
+      }
+      S[4 * q] = x0.x;
+      S[4 * q + 1] = x0.y;
+      S[4 * q + 2] = x1.x;
+      S[4 * q + 3] = x1.y;
     }
     store_state();
   }
@@ -348,34 +388,11 @@ __global__ void __launch_bounds__(kThreads6, 2)
         wait_bar(&sm.rk_bar, (uint32_t)c & 1u, &rk_done, c + 1);
         wait_bar(&sm.v_bar[c & 1], (uint32_t)(c >> 1) & 1u, &v_done, c + 1);
       }
-      // ---- C. bonus r_j . (u * k_j): lanes 4m .. 4m + 3 of warp g take
-      // token 8g + m, 16 channels each ----
-      {
-        const int j = tid >> 2, part = tid & 3;
-        float acc = 0.f;
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int chunk = 2 * part + cc;
-          const int phys = (chunk ^ (j & 7)) & 7;
-          const uint4 rv = *reinterpret_cast<const uint4*>(sm.r + j * 128 + phys * 16);
-          const uint4 kv = *reinterpret_cast<const uint4*>(sm.k + j * 128 + phys * 16);
-          const uint32_t rr[4] = {rv.x, rv.y, rv.z, rv.w}, kk[4] = {kv.x, kv.y, kv.z, kv.w};
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int i = chunk * 8 + 2 * q;
-            acc = fmaf(bf16lo(rr[q]) * sm.u[i], bf16lo(kk[q]), acc);
-            acc = fmaf(bf16hi(rr[q]) * sm.u[i + 1], bf16hi(kk[q]), acc);
-          }
-        }
-        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-        if (part == 0) sm.bonus[j] = (j >= off && j < off + len) ? acc : 0.f;
-      }
       // ---- C. pass 2 ----
       if (full)
-        wkv6_prepare<true>(sm, warp, lane, off, len, w0, w1, pre0, pre1, post0, post1);
+        wkv6_prepare<true>(sm, warp, lane, off, len, w0, w1, pre0, pre1, post0, post1, u0, u1);
       else
-        wkv6_prepare<false>(sm, warp, lane, off, len, w0, w1, pre0, pre1, post0, post1);
+        wkv6_prepare<false>(sm, warp, lane, off, len, w0, w1, pre0, pre1, post0, post1, u0, u1);
       fence_proxy_async_smem();
       if (__syncthreads_or(!ok)) {
         failed = true;
@@ -402,33 +419,35 @@ __global__ void __launch_bounds__(kThreads6, 2)
       // ---- F. mask(A) -> hi / lo tiles over K~; S = diag(E) S + dS ----
       wait_mma();
       {
-        const float bj = holder ? sm.bonus[row] : 0.f;
+        float a[16];
+        tmem_ld16x256b_x4(tl + kColA + 32 * ch, a);
+        tmem_wait_ld();
+        const float b0 = sm.bonus[r0], b1 = sm.bonus[r1];
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          float a[16];
-          tmem_ld16(tl + kColA + 32 * ch + 16 * q, a);
-          tmem_wait_ld();
-          if (holder) {
-            uint32_t ph[8], pl[8];
+        for (int q = 0; q < 4; ++q) {
+          const int s0 = cq + 8 * q;
 #pragma unroll
-            for (int e = 0; e < 16; e += 2) {
-              const int s = 32 * ch + 16 * q + e;
-              const float a0 = s < row ? a[e] : (s == row ? bj : 0.f);
-              const float a1 = s + 1 < row ? a[e + 1] : (s + 1 == row ? bj : 0.f);
-              split_bf16x2(a0, a1, ph[e / 2], pl[e / 2]);
-            }
-            tile_st_row16(sm.bt[0], row, 2 * ch + q, ph);
-            tile_st_row16(sm.bt[1], row, 2 * ch + q, pl);
+          for (int hh = 0; hh < 2; ++hh) {
+            const int rr = hh ? r1 : r0;
+            const float bb = hh ? b1 : b0;
+            const float x0 = s0 < rr ? a[4 * q + 2 * hh] : (s0 == rr ? bb : 0.f);
+            const float x1 = s0 + 1 < rr ? a[4 * q + 2 * hh + 1] : (s0 + 1 == rr ? bb : 0.f);
+            uint32_t ph, pl;
+            split_bf16x2(x0, x1, ph, pl);
+            tile_st_pair(sm.bt[0], rr, s0, ph);
+            tile_st_pair(sm.bt[1], rr, s0, pl);
           }
         }
-        const float dj = holder ? sm.dec[row] : 0.f;
+        float d[16];
+        tmem_ld16x256b_x4(tl + kColS + 32 * ch, d);
+        tmem_wait_ld();
+        const float d0 = sm.dec[r0], d1 = sm.dec[r1];
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          float d[16];
-          tmem_ld16(tl + kColS + 32 * ch + 16 * q, d);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) S[16 * q + e] = fmaf(dj, S[16 * q + e], d[e]);
+        for (int q = 0; q < 4; ++q) {
+          S[4 * q] = fmaf(d0, S[4 * q], d[4 * q]);
+          S[4 * q + 1] = fmaf(d0, S[4 * q + 1], d[4 * q + 1]);
+          S[4 * q + 2] = fmaf(d1, S[4 * q + 2], d[4 * q + 2]);
+          S[4 * q + 3] = fmaf(d1, S[4 * q + 3], d[4 * q + 3]);
         }
         store_state();
       }
@@ -473,10 +492,13 @@ __global__ void __launch_bounds__(kThreads6, 2)
       for (int cc = v_done; cc < v_issued; ++cc) mbar_wait_bounded(&sm.v_bar[cc & 1], (uint32_t)(cc >> 1) & 1u, err);
       if (mma_done < mma_issued) mbar_wait_bounded(&sm.mma_bar, (uint32_t)(mma_issued - 1) & 1u, err);
     }
-  } else if (final_state && holder) {
-    float* fs = final_state + ((int64_t)b * H + h) * kHead6 * kHead6 + row * kHead6 + 32 * ch;
+  } else if (final_state) {
+    float* fs = final_state + ((int64_t)b * H + h) * kHead6 * kHead6;
 #pragma unroll
-    for (int e = 0; e < 32; e += 4) *reinterpret_cast<float4*>(fs + e) = make_float4(S[e], S[e + 1], S[e + 2], S[e + 3]);
+    for (int q = 0; q < 4; ++q) {
+      *reinterpret_cast<float2*>(fs + r0 * kHead6 + cq + 8 * q) = make_float2(S[4 * q], S[4 * q + 1]);
+      *reinterpret_cast<float2*>(fs + r1 * kHead6 + cq + 8 * q) = make_float2(S[4 * q + 2], S[4 * q + 3]);
+    }
   }
   tc_fence_before_sync();
   __syncthreads();
