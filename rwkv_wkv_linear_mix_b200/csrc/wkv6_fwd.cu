@@ -32,7 +32,7 @@
 // Kernel shape: one CTA of 256 threads per (b, h), walking its chunks (and
 // sub-chunks: "units") in order; two CTAs share an SM. Per unit n:
 //   B. pass 1: product of w over each warp's 8 tokens, totals, split check
-//   C. bonus; pass 2: R^, K~ (fp32), K^ (bf16) into their tiles
+//   C. pass 2: R^, K~ (fp32), K^ = K~ E_{L-1} (bf16) and the bonus
 //   D. TMA starts the next chunk's r, k tiles; MMA12 and MMA4 issued
 //   E. epilogue of unit n - 1 (its O buffer) while those MMAs run
 //   F. mask(A) -> am tiles; S = diag(E) S + dS -> registers and the S^T rows
@@ -106,14 +106,14 @@ __device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uin
   lo = pack_bf16x2(a - bf16lo(hi), b - bf16hi(hi));
 }
 
-// Pass 2 for the tokens 8g .. 8g + 7 of warp g: R^ and K~ (fp32) forwards
-// from the prefix product `pre`, K^ (bf16) backwards from the suffix product
-// `post`, and the bonus r_j . (u * k_j) of each token (this lane's two
-// channels, then summed over the warp). FULL: the unit is the whole 64-token
-// chunk (no masking).
+// Pass 2 for the tokens 8g .. 8g + 7 of warp g: R^ = r E_{j-1} and
+// K~ = k / E_s (fp32) from the prefix product `pre`, K^ = K~ E_{L-1} =
+// k E_{L-1} / E_s (bf16; `tot` = E_{L-1}), and the bonus r_j . (u * k_j) of
+// each token (this lane's two channels, then summed over the warp). FULL: the
+// unit is the whole 64-token chunk (no masking).
 template <bool FULL>
 __device__ __forceinline__ void wkv6_prepare(Wkv6Smem& sm, int g, int lane, int off, int len, const float (&w0)[8],
-                                             const float (&w1)[8], float pre0, float pre1, float post0, float post1,
+                                             const float (&w1)[8], float pre0, float pre1, float tot0, float tot1,
                                              float u0, float u1) {
   const bool need_kb = FULL || len > 1;  // one token has no s < j pair
   float e0 = pre0, e1 = pre1;
@@ -128,12 +128,18 @@ __device__ __forceinline__ void wkv6_prepare(Wkv6Smem& sm, int g, int lane, int 
     e0 *= w0[jj];
     e1 *= w1[jj];
     float2 kb = make_float2(bf16lo(kx) * rcp(e0), bf16hi(kx) * rcp(e1));
+    // one token: E_{L-1} / E_s = 1, and K~ is not needed
+    uint32_t kh = need_kb ? pack_bf16x2(kb.x * tot0, kb.y * tot1) : kx;
     if (!FULL) {
-      if (!in) rh = make_float2(0.f, 0.f);
+      if (!in) {
+        rh = make_float2(0.f, 0.f);
+        kh = 0u;
+      }
       if (!(in && need_kb)) kb = make_float2(0.f, 0.f);
     }
     *reinterpret_cast<float2*>(sm.rf[0] + f32_pair_off(j, lane, kTile6)) = rh;
     *reinterpret_cast<float2*>(sm.bt[0] + f32_pair_off(j, lane, 2 * kTile6)) = kb;
+    tile_st2(sm.kh, j, lane, kh);
   }
   // sum the 8 bonus parts over the warp's 32 lanes at once: each exchange
   // halves the tokens a lane keeps, so lane l ends with token (l / 4) % 8
@@ -154,16 +160,6 @@ __device__ __forceinline__ void wkv6_prepare(Wkv6Smem& sm, int g, int lane, int 
     q1 += __shfl_xor_sync(0xffffffffu, q1, 2);
     q1 += __shfl_xor_sync(0xffffffffu, q1, 1);
     if ((lane & 3) == 0) sm.bonus[8 * g + ((lane >> 2) & 7)] = q1;
-  }
-  float g0 = post0, g1 = post1;
-#pragma unroll
-  for (int jj = 7; jj >= 0; --jj) {
-    const int j = 8 * g + jj;
-    const bool in = FULL || (j >= off && j < off + len);
-    const uint32_t kx = tile_ld2(sm.k, j, lane);
-    tile_st2(sm.kh, j, lane, in ? pack_bf16x2(bf16lo(kx) * g0, bf16hi(kx) * g1) : 0u);
-    g0 *= w0[jj];
-    g1 *= w1[jj];
   }
 }
 
@@ -348,7 +344,7 @@ __global__ void __launch_bounds__(kThreads6, 2)
         failed = true;
         break;
       }
-      float pre0 = 1.f, pre1 = 1.f, post0 = 1.f, post1 = 1.f, tot0 = 1.f, tot1 = 1.f;
+      float pre0 = 1.f, pre1 = 1.f, tot0 = 1.f, tot1 = 1.f;
       {
         const float* wq = reinterpret_cast<const float*>(sm.kh);
 #pragma unroll
@@ -357,10 +353,6 @@ __global__ void __launch_bounds__(kThreads6, 2)
           if (g < warp) {
             pre0 *= q.x;
             pre1 *= q.y;
-          }
-          if (g > warp) {
-            post0 *= q.x;
-            post1 *= q.y;
           }
           tot0 *= q.x;
           tot1 *= q.y;
@@ -390,9 +382,9 @@ __global__ void __launch_bounds__(kThreads6, 2)
       }
       // ---- C. pass 2 ----
       if (full)
-        wkv6_prepare<true>(sm, warp, lane, off, len, w0, w1, pre0, pre1, post0, post1, u0, u1);
+        wkv6_prepare<true>(sm, warp, lane, off, len, w0, w1, pre0, pre1, tot0, tot1, u0, u1);
       else
-        wkv6_prepare<false>(sm, warp, lane, off, len, w0, w1, pre0, pre1, post0, post1, u0, u1);
+        wkv6_prepare<false>(sm, warp, lane, off, len, w0, w1, pre0, pre1, tot0, tot1, u0, u1);
       fence_proxy_async_smem();
       if (__syncthreads_or(!ok)) {
         failed = true;
