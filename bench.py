@@ -24,6 +24,9 @@ RWKV-6 head-state forward.
 
 --impl reference times the fp64 CPU oracle (the only reference this project
 has) on the same workload and metric.
+
+--kernel NAME [--workload RECIPE[:B,T]] only runs one kernel --steps times
+(for profiler captures; prints no JSON line).
 """
 
 from __future__ import annotations
@@ -61,6 +64,11 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the secondary workloads (larger shapes, chunk step, RWKV-6)")
+    ap.add_argument("--kernel", choices=["wkv4_fwd", "wkv4_bwd", "wkv6_fwd", "wkv4_chunk"],
+                    help="profiling mode: run only this kernel --steps times on --workload (no JSON line)")
+    ap.add_argument("--workload", default=None,
+                    help="with --kernel: a recipe name of synth (RWKV-4 or RWKV-6), optionally resized "
+                         "as NAME:B,T (e.g. wkv4_fb_bf16_c4096:16,1024)")
     return ap.parse_args()
 
 
@@ -74,6 +82,23 @@ def dist_env():
 # ----------------------------------------------------------------------------
 # helpers
 # ----------------------------------------------------------------------------
+
+def max_over_ranks(ms, dev, world):
+    """The job's step time: the slowest rank's (every rank runs its own
+    replica, so the job is done when the last one is)."""
+    import torch
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank, world, ms):
+    """Whole-job throughput in G units/s: the units all ranks processed in one
+    step over the (max-over-ranks) step time."""
+    return units_per_rank * world / (ms * 1e-3) / 1e9
+
 
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -425,11 +450,8 @@ def run_ours(args):
     t_fwd = [a.elapsed_time(b) for a, b, _ in ev]
     t_bwd = [b.elapsed_time(c) for _, b, c in ev]
     step_ms = sum(f + b for f, b in zip(t_fwd, t_bwd)) / args.steps
-    t_local = torch.tensor([step_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_local, op=dist.ReduceOp.MAX)
-    step_ms_max = float(t_local.item())
-    value = tok_ch * world / (step_ms_max * 1e-3) / 1e9
+    step_ms_max = max_over_ranks(step_ms, dev, world)
+    value = job_throughput(tok_ch, world, step_ms_max)
 
     # ---- end to end through the C ABI with pinned host buffers ----
     # Every step copies its inputs host -> device, runs forward + backward and
@@ -493,11 +515,10 @@ def run_ours(args):
     s_out.wait_stream(s_comp)
     e_e.record(s_out)
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([e_s.elapsed_time(e_e) / e2e_steps], dtype=torch.float64, device=dev)
+    e2e_ms = max_over_ranks(e_s.elapsed_time(e_e) / e2e_steps, dev, world)
     if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
         dist.barrier()
-    e2e_val = tok_ch * world / (float(e2e_ms.item()) * 1e-3) / 1e9
+    e2e_val = job_throughput(tok_ch, world, e2e_ms)
     assert wkv.device_error(reset=True) == 0, "a kernel recorded a device-side error"
 
     # ---- roofline of the dominant kernel (the backward) ----
@@ -540,8 +561,79 @@ def run_ours(args):
     return 0
 
 
+def run_kernel_only(args):
+    """Profiling mode: the inputs are drawn on the device with the recipe's
+    distributions (as for the secondary workloads) and one kernel runs
+    --steps times back to back, so an ncu capture can pick a launch."""
+    import torch
+    from rwkv_wkv_linear_mix_b200 import synth, wkv
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    name, _, resize = (args.workload or "").partition(":")
+    if args.kernel == "wkv4_chunk":
+        S, C = 32, 4096
+        inp = synth.wkv4_slot_inputs(S=S, C=C, dtype="bf16", seed=0)
+        to_bf16 = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+        w, u = torch.from_numpy(inp["w"]).to(dev), torch.from_numpy(inp["u"]).to(dev)
+        kall, vall = to_bf16(inp["k"]), to_bf16(inp["v"])
+        calls, done = [], np.zeros(S, np.int64)
+        for take in synth.feed_schedule(inp["lengths"], 32):
+            idx = np.concatenate([np.arange(inp["offsets"][s] + done[s], inp["offsets"][s] + done[s] + take[s])
+                                  for s in range(S)])
+            it = torch.from_numpy(idx).to(dev)
+            cu = torch.from_numpy(np.concatenate([[0], np.cumsum(take)]).astype(np.int32)).to(dev)
+            calls.append((kall[it].contiguous(), vall[it].contiguous(), cu))
+            done += take
+        state = wkv.wkv4_state_init(S, C, dev)
+        for _ in range(args.steps):
+            wkv.wkv4_state_init(S, C, dev, state=state)
+            for kc, vc, cu in calls:
+                wkv.wkv4_chunk_step(w, u, kc, vc, cu, state)
+    elif args.kernel == "wkv6_fwd":
+        rec = synth.WKV6_RECIPES[name or "wkv6_fwd_bf16_c2048"]
+        if resize:
+            rec = rec.with_shape(*[int(x) for x in resize.split(",")])
+        B, T, HK = rec.B, rec.T, rec.H * rec.K
+        d = torch.randn(B, T, HK, device=dev, generator=g) * rec.d_std + rec.d_mean
+        w6 = torch.exp(-torch.exp(d)).to(torch.bfloat16)
+        del d
+        r6, k6, v6 = (torch.randn(B, T, HK, device=dev, generator=g).to(torch.bfloat16) for _ in range(3))
+        u6 = torch.rand(HK, device=dev, generator=g) * (rec.u_hi - rec.u_lo) + rec.u_lo
+        o6 = torch.empty_like(r6)
+        for _ in range(args.steps):
+            wkv.wkv6_forward(r6, k6, v6, w6, u6, o=o6)
+    else:
+        rec = synth.WKV4_RECIPES[name or WORKLOAD]
+        if resize:
+            rec = rec.with_shape(*[int(x) for x in resize.split(",")])
+        B, T, C = rec.B, rec.T, rec.C
+        dt = torch.float32 if rec.dtype == "f32" else torch.bfloat16
+        w = torch.exp(torch.rand(C, device=dev, generator=g) * (rec.td_hi - rec.td_lo) + rec.td_lo)
+        u = torch.rand(C, device=dev, generator=g) * (rec.u_hi - rec.u_lo) + rec.u_lo
+        k = (torch.randn(B, T, C, device=dev, generator=g) * rec.k_std).to(dt)
+        v = torch.randn(B, T, C, device=dev, generator=g).to(dt)
+        gy = torch.randn(B, T, C, device=dev, generator=g).to(dt)
+        y, gk, gv = torch.empty_like(k), torch.empty_like(k), torch.empty_like(k)
+        gw, gu = torch.empty(C, device=dev), torch.empty(C, device=dev)
+        ck = torch.empty(wkv.ckpt_shape(B, T, C), device=dev)
+        ws = torch.empty(max(16, wkv.wkv4_backward_workspace_bytes(B, T, C, True)), dtype=torch.uint8, device=dev)
+        wkv.wkv4_forward(w, u, k, v, y=y, ckpt=ck)
+        for _ in range(args.steps):
+            if args.kernel == "wkv4_fwd":
+                wkv.wkv4_forward(w, u, k, v, y=y, ckpt=ck)
+            else:
+                wkv.wkv4_backward(w, u, k, v, gy, ck, gk=gk, gv=gv, gw=gw, gu=gu, workspace=ws)
+    torch.cuda.synchronize()
+    assert wkv.device_error(reset=True) == 0, "a kernel recorded a device-side error"
+    print(f"{args.kernel} on {args.workload or 'default'}: {args.steps} runs ok", flush=True)
+    return 0
+
+
 def main():
     args = parse()
+    if args.kernel:
+        return run_kernel_only(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)
