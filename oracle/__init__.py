@@ -13,7 +13,9 @@ Definitions followed:
           / (sum_{i<t} e^{-(t-1-i)w+k_i} + e^{u+k_t}),  w = exp(time_decay).
   * RWKV-6 head-state WKV: RWKV6_OP (rwkv-ops package page, section
     "rwkv6op 使用方法"): o_t = r_t (S_{t-1} + diag(u) k_t^T v_t),
-    S_t = diag(w_t) S_{t-1} + k_t^T v_t.
+    S_t = diag(w_t) S_{t-1} + k_t^T v_t; the op is trainable (the page's
+    backend table lists its PyTorch CUDA backward), so its gradients are the
+    chain rule of this recurrence.
 """
 
 from __future__ import annotations
@@ -57,6 +59,8 @@ def _open(path):
     lib.oracle_wkv4_backward.restype = ctypes.c_int
     lib.oracle_wkv6_forward.argtypes = [i64, i64, i64, i64] + [dp] * 7 + [i64, dp, dp]
     lib.oracle_wkv6_forward.restype = ctypes.c_int
+    lib.oracle_wkv6_backward.argtypes = [i64, i64, i64, i64] + [dp] * 7 + [i64] + [dp] * 8
+    lib.oracle_wkv6_backward.restype = ctypes.c_int
     return lib
 
 
@@ -194,3 +198,44 @@ def wkv6_forward(r, k, v, w, u, init_state=None, state_map=None, _lib=None):
     if rc != 0:
         raise FloatingPointError(f"oracle_wkv6_forward failed (rc={rc})")
     return o, fs
+
+
+def wkv6_backward(r, k, v, w, u, dout, init_state=None, state_map=None, g_final=None, _lib=None):
+    """Gradients of sum(o * dout) + sum(final_state * g_final) for
+    wkv6_forward(r, k, v, w, u, init_state, state_map), in fp64.
+
+    u is [H, K] (or [H*K] with init_state fixing K). Returns
+    (gr, gk, gv, gw [B, T, H*K], gu [H*K] summed over samples and tokens,
+    g_init [B, H, K, K] = dL/dS_{-1} of each sample).
+    """
+    lib = _lib or _load()
+    u = np.asarray(u)
+    if u.ndim == 2:
+        H, K = u.shape
+    elif init_state is not None:
+        H, K = np.asarray(init_state).shape[1:3]
+    else:
+        raise ValueError("pass u as [H, K] or give init_state to fix the head size")
+    r, k, v, w, u, dout = _f64(r), _f64(k), _f64(v), _f64(w), _f64(u).reshape(-1), _f64(dout)
+    B, T, HK = r.shape
+    assert HK == H * K and k.shape == v.shape == w.shape == r.shape == dout.shape
+    n_state, s0, sm, gf = 0, None, None, None
+    if init_state is not None:
+        s0 = _f64(init_state)
+        n_state = s0.shape[0]
+        assert s0.shape == (n_state, H, K, K)
+    if state_map is not None:
+        sm = np.ascontiguousarray(state_map, dtype=np.int32)
+        assert sm.shape == (B,)
+    if g_final is not None:
+        gf = _f64(g_final)
+        assert gf.shape == (B, H, K, K)
+    gr, gk, gv, gw = (np.empty_like(r) for _ in range(4))
+    gu = np.empty(HK)
+    gi = np.empty((B, H, K, K))
+    rc = lib.oracle_wkv6_backward(B, T, H, K, _ptr(r), _ptr(k), _ptr(v), _ptr(w), _ptr(u), _ptr(s0), _ptr(sm),
+                                  n_state, _ptr(dout), _ptr(gf), _ptr(gr), _ptr(gk), _ptr(gv), _ptr(gw),
+                                  _ptr(gu), _ptr(gi))
+    if rc != 0:
+        raise FloatingPointError(f"oracle_wkv6_backward failed (rc={rc})")
+    return gr, gk, gv, gw, gu, gi

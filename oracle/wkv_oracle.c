@@ -304,3 +304,120 @@ int oracle_wkv6_forward(int64_t B, int64_t T, int64_t H, int64_t K,
     }
     return bad;
 }
+
+/* ------------------------------------------------------------------------ */
+/* RWKV-6 head-state backward                                                */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Gradients of L = sum(o * do) + sum(final_state * g_final) for the forward
+ * above (RWKV6_OP is a trainable operator: the rwkv-ops package page lists
+ * its PyTorch CUDA backward). The chain rule of the recurrence, written out
+ * with G_t = dL/dS_t walked from the last token back:
+ *
+ *   G_{T-1} = g_final (or 0),   G_{t-1} = diag(w_t) G_t + r_t^T do_t
+ *   gr_t[i] = sum_j S_{t-1}[i][j] do_t[j] + u[i] k_t[i] (v_t . do_t)
+ *   gk_t[i] = sum_j G_t[i][j] v_t[j]     + u[i] r_t[i] (v_t . do_t)
+ *   gv_t[j] = sum_i k_t[i] G_t[i][j]     + (sum_i r_t[i] u[i] k_t[i]) do_t[j]
+ *   gw_t[i] = sum_j G_t[i][j] S_{t-1}[i][j]
+ *   gu[i]  += r_t[i] k_t[i] (v_t . do_t)          (summed over samples, tokens)
+ *   g_init  = G_{-1}                                 (per sample: [B][H][K][K])
+ *
+ * Every S_{t-1} of a (sample, head) is kept (T * K * K doubles), so this is
+ * only for the test sizes. g_final, g_init may be NULL. gu gets the sum over
+ * samples and tokens, added per (sample, head) in a fixed order.
+ * Returns 0 on success, 1 on a non-finite result, 2 when out of memory,
+ * 3 on a bad state index.
+ */
+int oracle_wkv6_backward(int64_t B, int64_t T, int64_t H, int64_t K,
+                         const double *r, const double *k, const double *v,
+                         const double *w, const double *u,
+                         const double *init_state, const int32_t *state_map,
+                         int64_t n_state, const double *dout, const double *g_final,
+                         double *gr, double *gk, double *gv, double *gw,
+                         double *gu, double *g_init)
+{
+    const int64_t HK = H * K;
+    int bad = 0;
+    double *gu_part = (double *)calloc((size_t)(B * HK), sizeof(double));
+    if (!gu_part) return 2;
+    #pragma omp parallel reduction(|:bad)
+    {
+        double *Sh = (double *)malloc(sizeof(double) * (size_t)((T + 1) * K * K));
+        double *G = (double *)malloc(sizeof(double) * (size_t)(K * K));
+        if (!Sh || !G) bad |= 2;
+        #pragma omp for collapse(2) schedule(static)
+        for (int64_t bi = 0; bi < B; ++bi) {
+            for (int64_t h = 0; h < H; ++h) {
+                if (!Sh || !G) continue;
+                /* forward: Sh[t] = S_{t-1} */
+                if (init_state) {
+                    int64_t sidx;
+                    if (state_map) sidx = state_map[bi];
+                    else sidx = (n_state == 1) ? 0 : bi;
+                    if (sidx < 0 || sidx >= n_state) { bad |= 3; continue; }
+                    memcpy(Sh, init_state + (sidx * H + h) * K * K, sizeof(double) * (size_t)(K * K));
+                } else {
+                    memset(Sh, 0, sizeof(double) * (size_t)(K * K));
+                }
+                for (int64_t t = 0; t < T; ++t) {
+                    const int64_t row = (bi * T + t) * HK + h * K;
+                    const double *S = Sh + t * K * K;
+                    double *Sn = Sh + (t + 1) * K * K;
+                    for (int64_t i = 0; i < K; ++i)
+                        for (int64_t j = 0; j < K; ++j)
+                            Sn[i * K + j] = w[row + i] * S[i * K + j] + k[row + i] * v[row + j];
+                }
+                /* reverse */
+                if (g_final)
+                    memcpy(G, g_final + (bi * H + h) * K * K, sizeof(double) * (size_t)(K * K));
+                else
+                    memset(G, 0, sizeof(double) * (size_t)(K * K));
+                double *gup = gu_part + bi * HK + h * K;
+                for (int64_t t = T - 1; t >= 0; --t) {
+                    const int64_t row = (bi * T + t) * HK + h * K;
+                    const double *S = Sh + t * K * K; /* S_{t-1} */
+                    double vdo = 0.0, rku = 0.0;
+                    for (int64_t j = 0; j < K; ++j) vdo += v[row + j] * dout[row + j];
+                    for (int64_t i = 0; i < K; ++i) rku += r[row + i] * u[h * K + i] * k[row + i];
+                    for (int64_t i = 0; i < K; ++i) {
+                        double a = 0.0, b = 0.0, c = 0.0;
+                        for (int64_t j = 0; j < K; ++j) {
+                            a += S[i * K + j] * dout[row + j];
+                            b += G[i * K + j] * v[row + j];
+                            c += G[i * K + j] * S[i * K + j];
+                        }
+                        gr[row + i] = a + u[h * K + i] * k[row + i] * vdo;
+                        gk[row + i] = b + u[h * K + i] * r[row + i] * vdo;
+                        gw[row + i] = c;
+                        gup[i] += r[row + i] * k[row + i] * vdo;
+                    }
+                    for (int64_t j = 0; j < K; ++j) {
+                        double a = 0.0;
+                        for (int64_t i = 0; i < K; ++i) a += k[row + i] * G[i * K + j];
+                        gv[row + j] = a + rku * dout[row + j];
+                    }
+                    /* G_{t-1} = diag(w_t) G_t + r_t^T do_t */
+                    for (int64_t i = 0; i < K; ++i)
+                        for (int64_t j = 0; j < K; ++j)
+                            G[i * K + j] = w[row + i] * G[i * K + j] + r[row + i] * dout[row + j];
+                }
+                if (g_init)
+                    memcpy(g_init + (bi * H + h) * K * K, G, sizeof(double) * (size_t)(K * K));
+            }
+        }
+        free(Sh);
+        free(G);
+    }
+    for (int64_t c = 0; c < HK; ++c) {
+        double s = 0.0;
+        for (int64_t bi = 0; bi < B; ++bi) s += gu_part[bi * HK + c];
+        gu[c] = s;
+    }
+    free(gu_part);
+    const int64_t n = B * T * HK;
+    if (!all_finite(gr, n) || !all_finite(gk, n) || !all_finite(gv, n) || !all_finite(gw, n) ||
+        !all_finite(gu, HK))
+        bad |= 1;
+    return bad;
+}

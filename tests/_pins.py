@@ -140,3 +140,44 @@ def wkv4_fd_grads(fwd, w, u, k, v, gy):
     gw = np.array([fd(w, (c,)) for c in range(w.shape[0])])
     gu = np.array([fd(u, (c,)) for c in range(u.shape[0])])
     return gk, gv, gw, gu
+
+
+def wkv6_fd_grads(fwd, r, k, v, w, u, dout, init_state=None, g_final=None):
+    """Central finite differences of L = sum(o * dout) + sum(fs * g_final)
+    for (o, fs) = fwd(r, k, v, w, u, init_state=...). Step 1e-5 * max(1, |x|).
+    Returns (gr, gk, gv, gw, gu [flat H*K], g_init or None)."""
+    arrs = {n: np.array(a, dtype=np.float64) for n, a in
+            (("r", r), ("k", k), ("v", v), ("w", w), ("u", u))}
+    s0 = None if init_state is None else np.array(init_state, dtype=np.float64)
+
+    def loss():
+        kw = {} if s0 is None else {"init_state": s0}
+        o, fs = fwd(arrs["r"], arrs["k"], arrs["v"], arrs["w"], arrs["u"], **kw)
+        L = float((o * dout).sum())
+        if g_final is not None:
+            L += float((fs * g_final).sum())
+        return L
+
+    def fd(arr, idx):
+        x0 = arr[idx]
+        h = 1e-5 * max(1.0, abs(x0))
+        arr[idx] = x0 + h
+        lp = loss()
+        arr[idx] = x0 - h
+        lm = loss()
+        arr[idx] = x0
+        return (lp - lm) / (2 * h)
+
+    out = []
+    for n in ("r", "k", "v", "w", "u"):
+        a = arrs[n]
+        g = np.zeros_like(a)
+        for idx in np.ndindex(*a.shape):
+            g[idx] = fd(a, idx)
+        out.append(g.reshape(-1) if n == "u" else g)
+    gi = None
+    if s0 is not None:
+        gi = np.zeros_like(s0)
+        for idx in np.ndindex(*s0.shape):
+            gi[idx] = fd(s0, idx)
+    return tuple(out) + (gi,)

@@ -27,6 +27,14 @@ MUTATIONS = {
     "wkv6_u_index": ("u[h * K + i] * k[row + i] * v[row + j]", "u[h * K + j] * k[row + i] * v[row + j]"),
     # RWKV-6: decay indexed by the value dimension
     "wkv6_w_index": ("S[i * K + j] = w[row + i] * S[i * K + j]", "S[i * K + j] = w[row + j] * S[i * K + j]"),
+    # RWKV-6 backward: bonus term dropped from gk
+    "wkv6b_gk_bonus": ("gk[row + i] = b + u[h * K + i] * r[row + i] * vdo;", "gk[row + i] = b;"),
+    # RWKV-6 backward: transposed outer product in the adjoint update
+    "wkv6b_g_transpose": ("G[i * K + j] = w[row + i] * G[i * K + j] + r[row + i] * dout[row + j];",
+                          "G[i * K + j] = w[row + i] * G[i * K + j] + r[row + j] * dout[row + i];"),
+    # RWKV-6 backward: gw and gr against S_t instead of S_{t-1}
+    "wkv6b_state_index": ("const double *S = Sh + t * K * K; /* S_{t-1} */",
+                          "const double *S = Sh + (t + 1) * K * K;"),
 }
 
 
@@ -66,9 +74,23 @@ def _wkv6_pins_fail(var):
     return rel_err(o, wkv6_direct_sum(r, k, v, w, u, K)) > 1e-9
 
 
+def _wkv6b_pins_fail(var):
+    from _pins import wkv6_fd_grads
+    rng = np.random.default_rng(33)
+    B, T, H, K = 1, 5, 1, 3
+    r, k, v, dout = (rng.normal(size=(B, T, H * K)) for _ in range(4))
+    w = rng.uniform(0.3, 1.0, size=(B, T, H * K))
+    u = rng.uniform(-1, 1, size=(H, K))
+    s0, gf = rng.normal(size=(B, H, K, K)), rng.normal(size=(B, H, K, K))
+    got = var.wkv6_backward(r, k, v, w, u, dout, init_state=s0, g_final=gf)
+    num = wkv6_fd_grads(var.wkv6_forward, r, k, v, w, u, dout, init_state=s0, g_final=gf)
+    return any(rel_err(g, n) > 1e-6 for g, n in zip(got, num))
+
+
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
 def test_mutation_is_caught(variants, name):
-    check = _wkv4_pins_fail if name.startswith("wkv4") else _wkv6_pins_fail
+    check = (_wkv4_pins_fail if name.startswith("wkv4") else
+             _wkv6b_pins_fail if name.startswith("wkv6b") else _wkv6_pins_fail)
     assert check(variants[name]), f"planted mistake {name} passed every pin"
 
 
@@ -77,5 +99,7 @@ def test_unmutated_source_passes(oracle):
         wkv4_forward = staticmethod(oracle.wkv4_forward)
         wkv4_backward = staticmethod(oracle.wkv4_backward)
         wkv6_forward = staticmethod(oracle.wkv6_forward)
+        wkv6_backward = staticmethod(oracle.wkv6_backward)
     assert not _wkv4_pins_fail(_Orig)
     assert not _wkv6_pins_fail(_Orig)
+    assert not _wkv6b_pins_fail(_Orig)

@@ -121,3 +121,69 @@ def test_state_carry_and_mapping(oracle):
     # initial state enters the output as r_t diag(prod w) S_0
     oz, _ = oracle.wkv6_forward(r, k, v, w, u, init_state=np.zeros((1, H, K, K)))
     assert np.array_equal(oz, o)
+
+
+# --------------------------------------------------------------------------
+# backward (RWKV6_OP is trainable: the package page lists its CUDA backward)
+# --------------------------------------------------------------------------
+
+def _bwd_case(rng, B, T, H, K):
+    r, k, v, w, u = _case(rng, B, T, H, K, wlo=0.2)
+    dout = rng.normal(size=r.shape)
+    s0 = rng.normal(size=(B, H, K, K))
+    gf = rng.normal(size=(B, H, K, K))
+    return r, k, v, w, u, dout, s0, gf
+
+
+@pytest.mark.parametrize("B,T,H,K", [(1, 5, 1, 3), (2, 4, 2, 2), (1, 7, 1, 4)])
+def test_backward_finite_differences(oracle, B, T, H, K):
+    """Every gradient (r, k, v, w, u and the initial state) against central
+    differences of L = sum(o * dout) + sum(final_state * g_final)."""
+    from _pins import wkv6_fd_grads
+    rng = np.random.default_rng(300 + B * 10 + T)
+    r, k, v, w, u, dout, s0, gf = _bwd_case(rng, B, T, H, K)
+    got = oracle.wkv6_backward(r, k, v, w, u, dout, init_state=s0, g_final=gf)
+    num = wkv6_fd_grads(oracle.wkv6_forward, r, k, v, w, u, dout, init_state=s0, g_final=gf)
+    for name, g, n in zip(("gr", "gk", "gv", "gw", "gu", "g_init"), got, num):
+        assert rel_err(g, n) < 1e-6, name
+
+
+def test_backward_homogeneity(oracle):
+    """o and the final state are linear in r (o only), in k, in v, and affine
+    in the initial state; the bonus part of o is linear in u. Euler's theorem
+    then fixes sum(x * gx) for each, at any size."""
+    rng = np.random.default_rng(41)
+    B, T, H, K = 2, 40, 2, 8
+    r, k, v, w, u, dout, s0, gf = _bwd_case(rng, B, T, H, K)
+    gr, gk, gv, gw, gu, gi = oracle.wkv6_backward(r, k, v, w, u, dout, init_state=s0, g_final=gf)
+    o, fs = oracle.wkv6_forward(r, k, v, w, u, init_state=s0)
+    Lo, Lf = float((o * dout).sum()), float((fs * gf).sum())
+    assert np.isclose((r * gr).sum(), Lo, rtol=1e-11)
+    # with S_-1 = 0 the outputs are bilinear in k and v
+    o0, fs0 = oracle.wkv6_forward(r, k, v, w, u)
+    L0 = float((o0 * dout).sum() + (fs0 * gf).sum())
+    gr0, gk0, gv0, _, gu0, _ = oracle.wkv6_backward(r, k, v, w, u, dout, g_final=gf)
+    assert np.isclose((k * gk0).sum(), L0, rtol=1e-11)
+    assert np.isclose((v * gv0).sum(), L0, rtol=1e-11)
+    # the initial state's share of L
+    assert np.isclose((s0 * gi).sum(), Lo + Lf - L0, rtol=1e-11)
+    # the bonus share: sum_t r_t . (u * k_t) (v_t . do_t)
+    uu = u.reshape(1, 1, H * K)
+    vdo = (v * dout).reshape(B, T, H, K).sum(-1, keepdims=True)
+    bonus = ((r * uu * k).reshape(B, T, H, K) * vdo).sum()
+    assert np.isclose((u.reshape(-1) * gu).sum(), bonus, rtol=1e-11)
+
+
+def test_backward_state_map(oracle):
+    """With a state map every sample's g_init is dL/dS_-1 of that sample."""
+    rng = np.random.default_rng(42)
+    B, T, H, K = 3, 6, 1, 3
+    r, k, v, w, u, dout, _, gf = _bwd_case(rng, B, T, H, K)
+    init = rng.normal(size=(2, H, K, K))
+    smap = np.array([1, 0, 1], np.int32)
+    *_, gi = oracle.wkv6_backward(r, k, v, w, u, dout, init_state=init, state_map=smap, g_final=gf)
+    for b in range(B):
+        sub = lambda x: x[b:b + 1]
+        *_, gib = oracle.wkv6_backward(sub(r), sub(k), sub(v), sub(w), u, sub(dout),
+                                       init_state=init[smap[b]][None], g_final=sub(gf))
+        assert rel_err(gi[b], gib[0]) < 1e-14
