@@ -56,12 +56,13 @@ def test_version_and_strings(W):
 
 def test_size_helpers(W):
     L = W.lib()
-    assert L.wkv4_ckpt_floats(2, 64, 128) == 2 * 2 * 3 * 128
-    assert L.wkv4_ckpt_floats(1, 33, 8) == 1 * 2 * 3 * 8
+    n = lambda T: -(-T // W.CKPT_LEN)  # checkpoints of a T-token sequence
+    assert L.wkv4_ckpt_floats(2, 64, 128) == 2 * n(64) * 3 * 128
+    assert L.wkv4_ckpt_floats(1, 33, 8) == 1 * n(33) * 3 * 8
     assert L.wkv4_ckpt_floats(0, 10, 8) == 0
     ws = L.wkv4_backward_workspace_bytes(2, 64, 128, 1)
     assert ws >= 2 * 2 * 128 * 4
-    assert L.wkv4_backward_workspace_bytes(2, 64, 128, 0) >= ws + 2 * 2 * 3 * 128 * 4
+    assert L.wkv4_backward_workspace_bytes(2, 64, 128, 0) >= ws + 2 * n(64) * 3 * 128 * 4
 
 
 FAKE = 1 << 20  # 16-byte aligned, never dereferenced: every call below fails validation first
