@@ -27,10 +27,11 @@
 // (B~ the same with gy_i y_i). The carries stay bounded by sum |gy| and need
 // no exponent of their own; the loop-carried dependence is one multiply-add.
 //
-// Kernel shape. One warp = 32 channels of one sample; time is walked in
-// reverse one checkpoint interval (WKV4_CKPT_LEN = 16 steps) at a time: the
-// warp restarts the forward recurrence from the interval's checkpoint, keeps
-// the 32 states in registers, then runs the 32 reverse steps. k, v, gy of an
+// Kernel shape. One warp = 64 channels of one sample, a channel pair per
+// lane on the packed fp32 pair instructions; time is walked in reverse one
+// checkpoint interval (WKV4_CKPT_LEN = 16 steps) at a time: the warp restarts
+// the forward recurrence from the interval's checkpoint, keeps the 16 states
+// in registers, then runs the 16 reverse steps. k, v, gy of an
 // interval arrive as one TMA stage of a ring. When lanes are few, each lane's
 // sequence is split into NSEG segments handled by the NSEG one-warp CTAs of a
 // cluster: (1) each CTA folds its segment into a local carry starting from an
@@ -44,96 +45,157 @@
 
 namespace wkv {
 
+// 1: whole intervals take an unpredicated copy of the reverse steps (more
+// overlap between steps, more registers).
+#ifndef WKV4_BWD_WHOLE
+#define WKV4_BWD_WHOLE 1
+#endif
+
 constexpr int kBwdL = WKV4_CKPT_LEN;
+constexpr int kBwdCh = WKV4_WARP_CH;  // channels of one warp: a pair per lane
 
 template <bool V>
 struct BoolTag {
   static constexpr bool value = V;
 };
 
+// Where the recompute leaves the per-step forward quantities (state aa, bb
+// before the step and the absorb exponent z1) for the reverse steps: in
+// registers, or (bf16) in shared memory, which frees ~100 registers per
+// thread for the unpredicated reverse steps (float32 keeps them in registers:
+// its larger stages leave no room for the stash at 7 warps per SM).
+#ifndef WKV4_BWD_SMEM_STASH
+#define WKV4_BWD_SMEM_STASH 1
+#endif
+template <class E>
+constexpr bool bwd_smem_stash() {
+  return WKV4_BWD_SMEM_STASH && sizeof(E) == 2;
+}
+template <bool S>
+struct Wkv4Stash {
+  float4 ab[kBwdL][32];  // (aa.x, aa.y, bb.x, bb.y) of each step, per lane
+  float2 z[kBwdL][32];
+};
+template <>
+struct Wkv4Stash<false> {};
+
 template <class E, int STAGES>
 struct alignas(128) Wkv4BwdSmem {
-  E k[STAGES][kBwdL][32];
-  E v[STAGES][kBwdL][32];
-  E gy[STAGES][kBwdL][32];
+  E k[STAGES][kBwdL][kBwdCh];
+  E v[STAGES][kBwdL][kBwdCh];
+  E gy[STAGES][kBwdL][kBwdCh];
+  Wkv4Stash<bwd_smem_stash<E>()> stash;
   uint64_t full[STAGES];
-  float carry[5][32];  // this segment's local carry A, B, A', B' and its product of f1
+  float2 carry[5][32];  // this segment's local carry A, B, A', B' and its product of f1
 };
 
-// Carried future sums of one lane, normalised by 2^{P} of the forward state
-// at the point they refer to (see above).
-struct Wkv4Carry {
-  float A, B, Ap, Bp;
+// Carried future sums of a lane's channel pair, normalised by 2^{P} of the
+// forward state at the point they refer to (see above).
+struct Wkv4Carry2 {
+  float2 A, B, Ap, Bp;
 };
 
-// One checkpoint interval in reverse. FULL: also produce gk, gv, gw, gu;
-// otherwise only fold the interval into the carry.
-// fprod (fold-only pass) accumulates the product of the f1 factors. WHOLE
-// (n == kBwdL): the reverse steps are not predicated, so the compiler can
-// overlap the independent parts of consecutive steps; the recompute loop
-// always is (unpredicated, both loops together need too many registers).
-template <bool FULL, bool WHOLE, class E>
-__device__ __forceinline__ void wkv4_bwd_interval(const E (*ks)[32], const E (*vs)[32], const E (*gs)[32], int lane,
-                                                  int n, Wkv4State st, float ref, float u2, float w2, Wkv4Carry& cr,
-                                                  float& fprod, float& gw_acc, float& gu_acc, E* gkl, E* gvl,
+__device__ __forceinline__ float2 neg2(float2 a) { return make_float2(-a.x, -a.y); }
+
+// One checkpoint interval in reverse for a lane's channel pair. FULL: also
+// produce gk, gv, gw, gu; otherwise only fold the interval into the carry.
+// fprod (fold-only pass) accumulates the product of the f1 factors; gwn
+// accumulates -gw. WHOLE (n == kBwdL): the reverse steps are not
+// predicated, so the compiler can overlap the independent parts of
+// consecutive steps; the recompute loop always is.
+template <bool FULL, bool WHOLE, class E, bool S>
+__device__ __forceinline__ void wkv4_bwd_interval(const E (*ks)[kBwdCh], const E (*vs)[kBwdCh],
+                                                  const E (*gs)[kBwdCh], Wkv4Stash<S>& sx, int lane, int n,
+                                                  Wkv4State2 st, float2 ref, float2 uw2, float2 w2, Wkv4Carry2& cr,
+                                                  float2& fprod, float2& gwn, float2& gu_acc, E* gkl, E* gvl,
                                                   int C) {
-  // forward recompute over the interval: state before each token
-  float saa[kBwdL], sbb[kBwdL], spp[kBwdL];
+  // forward recompute over the interval: state before each token and the
+  // token's absorb exponent z1 (the forward's own rounding of it)
+  constexpr int kReg = S ? 1 : kBwdL;
+  float2 saa[kReg], sbb[kReg], sz[kReg];
 #pragma unroll
   for (int jj = 0; jj < kBwdL; ++jj) {
     if (jj < n) {
-      saa[jj] = st.aa;
-      sbb[jj] = st.bb;
-      spp[jj] = wkv4_exponent(st, w2);
-      wkv4_absorb(st, wkv4_key(Elem<E>::to_f32(ks[jj][lane]), ref), Elem<E>::to_f32(vs[jj][lane]), w2);
+      const float2 aa = st.aa, bb = st.bb;
+      const float2 z1 = wkv4_absorb2(st, wkv4_key2(ld_pair(&ks[jj][2 * lane]), ref), ld_pair(&vs[jj][2 * lane]), w2);
+      if constexpr (S) {
+        sx.ab[jj][lane] = make_float4(aa.x, aa.y, bb.x, bb.y);
+        sx.z[jj][lane] = z1;
+      } else {
+        saa[jj] = aa;
+        sbb[jj] = bb;
+        sz[jj] = z1;
+      }
     }
   }
-  float A = cr.A, B = cr.B, Ap = cr.Ap, Bp = cr.Bp;
+  float2 A = cr.A, B = cr.B, Ap = cr.Ap, Bp = cr.Bp;
 #pragma unroll
   for (int jj = kBwdL - 1; jj >= 0; --jj) {
     if (WHOLE || jj < n) {
-      const float k2 = wkv4_key(Elem<E>::to_f32(ks[jj][lane]), ref);
-      const float vv = Elem<E>::to_f32(vs[jj][lane]);
-      const float g = Elem<E>::to_f32(gs[jj][lane]);
-      const float P = spp[jj];
+      const float2 vv = ld_pair(&vs[jj][2 * lane]);
+      const float2 g = ld_pair(&gs[jj][2 * lane]);
+      float2 aa, bb, z;
+      if constexpr (S) {
+        const float4 ab = sx.ab[jj][lane];
+        aa = make_float2(ab.x, ab.y);
+        bb = make_float2(ab.z, ab.w);
+        z = sx.z[jj][lane];
+      } else {
+        aa = saa[jj];
+        bb = sbb[jj];
+        z = sz[jj];
+      }
       // output of token jj, in units of the past's exponent P: weight
-      // e = 2^{u + k - P} of the current token (capped as in the forward),
-      // D = 2^P (bb + e), y = (aa + e v) / (bb + e)
-      const float e = ex2(fminf(__fsub_rn(__fadd_rn(u2, k2), P), 64.f));
-      const float rd = rcp(__fadd_rn(sbb[jj], e));
-      const float yv = __fmul_rn(__fmaf_rn(e, vv, saa[jj]), rd);
+      // e = 2^{u + k - P} = 2^{z1 + u - w} of the current token (capped as in
+      // the forward), D = 2^P (bb + e), y = (aa + e v) / (bb + e)
+      const float2 zo = add2(z, uw2);
+      const float2 e = make_float2(ex2(fminf(zo.x, 64.f)), ex2(fminf(zo.y, 64.f)));
+      const float2 rd = rcp2(add2(bb, e));
+      const float2 yv = mul2(fma2(e, vv, aa), rd);
       // absorb pair of token jj: P' = max(P - w, k)
-      const float z = __fsub_rn(k2, __fsub_rn(P, w2));
-      const float ea = ex2(-fabsf(z));
-      const bool keep = z <= 0.f;
-      const float f1 = keep ? 1.f : ea;
-      const float f2 = keep ? ea : 1.f;
-      const float ag = __fmul_rn(g, rd);  // gy 2^P / D
+      const float2 ea = make_float2(ex2(-fabsf(z.x)), ex2(-fabsf(z.y)));
+      const bool kx = z.x <= 0.f, ky = z.y <= 0.f;
+      const float2 f1 = make_float2(kx ? 1.f : ea.x, ky ? 1.f : ea.y);
+      const float2 f2 = make_float2(kx ? ea.x : 1.f, ky ? ea.y : 1.f);
+      const float2 ag = mul2(g, rd);  // gy 2^P / D
       if constexpr (FULL) {
-        const float rg = __fmul_rn(ag, e);  // gy rho, rho = e^{u+k} / D
+        const float2 rg = mul2(ag, e);  // gy rho, rho = e^{u+k} / D
         // v - y = (bb v - aa) / (bb + e): no cancellation against v when the
         // current token dominates (y within rounding of v)
-        const float vmy = __fmul_rn(__fmaf_rn(sbb[jj], vv, -saa[jj]), rd);
-        const float gvv = __fmaf_rn(f2, A, rg);
-        const float gkv = __fmaf_rn(rg, vmy, __fmul_rn(f2, __fmaf_rn(vv, A, -B)));
-        gu_acc = __fmaf_rn(rg, vmy, gu_acc);
-        gw_acc = __fmaf_rn(-f2, __fmaf_rn(vv, Ap, -Bp), gw_acc);
-        gkl[(int64_t)jj * C] = Elem<E>::from_f32(gkv);
-        gvl[(int64_t)jj * C] = Elem<E>::from_f32(gvv);
+        const float2 vmy = mul2(fma2(bb, vv, neg2(aa)), rd);
+        const float2 gvv = fma2(f2, A, rg);
+        const float2 gkv = fma2(rg, vmy, mul2(f2, fma2(vv, A, neg2(B))));
+        gu_acc = fma2(rg, vmy, gu_acc);
+        gwn = fma2(f2, fma2(vv, Ap, neg2(Bp)), gwn);
+        st_pair(gkl + (int64_t)jj * C, gkv);
+        st_pair(gvl + (int64_t)jj * C, gvv);
       }
-      if constexpr (!FULL) fprod = __fmul_rn(fprod, f1);
+      if constexpr (!FULL) fprod = mul2(fprod, f1);
       // carries for token jj - 1
-      Ap = __fmul_rn(f1, __fadd_rn(Ap, A));
-      Bp = __fmul_rn(f1, __fadd_rn(Bp, B));
-      A = __fmaf_rn(f1, A, ag);
-      B = __fmaf_rn(f1, B, __fmul_rn(ag, yv));
+      Ap = mul2(f1, add2(Ap, A));
+      Bp = mul2(f1, add2(Bp, B));
+      A = fma2(f1, A, ag);
+      B = fma2(f1, B, mul2(ag, yv));
     }
   }
   cr = {A, B, Ap, Bp};
 }
 
+// One carry merge for one channel: the carry `in` entering segment r from
+// the later ones, folded through segment r (len steps, its local carry `own`
+// and product of f1 `f`).
+__device__ __forceinline__ void wkv4_carry_fold(float& A, float& B, float& Ap, float& Bp, float f, float m,
+                                                float oA, float oB, float oAp, float oBp) {
+  const float nA = __fmaf_rn(f, A, oA), nB = __fmaf_rn(f, B, oB);
+  const float nAp = __fmaf_rn(f, __fmaf_rn(m, A, Ap), oAp), nBp = __fmaf_rn(f, __fmaf_rn(m, B, Bp), oBp);
+  A = nA;
+  B = nB;
+  Ap = nAp;
+  Bp = nBp;
+}
+
 template <class E, int STAGES, int NSEG, int NW>
-__global__ void __launch_bounds__(32 * NW, NSEG == 1 ? 16 : 1) wkv4_bwd_kernel(const __grid_constant__ CUtensorMap tk,
+__global__ void __launch_bounds__(32 * NW, NSEG == 1 ? 8 : 1) wkv4_bwd_kernel(const __grid_constant__ CUtensorMap tk,
                                                            const __grid_constant__ CUtensorMap tv,
                                                            const __grid_constant__ CUtensorMap tg, int T, int C,
                                                            int ncb, int ngroups, const float* __restrict__ w,
@@ -144,7 +206,7 @@ __global__ void __launch_bounds__(32 * NW, NSEG == 1 ? 16 : 1) wkv4_bwd_kernel(c
   extern __shared__ __align__(128) unsigned char wkv4_bwd_dsmem[];
   // each warp is an independent lane group with its own ring and barriers
   Wkv4BwdSmem<E, STAGES>& sm = reinterpret_cast<Wkv4BwdSmem<E, STAGES>*>(wkv4_bwd_dsmem)[threadIdx.x / 32];
-  constexpr uint32_t kStageBytes = 3u * kBwdL * 32u * sizeof(E);
+  constexpr uint32_t kStageBytes = 3u * kBwdL * kBwdCh * sizeof(E);
   constexpr int kPasses = NSEG > 1 ? 2 : 1;
 
   const int lane = threadIdx.x % 32;
@@ -153,8 +215,8 @@ __global__ void __launch_bounds__(32 * NW, NSEG == 1 ? 16 : 1) wkv4_bwd_kernel(c
   const bool active = group < ngroups;  // a warp past the last group only joins the cluster barriers
   const int cb = group % ncb;
   const int b = group / ncb;
-  const int c0 = cb * 32;
-  const int c = c0 + lane;
+  const int c0 = cb * kBwdCh;
+  const int c = c0 + 2 * lane;  // this lane's channels c, c + 1
   const bool valid = active && c < C;
   const int nck = (T + kBwdL - 1) / kBwdL;
   const int i_beg = wkv4_seg_begin(seg, NSEG, nck);
@@ -181,16 +243,21 @@ __global__ void __launch_bounds__(32 * NW, NSEG == 1 ? 16 : 1) wkv4_bwd_kernel(c
   }
   __syncwarp();
 
-  const float w2 = valid ? __fmul_rn(w[c], kLog2e) : 0.f;
-  const float u2 = valid ? __fmul_rn(u[c], kLog2e) : 0.f;
+  const float2 w2 = valid ? mul2(ld_pair(w + c), splat2(kLog2e)) : splat2(0.f);
+  const float2 u2 = valid ? mul2(ld_pair(u + c), splat2(kLog2e)) : splat2(0.f);
+  const float2 uw2 = sub2(u2, w2);  // output exponent minus absorb exponent
   const int64_t lane_off = valid ? (int64_t)b * T * C + c : 0;
-  // lane reference exponent: the same value the forward derived from token 0
-  const float ref = valid ? wkv4_ref(Elem<E>::to_f32(kraw[lane_off])) : 0.f;
+  // lane reference exponents: the values the forward derived from token 0
+  float2 ref = splat2(0.f);
+  if (valid) {
+    const float2 kf = ld_pair(kraw + lane_off);
+    ref = make_float2(wkv4_ref(kf.x), wkv4_ref(kf.y));
+  }
   const float* ckl = ckpt + (valid ? (int64_t)b * nck * 3 * C + c : 0);
-  auto load_ckpt = [&](int i) -> Wkv4State {
-    if (!valid) return {0.f, 0.f, 0.f, 0.f};
+  auto load_ckpt = [&](int i) -> Wkv4State2 {
+    if (!valid) return {splat2(0.f), splat2(0.f), splat2(0.f), splat2(0.f)};
     const float* p = ckl + (int64_t)i * 3 * C;
-    return {p[0], p[C], p[2 * (int64_t)C], 0.f};
+    return {ld_pair(p), ld_pair(p + C), ld_pair(p + 2 * (int64_t)C), splat2(0.f)};
   };
 
   int qq = 0;
@@ -206,30 +273,31 @@ __global__ void __launch_bounds__(32 * NW, NSEG == 1 ? 16 : 1) wkv4_bwd_kernel(c
   };
 
   // reverse carries (normalised by the forward exponent, see above)
-  Wkv4Carry cr = {0.f, 0.f, 0.f, 0.f};
-  float gw_acc = 0.f, gu_acc = 0.f;
-  auto run_interval = [&](auto full_tag, int s, int i, const Wkv4State& st, float& fprod) {
+  Wkv4Carry2 cr = {splat2(0.f), splat2(0.f), splat2(0.f), splat2(0.f)};
+  float2 gwn = splat2(0.f), gu_acc = splat2(0.f);
+  auto run_interval = [&](auto full_tag, int s, int i, const Wkv4State2& st, float2& fprod) {
     constexpr bool kFull = decltype(full_tag)::value;
     const int n = min(kBwdL, T - i * kBwdL);
     const int64_t off = lane_off + (int64_t)i * kBwdL * C;
     E* gkp = kFull ? gk + off : nullptr;
     E* gvp = kFull ? gv + off : nullptr;
-    // unpredicated steps for whole bf16 intervals (float32 would spill)
-    if (sizeof(E) == 2 && n == kBwdL)
-      wkv4_bwd_interval<kFull, sizeof(E) == 2, E>(sm.k[s], sm.v[s], sm.gy[s], lane, n, st, ref, u2, w2, cr, fprod, gw_acc,
+#if WKV4_BWD_WHOLE
+    if (n == kBwdL)
+      wkv4_bwd_interval<kFull, true>(sm.k[s], sm.v[s], sm.gy[s], sm.stash, lane, n, st, ref, uw2, w2, cr, fprod, gwn,
                                         gu_acc, gkp, gvp, C);
     else
-      wkv4_bwd_interval<kFull, false, E>(sm.k[s], sm.v[s], sm.gy[s], lane, n, st, ref, u2, w2, cr, fprod, gw_acc,
+#endif
+      wkv4_bwd_interval<kFull, false>(sm.k[s], sm.v[s], sm.gy[s], sm.stash, lane, n, st, ref, uw2, w2, cr, fprod, gwn,
                                          gu_acc, gkp, gvp, C);
   };
 
   if constexpr (NSEG > 1) {
     // ---- phase 1: this segment's own carry, from an empty future ----
-    float fprod = 1.f;
-    Wkv4State nxt = nloc > 0 ? load_ckpt(interval(0)) : Wkv4State{0.f, 0.f, 0.f, 0.f};
+    float2 fprod = splat2(1.f);
+    Wkv4State2 nxt = nloc > 0 ? load_ckpt(interval(0)) : Wkv4State2{splat2(0.f), splat2(0.f), splat2(0.f), splat2(0.f)};
     for (; ok && qq < nloc; ++qq) {
       const int i = interval(qq);
-      const Wkv4State st = nxt;
+      const Wkv4State2 st = nxt;
       if (qq + 1 < nloc) nxt = load_ckpt(interval(qq + 1));
       if (!acquire(qq)) break;
       if (valid) run_interval(BoolTag<false>{}, qq % STAGES, i, st, fprod);
@@ -243,29 +311,32 @@ __global__ void __launch_bounds__(32 * NW, NSEG == 1 ? 16 : 1) wkv4_bwd_kernel(c
     cluster_arrive_release();
     cluster_wait_acquire();
     // ---- phase 2: the exact carry entering this segment from the later ones ----
-    Wkv4Carry in = {0.f, 0.f, 0.f, 0.f};
+    float in[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
     for (int r = NSEG - 1; r > seg; --r) {
       const int len = min(T, wkv4_seg_begin(r + 1, NSEG, nck) * kBwdL) - wkv4_seg_begin(r, NSEG, nck) * kBwdL;
-      const float f = ld_shared_cluster(map_shared_rank(&sm.carry[4][lane], r));
       const float m = (float)len;
-      in = {__fmaf_rn(f, in.A, ld_shared_cluster(map_shared_rank(&sm.carry[0][lane], r))),
-            __fmaf_rn(f, in.B, ld_shared_cluster(map_shared_rank(&sm.carry[1][lane], r))),
-            __fmaf_rn(f, __fmaf_rn(m, in.A, in.Ap), ld_shared_cluster(map_shared_rank(&sm.carry[2][lane], r))),
-            __fmaf_rn(f, __fmaf_rn(m, in.B, in.Bp), ld_shared_cluster(map_shared_rank(&sm.carry[3][lane], r)))};
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        auto peer = [&](int comp) {
+          return ld_shared_cluster(map_shared_rank(reinterpret_cast<const float*>(&sm.carry[comp][lane]) + h, r));
+        };
+        wkv4_carry_fold(in[h][0], in[h][1], in[h][2], in[h][3], peer(4), m, peer(0), peer(1), peer(2), peer(3));
+      }
     }
     cluster_arrive_release();  // done reading peers; waited for before exit
-    cr = in;
-    gw_acc = 0.f;
-    gu_acc = 0.f;
+    cr = {make_float2(in[0][0], in[1][0]), make_float2(in[0][1], in[1][1]), make_float2(in[0][2], in[1][2]),
+          make_float2(in[0][3], in[1][3])};
+    gwn = splat2(0.f);
+    gu_acc = splat2(0.f);
   }
 
   // ---- last pass: gradients ----
   {
-    float unused = 1.f;
-    Wkv4State nxt = nloc > 0 ? load_ckpt(interval(0)) : Wkv4State{0.f, 0.f, 0.f, 0.f};
+    float2 unused = splat2(1.f);
+    Wkv4State2 nxt = nloc > 0 ? load_ckpt(interval(0)) : Wkv4State2{splat2(0.f), splat2(0.f), splat2(0.f), splat2(0.f)};
     for (; ok && qq < total; ++qq) {
       const int i = interval(qq);
-      const Wkv4State st = nxt;
+      const Wkv4State2 st = nxt;
       if (qq + 1 < total) nxt = load_ckpt(interval(qq + 1));
       if (!acquire(qq)) break;
       if (valid) run_interval(BoolTag<true>{}, qq % STAGES, i, st, unused);
@@ -277,8 +348,8 @@ __global__ void __launch_bounds__(32 * NW, NSEG == 1 ? 16 : 1) wkv4_bwd_kernel(c
       for (int x = qq; x < total && x < qq + STAGES; ++x) mbar_wait_bounded(&sm.full[x % STAGES], (x / STAGES) & 1, err);
   } else if (valid) {
     const int64_t pi = ((int64_t)b * NSEG + seg) * C + c;
-    part_gw[pi] = gw_acc;
-    part_gu[pi] = gu_acc;
+    st_pair(part_gw + pi, neg2(gwn));
+    st_pair(part_gu + pi, gu_acc);
   }
   if constexpr (NSEG > 1) cluster_wait_acquire();  // peers may still read this CTA's carry
 }
@@ -321,11 +392,11 @@ template <class E, int STAGES, int NSEG, int NW>
 static wkv_status run_bwd(const Wkv4BwdArgs& a, cudaStream_t stream, unsigned* err, const char** why) {
   CUtensorMap tk, tv, tg;
   const CUtensorMapDataType ty = Elem<E>::tma_type;
-  if (!encode_tmap_3d(&tk, a.k, ty, sizeof(E), a.C, a.T, a.B, 32, kBwdL, 1, why) ||
-      !encode_tmap_3d(&tv, a.v, ty, sizeof(E), a.C, a.T, a.B, 32, kBwdL, 1, why) ||
-      !encode_tmap_3d(&tg, a.gy, ty, sizeof(E), a.C, a.T, a.B, 32, kBwdL, 1, why))
+  if (!encode_tmap_3d(&tk, a.k, ty, sizeof(E), a.C, a.T, a.B, kBwdCh, kBwdL, 1, why) ||
+      !encode_tmap_3d(&tv, a.v, ty, sizeof(E), a.C, a.T, a.B, kBwdCh, kBwdL, 1, why) ||
+      !encode_tmap_3d(&tg, a.gy, ty, sizeof(E), a.C, a.T, a.B, kBwdCh, kBwdL, 1, why))
     return WKV_ERR_INVALID_ARG;
-  const int ncb = (int)ceil_div(a.C, 32);
+  const int ncb = (int)ceil_div(a.C, kBwdCh);
   const int ngroups = (int)(ncb * a.B);
   const int64_t rows = a.B * NSEG;
   float* part_gw = a.part;
@@ -372,7 +443,7 @@ static wkv_status run_bwd(const Wkv4BwdArgs& a, cudaStream_t stream, unsigned* e
 }
 
 // Stages of the k/v/gy ring (one checkpoint interval each): four for bf16
-// (3 KB a stage), two for float32 (6 KB), so that the 14-16 one-warp CTAs an
+// (6 KB a stage), two for float32 (12 KB), so that the 7-8 one-warp CTAs an
 // SM holds still fit in shared memory.
 template <class E, int STAGES, int NSEG>
 static wkv_status run_bwd_nw(const Wkv4BwdArgs& a, cudaStream_t stream, unsigned* err, const char** why) {
@@ -385,7 +456,7 @@ static wkv_status run_bwd_nw(const Wkv4BwdArgs& a, cudaStream_t stream, unsigned
 
 template <class E>
 static wkv_status run_bwd_nseg(const Wkv4BwdArgs& a, cudaStream_t stream, unsigned* err, const char** why) {
-  constexpr int kStages = sizeof(E) == 2 ? 4 : 2;
+  constexpr int kStages = sizeof(E) == 2 ? (bwd_smem_stash<E>() ? 3 : 4) : 2;
   switch (wkv4_bwd_segments(a.B, a.T, a.C)) {
 #if WKV4_MAX_SEGMENTS_ANY > 8
     case 16: return run_bwd_nw<E, kStages, 16>(a, stream, err, why);

@@ -5,8 +5,9 @@
 // running-max recurrence of wkv_device.cuh.
 //
 // Design. The recurrence is sequential in t and independent per lane (b, c).
-// A warp owns 32 consecutive channels of one sample and keeps their states in
-// registers. When there are too few lanes to fill the GPU, each lane's
+// A warp owns 64 consecutive channels of one sample, a pair per thread, and
+// keeps their states in registers; the pair runs on the packed fp32
+// instructions (wkv4_token2). When there are too few lanes to fill the GPU, each lane's
 // sequence is split into NSEG segments of whole checkpoint intervals, one
 // one-warp CTA per segment, the NSEG CTAs forming a thread-block cluster:
 //   1. every CTA runs its segment from the empty past (absorb only) and leaves
@@ -18,7 +19,7 @@
 //      checkpoints (the second read of k, v mostly hits L2).
 // With NSEG = 1 phases 1-2 vanish and the kernel is the plain sequential scan.
 // k and v stream through a ring of STAGES shared-memory tiles of LT steps,
-// filled by 3-D TMA loads (box {32 ch, LT steps, 1 sample}; rows past the
+// filled by 3-D TMA loads (box {64 ch, LT steps, 1 sample}; rows past the
 // segment are ignored) that complete on per-stage mbarriers; lane 0 refills a
 // stage as soon as the warp has consumed it. y is written straight from
 // registers. Every WKV4_CKPT_LEN steps the state (aa, bb, P) goes to the
@@ -29,12 +30,15 @@
 
 namespace wkv {
 
+// Channels one warp covers: 32 lanes x a pair each.
+constexpr int kFwdCh = WKV4_WARP_CH;
+
 template <class E, int LT, int STAGES>
 struct alignas(128) Wkv4FwdSmem {
-  E k[STAGES][LT][32];
-  E v[STAGES][LT][32];
+  E k[STAGES][LT][kFwdCh];
+  E v[STAGES][LT][kFwdCh];
   uint64_t full[STAGES];
-  float seg_aa[32], seg_bb[32], seg_P[32];  // this segment's own state (phase 1)
+  float2 seg_aa[32], seg_bb[32], seg_P[32];  // this segment's own state (phase 1)
 };
 
 template <class E, int LT, int STAGES, int NSEG, int NW>
@@ -48,7 +52,7 @@ __global__ void __launch_bounds__(32 * NW) wkv4_fwd_kernel(const __grid_constant
   extern __shared__ __align__(128) unsigned char wkv4_fwd_dsmem[];
   // each warp is an independent lane group with its own ring and barriers
   Wkv4FwdSmem<E, LT, STAGES>& sm = reinterpret_cast<Wkv4FwdSmem<E, LT, STAGES>*>(wkv4_fwd_dsmem)[threadIdx.x / 32];
-  constexpr uint32_t kStageBytes = 2u * LT * 32u * sizeof(E);
+  constexpr uint32_t kStageBytes = 2u * LT * kFwdCh * sizeof(E);
   constexpr int kPasses = NSEG > 1 ? 2 : 1;
 
   const int lane = threadIdx.x % 32;
@@ -57,8 +61,8 @@ __global__ void __launch_bounds__(32 * NW) wkv4_fwd_kernel(const __grid_constant
   const bool active = group < ngroups;  // a warp past the last group only joins the cluster barriers
   const int cb = group % ncb;
   const int b = group / ncb;
-  const int c0 = cb * 32;
-  const int c = c0 + lane;
+  const int c0 = cb * kFwdCh;
+  const int c = c0 + 2 * lane;  // this lane's channels c, c + 1
   const bool valid = active && c < C;
   const int nck = (T + WKV4_CKPT_LEN - 1) / WKV4_CKPT_LEN;
   const int t_beg = wkv4_seg_begin(seg, NSEG, nck) * WKV4_CKPT_LEN;
@@ -83,9 +87,13 @@ __global__ void __launch_bounds__(32 * NW) wkv4_fwd_kernel(const __grid_constant
   __syncwarp();
 
   const int64_t lane_off = valid ? (int64_t)b * T * C + c : 0;
-  const float w2 = valid ? __fmul_rn(w[c], kLog2e) : 0.f;
-  const float u2 = valid ? __fmul_rn(u[c], kLog2e) : 0.f;
-  const float ref = valid ? wkv4_ref(Elem<E>::to_f32(kraw[lane_off])) : 0.f;
+  const float2 w2 = valid ? mul2(ld_pair(w + c), splat2(kLog2e)) : splat2(0.f);
+  const float2 u2 = valid ? mul2(ld_pair(u + c), splat2(kLog2e)) : splat2(0.f);
+  float2 ref = splat2(0.f);
+  if (valid) {
+    const float2 kf = ld_pair(kraw + lane_off);
+    ref = make_float2(wkv4_ref(kf.x), wkv4_ref(kf.y));
+  }
   float* ckl = ckpt ? ckpt + (int64_t)b * nck * 3 * C + c : nullptr;
 
   int q = 0;          // next tile to consume
@@ -100,7 +108,7 @@ __global__ void __launch_bounds__(32 * NW) wkv4_fwd_kernel(const __grid_constant
     if (lane == 0 && qq + STAGES < total) issue(qq + STAGES);
   };
 
-  Wkv4State st = wkv4_empty_state();
+  Wkv4State2 st = wkv4_empty_state2();
   if constexpr (NSEG > 1) {
     // ---- phase 1: this segment from the empty past ----
     for (; ok && q < ntile; ++q) {
@@ -110,28 +118,36 @@ __global__ void __launch_bounds__(32 * NW) wkv4_fwd_kernel(const __grid_constant
       if (valid) {
 #pragma unroll 4
         for (int j = 0; j < n; ++j)
-          wkv4_absorb(st, wkv4_key(Elem<E>::to_f32(sm.k[s][j][lane]), ref), Elem<E>::to_f32(sm.v[s][j][lane]), w2);
+          wkv4_absorb2(st, wkv4_key2(ld_pair(&sm.k[s][j][2 * lane]), ref), ld_pair(&sm.v[s][j][2 * lane]), w2);
       }
       release(q);
     }
     sm.seg_aa[lane] = st.aa;
     sm.seg_bb[lane] = st.bb;
-    sm.seg_P[lane] = wkv4_exponent(st, w2);
+    sm.seg_P[lane] = wkv4_exponent2(st, w2);
     cluster_arrive_release();
     cluster_wait_acquire();
     // ---- phase 2: fold the segments before this one into the incoming state ----
-    Wkv4Sum in = {0.f, 0.f, kEmptyPP};
+    Wkv4Sum inx = {0.f, 0.f, kEmptyPP}, iny = inx;
     for (int r = 0; r < seg; ++r) {
       const int len = min(T, wkv4_seg_begin(r + 1, NSEG, nck) * WKV4_CKPT_LEN) -
                       wkv4_seg_begin(r, NSEG, nck) * WKV4_CKPT_LEN;
-      const Wkv4Sum own = {ld_shared_cluster(map_shared_rank(&sm.seg_aa[lane], r)),
-                           ld_shared_cluster(map_shared_rank(&sm.seg_bb[lane], r)),
-                           ld_shared_cluster(map_shared_rank(&sm.seg_P[lane], r))};
-      in.P = __fmaf_rn(-(float)len, w2, in.P);  // decay the earlier part across segment r
-      in = wkv4_merge(in, own);
+      const float* pa = reinterpret_cast<const float*>(&sm.seg_aa[lane]);
+      const float* pb = reinterpret_cast<const float*>(&sm.seg_bb[lane]);
+      const float* pp = reinterpret_cast<const float*>(&sm.seg_P[lane]);
+      const Wkv4Sum ownx = {ld_shared_cluster(map_shared_rank(pa, r)), ld_shared_cluster(map_shared_rank(pb, r)),
+                            ld_shared_cluster(map_shared_rank(pp, r))};
+      const Wkv4Sum owny = {ld_shared_cluster(map_shared_rank(pa + 1, r)),
+                            ld_shared_cluster(map_shared_rank(pb + 1, r)),
+                            ld_shared_cluster(map_shared_rank(pp + 1, r))};
+      // decay the earlier part across segment r
+      inx.P = __fmaf_rn(-(float)len, w2.x, inx.P);
+      iny.P = __fmaf_rn(-(float)len, w2.y, iny.P);
+      inx = wkv4_merge(inx, ownx);
+      iny = wkv4_merge(iny, owny);
     }
     cluster_arrive_release();  // done reading peers; waited for before exit
-    st = {in.aa, in.bb, in.P, 0.f};
+    st = {make_float2(inx.aa, iny.aa), make_float2(inx.bb, iny.bb), make_float2(inx.P, iny.P), splat2(0.f)};
   }
 
   // ---- last pass: outputs and checkpoints ----
@@ -139,9 +155,9 @@ __global__ void __launch_bounds__(32 * NW) wkv4_fwd_kernel(const __grid_constant
   // state before token t (t a multiple of WKV4_CKPT_LEN) to the checkpoints
   auto write_ckpt = [&](int t) {
     float* p = ckl + (int64_t)(t / WKV4_CKPT_LEN) * 3 * C;
-    p[0] = st.aa;
-    p[C] = st.bb;
-    p[2 * (int64_t)C] = wkv4_exponent(st, w2);
+    st_pair(p, st.aa);
+    st_pair(p + C, st.bb);
+    st_pair(p + 2 * (int64_t)C, wkv4_exponent2(st, w2));
   };
   for (; ok && q < total; ++q) {
     const int t0 = t_beg + (q % ntile) * LT;  // a multiple of WKV4_CKPT_LEN
@@ -158,17 +174,17 @@ __global__ void __launch_bounds__(32 * NW) wkv4_fwd_kernel(const __grid_constant
 #pragma unroll 8
           for (int j2 = 0; j2 < WKV4_CKPT_LEN; ++j2) {
             const int j = jc + j2;
-            const float yv = wkv4_token(st, wkv4_key(Elem<E>::to_f32(sm.k[s][j][lane]), ref),
-                                        Elem<E>::to_f32(sm.v[s][j][lane]), u2, w2);
-            if (yt) yt[(int64_t)j * C] = Elem<E>::from_f32(yv);
+            const float2 yv = wkv4_token2(st, wkv4_key2(ld_pair(&sm.k[s][j][2 * lane]), ref),
+                                          ld_pair(&sm.v[s][j][2 * lane]), u2, w2);
+            if (yt) st_pair(yt + (int64_t)j * C, yv);
           }
         }
       } else {
         for (int j = 0; j < n; ++j) {
           if (j > 0 && j % WKV4_CKPT_LEN == 0 && ckl) write_ckpt(t0 + j);
-          const float yv = wkv4_token(st, wkv4_key(Elem<E>::to_f32(sm.k[s][j][lane]), ref),
-                                      Elem<E>::to_f32(sm.v[s][j][lane]), u2, w2);
-          if (yt) yt[(int64_t)j * C] = Elem<E>::from_f32(yv);
+          const float2 yv = wkv4_token2(st, wkv4_key2(ld_pair(&sm.k[s][j][2 * lane]), ref),
+                                        ld_pair(&sm.v[s][j][2 * lane]), u2, w2);
+          if (yt) st_pair(yt + (int64_t)j * C, yv);
         }
       }
     }
@@ -187,10 +203,10 @@ template <class E, int LT, int STAGES, int NSEG, int NW>
 static wkv_status run_fwd(const Wkv4FwdArgs& a, cudaStream_t stream, unsigned* err, const char** why) {
   CUtensorMap tk, tv;
   const CUtensorMapDataType ty = Elem<E>::tma_type;
-  if (!encode_tmap_3d(&tk, a.k, ty, sizeof(E), a.C, a.T, a.B, 32, LT, 1, why) ||
-      !encode_tmap_3d(&tv, a.v, ty, sizeof(E), a.C, a.T, a.B, 32, LT, 1, why))
+  if (!encode_tmap_3d(&tk, a.k, ty, sizeof(E), a.C, a.T, a.B, kFwdCh, LT, 1, why) ||
+      !encode_tmap_3d(&tv, a.v, ty, sizeof(E), a.C, a.T, a.B, kFwdCh, LT, 1, why))
     return WKV_ERR_INVALID_ARG;
-  const int ncb = (int)ceil_div(a.C, 32);
+  const int ncb = (int)ceil_div(a.C, kFwdCh);
   const int ngroups = (int)(ncb * a.B);
   auto kern = wkv4_fwd_kernel<E, LT, STAGES, NSEG, NW>;
   const size_t smem = NW * sizeof(Wkv4FwdSmem<E, LT, STAGES>);

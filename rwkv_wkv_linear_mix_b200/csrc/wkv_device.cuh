@@ -391,4 +391,84 @@ __device__ __forceinline__ void wkv4_absorb(Wkv4State& s, float kk, float v, flo
   s.n = pa ? n1 : 0.f;
 }
 
+// ----------------------------------------------------------------------------
+// Two channels per lane. The RWKV-4 kernels give each lane an adjacent pair
+// of channels and run the step above on float2 with the packed fp32 pair
+// instructions of sm_100 (FFMA2 / FADD2 / FMUL2 behind __ffma2_rn and
+// friends): one issue slot does the arithmetic of both channels, and every
+// component is rounded exactly as its scalar counterpart, so a pair step is
+// bit for bit two scalar steps. k, v and y move as 4-byte (bf16) or 8-byte
+// (float32) pairs. C is even (see the ABI), so a pair never straddles C.
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ float2 splat2(float a) { return make_float2(a, a); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+// a - b with one rounding: fma(b, -1, a) is exact before it rounds, so it
+// equals the scalar __fsub_rn(a, b)
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __ffma2_rn(b, make_float2(-1.f, -1.f), a); }
+__device__ __forceinline__ float2 ex2_2(float2 a) { return make_float2(ex2(a.x), ex2(a.y)); }
+__device__ __forceinline__ float2 rcp2(float2 a) { return make_float2(rcp(a.x), rcp(a.y)); }
+
+__device__ __forceinline__ float2 ld_pair(const float* p) { return *reinterpret_cast<const float2*>(p); }
+__device__ __forceinline__ float2 ld_pair(const __nv_bfloat16* p) {
+  const uint32_t x = *reinterpret_cast<const uint32_t*>(p);  // channel c in the low half
+  return make_float2(__uint_as_float(x << 16), __uint_as_float(x & 0xFFFF0000u));
+}
+__device__ __forceinline__ void st_pair(float* p, float2 v) { *reinterpret_cast<float2*>(p) = v; }
+__device__ __forceinline__ void st_pair(__nv_bfloat16* p, float2 v) {
+  *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(v.x, v.y);
+}
+
+struct Wkv4State2 {
+  float2 aa, bb, base, n;
+};
+
+__device__ __forceinline__ Wkv4State2 wkv4_empty_state2() {
+  return {splat2(0.f), splat2(0.f), splat2(kEmptyPP), splat2(0.f)};
+}
+__device__ __forceinline__ float2 wkv4_key2(float2 k, float2 ref) {
+  return fma2(k, splat2(kLog2e), make_float2(-ref.x, -ref.y));
+}
+__device__ __forceinline__ float2 wkv4_exponent2(const Wkv4State2& s, float2 w2) {
+  return fma2(make_float2(-s.n.x, -s.n.y), w2, s.base);
+}
+
+// Pair form of wkv4_token (same operations in the same order).
+__device__ __forceinline__ float2 wkv4_token2(Wkv4State2& s, float2 kk, float2 v, float2 u2, float2 w2) {
+  const float2 y0 = sub2(kk, s.base);
+  const float2 zo = fma2(s.n, w2, add2(y0, u2));
+  const float2 e = make_float2(ex2(fminf(zo.x, 64.f)), ex2(fminf(zo.y, 64.f)));
+  const float2 y = mul2(fma2(e, v, s.aa), rcp2(add2(s.bb, e)));
+  const float2 n1 = add2(s.n, splat2(1.f));
+  const float2 z1 = fma2(n1, w2, y0);
+  const float2 ea = make_float2(ex2(-fabsf(z1.x)), ex2(-fabsf(z1.y)));
+  const bool px = z1.x <= 0.f, py = z1.y <= 0.f;
+  const float2 f1 = make_float2(px ? 1.f : ea.x, py ? 1.f : ea.y);
+  const float2 f2 = make_float2(px ? ea.x : 1.f, py ? ea.y : 1.f);
+  s.aa = fma2(f1, s.aa, mul2(f2, v));
+  s.bb = fma2(f1, s.bb, f2);
+  s.base = make_float2(px ? s.base.x : kk.x, py ? s.base.y : kk.y);
+  s.n = make_float2(px ? n1.x : 0.f, py ? n1.y : 0.f);
+  return y;
+}
+
+// Pair form of wkv4_absorb. Returns z1, the exponent of the token against
+// the decayed past (2^{-|z1|} is the absorb factor; z1 <= 0 keeps the past's
+// maximum).
+__device__ __forceinline__ float2 wkv4_absorb2(Wkv4State2& s, float2 kk, float2 v, float2 w2) {
+  const float2 y0 = sub2(kk, s.base);
+  const float2 n1 = add2(s.n, splat2(1.f));
+  const float2 z1 = fma2(n1, w2, y0);
+  const float2 ea = make_float2(ex2(-fabsf(z1.x)), ex2(-fabsf(z1.y)));
+  const bool px = z1.x <= 0.f, py = z1.y <= 0.f;
+  const float2 f1 = make_float2(px ? 1.f : ea.x, py ? 1.f : ea.y);
+  const float2 f2 = make_float2(px ? ea.x : 1.f, py ? ea.y : 1.f);
+  s.aa = fma2(f1, s.aa, mul2(f2, v));
+  s.bb = fma2(f1, s.bb, f2);
+  s.base = make_float2(px ? s.base.x : kk.x, py ? s.base.y : kk.y);
+  s.n = make_float2(px ? n1.x : 0.f, py ? n1.y : 0.f);
+  return z1;
+}
+
 }  // namespace wkv

@@ -13,9 +13,12 @@ namespace wkv {
 
 __host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// Channels of one RWKV-4 warp (32 lanes x a channel pair each).
+#define WKV4_WARP_CH 64
+
 // Launch-shape constants of the RWKV-4 kernels (build-time tunables).
 #ifndef WKV4_TARGET_WARPS
-#define WKV4_TARGET_WARPS (148 * 8)  // warps wanted in flight: 8 per SM of a B200
+#define WKV4_TARGET_WARPS (148 * 4)  // warps wanted in flight: 4 per SM of a B200 (8 channels each)
 #endif
 #ifndef WKV4_FWD_MAX_SEGMENTS
 #define WKV4_FWD_MAX_SEGMENTS 8
@@ -36,14 +39,14 @@ __host__ __device__ __forceinline__ int64_t ceil_div(int64_t a, int64_t b) { ret
 #define WKV4_MIN_SEG_STEPS 64
 #endif
 inline int wkv4_segments_capped(int64_t B, int64_t T, int64_t C, int max_seg) {
-  const int64_t groups = B * ceil_div(C, 32);
+  const int64_t groups = B * ceil_div(C, WKV4_WARP_CH);
   const int64_t steps = ceil_div(T, WKV4_CKPT_LEN) * WKV4_CKPT_LEN;
   int nseg = 1;
   while (nseg < max_seg && groups * nseg < (int64_t)(WKV4_TARGET_WARPS) && steps >= 2 * WKV4_MIN_SEG_STEPS * nseg)
     nseg *= 2;
   return nseg;
 }
-// Warps (independent 32-channel lane groups) per CTA of a split launch: the
+// Warps (independent 64-channel lane groups) per CTA of a split launch: the
 // GPU keeps only ~140 clusters resident at once, so a split launch packs
 // several lane groups into each CTA to stay within one wave of clusters.
 #ifndef WKV4_MAX_CLUSTERS
@@ -51,7 +54,7 @@ inline int wkv4_segments_capped(int64_t B, int64_t T, int64_t C, int max_seg) {
 #endif
 inline int wkv4_warps_per_cta(int64_t B, int64_t C, int nseg) {
   if (nseg == 1) return 1;
-  const int64_t groups = B * ceil_div(C, 32);
+  const int64_t groups = B * ceil_div(C, WKV4_WARP_CH);
   int nw = 1;
   while (nw < 4 && ceil_div(groups, nw) > WKV4_MAX_CLUSTERS) nw *= 2;
   return nw;
