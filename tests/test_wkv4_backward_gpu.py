@@ -116,3 +116,14 @@ def test_special_cases(W, oracle):
     assert np.max(np.abs(gk)) < 1e-4 and np.max(np.abs(gu)) < 1e-3 and np.max(np.abs(gw)) < 1e-2
     np.testing.assert_allclose(gv.sum(axis=1), inp["gy32"].sum(axis=1), rtol=1e-4, atol=1e-3)
     assert_no_device_error()
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_extreme_bonus_and_decay_groups(W, oracle, dtype):
+    from test_wkv4_forward_gpu import extreme_channels
+    rec = dataclasses.replace(synth.WKV4_RECIPES["wkv4_fb_f32_169m"].with_shape(2, 300, 200), dtype=dtype)
+    inp = extreme_channels(synth.wkv4_inputs(rec, seed=5))
+    grads = run_bwd(W, inp)
+    ref = oracle.wkv4_backward(inp["w"], inp["u"], inp["k32"], inp["v32"], inp["gy32"])
+    check(grads, ref, dtype)
+    assert_no_device_error()

@@ -142,3 +142,32 @@ def test_checkpoint_state_matches_oracle(W, oracle):
         aa, bb, pp = ck[:, n, 0], ck[:, n, 1], ck[:, n, 2]
         np.testing.assert_allclose(np.log(bb) + (pp + ref_exp) * np.log(2.0), log_b, rtol=0, atol=1e-4)
         assert rel_err(aa / bb, ratio) < 1e-4
+
+
+def extreme_channels(inp):
+    """Give channel group 1 (channels 64..127) a bonus u far above the decay
+    and group 2 a decay w far above the bonus (|u - w| beyond 44 nats, where
+    the kernels switch that 64-channel group to the capped-weight output
+    evaluation); group 0 keeps the recipe's values (the fast evaluation)."""
+    inp = dict(inp)
+    inp["u"], inp["w"] = inp["u"].copy(), inp["w"].copy()
+    inp["u"][64 + 5] = 60.0
+    inp["u"][64 + 40] = 35.0
+    inp["w"][128 + 7] = 90.0
+    inp["u"][128 + 8] = -50.0
+    return inp
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("B,T", [(2, 150), (1, 700)])
+def test_extreme_bonus_and_decay_groups(W, oracle, dtype, B, T):
+    rec = synth.WKV4_RECIPES["wkv4_fwd_f32_small"].with_shape(B, T, 200)
+    rec = dataclasses.replace(rec, dtype=dtype, k_std=2.0)
+    inp = extreme_channels(synth.wkv4_inputs(rec, seed=11 + T))
+    y = host64(run_fwd(W, inp))
+    ref = oracle.wkv4_forward(inp["w"], inp["u"], inp["k32"], inp["v32"])
+    assert rel_err(y, ref) < TOL[dtype]
+    # the big-bonus channel follows v closely; the fast-decay channel too
+    assert rel_err(y[..., 64 + 5], ref[..., 64 + 5]) < TOL[dtype]
+    assert rel_err(y[..., 128 + 7], ref[..., 128 + 7]) < TOL[dtype]
+    assert_no_device_error()
