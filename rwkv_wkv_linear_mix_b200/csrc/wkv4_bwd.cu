@@ -64,12 +64,18 @@ struct BoolTag {
 // registers, or (bf16) in shared memory, which frees ~100 registers per
 // thread for the unpredicated reverse steps (float32 keeps them in registers:
 // its larger stages leave no room for the stash at 7 warps per SM).
+#ifndef WKV4_BWD_WHOLE_RECOMPUTE
+#define WKV4_BWD_WHOLE_RECOMPUTE 1
+#endif
+#ifndef WKV4_BWD_SMEM_STASH_F32
+#define WKV4_BWD_SMEM_STASH_F32 0
+#endif
 #ifndef WKV4_BWD_SMEM_STASH
 #define WKV4_BWD_SMEM_STASH 1
 #endif
 template <class E>
 constexpr bool bwd_smem_stash() {
-  return WKV4_BWD_SMEM_STASH && sizeof(E) == 2;
+  return WKV4_BWD_SMEM_STASH && (sizeof(E) == 2 || WKV4_BWD_SMEM_STASH_F32);
 }
 template <bool S>
 struct Wkv4Stash {
@@ -115,7 +121,7 @@ __device__ __forceinline__ void wkv4_bwd_interval(const E (*ks)[kBwdCh], const E
   float2 saa[kReg], sbb[kReg], sz[kReg];
 #pragma unroll
   for (int jj = 0; jj < kBwdL; ++jj) {
-    if (jj < n) {
+    if (WKV4_BWD_WHOLE_RECOMPUTE && WHOLE || jj < n) {
       const float2 aa = st.aa, bb = st.bb;
       const float2 z1 = wkv4_absorb2(st, wkv4_key2(ld_pair(&ks[jj][2 * lane]), ref), ld_pair(&vs[jj][2 * lane]), w2);
       if constexpr (S) {
@@ -222,7 +228,9 @@ __global__ void __launch_bounds__(32 * NW, NSEG == 1 ? 8 : 1) wkv4_bwd_kernel(co
   const int i_beg = wkv4_seg_begin(seg, NSEG, nck);
   const int i_end = wkv4_seg_begin(seg + 1, NSEG, nck);
   const int nloc = active ? i_end - i_beg : 0;  // intervals of this segment, walked last to first
-  const int total = kPasses * nloc;
+  // segment 0's own carry is read by no other segment: no phase 1 there
+  const bool own_pass = kPasses > 1 && seg > 0;
+  const int total = (own_pass ? 2 : 1) * nloc;
   auto interval = [&](int qq) { return i_end - 1 - (qq % nloc); };
 
   auto issue = [&](int qq) {
@@ -295,7 +303,7 @@ __global__ void __launch_bounds__(32 * NW, NSEG == 1 ? 8 : 1) wkv4_bwd_kernel(co
     // ---- phase 1: this segment's own carry, from an empty future ----
     float2 fprod = splat2(1.f);
     Wkv4State2 nxt = nloc > 0 ? load_ckpt(interval(0)) : Wkv4State2{splat2(0.f), splat2(0.f), splat2(0.f), splat2(0.f)};
-    for (; ok && qq < nloc; ++qq) {
+    for (; own_pass && ok && qq < nloc; ++qq) {
       const int i = interval(qq);
       const Wkv4State2 st = nxt;
       if (qq + 1 < nloc) nxt = load_ckpt(interval(qq + 1));
@@ -456,7 +464,7 @@ static wkv_status run_bwd_nw(const Wkv4BwdArgs& a, cudaStream_t stream, unsigned
 
 template <class E>
 static wkv_status run_bwd_nseg(const Wkv4BwdArgs& a, cudaStream_t stream, unsigned* err, const char** why) {
-  constexpr int kStages = sizeof(E) == 2 ? (bwd_smem_stash<E>() ? 3 : 4) : 2;
+  constexpr int kStages = sizeof(E) == 2 ? (bwd_smem_stash<E>() ? 3 : 4) : 2;  // f32: 2 either way
   switch (wkv4_bwd_segments(a.B, a.T, a.C)) {
 #if WKV4_MAX_SEGMENTS_ANY > 8
     case 16: return run_bwd_nw<E, kStages, 16>(a, stream, err, why);

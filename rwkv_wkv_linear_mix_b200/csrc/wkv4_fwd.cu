@@ -68,7 +68,9 @@ __global__ void __launch_bounds__(32 * NW) wkv4_fwd_kernel(const __grid_constant
   const int t_beg = wkv4_seg_begin(seg, NSEG, nck) * WKV4_CKPT_LEN;
   const int t_end = min(T, wkv4_seg_begin(seg + 1, NSEG, nck) * WKV4_CKPT_LEN);
   const int ntile = (active && t_end > t_beg) ? (t_end - t_beg + LT - 1) / LT : 0;
-  const int total = kPasses * ntile;  // tiles streamed through the ring
+  // the last segment's own state is read by no other segment: no phase 1 there
+  const bool own_pass = kPasses > 1 && seg < NSEG - 1;
+  const int total = (own_pass ? 2 : 1) * ntile;  // tiles streamed through the ring
 
   auto issue = [&](int q) {
     const int s = q % STAGES;
@@ -111,7 +113,7 @@ __global__ void __launch_bounds__(32 * NW) wkv4_fwd_kernel(const __grid_constant
   Wkv4State2 st = wkv4_empty_state2();
   if constexpr (NSEG > 1) {
     // ---- phase 1: this segment from the empty past ----
-    for (; ok && q < ntile; ++q) {
+    for (; own_pass && ok && q < ntile; ++q) {
       if (!acquire(q)) break;
       const int s = q % STAGES;
       const int n = min(LT, t_end - (t_beg + q * LT));
