@@ -64,6 +64,10 @@ struct BoolTag {
 // registers, or (bf16) in shared memory, which frees ~100 registers per
 // thread for the unpredicated reverse steps (float32 keeps them in registers:
 // its larger stages leave no room for the stash at 7 warps per SM).
+// Ring depth of the bf16 kernel next to the 16 KB stash (7 warps per SM).
+#ifndef WKV4_BWD_STAGES_STASH
+#define WKV4_BWD_STAGES_STASH 2
+#endif
 #ifndef WKV4_BWD_WHOLE_RECOMPUTE
 #define WKV4_BWD_WHOLE_RECOMPUTE 1
 #endif
@@ -80,7 +84,7 @@ constexpr bool bwd_smem_stash() {
 template <bool S>
 struct Wkv4Stash {
   float4 ab[kBwdL][32];  // (aa.x, aa.y, bb.x, bb.y) of each step, per lane
-  float2 z[kBwdL][32];
+  float4 zv[kBwdL][32];  // (z1.x, z1.y, v.x, v.y): v unpacked once
 };
 template <>
 struct Wkv4Stash<false> {};
@@ -103,6 +107,48 @@ struct Wkv4Carry2 {
 
 __device__ __forceinline__ float2 neg2(float2 a) { return make_float2(-a.x, -a.y); }
 
+// One reverse step of a lane's channel pair (token t, walking down), from
+// the forward quantities of the token: the state (aa, bb) before it, its
+// absorb exponent z (z1 of the forward), v and gy. FULL: also write gk, gv
+// at gkp, gvp and add the token's gw, gu terms (gwn holds -gw); otherwise
+// only fold the token into the carries and fprod.
+template <bool FULL, class E>
+__device__ __forceinline__ void wkv4_bwd_rstep(float2& A, float2& B, float2& Ap, float2& Bp, float2& fprod,
+                                               float2& gwn, float2& gu_acc, float2 vv, float2 g, float2 aa,
+                                               float2 bb, float2 z, float2 uw2, E* gkp, E* gvp) {
+  // output of the token, in units of the past's exponent P: weight
+  // e = 2^{u + k - P} = 2^{z1 + u - w} of the current token (capped as in
+  // the forward), D = 2^P (bb + e), y = (aa + e v) / (bb + e)
+  const float2 zo = add2(z, uw2);
+  const float2 e = make_float2(ex2(fminf(zo.x, 64.f)), ex2(fminf(zo.y, 64.f)));
+  const float2 rd = rcp2(add2(bb, e));
+  const float2 yv = mul2(fma2(e, vv, aa), rd);
+  // absorb pair of the token: P' = max(P - w, k)
+  const float2 ea = make_float2(ex2(-fabsf(z.x)), ex2(-fabsf(z.y)));
+  const bool kx = z.x <= 0.f, ky = z.y <= 0.f;
+  const float2 f1 = make_float2(kx ? 1.f : ea.x, ky ? 1.f : ea.y);
+  const float2 f2 = make_float2(kx ? ea.x : 1.f, ky ? ea.y : 1.f);
+  const float2 ag = mul2(g, rd);  // gy 2^P / D
+  if constexpr (FULL) {
+    const float2 rg = mul2(ag, e);  // gy rho, rho = e^{u+k} / D
+    // v - y = (bb v - aa) / (bb + e): no cancellation against v when the
+    // current token dominates (y within rounding of v)
+    const float2 vmy = mul2(fma2(bb, vv, neg2(aa)), rd);
+    const float2 gvv = fma2(f2, A, rg);
+    const float2 gkv = fma2(rg, vmy, mul2(f2, fma2(vv, A, neg2(B))));
+    gu_acc = fma2(rg, vmy, gu_acc);
+    gwn = fma2(f2, fma2(vv, Ap, neg2(Bp)), gwn);
+    st_pair(gkp, gkv);
+    st_pair(gvp, gvv);
+  }
+  if constexpr (!FULL) fprod = mul2(fprod, f1);
+  // carries for the token before
+  Ap = mul2(f1, add2(Ap, A));
+  Bp = mul2(f1, add2(Bp, B));
+  A = fma2(f1, A, ag);
+  B = fma2(f1, B, mul2(ag, yv));
+}
+
 // One checkpoint interval in reverse for a lane's channel pair. FULL: also
 // produce gk, gv, gw, gu; otherwise only fold the interval into the carry.
 // fprod (fold-only pass) accumulates the product of the f1 factors; gwn
@@ -123,10 +169,11 @@ __device__ __forceinline__ void wkv4_bwd_interval(const E (*ks)[kBwdCh], const E
   for (int jj = 0; jj < kBwdL; ++jj) {
     if (WKV4_BWD_WHOLE_RECOMPUTE && WHOLE || jj < n) {
       const float2 aa = st.aa, bb = st.bb;
-      const float2 z1 = wkv4_absorb2(st, wkv4_key2(ld_pair(&ks[jj][2 * lane]), ref), ld_pair(&vs[jj][2 * lane]), w2);
+      const float2 vj = ld_pair(&vs[jj][2 * lane]);
+      const float2 z1 = wkv4_absorb2(st, wkv4_key2(ld_pair(&ks[jj][2 * lane]), ref), vj, w2);
       if constexpr (S) {
         sx.ab[jj][lane] = make_float4(aa.x, aa.y, bb.x, bb.y);
-        sx.z[jj][lane] = z1;
+        sx.zv[jj][lane] = make_float4(z1.x, z1.y, vj.x, vj.y);
       } else {
         saa[jj] = aa;
         sbb[jj] = bb;
@@ -138,50 +185,23 @@ __device__ __forceinline__ void wkv4_bwd_interval(const E (*ks)[kBwdCh], const E
 #pragma unroll
   for (int jj = kBwdL - 1; jj >= 0; --jj) {
     if (WHOLE || jj < n) {
-      const float2 vv = ld_pair(&vs[jj][2 * lane]);
       const float2 g = ld_pair(&gs[jj][2 * lane]);
-      float2 aa, bb, z;
+      float2 aa, bb, z, vv;
       if constexpr (S) {
         const float4 ab = sx.ab[jj][lane];
+        const float4 zv = sx.zv[jj][lane];
         aa = make_float2(ab.x, ab.y);
         bb = make_float2(ab.z, ab.w);
-        z = sx.z[jj][lane];
+        z = make_float2(zv.x, zv.y);
+        vv = make_float2(zv.z, zv.w);
       } else {
         aa = saa[jj];
         bb = sbb[jj];
         z = sz[jj];
+        vv = ld_pair(&vs[jj][2 * lane]);
       }
-      // output of token jj, in units of the past's exponent P: weight
-      // e = 2^{u + k - P} = 2^{z1 + u - w} of the current token (capped as in
-      // the forward), D = 2^P (bb + e), y = (aa + e v) / (bb + e)
-      const float2 zo = add2(z, uw2);
-      const float2 e = make_float2(ex2(fminf(zo.x, 64.f)), ex2(fminf(zo.y, 64.f)));
-      const float2 rd = rcp2(add2(bb, e));
-      const float2 yv = mul2(fma2(e, vv, aa), rd);
-      // absorb pair of token jj: P' = max(P - w, k)
-      const float2 ea = make_float2(ex2(-fabsf(z.x)), ex2(-fabsf(z.y)));
-      const bool kx = z.x <= 0.f, ky = z.y <= 0.f;
-      const float2 f1 = make_float2(kx ? 1.f : ea.x, ky ? 1.f : ea.y);
-      const float2 f2 = make_float2(kx ? ea.x : 1.f, ky ? ea.y : 1.f);
-      const float2 ag = mul2(g, rd);  // gy 2^P / D
-      if constexpr (FULL) {
-        const float2 rg = mul2(ag, e);  // gy rho, rho = e^{u+k} / D
-        // v - y = (bb v - aa) / (bb + e): no cancellation against v when the
-        // current token dominates (y within rounding of v)
-        const float2 vmy = mul2(fma2(bb, vv, neg2(aa)), rd);
-        const float2 gvv = fma2(f2, A, rg);
-        const float2 gkv = fma2(rg, vmy, mul2(f2, fma2(vv, A, neg2(B))));
-        gu_acc = fma2(rg, vmy, gu_acc);
-        gwn = fma2(f2, fma2(vv, Ap, neg2(Bp)), gwn);
-        st_pair(gkl + (int64_t)jj * C, gkv);
-        st_pair(gvl + (int64_t)jj * C, gvv);
-      }
-      if constexpr (!FULL) fprod = mul2(fprod, f1);
-      // carries for token jj - 1
-      Ap = mul2(f1, add2(Ap, A));
-      Bp = mul2(f1, add2(Bp, B));
-      A = fma2(f1, A, ag);
-      B = fma2(f1, B, mul2(ag, yv));
+      wkv4_bwd_rstep<FULL>(A, B, Ap, Bp, fprod, gwn, gu_acc, vv, g, aa, bb, z, uw2, gkl + (int64_t)jj * C,
+                           gvl + (int64_t)jj * C);
     }
   }
   cr = {A, B, Ap, Bp};
@@ -464,7 +484,7 @@ static wkv_status run_bwd_nw(const Wkv4BwdArgs& a, cudaStream_t stream, unsigned
 
 template <class E>
 static wkv_status run_bwd_nseg(const Wkv4BwdArgs& a, cudaStream_t stream, unsigned* err, const char** why) {
-  constexpr int kStages = sizeof(E) == 2 ? (bwd_smem_stash<E>() ? 3 : 4) : 2;  // f32: 2 either way
+  constexpr int kStages = sizeof(E) == 2 ? (bwd_smem_stash<E>() ? WKV4_BWD_STAGES_STASH : 4) : 2;
   switch (wkv4_bwd_segments(a.B, a.T, a.C)) {
 #if WKV4_MAX_SEGMENTS_ANY > 8
     case 16: return run_bwd_nw<E, kStages, 16>(a, stream, err, why);
