@@ -231,6 +231,45 @@ wkv_status wkv6_forward(int64_t B, int64_t T, int64_t H, int64_t K, int dtype,
                         const float *init_state, const int32_t *state_map, int64_t n_state,
                         float *final_state, void *o, void *stream);
 
+/* Bytes of workspace wkv6_backward needs: 4 * (68*B*H*T + 128*B*H) for
+ * K = 64 (per token and head the row products x_t and two scalars, per head
+ * P_{T-1} and the gu partials); 0 for another K. */
+size_t wkv6_backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K);
+
+/*
+ * RWKV-6 head-state WKV backward: the gradients of
+ *   L = sum(dout * o) + sum(g_final * S_final)
+ * for wkv6_forward with the same arguments (RWKV6_OP on the rwkv-ops package
+ * page is a trained operator; its table lists the PyTorch CUDA version).
+ *   K, dtype, r, k, v, w, u, init_state, state_map, n_state
+ *                as wkv6_forward (K = 64, bf16 only).
+ *   dout         [B][T][H*K] bf16: dL/do.
+ *   g_final      NULL (zero) or [B][H][K][K] float32: dL/dS after the last token.
+ *   gr, gk, gv   [B][T][H*K] bf16, written.
+ *   glogw        [B][T][H*K] bf16, written: w * dL/dw, the gradient with
+ *                respect to log w (w = exp(-exp(d)) gives dL/dd = -exp(d) glogw).
+ *                It is formed without dividing by w, so it stays accurate
+ *                where w is tiny; dL/dw itself is glogw / w.
+ *   gu           [H*K] float32, written: summed over samples and tokens in a
+ *                fixed order (deterministic).
+ *   g_init       NULL or [B][H][K][K] float32, written: dL/dS_{-1} of each
+ *                sample (adding rows that share an init_state entry is the
+ *                caller's).
+ *   workspace    device memory of workspace_bytes >= wkv6_backward_workspace_bytes,
+ *                16-byte aligned; overwritten, nothing in it needs clearing.
+ * Every device pointer must be 16-byte aligned. Two kernels walk each head's
+ * sequence up and then down (256 threads per head), a third sums gu.
+ * Returns WKV_ERR_INVALID_ARG for a missing pointer or a short workspace,
+ * WKV_ERR_UNSUPPORTED for K != 64 or a dtype other than WKV_BF16.
+ */
+wkv_status wkv6_backward(int64_t B, int64_t T, int64_t H, int64_t K, int dtype,
+                         const void *r, const void *k, const void *v, const void *w,
+                         const float *u,
+                         const float *init_state, const int32_t *state_map, int64_t n_state,
+                         const void *dout, const float *g_final,
+                         void *gr, void *gk, void *gv, void *glogw, float *gu, float *g_init,
+                         void *workspace, size_t workspace_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -295,3 +295,53 @@ WKV_EXPORT wkv_status wkv6_forward(int64_t B, int64_t T, int64_t H, int64_t K, i
   wkv_status s = launch_wkv6_forward(a, static_cast<cudaStream_t>(stream), err, &why);
   return s == WKV_OK ? s : fail(s, why);
 }
+
+WKV_EXPORT size_t wkv6_backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K) {
+  if (B < 0 || T < 0 || H < 0 || K != 64) return 0;
+  return wkv6_bwd_workspace_bytes(B, T, H);
+}
+
+WKV_EXPORT wkv_status wkv6_backward(int64_t B, int64_t T, int64_t H, int64_t K, int dtype, const void* r,
+                                    const void* k, const void* v, const void* w, const float* u,
+                                    const float* init_state, const int32_t* state_map, int64_t n_state,
+                                    const void* dout, const float* g_final, void* gr, void* gk, void* gv,
+                                    void* glogw, float* gu, float* g_init, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  if (B < 0 || T < 0 || H < 0 || K < 0 || n_state < 0) return fail(WKV_ERR_INVALID_ARG, "negative size");
+  if (dtype != WKV_F32 && dtype != WKV_BF16) return fail(WKV_ERR_INVALID_ARG, "unknown dtype");
+  if (dtype != WKV_BF16) return fail(WKV_ERR_UNSUPPORTED, "wkv6_backward supports bf16 only");
+  if (K != 64) return fail(WKV_ERR_UNSUPPORTED, "wkv6_backward supports head size 64 only");
+  if (B == 0 || H == 0) return WKV_OK;
+  if (T > INT32_MAX || H > 65535 || B * H > INT32_MAX) return fail(WKV_ERR_UNSUPPORTED, "size out of range");
+  WKV_REQUIRE_PTR(u, "u");
+  WKV_REQUIRE_PTR(gu, "gu");
+  WKV_REQUIRE_PTR(workspace, "workspace");
+  WKV_OPTIONAL_PTR(init_state, "init_state");
+  WKV_OPTIONAL_PTR(state_map, "state_map");
+  WKV_OPTIONAL_PTR(g_final, "g_final");
+  WKV_OPTIONAL_PTR(g_init, "g_init");
+  if (init_state) {
+    if (n_state < 1) return fail(WKV_ERR_INVALID_ARG, "init_state given with n_state < 1");
+    if (!state_map && n_state != 1 && n_state != B)
+      return fail(WKV_ERR_INVALID_ARG, "without state_map, n_state must be 1 or B");
+  }
+  if (T > 0) {
+    WKV_REQUIRE_PTR(r, "r");
+    WKV_REQUIRE_PTR(k, "k");
+    WKV_REQUIRE_PTR(v, "v");
+    WKV_REQUIRE_PTR(w, "w");
+    WKV_REQUIRE_PTR(dout, "dout");
+    WKV_REQUIRE_PTR(gr, "gr");
+    WKV_REQUIRE_PTR(gk, "gk");
+    WKV_REQUIRE_PTR(gv, "gv");
+    WKV_REQUIRE_PTR(glogw, "glogw");
+  }
+  if (workspace_bytes < wkv6_bwd_workspace_bytes(B, T, H)) return fail(WKV_ERR_INVALID_ARG, "workspace too small");
+  unsigned* err = nullptr;
+  if (wkv_status s = device_error_ptr(&err)) return s;
+  const char* why = "";
+  Wkv6BwdArgs a{B, T, H, K, r, k, v, w, u, init_state, state_map, init_state ? n_state : 0, dout, g_final,
+                gr, gk, gv, glogw, gu, g_init, workspace};
+  wkv_status s = launch_wkv6_backward(a, static_cast<cudaStream_t>(stream), err, &why);
+  return s == WKV_OK ? s : fail(s, why);
+}

@@ -136,6 +136,28 @@ struct Wkv6FwdArgs {
   void* o;
 };
 
+struct Wkv6BwdArgs {
+  int64_t B, T, H, K;
+  const void* r;
+  const void* k;
+  const void* v;
+  const void* w;
+  const float* u;
+  const float* init_state;
+  const int32_t* state_map;
+  int64_t n_state;
+  const void* dout;
+  const float* g_final;
+  void* gr;
+  void* gk;
+  void* gv;
+  void* glogw;
+  float* gu;
+  float* g_init;
+  void* workspace;
+};
+size_t wkv6_bwd_workspace_bytes(int64_t B, int64_t T, int64_t H);
+
 // Record `why` as the calling thread's wkv_last_error() message.
 void set_last_error(const char* why);
 
@@ -146,5 +168,6 @@ wkv_status launch_wkv4_backward(const Wkv4BwdArgs& a, cudaStream_t stream, unsig
 wkv_status launch_wkv4_state_init(int64_t S, int64_t C, float* state, cudaStream_t stream, const char** why);
 wkv_status launch_wkv4_chunk_step(const Wkv4ChunkArgs& a, cudaStream_t stream, unsigned* err, const char** why);
 wkv_status launch_wkv6_forward(const Wkv6FwdArgs& a, cudaStream_t stream, unsigned* err, const char** why);
+wkv_status launch_wkv6_backward(const Wkv6BwdArgs& a, cudaStream_t stream, unsigned* err, const char** why);
 
 }  // namespace wkv

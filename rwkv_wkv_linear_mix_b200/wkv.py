@@ -38,6 +38,8 @@ SIGNATURES = {
     "wkv4_chunk_step": (_int, [_i64, _i64, _int, _vp, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp]),
     "wkv6_forward": (_int, [_i64, _i64, _i64, _i64, _int] + [_vp] * 7 + [_i64, _vp, _vp, _vp]),
     "wkv4_backward_noalloc": (_int, [_i64, _i64, _i64, _int] + [_vp] * 11),
+    "wkv6_backward_workspace_bytes": (_sz, [_i64, _i64, _i64, _i64]),
+    "wkv6_backward": (_int, [_i64, _i64, _i64, _i64, _int] + [_vp] * 7 + [_i64] + [_vp] * 9 + [_sz, _vp]),
 }
 
 
@@ -270,3 +272,53 @@ def wkv6_forward(r, k, v, w, u, init_state: Optional[torch.Tensor] = None,
                              _ptr(init_state), _ptr(state_map), n_state, _ptr(final_state), _ptr(o),
                              _stream(r)), "wkv6_forward")
     return o, final_state
+
+
+def wkv6_backward_workspace_bytes(B: int, T: int, H: int, K: int = 64) -> int:
+    return int(_lib.wkv6_backward_workspace_bytes(B, T, H, K))
+
+
+def wkv6_backward(r, k, v, w, u, dout, init_state: Optional[torch.Tensor] = None,
+                  state_map: Optional[torch.Tensor] = None, g_final: Optional[torch.Tensor] = None, *,
+                  head_size: int = 64, want_g_init: bool = True, workspace: Optional[torch.Tensor] = None,
+                  gr=None, gk=None, gv=None, glogw=None, gu=None, g_init=None):
+    """RWKV-6 head-state backward of wkv6_forward(r, k, v, w, u, init_state,
+    state_map). dout: [B, T, H*K] bf16; g_final: [B, H, K, K] float32 or None.
+    Returns (gr, gk, gv, glogw, gu, g_init or None); glogw = w * dL/dw."""
+    B, T, HK = r.shape
+    K = head_size
+    if HK % K:
+        raise ValueError("hidden size must be a multiple of head_size")
+    H = HK // K
+    dev = r.device
+    for name, t in (("r", r), ("k", k), ("v", v), ("w", w), ("dout", dout)):
+        _want(t, name, dtype=r.dtype, shape=r.shape, device=dev)
+    _want(u, "u", dtype=torch.float32, device=dev)
+    if u.numel() != HK:
+        raise ValueError("u must hold H*K values")
+    n_state = 0
+    if init_state is not None:
+        _want(init_state, "init_state", dtype=torch.float32, device=dev)
+        n_state = init_state.shape[0]
+        if tuple(init_state.shape[1:]) != (H, K, K):
+            raise ValueError("init_state must be [n_state, H, K, K]")
+    if state_map is not None:
+        _want(state_map, "state_map", dtype=torch.int32, shape=(B,), device=dev)
+    if g_final is not None:
+        _want(g_final, "g_final", dtype=torch.float32, shape=(B, H, K, K), device=dev)
+    gr = torch.empty_like(r) if gr is None else gr
+    gk = torch.empty_like(r) if gk is None else gk
+    gv = torch.empty_like(r) if gv is None else gv
+    glogw = torch.empty_like(r) if glogw is None else glogw
+    gu = torch.empty(HK, dtype=torch.float32, device=dev) if gu is None else gu
+    if want_g_init and g_init is None:
+        g_init = torch.empty((B, H, K, K), dtype=torch.float32, device=dev)
+    need = wkv6_backward_workspace_bytes(B, T, H, K)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _check(_lib.wkv6_backward(B, T, H, K, _dtype_code(r), _ptr(r), _ptr(k), _ptr(v), _ptr(w), _ptr(u),
+                              _ptr(init_state), _ptr(state_map), n_state, _ptr(dout), _ptr(g_final),
+                              _ptr(gr), _ptr(gk), _ptr(gv), _ptr(glogw), _ptr(gu), _ptr(g_init),
+                              _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(r)),
+           "wkv6_backward")
+    return gr, gk, gv, glogw, gu, g_init

@@ -35,7 +35,7 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("wkv4_forward", "wkv4_backward", "wkv4_chunk_step", "wkv4_state_init", "wkv6_forward",
               "wkv4_backward_workspace_bytes", "wkv4_ckpt_floats", "wkv_status_string", "wkv_last_error",
-              "wkv_device_error", "wkv_abi_version"):
+              "wkv_device_error", "wkv_abi_version", "wkv6_backward", "wkv6_backward_workspace_bytes"):
         assert n in names
 
 
@@ -113,6 +113,19 @@ def test_chunk_and_wkv6_argument_errors(W):
     assert wk6(B=3, init=FAKE, ns=2) == W.WKV_ERR_INVALID_ARG     # n_state neither 1 nor B
     assert wk6(B=3, init=FAKE, ns=0) == W.WKV_ERR_INVALID_ARG
     assert wk6(B=0) == W.WKV_OK
+    need = L.wkv6_backward_workspace_bytes(2, 40, 3, 64)
+    assert need == 4 * (68 * 2 * 3 * 40 + 128 * 2 * 3)
+    assert L.wkv6_backward_workspace_bytes(2, 40, 3, 32) == 0
+    wb6 = lambda B=2, T=40, H=3, K=64, dt=1, init=None, ns=0, ws=need, wsp=FAKE: L.wkv6_backward(
+        B, T, H, K, dt, FAKE, FAKE, FAKE, FAKE, FAKE, init, None, ns, FAKE, None,
+        FAKE, FAKE, FAKE, FAKE, FAKE, None, wsp, ws, None)
+    assert wb6(K=32) == W.WKV_ERR_UNSUPPORTED
+    assert wb6(dt=0) == W.WKV_ERR_UNSUPPORTED
+    assert wb6(T=-1) == W.WKV_ERR_INVALID_ARG
+    assert wb6(ws=need - 1) == W.WKV_ERR_INVALID_ARG
+    assert wb6(wsp=None) == W.WKV_ERR_INVALID_ARG
+    assert wb6(init=FAKE, ns=3) == W.WKV_ERR_INVALID_ARG      # n_state neither 1 nor B
+    assert wb6(H=0) == W.WKV_OK
 
 
 def test_binding_refuses_cpu_tensors(W):
