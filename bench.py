@@ -64,7 +64,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the secondary workloads (larger shapes, chunk step, RWKV-6)")
-    ap.add_argument("--kernel", choices=["wkv4_fwd", "wkv4_bwd", "wkv6_fwd", "wkv4_chunk"],
+    ap.add_argument("--kernel", choices=["wkv4_fwd", "wkv4_bwd", "wkv6_fwd", "wkv6_bwd", "wkv4_chunk"],
                     help="profiling mode: run only this kernel --steps times on --workload (no JSON line)")
     ap.add_argument("--workload", default=None,
                     help="with --kernel: a recipe name of synth (RWKV-4 or RWKV-6), optionally resized "
@@ -374,9 +374,22 @@ def secondary(dev, flush, peak):
     f6()
     t6 = _events_ms(f6, 3, flush, stream)
     n6 = B * T * HK
+    # RWKV-6 backward on the same inputs (dout ~ N(0, 1)); bytes: r, k, v, w, dout in and
+    # gr, gk, gv, glogw out, bf16 (9 x 2 B per token-channel)
+    do6 = torch.randn(B, T, HK, device=dev, generator=g).to(torch.bfloat16)
+    ws6 = torch.empty(wkv.wkv6_backward_workspace_bytes(B, T, H), dtype=torch.uint8, device=dev)
+    go6 = [torch.empty_like(r6) for _ in range(4)]
+    gu6 = torch.empty(HK, device=dev)
+    b6 = lambda: wkv.wkv6_backward(r6, k6, v6, w6, u6, do6, want_g_init=False, workspace=ws6, gr=go6[0],
+                                   gk=go6[1], gv=go6[2], glogw=go6[3], gu=gu6)
+    b6()
+    tb6 = _events_ms(b6, 3, flush, stream)
     res["wkv6_fwd_bf16_c2048"] = {"B": B, "T": T, "H": H, "K": 64, "fwd_ms": t6,
                                   "GBps": 10 * n6 / (t6 * 1e-3) / 1e9, "frac": 10 * n6 / (t6 * 1e-3) / 1e9 / peak,
-                                  "Gtokch_per_s": n6 / (t6 * 1e-3) / 1e9}
+                                  "Gtokch_per_s": n6 / (t6 * 1e-3) / 1e9,
+                                  "bwd_ms": tb6, "bwd_GBps": 18 * n6 / (tb6 * 1e-3) / 1e9,
+                                  "bwd_frac": 18 * n6 / (tb6 * 1e-3) / 1e9 / peak}
+    del do6, ws6, go6
     assert wkv.device_error(reset=True) == 0, "a kernel recorded a device-side error"
     return res
 
@@ -590,7 +603,7 @@ def run_kernel_only(args):
             wkv.wkv4_state_init(S, C, dev, state=state)
             for kc, vc, cu in calls:
                 wkv.wkv4_chunk_step(w, u, kc, vc, cu, state)
-    elif args.kernel == "wkv6_fwd":
+    elif args.kernel in ("wkv6_fwd", "wkv6_bwd"):
         rec = synth.WKV6_RECIPES[name or "wkv6_fwd_bf16_c2048"]
         if resize:
             rec = rec.with_shape(*[int(x) for x in resize.split(",")])
@@ -601,8 +614,14 @@ def run_kernel_only(args):
         r6, k6, v6 = (torch.randn(B, T, HK, device=dev, generator=g).to(torch.bfloat16) for _ in range(3))
         u6 = torch.rand(HK, device=dev, generator=g) * (rec.u_hi - rec.u_lo) + rec.u_lo
         o6 = torch.empty_like(r6)
-        for _ in range(args.steps):
-            wkv.wkv6_forward(r6, k6, v6, w6, u6, o=o6)
+        if args.kernel == "wkv6_fwd":
+            for _ in range(args.steps):
+                wkv.wkv6_forward(r6, k6, v6, w6, u6, o=o6)
+        else:
+            do6 = torch.randn(B, T, HK, device=dev, generator=g).to(torch.bfloat16)
+            ws6 = torch.empty(wkv.wkv6_backward_workspace_bytes(B, T, rec.H), dtype=torch.uint8, device=dev)
+            for _ in range(args.steps):
+                wkv.wkv6_backward(r6, k6, v6, w6, u6, do6, want_g_init=False, workspace=ws6)
     else:
         rec = synth.WKV4_RECIPES[name or WORKLOAD]
         if resize:

@@ -30,11 +30,13 @@
 //                    by columns (k G becomes a row product as well, so no
 //                    64-way reduction across threads); writes gk, gv, glogw
 //                    and per-(b, h) gu partials.
-// Inputs arrive per 32-token chunk by TMA (one stage) and are widened to fp32
-// in shared memory; the stage is free once widened, so the next chunk's load
-// overlaps this chunk's steps. Outputs leave through shared-memory tiles as
-// coalesced 16-byte stores. The 16-wide row work runs on packed fp32 pairs.
-// gu is summed over samples by a fixed-order reduction.
+// Inputs arrive per 32-token chunk by TMA into two stages (the next chunk
+// loads while this one runs). Each step reads its 16-wide slices as bf16
+// (32 bytes per vector: the 64 threads that share a slice make shared-memory
+// bandwidth, not arithmetic, the limit) one step ahead of use, and widens
+// them in registers. Outputs leave through shared-memory tiles as coalesced
+// 16-byte stores. The 16-wide row work runs on packed fp32 pairs. gu is
+// summed over samples by a fixed-order reduction.
 #include <string.h>
 
 #include "wkv_device.cuh"
@@ -49,37 +51,42 @@ constexpr int kIn6b = 5;       // r, k, v, w, do
 enum { kR = 0, kKk = 1, kV = 2, kW = 3, kDo = 4 };
 
 struct alignas(128) Wkv6Bwd1Smem {
-  __nv_bfloat16 in[kIn6b][kL6b][kK6b];  // TMA stage
-  float f[kIn6b][kL6b][kK6b];           // widened copies
-  float cv[kL6b][4];                    // per token: c_t, v_t . do_t
-  float xo[kL6b][kK6b];                 // x_t rows for the workspace
-  __nv_bfloat16 gro[kL6b][kK6b];        // gr tile
-  uint64_t full;
+  __nv_bfloat16 in[2][kIn6b][kL6b][kK6b];  // two TMA stages
+  float cv[2][kL6b][4];                    // per stage and token: c_t, v_t . do_t
+  float xo[kL6b][kK6b];                    // x_t rows for the workspace
+  __nv_bfloat16 gro[kL6b][kK6b];           // gr tile
+  uint64_t full[2];
+};
+
+struct alignas(128) Wkv6Bwd2Stage {
+  __nv_bfloat16 in[kIn6b][kL6b][kK6b];
+  float x[kL6b][kK6b];   // x_t rows
+  float cv[kL6b][4];     // (c_t, v_t . do_t, -, -)
 };
 
 struct alignas(128) Wkv6Bwd2Smem {
-  __nv_bfloat16 in[kIn6b][kL6b][kK6b];  // TMA stage
-  float xin[kL6b][kK6b];                // TMA stage: x_t rows
-  float cvin[kL6b][4];                  // TMA stage: (c_t, v_t . do_t, -, -)
-  float f[kIn6b][kL6b][kK6b];
-  float xf[kL6b][kK6b];
-  float cvf[kL6b][4];
+  Wkv6Bwd2Stage st[2];                  // two TMA stages
   __nv_bfloat16 out[3][kL6b][kK6b];     // gk, gv, glogw tiles
-  uint64_t full;
+  uint64_t full[2];
 };
 
-// Widen the bf16 stage into fp32 (all threads; 8 values per 16-byte piece).
-__device__ __forceinline__ void wkv6_widen(const __nv_bfloat16* src, float* dst, int tid) {
-  constexpr int kPieces = kIn6b * kL6b * kK6b / 8;
-  for (int g = tid; g < kPieces; g += kT6b) {
-    const uint4 raw = reinterpret_cast<const uint4*>(src)[g];
-    float4* d = reinterpret_cast<float4*>(dst) + 2 * g;
-    d[0] = make_float4(bf16lo(raw.x), bf16hi(raw.x), bf16lo(raw.y), bf16hi(raw.y));
-    d[1] = make_float4(bf16lo(raw.z), bf16hi(raw.z), bf16lo(raw.w), bf16hi(raw.w));
-  }
+// 16 consecutive bf16 of shared memory (two 16-byte loads), and their
+// widening to 8 fp32 pairs (element 2m in the low half of word m).
+struct Bf16x16 {
+  uint4 a, b;
+};
+__device__ __forceinline__ Bf16x16 ld16b(const __nv_bfloat16* p) {
+  const uint4* p4 = reinterpret_cast<const uint4*>(p);
+  return {p4[0], p4[1]};
 }
+__device__ __forceinline__ void widen16(const Bf16x16& x, float2 (&y)[8]) {
+  const uint32_t wds[8] = {x.a.x, x.a.y, x.a.z, x.a.w, x.b.x, x.b.y, x.b.z, x.b.w};
+#pragma unroll
+  for (int m = 0; m < 8; ++m) y[m] = make_float2(bf16lo(wds[m]), bf16hi(wds[m]));
+}
+__device__ __forceinline__ float bf(const __nv_bfloat16& x) { return __bfloat162float(x); }
 
-// 16 consecutive fp32 of shared memory as 8 pairs.
+// 16 consecutive fp32 of global memory as 8 pairs.
 __device__ __forceinline__ void ld16(const float* p, float2 (&x)[8]) {
   const float4* p4 = reinterpret_cast<const float4*>(p);
 #pragma unroll
@@ -98,9 +105,13 @@ __device__ __forceinline__ float row_sum4(float x) {
 }
 
 __device__ __forceinline__ float dot16(const float2 (&a)[8], const float2 (&b)[8]) {
-  float2 s = make_float2(0.f, 0.f);
+  float2 s0 = make_float2(0.f, 0.f), s1 = s0;
 #pragma unroll
-  for (int m = 0; m < 8; ++m) s = fma2(a[m], b[m], s);
+  for (int m = 0; m < 8; m += 2) {
+    s0 = fma2(a[m], b[m], s0);
+    s1 = fma2(a[m + 1], b[m + 1], s1);
+  }
+  const float2 s = add2(s0, s1);
   return __fadd_rn(s.x, s.y);
 }
 
@@ -131,16 +142,17 @@ __global__ void __launch_bounds__(kT6b, 2) wkv6_bwd_pass1_kernel(
   constexpr uint32_t kStageBytes = kIn6b * kL6b * kK6b * sizeof(__nv_bfloat16);
   const CUtensorMap* maps[kIn6b] = {&tr, &tk, &tv, &tw, &tdo};
   auto issue = [&](int ch) {
-    mbar_arrive_expect_tx(&sm.full, kStageBytes);
-    for (int m = 0; m < kIn6b; ++m) tma_load_3d(&sm.in[m][0][0], maps[m], &sm.full, h * kK6b, ch * kL6b, b);
+    const int s = ch & 1;
+    mbar_arrive_expect_tx(&sm.full[s], kStageBytes);
+    for (int m = 0; m < kIn6b; ++m) tma_load_3d(&sm.in[s][m][0][0], maps[m], &sm.full[s], h * kK6b, ch * kL6b, b);
   };
   if (tid == 0) {
-    mbar_init(&sm.full, 1);
+    mbar_init(&sm.full[0], 1);
+    mbar_init(&sm.full[1], 1);
     mbar_init_fence();
-    if (nchunk > 0) {
+    if (nchunk > 0)
       for (int m = 0; m < kIn6b; ++m) tma_prefetch_desc(maps[m]);
-      issue(0);
-    }
+    for (int ch = 0; ch < 2 && ch < nchunk; ++ch) issue(ch);
   }
   // S_{-1}: init_state[state_map[b]] (or the n_state rule), else zero
   float2 S[8];
@@ -160,15 +172,14 @@ __global__ void __launch_bounds__(kT6b, 2) wkv6_bwd_pass1_kernel(
   bool ok = true;
   int ch = 0;
   for (; ch < nchunk; ++ch) {
+    const int s = ch & 1;
     const int t0 = ch * kL6b, n = min(kL6b, T - t0);
-    const bool got = mbar_wait_bounded(&sm.full, ch & 1, err);
+    const bool got = mbar_wait_bounded(&sm.full[s], (ch >> 1) & 1, err);
     if (!__syncthreads_and(got)) {
       ok = false;
       break;
     }
-    wkv6_widen(&sm.in[0][0][0], &sm.f[0][0][0], tid);
-    __syncthreads();
-    if (tid == 0 && ch + 1 < nchunk) issue(ch + 1);  // every read of the stage is done
+    const __nv_bfloat16(*in)[kL6b][kK6b] = sm.in[s];
     {
       // per token: c_t = r . (u o k) and v . do, 8 threads per token
       const int jt = tid >> 3, part = tid & 7;
@@ -176,28 +187,34 @@ __global__ void __launch_bounds__(kT6b, 2) wkv6_bwd_pass1_kernel(
 #pragma unroll
       for (int m = 0; m < 8; ++m) {
         const int e = part * 8 + m;
-        c = __fmaf_rn(sm.f[kR][jt][e] * u[h * kK6b + e], sm.f[kKk][jt][e], c);
-        vd = __fmaf_rn(sm.f[kV][jt][e], sm.f[kDo][jt][e], vd);
+        c = __fmaf_rn(bf(in[kR][jt][e]) * u[h * kK6b + e], bf(in[kKk][jt][e]), c);
+        vd = __fmaf_rn(bf(in[kV][jt][e]), bf(in[kDo][jt][e]), vd);
       }
 #pragma unroll
       for (int o = 1; o < 8; o <<= 1) {
         c += __shfl_xor_sync(0xffffffffu, c, o);
         vd += __shfl_xor_sync(0xffffffffu, vd, o);
       }
-      if (part == 0) {
-        sm.cv[jt][0] = c;
-        sm.cv[jt][1] = vd;
-        sm.cv[jt][2] = 0.f;
-        sm.cv[jt][3] = 0.f;
-      }
+      if (part == 0) reinterpret_cast<float4*>(&sm.cv[s][jt][0])[0] = make_float4(c, vd, 0.f, 0.f);
     }
     __syncthreads();
+    // the step's vectors are fetched one step ahead
+    Bf16x16 vn = ld16b(&in[kV][0][16 * q]), dn = ld16b(&in[kDo][0][16 * q]);
+    float wn = bf(in[kW][0][i]), kn = bf(in[kKk][0][i]), rn = bf(in[kR][0][i]), vdn = sm.cv[s][0][1];
     for (int jt = 0; jt < n; ++jt) {
+      const Bf16x16 vc = vn, dc = dn;
+      const float wi = wn, ki = kn, ri = rn, vdo = vdn;
+      if (jt + 1 < n) {
+        vn = ld16b(&in[kV][jt + 1][16 * q]);
+        dn = ld16b(&in[kDo][jt + 1][16 * q]);
+        wn = bf(in[kW][jt + 1][i]);
+        kn = bf(in[kKk][jt + 1][i]);
+        rn = bf(in[kR][jt + 1][i]);
+        vdn = sm.cv[s][jt + 1][1];
+      }
       float2 vv[8], dd[8];
-      ld16(&sm.f[kV][jt][16 * q], vv);
-      ld16(&sm.f[kDo][jt][16 * q], dd);
-      const float wi = sm.f[kW][jt][i], ki = sm.f[kKk][jt][i], ri = sm.f[kR][jt][i];
-      const float vdo = sm.cv[jt][1];
+      widen16(vc, vv);
+      widen16(dc, dd);
       const float acc = row_sum4(dot16(S, dd));  // (S_{t-1} do_t)[i]
       if (q == 0) {
         sm.gro[jt][i] = __float2bfloat16_rn(__fmaf_rn(ui * ki, vdo, acc));
@@ -208,6 +225,7 @@ __global__ void __launch_bounds__(kT6b, 2) wkv6_bwd_pass1_kernel(
       for (int m = 0; m < 8; ++m) S[m] = fma2(S[m], w2, mul2(k2, vv[m]));
     }
     __syncthreads();
+    if (tid == 0 && ch + 2 < nchunk) issue(ch + 2);  // every read of stage s is done
     wkv6_store_tile(sm.gro, gr, b, T, HK, h, t0, n, tid);
     float* xrow = xws + ((int64_t)bh * T + t0) * kK6b;
     for (int g = tid; g < kL6b * kK6b / 4; g += kT6b) {
@@ -215,11 +233,12 @@ __global__ void __launch_bounds__(kT6b, 2) wkv6_bwd_pass1_kernel(
       if (row < n) reinterpret_cast<float4*>(xrow)[g] = reinterpret_cast<const float4*>(&sm.xo[0][0])[g];
     }
     if (tid < n) reinterpret_cast<float4*>(cvws + ((int64_t)bh * T + t0) * 4)[tid] =
-        reinterpret_cast<const float4*>(&sm.cv[0][0])[tid];
+        reinterpret_cast<const float4*>(&sm.cv[s][0][0])[tid];
   }
   if (!ok) {
-    // a wait gave up: let the copy in flight land before the CTA exits
-    if (tid == 0 && ch < nchunk) mbar_wait_bounded(&sm.full, ch & 1, err);
+    // a wait gave up: let the copies in flight land before the CTA exits
+    if (tid == 0)
+      for (int x = ch; x < nchunk && x < ch + 2; ++x) mbar_wait_bounded(&sm.full[x & 1], (x >> 1) & 1, err);
     return;
   }
   // P_{T-1}[i] = sum_j g_final[i][j] S_{T-1}[i][j]
@@ -251,21 +270,23 @@ __global__ void __launch_bounds__(kT6b, 2) wkv6_bwd_pass2_kernel(
       kIn6b * kL6b * kK6b * sizeof(__nv_bfloat16) + kL6b * kK6b * sizeof(float) + kL6b * 4 * sizeof(float);
   const CUtensorMap* maps[kIn6b] = {&tr, &tk, &tv, &tw, &tdo};
   auto issue = [&](int ch) {  // ch counts chunks from the end
+    const int s = ch & 1;
     const int t0 = (nchunk - 1 - ch) * kL6b;
-    mbar_arrive_expect_tx(&sm.full, kStageBytes);
-    for (int m = 0; m < kIn6b; ++m) tma_load_3d(&sm.in[m][0][0], maps[m], &sm.full, h * kK6b, t0, b);
-    tma_load_3d(&sm.xin[0][0], &tx, &sm.full, 0, t0, bh);
-    tma_load_3d(&sm.cvin[0][0], &tcv, &sm.full, 0, t0, bh);
+    mbar_arrive_expect_tx(&sm.full[s], kStageBytes);
+    for (int m = 0; m < kIn6b; ++m) tma_load_3d(&sm.st[s].in[m][0][0], maps[m], &sm.full[s], h * kK6b, t0, b);
+    tma_load_3d(&sm.st[s].x[0][0], &tx, &sm.full[s], 0, t0, bh);
+    tma_load_3d(&sm.st[s].cv[0][0], &tcv, &sm.full[s], 0, t0, bh);
   };
   if (tid == 0) {
-    mbar_init(&sm.full, 1);
+    mbar_init(&sm.full[0], 1);
+    mbar_init(&sm.full[1], 1);
     mbar_init_fence();
     if (nchunk > 0) {
       for (int m = 0; m < kIn6b; ++m) tma_prefetch_desc(maps[m]);
       tma_prefetch_desc(&tx);
       tma_prefetch_desc(&tcv);
-      issue(0);
     }
+    for (int ch = 0; ch < 2 && ch < nchunk; ++ch) issue(ch);
   }
   // G_{T-1} = g_final, by rows (G[i][16q ..]) and by columns (G[16q ..][i])
   float2 G[8], Gc[8];
@@ -286,38 +307,55 @@ __global__ void __launch_bounds__(kT6b, 2) wkv6_bwd_pass2_kernel(
   bool ok = true;
   int ch = 0;
   for (; ch < nchunk; ++ch) {
+    const int s = ch & 1;
     const int t0 = (nchunk - 1 - ch) * kL6b, n = min(kL6b, T - t0);
-    const bool got = mbar_wait_bounded(&sm.full, ch & 1, err);
+    const bool got = mbar_wait_bounded(&sm.full[s], (ch >> 1) & 1, err);
     if (!__syncthreads_and(got)) {
       ok = false;
       break;
     }
-    wkv6_widen(&sm.in[0][0][0], &sm.f[0][0][0], tid);
-    for (int g = tid; g < kL6b * kK6b / 4; g += kT6b)
-      reinterpret_cast<float4*>(&sm.xf[0][0])[g] = reinterpret_cast<const float4*>(&sm.xin[0][0])[g];
-    if (tid < kL6b) reinterpret_cast<float4*>(&sm.cvf[0][0])[tid] = reinterpret_cast<const float4*>(&sm.cvin[0][0])[tid];
-    __syncthreads();
-    if (tid == 0 && ch + 1 < nchunk) issue(ch + 1);
+    const Wkv6Bwd2Stage& st = sm.st[s];
+    struct Tok {
+      Bf16x16 v, d, r, k, w;
+      float wi, ri, ki, dj, c, vdo, xi;
+    };
+    auto fetch = [&](int jt) {
+      Tok x;
+      x.v = ld16b(&st.in[kV][jt][16 * q]);
+      x.d = ld16b(&st.in[kDo][jt][16 * q]);
+      x.r = ld16b(&st.in[kR][jt][16 * q]);
+      x.k = ld16b(&st.in[kKk][jt][16 * q]);
+      x.w = ld16b(&st.in[kW][jt][16 * q]);
+      x.wi = bf(st.in[kW][jt][i]);
+      x.ri = bf(st.in[kR][jt][i]);
+      x.ki = bf(st.in[kKk][jt][i]);
+      x.dj = bf(st.in[kDo][jt][i]);
+      x.c = st.cv[jt][0];
+      x.vdo = st.cv[jt][1];
+      x.xi = st.x[jt][i];
+      return x;
+    };
+    Tok nx = fetch(n - 1);
     for (int jt = n - 1; jt >= 0; --jt) {
+      const Tok cu = nx;
+      if (jt > 0) nx = fetch(jt - 1);
       float2 vv[8], dd[8], rr[8], kk[8], ww[8];
-      ld16(&sm.f[kV][jt][16 * q], vv);
-      ld16(&sm.f[kDo][jt][16 * q], dd);
-      ld16(&sm.f[kR][jt][16 * q], rr);
-      ld16(&sm.f[kKk][jt][16 * q], kk);
-      ld16(&sm.f[kW][jt][16 * q], ww);
-      const float wi = sm.f[kW][jt][i], ri = sm.f[kR][jt][i], ki = sm.f[kKk][jt][i], dj = sm.f[kDo][jt][i];
-      const float c = sm.cvf[jt][0], vdo = sm.cvf[jt][1], xi = sm.xf[jt][i];
+      widen16(cu.v, vv);
+      widen16(cu.d, dd);
+      widen16(cu.r, rr);
+      widen16(cu.k, kk);
+      widen16(cu.w, ww);
       const float gki = row_sum4(dot16(G, vv));   // (G_t v_t)[i]
       const float gvj = row_sum4(dot16(kk, Gc));  // (k_t G_t)[i]
-      const float gl = __fsub_rn(P, __fmul_rn(ki, gki));  // w_t gw_t
-      P = __fadd_rn(gl, xi);                                 // P_{t-1}
+      const float gl = __fsub_rn(P, __fmul_rn(cu.ki, gki));  // w_t gw_t
+      P = __fadd_rn(gl, cu.xi);                              // P_{t-1}
       if (q == 0) {
-        sm.out[0][jt][i] = __float2bfloat16_rn(__fmaf_rn(ui * ri, vdo, gki));
-        sm.out[1][jt][i] = __float2bfloat16_rn(__fmaf_rn(c, dj, gvj));
+        sm.out[0][jt][i] = __float2bfloat16_rn(__fmaf_rn(ui * cu.ri, cu.vdo, gki));
+        sm.out[1][jt][i] = __float2bfloat16_rn(__fmaf_rn(cu.c, cu.dj, gvj));
         sm.out[2][jt][i] = __float2bfloat16_rn(gl);
       }
-      gu_i = __fmaf_rn(ri * ki, vdo, gu_i);
-      const float2 w2 = make_float2(wi, wi), r2 = make_float2(ri, ri), d2 = make_float2(dj, dj);
+      gu_i = __fmaf_rn(cu.ri * cu.ki, cu.vdo, gu_i);
+      const float2 w2 = make_float2(cu.wi, cu.wi), r2 = make_float2(cu.ri, cu.ri), d2 = make_float2(cu.dj, cu.dj);
 #pragma unroll
       for (int m = 0; m < 8; ++m) {
         G[m] = fma2(G[m], w2, mul2(r2, dd[m]));
@@ -325,12 +363,14 @@ __global__ void __launch_bounds__(kT6b, 2) wkv6_bwd_pass2_kernel(
       }
     }
     __syncthreads();
+    if (tid == 0 && ch + 2 < nchunk) issue(ch + 2);  // every read of stage s is done
     wkv6_store_tile(sm.out[0], gk, b, T, HK, h, t0, n, tid);
     wkv6_store_tile(sm.out[1], gv, b, T, HK, h, t0, n, tid);
     wkv6_store_tile(sm.out[2], glogw, b, T, HK, h, t0, n, tid);
   }
   if (!ok) {
-    if (tid == 0 && ch < nchunk) mbar_wait_bounded(&sm.full, ch & 1, err);
+    if (tid == 0)
+      for (int x = ch; x < nchunk && x < ch + 2; ++x) mbar_wait_bounded(&sm.full[x & 1], (x >> 1) & 1, err);
     return;
   }
   if (g_init) {
