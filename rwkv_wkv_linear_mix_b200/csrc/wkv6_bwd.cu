@@ -21,22 +21,23 @@
 // consumes: dL/dd = -exp(d) glogw); it stays accurate where w_t is tiny,
 // where gw itself would be a difference of large terms divided by w_t.
 //
-// Two passes, one CTA of 256 threads per (b, h); thread (i = tid / 4,
-// q = tid % 4) holds row i, columns 16q .. 16q + 15:
+// Two passes, one CTA of 128 threads per (b, h); thread (p = tid / 4,
+// q = tid % 4) holds rows 2p and 2p + 1, columns 16q .. 16q + 15 (each slice
+// of a token's vectors it reads serves two rows):
 //   pass 1 (t up):   S; writes gr and, per token, x_t = r_t o (S_{t-1} do_t)
 //                    and (c_t = r_t . (u o k_t), v_t . do_t) to the workspace;
 //                    at the end P_{T-1} = sum_j g_final S_{T-1}.
 //   pass 2 (t down): G in two copies, by rows (G v, the P walk, g_init) and
-//                    by columns (k G becomes a row product as well, so no
-//                    64-way reduction across threads); writes gk, gv, glogw
-//                    and per-(b, h) gu partials.
+//                    by columns 2p, 2p + 1 (rows 16q ..: k G becomes a row
+//                    product as well, so no 64-way reduction across
+//                    threads); writes gk, gv, glogw and per-(b, h) gu
+//                    partials.
 // Inputs arrive per 32-token chunk by TMA into two stages (the next chunk
-// loads while this one runs). Each step reads its 16-wide slices as bf16
-// (32 bytes per vector: the 64 threads that share a slice make shared-memory
-// bandwidth, not arithmetic, the limit) one step ahead of use, and widens
-// them in registers. Outputs leave through shared-memory tiles as coalesced
-// 16-byte stores. The 16-wide row work runs on packed fp32 pairs. gu is
-// summed over samples by a fixed-order reduction.
+// loads while this one runs). Each step reads its 16-wide slices as bf16 (32
+// bytes per vector) one step ahead of use and widens them in registers.
+// Outputs leave through shared-memory tiles as coalesced 16-byte stores. The
+// 16-wide row work runs on packed fp32 pairs. gu is summed over samples by a
+// fixed-order reduction.
 #include <string.h>
 
 #include "wkv_device.cuh"
@@ -46,7 +47,7 @@ namespace wkv {
 
 constexpr int kK6b = 64;       // head size
 constexpr int kL6b = 32;       // tokens per chunk
-constexpr int kT6b = 256;      // threads per CTA
+constexpr int kT6b = 128;      // threads per CTA (2 rows per thread)
 constexpr int kIn6b = 5;       // r, k, v, w, do
 enum { kR = 0, kKk = 1, kV = 2, kW = 3, kDo = 4 };
 
@@ -115,14 +116,22 @@ __device__ __forceinline__ float dot16(const float2 (&a)[8], const float2 (&b)[8
   return __fadd_rn(s.x, s.y);
 }
 
+// Two adjacent bf16 of shared memory as a pair.
+__device__ __forceinline__ float2 ld2b(const __nv_bfloat16* p) {
+  const uint32_t x = *reinterpret_cast<const uint32_t*>(p);
+  return make_float2(bf16lo(x), bf16hi(x));
+}
+
 // Store a [kL6b][kK6b] bf16 tile to rows t0 .. t0 + n - 1 of a [B][T][HK]
-// tensor at column h * 64 (one 16-byte piece per thread).
+// tensor at column h * 64 (16-byte pieces).
 __device__ __forceinline__ void wkv6_store_tile(const __nv_bfloat16 (*tile)[kK6b], __nv_bfloat16* dst, int b, int T,
                                                 int HK, int h, int t0, int n, int tid) {
-  const int row = tid / 8, piece = tid % 8;
-  if (row < n) {
-    const uint4 val = reinterpret_cast<const uint4*>(&tile[row][0])[piece];
-    *reinterpret_cast<uint4*>(dst + ((int64_t)b * T + t0 + row) * HK + (int64_t)h * kK6b + piece * 8) = val;
+  for (int g = tid; g < kL6b * 8; g += kT6b) {
+    const int row = g / 8, piece = g % 8;
+    if (row < n) {
+      const uint4 val = reinterpret_cast<const uint4*>(&tile[row][0])[piece];
+      *reinterpret_cast<uint4*>(dst + ((int64_t)b * T + t0 + row) * HK + (int64_t)h * kK6b + piece * 8) = val;
+    }
   }
 }
 
@@ -135,7 +144,7 @@ __global__ void __launch_bounds__(kT6b, 2) wkv6_bwd_pass1_kernel(
     float* __restrict__ cvws, float* __restrict__ p0, unsigned* err) {
   extern __shared__ __align__(128) unsigned char wkv6_bwd1_dsmem[];
   Wkv6Bwd1Smem& sm = *reinterpret_cast<Wkv6Bwd1Smem*>(wkv6_bwd1_dsmem);
-  const int tid = threadIdx.x, i = tid >> 2, q = tid & 3;
+  const int tid = threadIdx.x, q = tid & 3, i0 = 2 * (tid >> 2);  // rows i0, i0 + 1
   const int bh = (int)blockIdx.x, b = bh / H, h = bh % H;
   const int HK = H * kK6b;
   const int nchunk = (T + kL6b - 1) / kL6b;
@@ -155,18 +164,20 @@ __global__ void __launch_bounds__(kT6b, 2) wkv6_bwd_pass1_kernel(
     for (int ch = 0; ch < 2 && ch < nchunk; ++ch) issue(ch);
   }
   // S_{-1}: init_state[state_map[b]] (or the n_state rule), else zero
-  float2 S[8];
+  float2 S0[8], S1[8];
 #pragma unroll
-  for (int m = 0; m < 8; ++m) S[m] = make_float2(0.f, 0.f);
+  for (int m = 0; m < 8; ++m) S0[m] = S1[m] = make_float2(0.f, 0.f);
   if (init_state) {
     const int sidx = state_map ? state_map[b] : (n_state == 1 ? 0 : b);
     if (sidx < 0 || sidx >= n_state) {
       if (tid == 0) record_error(err, WKV_DEVERR_BAD_STATE);
     } else {
-      ld16(init_state + (((int64_t)sidx * H + h) * kK6b + i) * kK6b + 16 * q, S);
+      const float* base = init_state + (((int64_t)sidx * H + h) * kK6b + i0) * kK6b + 16 * q;
+      ld16(base, S0);
+      ld16(base + kK6b, S1);
     }
   }
-  const float ui = u[h * kK6b + i];
+  const float2 uu = make_float2(u[h * kK6b + i0], u[h * kK6b + i0 + 1]);
   __syncthreads();
 
   bool ok = true;
@@ -181,48 +192,53 @@ __global__ void __launch_bounds__(kT6b, 2) wkv6_bwd_pass1_kernel(
     }
     const __nv_bfloat16(*in)[kL6b][kK6b] = sm.in[s];
     {
-      // per token: c_t = r . (u o k) and v . do, 8 threads per token
-      const int jt = tid >> 3, part = tid & 7;
+      // per token: c_t = r . (u o k) and v . do, 4 threads per token
+      const int jt = tid >> 2, part = tid & 3;
       float c = 0.f, vd = 0.f;
 #pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const int e = part * 8 + m;
+      for (int m = 0; m < 16; ++m) {
+        const int e = part * 16 + m;
         c = __fmaf_rn(bf(in[kR][jt][e]) * u[h * kK6b + e], bf(in[kKk][jt][e]), c);
         vd = __fmaf_rn(bf(in[kV][jt][e]), bf(in[kDo][jt][e]), vd);
       }
-#pragma unroll
-      for (int o = 1; o < 8; o <<= 1) {
-        c += __shfl_xor_sync(0xffffffffu, c, o);
-        vd += __shfl_xor_sync(0xffffffffu, vd, o);
-      }
+      c = row_sum4(c);
+      vd = row_sum4(vd);
       if (part == 0) reinterpret_cast<float4*>(&sm.cv[s][jt][0])[0] = make_float4(c, vd, 0.f, 0.f);
     }
     __syncthreads();
     // the step's vectors are fetched one step ahead
     Bf16x16 vn = ld16b(&in[kV][0][16 * q]), dn = ld16b(&in[kDo][0][16 * q]);
-    float wn = bf(in[kW][0][i]), kn = bf(in[kKk][0][i]), rn = bf(in[kR][0][i]), vdn = sm.cv[s][0][1];
+    float2 wn = ld2b(&in[kW][0][i0]), kn = ld2b(&in[kKk][0][i0]), rn = ld2b(&in[kR][0][i0]);
+    float vdn = sm.cv[s][0][1];
     for (int jt = 0; jt < n; ++jt) {
       const Bf16x16 vc = vn, dc = dn;
-      const float wi = wn, ki = kn, ri = rn, vdo = vdn;
+      const float2 w2 = wn, k2 = kn, r2 = rn;
+      const float vdo = vdn;
       if (jt + 1 < n) {
         vn = ld16b(&in[kV][jt + 1][16 * q]);
         dn = ld16b(&in[kDo][jt + 1][16 * q]);
-        wn = bf(in[kW][jt + 1][i]);
-        kn = bf(in[kKk][jt + 1][i]);
-        rn = bf(in[kR][jt + 1][i]);
+        wn = ld2b(&in[kW][jt + 1][i0]);
+        kn = ld2b(&in[kKk][jt + 1][i0]);
+        rn = ld2b(&in[kR][jt + 1][i0]);
         vdn = sm.cv[s][jt + 1][1];
       }
       float2 vv[8], dd[8];
       widen16(vc, vv);
       widen16(dc, dd);
-      const float acc = row_sum4(dot16(S, dd));  // (S_{t-1} do_t)[i]
+      // (S_{t-1} do_t) for both rows
+      const float a0 = row_sum4(dot16(S0, dd)), a1 = row_sum4(dot16(S1, dd));
       if (q == 0) {
-        sm.gro[jt][i] = __float2bfloat16_rn(__fmaf_rn(ui * ki, vdo, acc));
-        sm.xo[jt][i] = __fmul_rn(ri, acc);
+        *reinterpret_cast<__nv_bfloat162*>(&sm.gro[jt][i0]) =
+            __floats2bfloat162_rn(__fmaf_rn(uu.x * k2.x, vdo, a0), __fmaf_rn(uu.y * k2.y, vdo, a1));
+        *reinterpret_cast<float2*>(&sm.xo[jt][i0]) = make_float2(__fmul_rn(r2.x, a0), __fmul_rn(r2.y, a1));
       }
-      const float2 w2 = make_float2(wi, wi), k2 = make_float2(ki, ki);
+      const float2 wa = make_float2(w2.x, w2.x), ka = make_float2(k2.x, k2.x);
+      const float2 wb = make_float2(w2.y, w2.y), kb = make_float2(k2.y, k2.y);
 #pragma unroll
-      for (int m = 0; m < 8; ++m) S[m] = fma2(S[m], w2, mul2(k2, vv[m]));
+      for (int m = 0; m < 8; ++m) {
+        S0[m] = fma2(S0[m], wa, mul2(ka, vv[m]));
+        S1[m] = fma2(S1[m], wb, mul2(kb, vv[m]));
+      }
     }
     __syncthreads();
     if (tid == 0 && ch + 2 < nchunk) issue(ch + 2);  // every read of stage s is done
@@ -242,14 +258,18 @@ __global__ void __launch_bounds__(kT6b, 2) wkv6_bwd_pass1_kernel(
     return;
   }
   // P_{T-1}[i] = sum_j g_final[i][j] S_{T-1}[i][j]
-  float pp = 0.f;
+  float p0a = 0.f, p0b = 0.f;
   if (g_final) {
     float2 gf[8];
-    ld16(g_final + ((int64_t)bh * kK6b + i) * kK6b + 16 * q, gf);
-    pp = dot16(gf, S);
+    const float* base = g_final + ((int64_t)bh * kK6b + i0) * kK6b + 16 * q;
+    ld16(base, gf);
+    p0a = dot16(gf, S0);
+    ld16(base + kK6b, gf);
+    p0b = dot16(gf, S1);
   }
-  pp = row_sum4(pp);
-  if (q == 0) p0[(int64_t)bh * kK6b + i] = pp;
+  p0a = row_sum4(p0a);
+  p0b = row_sum4(p0b);
+  if (q == 0) *reinterpret_cast<float2*>(&p0[(int64_t)bh * kK6b + i0]) = make_float2(p0a, p0b);
 }
 
 __global__ void __launch_bounds__(kT6b, 2) wkv6_bwd_pass2_kernel(
@@ -262,7 +282,8 @@ __global__ void __launch_bounds__(kT6b, 2) wkv6_bwd_pass2_kernel(
     float* __restrict__ gu_part, unsigned* err) {
   extern __shared__ __align__(128) unsigned char wkv6_bwd2_dsmem[];
   Wkv6Bwd2Smem& sm = *reinterpret_cast<Wkv6Bwd2Smem*>(wkv6_bwd2_dsmem);
-  const int tid = threadIdx.x, i = tid >> 2, q = tid & 3;  // row i of G; column i of G^T
+  // rows i0, i0 + 1 of G and columns i0, i0 + 1 of G (rows 16q .. 16q + 15)
+  const int tid = threadIdx.x, q = tid & 3, i0 = 2 * (tid >> 2);
   const int bh = (int)blockIdx.x, b = bh / H, h = bh % H;
   const int HK = H * kK6b;
   const int nchunk = (T + kL6b - 1) / kL6b;
@@ -289,19 +310,24 @@ __global__ void __launch_bounds__(kT6b, 2) wkv6_bwd_pass2_kernel(
     for (int ch = 0; ch < 2 && ch < nchunk; ++ch) issue(ch);
   }
   // G_{T-1} = g_final, by rows (G[i][16q ..]) and by columns (G[16q ..][i])
-  float2 G[8], Gc[8];
+  float2 G0[8], G1[8], C0[8], C1[8];
 #pragma unroll
-  for (int m = 0; m < 8; ++m) G[m] = Gc[m] = make_float2(0.f, 0.f);
+  for (int m = 0; m < 8; ++m) G0[m] = G1[m] = C0[m] = C1[m] = make_float2(0.f, 0.f);
   if (g_final) {
     const float* gf = g_final + (int64_t)bh * kK6b * kK6b;
-    ld16(gf + i * kK6b + 16 * q, G);
+    ld16(gf + i0 * kK6b + 16 * q, G0);
+    ld16(gf + (i0 + 1) * kK6b + 16 * q, G1);
 #pragma unroll
-    for (int m = 0; m < 8; ++m)
-      Gc[m] = make_float2(gf[(16 * q + 2 * m) * kK6b + i], gf[(16 * q + 2 * m + 1) * kK6b + i]);
+    for (int m = 0; m < 8; ++m) {
+      const float2 top = *reinterpret_cast<const float2*>(gf + (16 * q + 2 * m) * kK6b + i0);
+      const float2 bot = *reinterpret_cast<const float2*>(gf + (16 * q + 2 * m + 1) * kK6b + i0);
+      C0[m] = make_float2(top.x, bot.x);
+      C1[m] = make_float2(top.y, bot.y);
+    }
   }
-  float P = p0[(int64_t)bh * kK6b + i];
-  const float ui = u[h * kK6b + i];
-  float gu_i = 0.f;
+  float2 P = *reinterpret_cast<const float2*>(&p0[(int64_t)bh * kK6b + i0]);
+  const float2 uu = make_float2(u[h * kK6b + i0], u[h * kK6b + i0 + 1]);
+  float2 gu2 = make_float2(0.f, 0.f);
   __syncthreads();
 
   bool ok = true;
@@ -317,7 +343,7 @@ __global__ void __launch_bounds__(kT6b, 2) wkv6_bwd_pass2_kernel(
     const Wkv6Bwd2Stage& st = sm.st[s];
     struct Tok {
       Bf16x16 v, d, r, k, w;
-      float wi, ri, ki, dj, c, vdo, xi;
+      float2 w2, r2, k2, d2, cvd, x2;
     };
     auto fetch = [&](int jt) {
       Tok x;
@@ -326,13 +352,12 @@ __global__ void __launch_bounds__(kT6b, 2) wkv6_bwd_pass2_kernel(
       x.r = ld16b(&st.in[kR][jt][16 * q]);
       x.k = ld16b(&st.in[kKk][jt][16 * q]);
       x.w = ld16b(&st.in[kW][jt][16 * q]);
-      x.wi = bf(st.in[kW][jt][i]);
-      x.ri = bf(st.in[kR][jt][i]);
-      x.ki = bf(st.in[kKk][jt][i]);
-      x.dj = bf(st.in[kDo][jt][i]);
-      x.c = st.cv[jt][0];
-      x.vdo = st.cv[jt][1];
-      x.xi = st.x[jt][i];
+      x.w2 = ld2b(&st.in[kW][jt][i0]);
+      x.r2 = ld2b(&st.in[kR][jt][i0]);
+      x.k2 = ld2b(&st.in[kKk][jt][i0]);
+      x.d2 = ld2b(&st.in[kDo][jt][i0]);
+      x.cvd = *reinterpret_cast<const float2*>(&st.cv[jt][0]);  // (c_t, v_t . do_t)
+      x.x2 = *reinterpret_cast<const float2*>(&st.x[jt][i0]);
       return x;
     };
     Tok nx = fetch(n - 1);
@@ -345,21 +370,29 @@ __global__ void __launch_bounds__(kT6b, 2) wkv6_bwd_pass2_kernel(
       widen16(cu.r, rr);
       widen16(cu.k, kk);
       widen16(cu.w, ww);
-      const float gki = row_sum4(dot16(G, vv));   // (G_t v_t)[i]
-      const float gvj = row_sum4(dot16(kk, Gc));  // (k_t G_t)[i]
-      const float gl = __fsub_rn(P, __fmul_rn(cu.ki, gki));  // w_t gw_t
-      P = __fadd_rn(gl, cu.xi);                              // P_{t-1}
+      // (G_t v_t) for rows i0, i0 + 1 and (k_t G_t) for columns i0, i0 + 1
+      const float g0 = row_sum4(dot16(G0, vv)), g1 = row_sum4(dot16(G1, vv));
+      const float h0 = row_sum4(dot16(kk, C0)), h1 = row_sum4(dot16(kk, C1));
+      const float c = cu.cvd.x, vdo = cu.cvd.y;
+      const float2 gl = make_float2(__fsub_rn(P.x, __fmul_rn(cu.k2.x, g0)), __fsub_rn(P.y, __fmul_rn(cu.k2.y, g1)));
+      P = add2(gl, cu.x2);  // P_{t-1}
       if (q == 0) {
-        sm.out[0][jt][i] = __float2bfloat16_rn(__fmaf_rn(ui * cu.ri, cu.vdo, gki));
-        sm.out[1][jt][i] = __float2bfloat16_rn(__fmaf_rn(cu.c, cu.dj, gvj));
-        sm.out[2][jt][i] = __float2bfloat16_rn(gl);
+        *reinterpret_cast<__nv_bfloat162*>(&sm.out[0][jt][i0]) =
+            __floats2bfloat162_rn(__fmaf_rn(uu.x * cu.r2.x, vdo, g0), __fmaf_rn(uu.y * cu.r2.y, vdo, g1));
+        *reinterpret_cast<__nv_bfloat162*>(&sm.out[1][jt][i0]) =
+            __floats2bfloat162_rn(__fmaf_rn(c, cu.d2.x, h0), __fmaf_rn(c, cu.d2.y, h1));
+        *reinterpret_cast<__nv_bfloat162*>(&sm.out[2][jt][i0]) = __floats2bfloat162_rn(gl.x, gl.y);
       }
-      gu_i = __fmaf_rn(cu.ri * cu.ki, cu.vdo, gu_i);
-      const float2 w2 = make_float2(cu.wi, cu.wi), r2 = make_float2(cu.ri, cu.ri), d2 = make_float2(cu.dj, cu.dj);
+      gu2 = fma2(mul2(cu.r2, cu.k2), make_float2(vdo, vdo), gu2);
+      const float2 wa = make_float2(cu.w2.x, cu.w2.x), ra = make_float2(cu.r2.x, cu.r2.x);
+      const float2 wb = make_float2(cu.w2.y, cu.w2.y), rb = make_float2(cu.r2.y, cu.r2.y);
+      const float2 da = make_float2(cu.d2.x, cu.d2.x), db = make_float2(cu.d2.y, cu.d2.y);
 #pragma unroll
       for (int m = 0; m < 8; ++m) {
-        G[m] = fma2(G[m], w2, mul2(r2, dd[m]));
-        Gc[m] = fma2(Gc[m], ww[m], mul2(rr[m], d2));
+        G0[m] = fma2(G0[m], wa, mul2(ra, dd[m]));
+        G1[m] = fma2(G1[m], wb, mul2(rb, dd[m]));
+        C0[m] = fma2(C0[m], ww[m], mul2(rr[m], da));
+        C1[m] = fma2(C1[m], ww[m], mul2(rr[m], db));
       }
     }
     __syncthreads();
@@ -374,11 +407,16 @@ __global__ void __launch_bounds__(kT6b, 2) wkv6_bwd_pass2_kernel(
     return;
   }
   if (g_init) {
-    float4* d = reinterpret_cast<float4*>(g_init + ((int64_t)bh * kK6b + i) * kK6b + 16 * q);
+    float* base = g_init + ((int64_t)bh * kK6b + i0) * kK6b + 16 * q;
+    float4* d0 = reinterpret_cast<float4*>(base);
+    float4* d1 = reinterpret_cast<float4*>(base + kK6b);
 #pragma unroll
-    for (int m = 0; m < 4; ++m) d[m] = make_float4(G[2 * m].x, G[2 * m].y, G[2 * m + 1].x, G[2 * m + 1].y);
+    for (int m = 0; m < 4; ++m) {
+      d0[m] = make_float4(G0[2 * m].x, G0[2 * m].y, G0[2 * m + 1].x, G0[2 * m + 1].y);
+      d1[m] = make_float4(G1[2 * m].x, G1[2 * m].y, G1[2 * m + 1].x, G1[2 * m + 1].y);
+    }
   }
-  if (q == 0) gu_part[(int64_t)bh * kK6b + i] = gu_i;
+  if (q == 0) *reinterpret_cast<float2*>(&gu_part[(int64_t)bh * kK6b + i0]) = gu2;
 }
 
 // gu[c] = sum over samples b (ascending) of gu_part[b][c]: fixed order.
