@@ -358,6 +358,37 @@ def secondary(dev, flush, peak):
     del graph
     torch.cuda.empty_cache()
 
+    # decode: 256 slots, one token each per call (the T = 1 path of the chunk step), 64 calls
+    # captured in one CUDA graph
+    S, C, steps = 256, 4096, 64
+    g.manual_seed(0)
+    kd = torch.randn(steps, S, C, device=dev, generator=g).to(torch.bfloat16)
+    vd = torch.randn(steps, S, C, device=dev, generator=g).to(torch.bfloat16)
+    yd = torch.empty_like(kd)
+    cud = torch.arange(S + 1, dtype=torch.int32, device=dev)
+    stated = wkv.wkv4_state_init(S, C, dev)
+
+    def decode_calls():
+        wkv.wkv4_state_init(S, C, dev, state=stated)
+        for t in range(steps):
+            wkv.wkv4_chunk_step(w, u, kd[t], vd[t], cud, stated, y=yd[t])
+
+    decode_calls()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        decode_calls()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph, stream=side):
+            decode_calls()
+    torch.cuda.synchronize()
+    t_dec = _events_ms(graph.replay, 5, flush, stream)
+    res["wkv4_decode_bf16_slots256"] = {
+        "S": S, "C": C, "calls": steps, "graph_ms": t_dec, "per_call_us_graph": 1e3 * t_dec / steps,
+        "Gtokch_per_s_graph": steps * S * C / (t_dec * 1e-3) / 1e9,
+        "GBps_graph": (6 + 40) * steps * S * C / (t_dec * 1e-3) / 1e9}
+    del graph, kd, vd, yd
+    torch.cuda.empty_cache()
+
     # RWKV-6 head-state forward
     rec = synth.WKV6_RECIPES["wkv6_fwd_bf16_c2048"]
     B, T, H = rec.B, rec.T, rec.H

@@ -49,6 +49,17 @@ def test_chunked_equals_whole_bitwise(W, slots):
     y7, s7 = feed(W, slots, 7, w, u, k, v)
     assert torch.equal(y32, yall) and torch.equal(s32, sall)
     assert torch.equal(y7, yall) and torch.equal(s7, sall)
+    # one token per slot per call: the decode path
+    short = dict(slots)
+    short["lengths"] = np.minimum(slots["lengths"], 40)
+    short["offsets"] = np.concatenate([[0], np.cumsum(short["lengths"])])
+    idx = np.concatenate([np.arange(slots["offsets"][s], slots["offsets"][s] + short["lengths"][s])
+                          for s in range(len(short["lengths"]))])
+    it = torch.from_numpy(idx).cuda()
+    ks, vs = k[it].contiguous(), v[it].contiguous()
+    y1, s1 = feed(W, short, 1, w, u, ks, vs)
+    ya, sa = feed(W, short, 1 << 30, w, u, ks, vs)
+    assert torch.equal(y1, ya) and torch.equal(s1, sa)
     assert W.device_error(reset=True) == 0
 
 
