@@ -30,6 +30,8 @@ SHAPES = [
     (2, 64, 128), (3, 100, 72), (1, 1, 8), (2, 33, 40), (1, 257, 264), (4, 31, 96), (1, 1000, 32),
     # 257 lane groups split 4 ways: 4 warps per CTA, the last CTA with one active warp
     (1, 300, 8200),
+    # few lane groups, long ragged sequence: 8-CTA clusters, two sub-segments per CTA
+    (2, 1500, 96),
 ]
 
 
