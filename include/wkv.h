@@ -204,6 +204,17 @@ wkv_status wkv4_backward_noalloc(int64_t B, int64_t T, int64_t C, int dtype,
                                  const float *ckpt,
                                  void *gk, void *gv, float *gw, float *gu, void *stream);
 
+/*
+ * The failure path of the bounded waits, on demand: launches one warp that
+ * waits on a barrier nothing will complete, giving up after limit_ns
+ * nanoseconds (1000 .. 10^10). It records WKV_DEVERR_WAIT_TIMEOUT in the
+ * device error word -- what every kernel does if a copy it waits on never
+ * lands -- and returns; the context stays usable. For tests of the error
+ * reporting (read it with wkv_device_error). Returns WKV_ERR_INVALID_ARG for
+ * a limit outside the range.
+ */
+wkv_status wkv_wait_selfcheck(int64_t limit_ns, void *stream);
+
 /* ------------------------------------------------------------------------ */
 /* RWKV-6                                                                    */
 /* ------------------------------------------------------------------------ */

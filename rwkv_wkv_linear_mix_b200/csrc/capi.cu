@@ -296,6 +296,15 @@ WKV_EXPORT wkv_status wkv6_forward(int64_t B, int64_t T, int64_t H, int64_t K, i
   return s == WKV_OK ? s : fail(s, why);
 }
 
+WKV_EXPORT wkv_status wkv_wait_selfcheck(int64_t limit_ns, void* stream) {
+  if (limit_ns < 1000 || limit_ns > 10000000000ll) return fail(WKV_ERR_INVALID_ARG, "limit_ns outside 1 us .. 10 s");
+  unsigned* err = nullptr;
+  if (wkv_status s = device_error_ptr(&err)) return s;
+  const char* why = "";
+  wkv_status s = launch_wait_selfcheck(limit_ns, static_cast<cudaStream_t>(stream), err, &why);
+  return s == WKV_OK ? s : fail(s, why);
+}
+
 WKV_EXPORT size_t wkv6_backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K) {
   if (B < 0 || T < 0 || H < 0 || K != 64) return 0;
   return wkv6_bwd_workspace_bytes(B, T, H);

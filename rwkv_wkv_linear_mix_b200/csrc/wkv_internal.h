@@ -169,5 +169,6 @@ wkv_status launch_wkv4_state_init(int64_t S, int64_t C, float* state, cudaStream
 wkv_status launch_wkv4_chunk_step(const Wkv4ChunkArgs& a, cudaStream_t stream, unsigned* err, const char** why);
 wkv_status launch_wkv6_forward(const Wkv6FwdArgs& a, cudaStream_t stream, unsigned* err, const char** why);
 wkv_status launch_wkv6_backward(const Wkv6BwdArgs& a, cudaStream_t stream, unsigned* err, const char** why);
+wkv_status launch_wait_selfcheck(int64_t limit_ns, cudaStream_t stream, unsigned* err, const char** why);
 
 }  // namespace wkv

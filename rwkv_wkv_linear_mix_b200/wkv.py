@@ -39,6 +39,7 @@ SIGNATURES = {
     "wkv6_forward": (_int, [_i64, _i64, _i64, _i64, _int] + [_vp] * 7 + [_i64, _vp, _vp, _vp]),
     "wkv4_backward_noalloc": (_int, [_i64, _i64, _i64, _int] + [_vp] * 11),
     "wkv6_backward_workspace_bytes": (_sz, [_i64, _i64, _i64, _i64]),
+    "wkv_wait_selfcheck": (_int, [_i64, _vp]),
     "wkv6_backward": (_int, [_i64, _i64, _i64, _i64, _int] + [_vp] * 7 + [_i64] + [_vp] * 9 + [_sz, _vp]),
 }
 
@@ -272,6 +273,14 @@ def wkv6_forward(r, k, v, w, u, init_state: Optional[torch.Tensor] = None,
                              _ptr(init_state), _ptr(state_map), n_state, _ptr(final_state), _ptr(o),
                              _stream(r)), "wkv6_forward")
     return o, final_state
+
+
+def wait_selfcheck(limit_ns: int = 2_000_000, device=None) -> None:
+    """Run the bounded-wait failure path once (see wkv_wait_selfcheck)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        _check(_lib.wkv_wait_selfcheck(int(limit_ns), ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)),
+               "wkv_wait_selfcheck")
 
 
 def wkv6_backward_workspace_bytes(B: int, T: int, H: int, K: int = 64) -> int:

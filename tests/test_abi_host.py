@@ -126,6 +126,8 @@ def test_chunk_and_wkv6_argument_errors(W):
     assert wb6(wsp=None) == W.WKV_ERR_INVALID_ARG
     assert wb6(init=FAKE, ns=3) == W.WKV_ERR_INVALID_ARG      # n_state neither 1 nor B
     assert wb6(H=0) == W.WKV_OK
+    assert L.wkv_wait_selfcheck(0, None) == W.WKV_ERR_INVALID_ARG
+    assert L.wkv_wait_selfcheck(20_000_000_000, None) == W.WKV_ERR_INVALID_ARG
 
 
 def test_binding_refuses_cpu_tensors(W):
