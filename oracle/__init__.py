@@ -60,6 +60,8 @@ def _open(path):
     lib.oracle_wkv6_forward.argtypes = [i64, i64, i64, i64] + [dp] * 7 + [i64, dp, dp]
     lib.oracle_wkv6_forward.restype = ctypes.c_int
     lib.oracle_wkv6_backward.argtypes = [i64, i64, i64, i64] + [dp] * 7 + [i64] + [dp] * 8
+    lib.oracle_wkv7_forward.argtypes = [i64, i64, i64, i64] + [dp] * 9
+    lib.oracle_wkv7_forward.restype = ctypes.c_int
     lib.oracle_wkv6_backward.restype = ctypes.c_int
     return lib
 
@@ -239,3 +241,29 @@ def wkv6_backward(r, k, v, w, u, dout, init_state=None, state_map=None, g_final=
     if rc != 0:
         raise FloatingPointError(f"oracle_wkv6_backward failed (rc={rc})")
     return gr, gk, gv, gw, gu, gi
+
+
+def wkv7_forward(r, w, k, v, a, b, init_state=None, head_size: int = 64, _lib=None):
+    """RWKV-7 generalized delta rule forward in fp64 (see oracle_wkv7_forward).
+
+    r, w, k, v, a, b: [B, T, H*K] (w the decay in log space); init_state:
+    [B, H, K, K] indexed [b][h][key][value] or None. Returns (o [B, T, H*K],
+    final_state [B, H, K, K]).
+    """
+    lib = _lib or _load()
+    r, w, k, v, a, b = (_f64(x) for x in (r, w, k, v, a, b))
+    B, T, HK = r.shape
+    K = head_size
+    assert HK % K == 0 and all(x.shape == r.shape for x in (w, k, v, a, b))
+    H = HK // K
+    s0 = None
+    if init_state is not None:
+        s0 = _f64(init_state)
+        assert s0.shape == (B, H, K, K)
+    o = np.empty_like(r)
+    fs = np.empty((B, H, K, K))
+    rc = lib.oracle_wkv7_forward(B, T, H, K, _ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(s0),
+                                 _ptr(o), _ptr(fs))
+    if rc != 0:
+        raise FloatingPointError(f"oracle_wkv7_forward failed (rc={rc})")
+    return o, fs

@@ -32,7 +32,14 @@
  *      o_t[j]    = sum_i r_t[i] * ( S_{t-1}[i][j] + u[i] k_t[i] v_t[j] )
  *      S_t[i][j] = w_t[i] * S_{t-1}[i][j] + k_t[i] v_t[j]
  *
- *  with S_{-1} = 0 or a caller-given initial state.
+ *  with S_{-1} = 0 or a caller-given initial state, and its backward (the
+ *  chain rule with G_t = dL/dS_t walked down).
+ *
+ *  RWKV-7 generalized delta rule (generalized_delta_rule / rwkv7_op of the
+ *  rwkv-ops package page; the page gives the interface, the recurrence is
+ *  the diagonal-plus-rank-one transition written at oracle_wkv7_forward):
+ *
+ *      S_t = (diag(e^{w_t}) + b_t a_t^T) S_{t-1} + k_t^T v_t,    o_t = r_t S_t
  *
  * Layouts: activations [B][T][C] row-major, C fastest. All inputs are fp64
  * (the Python wrapper widens float32 / bf16 inputs exactly).
@@ -419,5 +426,76 @@ int oracle_wkv6_backward(int64_t B, int64_t T, int64_t H, int64_t K,
     if (!all_finite(gr, n) || !all_finite(gk, n) || !all_finite(gv, n) || !all_finite(gw, n) ||
         !all_finite(gu, HK))
         bad |= 1;
+    return bad;
+}
+
+/* ------------------------------------------------------------------------ */
+/* RWKV-7 generalized delta rule, forward                                    */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * generalized_delta_rule(r, w, k, v, a, b, initial_state, output_final_state)
+ * of the rwkv-ops package page (section on rwkv7_op / generalized_delta_rule):
+ * inputs [B][T][H][K] (w the decay in log space), state [N][H][K][V] with
+ * N = B sequences, outputs o [B][T][H][V] and the final state. The page
+ * prints the interface only; the recurrence taken is the plain
+ * diagonal-plus-rank-one state transition of a "generalized delta rule",
+ * per head with key index j and value index i (V = K here):
+ *
+ *   sa[i]     = sum_j a_t[j] S_{t-1}[j][i]
+ *   S_t[j][i] = e^{w_t[j]} S_{t-1}[j][i] + b_t[j] sa[i] + k_t[j] v_t[i]
+ *   o_t[i]    = sum_j r_t[j] S_t[j][i]          (the state after the token)
+ *
+ * i.e. S_t = (diag(e^{w_t}) + b_t a_t^T) S_{t-1} + k_t^T v_t, o_t = r_t S_t.
+ * r, w, k, v, a, b: [B][T][H*K]; init_state (nullable): [B][H][K][K] indexed
+ * [b][h][j][i]; o: [B][T][H*K]; final_state (nullable): [B][H][K][K].
+ * Returns 0 on success, 1 on a non-finite output, 2 on allocation failure.
+ */
+int oracle_wkv7_forward(int64_t B, int64_t T, int64_t H, int64_t K,
+                        const double *r, const double *w, const double *k, const double *v,
+                        const double *a, const double *b, const double *init_state,
+                        double *o, double *final_state)
+{
+    const int64_t HK = H * K;
+    int bad = 0;
+    #pragma omp parallel reduction(|:bad)
+    {
+        double *S = (double *)malloc(sizeof(double) * (size_t)(K * K));
+        double *sa = (double *)malloc(sizeof(double) * (size_t)K);
+        if (!S || !sa) bad = 2;
+        #pragma omp for collapse(2) schedule(static)
+        for (int64_t bi = 0; bi < B; ++bi) {
+            for (int64_t h = 0; h < H; ++h) {
+                if (!S || !sa) continue;
+                if (init_state)
+                    memcpy(S, init_state + (bi * H + h) * K * K, sizeof(double) * (size_t)(K * K));
+                else
+                    memset(S, 0, sizeof(double) * (size_t)(K * K));
+                for (int64_t t = 0; t < T; ++t) {
+                    const int64_t row = (bi * T + t) * HK + h * K;
+                    for (int64_t i = 0; i < K; ++i) {
+                        double acc = 0.0;
+                        for (int64_t j = 0; j < K; ++j) acc += a[row + j] * S[j * K + i];
+                        sa[i] = acc;
+                    }
+                    for (int64_t j = 0; j < K; ++j) {
+                        const double d = exp(w[row + j]);
+                        for (int64_t i = 0; i < K; ++i)
+                            S[j * K + i] = d * S[j * K + i] + b[row + j] * sa[i] + k[row + j] * v[row + i];
+                    }
+                    for (int64_t i = 0; i < K; ++i) {
+                        double acc = 0.0;
+                        for (int64_t j = 0; j < K; ++j) acc += r[row + j] * S[j * K + i];
+                        o[row + i] = acc;
+                        if (!isfinite(acc)) bad |= 1;
+                    }
+                }
+                if (final_state)
+                    memcpy(final_state + (bi * H + h) * K * K, S, sizeof(double) * (size_t)(K * K));
+            }
+        }
+        free(S);
+        free(sa);
+    }
     return bad;
 }

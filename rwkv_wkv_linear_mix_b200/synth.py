@@ -34,6 +34,9 @@ __all__ = [
     "wkv6_inputs",
     "WKV4_RECIPES",
     "WKV6_RECIPES",
+    "Wkv7Recipe",
+    "WKV7_RECIPES",
+    "wkv7_inputs",
     "feed_schedule",
 ]
 
@@ -241,6 +244,61 @@ def wkv6_inputs(recipe: Wkv6Recipe, seed: int = 0) -> dict:
     out = {"u": u}
     out["w"], out["w32"] = _store(w, "bf16")
     del w
+    for name in ("r", "k", "v"):
+        x = rng.standard_normal(size=(B, T, HK), dtype=np.float32)
+        out[name], out[name + "32"] = _store(x, "bf16")
+    return out
+
+
+# ----------------------------------------------------------------------------
+# RWKV-7 (generalized delta rule) recipes
+# ----------------------------------------------------------------------------
+
+@dataclasses.dataclass(frozen=True)
+class Wkv7Recipe:
+    name: str
+    B: int
+    T: int
+    H: int
+    K: int = 64
+    d_mean: float = -1.0   # decay in log space w = -exp(d), d ~ N(d_mean, d_std^2)
+    d_std: float = 0.5
+    lr_lo: float = 0.0     # b = kappa * alpha with alpha ~ U(lr_lo, lr_hi) per (t, channel)
+    lr_hi: float = 1.0
+
+    def with_shape(self, B=None, T=None, H=None, name=None):
+        return dataclasses.replace(
+            self, B=self.B if B is None else B, T=self.T if T is None else T,
+            H=self.H if H is None else H, name=name or self.name)
+
+
+WKV7_RECIPES = {
+    "wkv7_fwd_bf16_c2048": Wkv7Recipe("wkv7_fwd_bf16_c2048", 8, 4096, 32),
+}
+
+
+def wkv7_inputs(recipe: Wkv7Recipe, seed: int = 0) -> dict:
+    """Draw one RWKV-7 workload: r, w, k, v, a, b as bf16 [B,T,H*K] (and their
+    exact float32 decodings r32, ...). w = -exp(d) is the decay in log space;
+    per (sample, token, head) a unit vector kappa is drawn (normalised
+    N(0,1)), a = -kappa and b = kappa * alpha (the in-context removal and its
+    rate, as in the delta rule); r, k, v ~ N(0,1). Draw order: d, kappa,
+    alpha, r, k, v.
+    """
+    B, T, H, K = recipe.B, recipe.T, recipe.H, recipe.K
+    HK = H * K
+    rng = np.random.Generator(np.random.PCG64(seed))
+    d = rng.standard_normal(size=(B, T, HK), dtype=np.float32).astype(np.float64) * recipe.d_std + recipe.d_mean
+    out = {}
+    out["w"], out["w32"] = _store((-np.exp(d)).astype(np.float32), "bf16")
+    del d
+    kap = rng.standard_normal(size=(B, T, H, K), dtype=np.float32).astype(np.float64)
+    kap /= np.sqrt(np.sum(kap * kap, axis=-1, keepdims=True))
+    kap = kap.reshape(B, T, HK)
+    alpha = rng.uniform(recipe.lr_lo, recipe.lr_hi, size=(B, T, HK))
+    out["a"], out["a32"] = _store((-kap).astype(np.float32), "bf16")
+    out["b"], out["b32"] = _store((kap * alpha).astype(np.float32), "bf16")
+    del kap, alpha
     for name in ("r", "k", "v"):
         x = rng.standard_normal(size=(B, T, HK), dtype=np.float32)
         out[name], out[name + "32"] = _store(x, "bf16")

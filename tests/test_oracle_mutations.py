@@ -35,6 +35,20 @@ MUTATIONS = {
     # RWKV-6 backward: gw and gr against S_t instead of S_{t-1}
     "wkv6b_state_index": ("const double *S = Sh + t * K * K; /* S_{t-1} */",
                           "const double *S = Sh + (t + 1) * K * K;"),
+    # RWKV-7: the log decay used as the decay itself
+    "wkv7_no_exp": ("const double d = exp(w[row + j]);", "const double d = w[row + j];"),
+    # RWKV-7: the removal projection taken with b instead of a
+    "wkv7_ab_swap": ("for (int64_t j = 0; j < K; ++j) acc += a[row + j] * S[j * K + i];",
+                     "for (int64_t j = 0; j < K; ++j) acc += b[row + j] * S[j * K + i];"),
+    # RWKV-7: transposed outer product k v^T
+    "wkv7_kv_transpose": ("b[row + j] * sa[i] + k[row + j] * v[row + i];",
+                          "b[row + j] * sa[i] + k[row + i] * v[row + j];"),
+    # RWKV-7: wrong sign on the rank-one term
+    "wkv7_rank_one_sign": ("S[j * K + i] = d * S[j * K + i] + b[row + j] * sa[i]",
+                           "S[j * K + i] = d * S[j * K + i] - b[row + j] * sa[i]"),
+    # RWKV-7: the read leaves out the current token's write
+    "wkv7_read_without_token": ("for (int64_t j = 0; j < K; ++j) acc += r[row + j] * S[j * K + i];",
+                                "for (int64_t j = 0; j < K; ++j) acc += r[row + j] * (S[j * K + i] - k[row + j] * v[row + i]);"),
 }
 
 
@@ -87,9 +101,24 @@ def _wkv6b_pins_fail(var):
     return any(rel_err(g, n) > 1e-6 for g, n in zip(got, num))
 
 
+def _wkv7_pins_fail(var):
+    import test_oracle_wkv7 as p7
+
+    class _Adapter:  # the pin functions take the oracle module; give them the variant
+        wkv7_forward = staticmethod(var.wkv7_forward)
+    for pin in (p7.test_delta_rule_stores_and_reads_back, p7.test_hand_worked_two_steps,
+                lambda o: p7.test_without_the_rank_one_term(o, "b_zero")):
+        try:
+            pin(_Adapter)
+        except AssertionError:
+            return True
+    return False
+
+
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
 def test_mutation_is_caught(variants, name):
     check = (_wkv4_pins_fail if name.startswith("wkv4") else
+             _wkv7_pins_fail if name.startswith("wkv7") else
              _wkv6b_pins_fail if name.startswith("wkv6b") else _wkv6_pins_fail)
     assert check(variants[name]), f"planted mistake {name} passed every pin"
 
@@ -100,6 +129,8 @@ def test_unmutated_source_passes(oracle):
         wkv4_backward = staticmethod(oracle.wkv4_backward)
         wkv6_forward = staticmethod(oracle.wkv6_forward)
         wkv6_backward = staticmethod(oracle.wkv6_backward)
+        wkv7_forward = staticmethod(oracle.wkv7_forward)
     assert not _wkv4_pins_fail(_Orig)
+    assert not _wkv7_pins_fail(_Orig)
     assert not _wkv6_pins_fail(_Orig)
     assert not _wkv6b_pins_fail(_Orig)
