@@ -281,6 +281,33 @@ wkv_status wkv6_backward(int64_t B, int64_t T, int64_t H, int64_t K, int dtype,
                          void *gr, void *gk, void *gv, void *glogw, float *gu, float *g_init,
                          void *workspace, size_t workspace_bytes, void *stream);
 
+/* ------------------------------------------------------------------------ */
+/* RWKV-7                                                                    */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * RWKV-7 generalized delta rule forward (generalized_delta_rule / rwkv7_op on
+ * the rwkv-ops package page: r, w, k, v, a, b with w the decay in log space,
+ * initial and final state [N, H, K, V]). Per head, with the key index j and
+ * the value index i of the state S[j][i]:
+ *   S_t = (diag(e^{w_t}) + b_t a_t^T) S_{t-1} + k_t^T v_t,    o_t = r_t S_t
+ * (the page gives the interface; this diagonal-plus-rank-one transition is
+ * the recurrence taken for it).
+ *   K            head size (= value size); 64 is the supported value.
+ *   dtype        WKV_BF16 (else UNSUPPORTED).
+ *   r, w, k, v, a, b  [B][T][H*K] bf16.
+ *   init_state   NULL (every sample starts from S = 0) or [B][H][K][K]
+ *                float32 indexed [b][h][j][i] (one sequence per sample).
+ *   final_state  NULL or [B][H][K][K] float32, written: S after the last token.
+ *   o            [B][T][H*K] bf16, written.
+ * One CTA of 128 threads walks each head's sequence in order (fp32 state).
+ * T = 1 is the decode step of rwkv7_op_rnn.
+ */
+wkv_status wkv7_forward(int64_t B, int64_t T, int64_t H, int64_t K, int dtype,
+                        const void *r, const void *w, const void *k, const void *v,
+                        const void *a, const void *b,
+                        const float *init_state, float *final_state, void *o, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

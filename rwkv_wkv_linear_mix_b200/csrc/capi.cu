@@ -296,6 +296,34 @@ WKV_EXPORT wkv_status wkv6_forward(int64_t B, int64_t T, int64_t H, int64_t K, i
   return s == WKV_OK ? s : fail(s, why);
 }
 
+WKV_EXPORT wkv_status wkv7_forward(int64_t B, int64_t T, int64_t H, int64_t K, int dtype, const void* r,
+                                   const void* w, const void* k, const void* v, const void* a, const void* b,
+                                   const float* init_state, float* final_state, void* o, void* stream) {
+  if (B < 0 || T < 0 || H < 0 || K < 0) return fail(WKV_ERR_INVALID_ARG, "negative size");
+  if (dtype != WKV_F32 && dtype != WKV_BF16) return fail(WKV_ERR_INVALID_ARG, "unknown dtype");
+  if (dtype != WKV_BF16) return fail(WKV_ERR_UNSUPPORTED, "wkv7_forward supports bf16 only");
+  if (K != 64) return fail(WKV_ERR_UNSUPPORTED, "wkv7_forward supports head size 64 only");
+  if (B == 0 || H == 0) return WKV_OK;
+  if (T > INT32_MAX || H > 65535 || B * H > INT32_MAX) return fail(WKV_ERR_UNSUPPORTED, "size out of range");
+  WKV_OPTIONAL_PTR(init_state, "init_state");
+  WKV_OPTIONAL_PTR(final_state, "final_state");
+  if (T > 0) {
+    WKV_REQUIRE_PTR(r, "r");
+    WKV_REQUIRE_PTR(w, "w");
+    WKV_REQUIRE_PTR(k, "k");
+    WKV_REQUIRE_PTR(v, "v");
+    WKV_REQUIRE_PTR(a, "a");
+    WKV_REQUIRE_PTR(b, "b");
+    WKV_REQUIRE_PTR(o, "o");
+  }
+  unsigned* err = nullptr;
+  if (wkv_status s = device_error_ptr(&err)) return s;
+  const char* why = "";
+  Wkv7FwdArgs args{B, T, H, K, r, w, k, v, a, b, init_state, final_state, o};
+  wkv_status s = launch_wkv7_forward(args, static_cast<cudaStream_t>(stream), err, &why);
+  return s == WKV_OK ? s : fail(s, why);
+}
+
 WKV_EXPORT wkv_status wkv_wait_selfcheck(int64_t limit_ns, void* stream) {
   if (limit_ns < 1000 || limit_ns > 10000000000ll) return fail(WKV_ERR_INVALID_ARG, "limit_ns outside 1 us .. 10 s");
   unsigned* err = nullptr;

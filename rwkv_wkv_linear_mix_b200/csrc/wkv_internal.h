@@ -158,6 +158,19 @@ struct Wkv6BwdArgs {
 };
 size_t wkv6_bwd_workspace_bytes(int64_t B, int64_t T, int64_t H);
 
+struct Wkv7FwdArgs {
+  int64_t B, T, H, K;
+  const void* r;
+  const void* w;
+  const void* k;
+  const void* v;
+  const void* a;
+  const void* b;
+  const float* init_state;
+  float* final_state;
+  void* o;
+};
+
 // Record `why` as the calling thread's wkv_last_error() message.
 void set_last_error(const char* why);
 
@@ -169,6 +182,7 @@ wkv_status launch_wkv4_state_init(int64_t S, int64_t C, float* state, cudaStream
 wkv_status launch_wkv4_chunk_step(const Wkv4ChunkArgs& a, cudaStream_t stream, unsigned* err, const char** why);
 wkv_status launch_wkv6_forward(const Wkv6FwdArgs& a, cudaStream_t stream, unsigned* err, const char** why);
 wkv_status launch_wkv6_backward(const Wkv6BwdArgs& a, cudaStream_t stream, unsigned* err, const char** why);
+wkv_status launch_wkv7_forward(const Wkv7FwdArgs& a, cudaStream_t stream, unsigned* err, const char** why);
 wkv_status launch_wait_selfcheck(int64_t limit_ns, cudaStream_t stream, unsigned* err, const char** why);
 
 }  // namespace wkv

@@ -40,6 +40,7 @@ SIGNATURES = {
     "wkv4_backward_noalloc": (_int, [_i64, _i64, _i64, _int] + [_vp] * 11),
     "wkv6_backward_workspace_bytes": (_sz, [_i64, _i64, _i64, _i64]),
     "wkv_wait_selfcheck": (_int, [_i64, _vp]),
+    "wkv7_forward": (_int, [_i64, _i64, _i64, _i64, _int] + [_vp] * 10),
     "wkv6_backward": (_int, [_i64, _i64, _i64, _i64, _int] + [_vp] * 7 + [_i64] + [_vp] * 9 + [_sz, _vp]),
 }
 
@@ -331,3 +332,26 @@ def wkv6_backward(r, k, v, w, u, dout, init_state: Optional[torch.Tensor] = None
                               _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(r)),
            "wkv6_backward")
     return gr, gk, gv, glogw, gu, g_init
+
+
+def wkv7_forward(r, w, k, v, a, b, init_state: Optional[torch.Tensor] = None, *, head_size: int = 64,
+                 want_final_state: bool = True, o=None, final_state=None):
+    """RWKV-7 generalized delta rule forward. r, w, k, v, a, b: [B, T, H*K]
+    bf16 (w the decay in log space); init_state: [B, H, K, K] float32
+    (indexed [b][h][key][value]) or None. Returns (o, final_state or None)."""
+    B, T, HK = r.shape
+    K = head_size
+    if HK % K:
+        raise ValueError("hidden size must be a multiple of head_size")
+    H = HK // K
+    dev = r.device
+    for name, t in (("r", r), ("w", w), ("k", k), ("v", v), ("a", a), ("b", b)):
+        _want(t, name, dtype=r.dtype, shape=r.shape, device=dev)
+    if init_state is not None:
+        _want(init_state, "init_state", dtype=torch.float32, shape=(B, H, K, K), device=dev)
+    o = torch.empty_like(r) if o is None else o
+    if want_final_state and final_state is None:
+        final_state = torch.empty((B, H, K, K), dtype=torch.float32, device=dev)
+    _check(_lib.wkv7_forward(B, T, H, K, _dtype_code(r), _ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(a), _ptr(b),
+                             _ptr(init_state), _ptr(final_state), _ptr(o), _stream(r)), "wkv7_forward")
+    return o, final_state

@@ -126,6 +126,12 @@ def test_chunk_and_wkv6_argument_errors(W):
     assert wb6(wsp=None) == W.WKV_ERR_INVALID_ARG
     assert wb6(init=FAKE, ns=3) == W.WKV_ERR_INVALID_ARG      # n_state neither 1 nor B
     assert wb6(H=0) == W.WKV_OK
+    wk7 = lambda B=1, T=4, H=2, K=64, dt=1: L.wkv7_forward(B, T, H, K, dt, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                                           None, None, FAKE, None)
+    assert wk7(K=32) == W.WKV_ERR_UNSUPPORTED
+    assert wk7(dt=0) == W.WKV_ERR_UNSUPPORTED
+    assert wk7(T=-1) == W.WKV_ERR_INVALID_ARG
+    assert wk7(B=0) == W.WKV_OK
     assert L.wkv_wait_selfcheck(0, None) == W.WKV_ERR_INVALID_ARG
     assert L.wkv_wait_selfcheck(20_000_000_000, None) == W.WKV_ERR_INVALID_ARG
 
