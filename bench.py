@@ -64,7 +64,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the secondary workloads (larger shapes, chunk step, RWKV-6)")
-    ap.add_argument("--kernel", choices=["wkv4_fwd", "wkv4_bwd", "wkv6_fwd", "wkv6_bwd", "wkv4_chunk"],
+    ap.add_argument("--kernel", choices=["wkv4_fwd", "wkv4_bwd", "wkv6_fwd", "wkv6_bwd", "wkv7_fwd", "wkv4_chunk"],
                     help="profiling mode: run only this kernel --steps times on --workload (no JSON line)")
     ap.add_argument("--workload", default=None,
                     help="with --kernel: a recipe name of synth (RWKV-4 or RWKV-6), optionally resized "
@@ -421,6 +421,29 @@ def secondary(dev, flush, peak):
                                   "bwd_ms": tb6, "bwd_GBps": 18 * n6 / (tb6 * 1e-3) / 1e9,
                                   "bwd_frac": 18 * n6 / (tb6 * 1e-3) / 1e9 / peak}
     del do6, ws6, go6
+
+    # RWKV-7 generalized delta rule forward (same shape); bytes: r, w, k, v, a, b in, o out (bf16)
+    rec7 = synth.WKV7_RECIPES["wkv7_fwd_bf16_c2048"]
+    g.manual_seed(0)
+    mk7 = lambda: torch.randn(rec7.B, rec7.T, rec7.H * rec7.K, device=dev, generator=g)
+    w7 = (-torch.exp(mk7() * rec7.d_std + rec7.d_mean)).to(torch.bfloat16)
+    kap = torch.randn(rec7.B, rec7.T, rec7.H, rec7.K, device=dev, generator=g)
+    kap = (kap / kap.norm(dim=-1, keepdim=True)).reshape(rec7.B, rec7.T, rec7.H * rec7.K)
+    a7 = (-kap).to(torch.bfloat16)
+    b7 = (kap * (torch.rand(kap.shape, device=dev, generator=g) * (rec7.lr_hi - rec7.lr_lo) + rec7.lr_lo)).to(
+        torch.bfloat16)
+    del kap
+    r7, k7, v7 = (mk7().to(torch.bfloat16) for _ in range(3))
+    o7 = torch.empty_like(r7)
+    fs7 = torch.empty(rec7.B, rec7.H, rec7.K, rec7.K, device=dev)
+    f7 = lambda: wkv.wkv7_forward(r7, w7, k7, v7, a7, b7, o=o7, final_state=fs7)
+    f7()
+    t7 = _events_ms(f7, 3, flush, stream)
+    n7 = rec7.B * rec7.T * rec7.H * rec7.K
+    res["wkv7_fwd_bf16_c2048"] = {"B": rec7.B, "T": rec7.T, "H": rec7.H, "K": rec7.K, "fwd_ms": t7,
+                                  "GBps": 14 * n7 / (t7 * 1e-3) / 1e9, "frac": 14 * n7 / (t7 * 1e-3) / 1e9 / peak,
+                                  "Gtokch_per_s": n7 / (t7 * 1e-3) / 1e9}
+    del r7, k7, v7, w7, a7, b7, o7, fs7
     assert wkv.device_error(reset=True) == 0, "a kernel recorded a device-side error"
     return res
 
@@ -634,6 +657,18 @@ def run_kernel_only(args):
             wkv.wkv4_state_init(S, C, dev, state=state)
             for kc, vc, cu in calls:
                 wkv.wkv4_chunk_step(w, u, kc, vc, cu, state)
+    elif args.kernel == "wkv7_fwd":
+        rec7 = synth.WKV7_RECIPES[name or "wkv7_fwd_bf16_c2048"]
+        if resize:
+            rec7 = rec7.with_shape(*[int(x) for x in resize.split(",")])
+        shape = (rec7.B, rec7.T, rec7.H * rec7.K)
+        w7 = (-torch.exp(torch.randn(shape, device=dev, generator=g) * rec7.d_std + rec7.d_mean)).to(torch.bfloat16)
+        kap = torch.randn(rec7.B, rec7.T, rec7.H, rec7.K, device=dev, generator=g)
+        kap = (kap / kap.norm(dim=-1, keepdim=True)).reshape(shape)
+        a7, b7 = (-kap).to(torch.bfloat16), (kap * torch.rand(shape, device=dev, generator=g)).to(torch.bfloat16)
+        r7, k7, v7 = (torch.randn(shape, device=dev, generator=g).to(torch.bfloat16) for _ in range(3))
+        for _ in range(args.steps):
+            wkv.wkv7_forward(r7, w7, k7, v7, a7, b7)
     elif args.kernel in ("wkv6_fwd", "wkv6_bwd"):
         rec = synth.WKV6_RECIPES[name or "wkv6_fwd_bf16_c2048"]
         if resize:
