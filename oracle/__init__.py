@@ -164,6 +164,28 @@ def wkv4_backward(w, u, k, v, gy, return_reverse_gw: bool = False, _lib=None):
     return (gk, gv, gw, gu, gwr) if return_reverse_gw else (gk, gv, gw, gu)
 
 
+def _sigmoid(x):
+    return 1.0 / (1.0 + np.exp(-x))
+
+
+def wkv4_forward_gated(w, u, k, v, r, _lib=None):
+    """The gated output of RWKV_TimeMix.forward ("代码连连看——RWKV", section
+    RWKV_TimeMix: rwkv = sigmoid(r) * RUN_CUDA(...)): sigmoid(r) * y in fp64,
+    y the WKV above. r: [B, T, C]."""
+    return _sigmoid(_f64(r)) * wkv4_forward(w, u, k, v, _lib=_lib)
+
+
+def wkv4_backward_gated(w, u, k, v, r, g, _lib=None):
+    """Gradients of L = sum(g * sigmoid(r) * y) in fp64 by the chain rule:
+    with s = sigmoid(r), the WKV sees gy = g * s, and dL/dr = g * y * s (1 - s).
+    Returns (gk, gv, gr, gw, gu)."""
+    r, g = _f64(r), _f64(g)
+    s = _sigmoid(r)
+    y = wkv4_forward(w, u, k, v, _lib=_lib)
+    gk, gv, gw, gu = wkv4_backward(w, u, k, v, g * s, _lib=_lib)
+    return gk, gv, g * y * s * (1.0 - s), gw, gu
+
+
 def wkv6_forward(r, k, v, w, u, init_state=None, state_map=None, _lib=None):
     """RWKV-6 head-state WKV forward in fp64.
 

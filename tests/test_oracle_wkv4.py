@@ -201,3 +201,46 @@ def test_final_state(oracle):
             sc = np.exp(st["kmax"][b, c])
             np.testing.assert_allclose(st["a_end"][b, c] * sc, a, rtol=1e-12)
             np.testing.assert_allclose(st["b_end"][b, c] * sc, bb, rtol=1e-12)
+
+
+def test_gated_backward_matches_finite_differences(oracle):
+    """sigmoid(r) * WKV (the gate of RWKV_TimeMix.forward): every gradient of
+    L = sum(g * sigmoid(r) * y), r included, against central differences."""
+    rng = np.random.default_rng(41)
+    B, T, C = 1, 6, 3
+    w = np.exp(rng.uniform(-3, 1, size=C))
+    u = rng.uniform(-1, 1, size=C)
+    k, v, r, g = (rng.normal(size=(B, T, C)) for _ in range(4))
+    gk, gv, gr, gw, gu = oracle.wkv4_backward_gated(w, u, k, v, r, g)
+
+    def loss(w_, u_, k_, v_, r_):
+        return float((g * oracle.wkv4_forward_gated(w_, u_, k_, v_, r_)).sum())
+
+    def fd(args, i, idx):
+        a = [np.array(x, dtype=np.float64) for x in args]
+        x0 = a[i][idx]
+        hh = 1e-5 * max(1.0, abs(x0))
+        a[i][idx] = x0 + hh
+        lp = loss(*a)
+        a[i][idx] = x0 - hh
+        lm = loss(*a)
+        return (lp - lm) / (2 * hh)
+
+    args = (w, u, k, v, r)
+    for name, got, i in (("gk", gk, 2), ("gv", gv, 3), ("gr", gr, 4)):
+        num = np.array([fd(args, i, idx) for idx in np.ndindex(*k.shape)]).reshape(k.shape)
+        assert _rel(got, num) < 1e-6, name
+    assert _rel(gw, np.array([fd(args, 0, (c,)) for c in range(C)])) < 1e-6
+    assert _rel(gu, np.array([fd(args, 1, (c,)) for c in range(C)])) < 1e-6
+
+
+def test_gate_limits(oracle):
+    """r -> +inf leaves the WKV unchanged; r = 0 halves it."""
+    rng = np.random.default_rng(42)
+    B, T, C = 2, 9, 4
+    w = np.exp(rng.uniform(-3, 1, size=C))
+    u = rng.uniform(-1, 1, size=C)
+    k, v = rng.normal(size=(B, T, C)), rng.normal(size=(B, T, C))
+    y = oracle.wkv4_forward(w, u, k, v)
+    assert _rel(oracle.wkv4_forward_gated(w, u, k, v, np.full(k.shape, 60.0)), y) < 1e-15
+    assert _rel(oracle.wkv4_forward_gated(w, u, k, v, np.zeros(k.shape)), 0.5 * y) < 1e-15
