@@ -64,7 +64,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the secondary workloads (larger shapes, chunk step, RWKV-6)")
-    ap.add_argument("--kernel", choices=["wkv4_fwd", "wkv4_bwd", "wkv6_fwd", "wkv6_bwd", "wkv7_fwd", "wkv4_chunk"],
+    ap.add_argument("--kernel", choices=["wkv4_fwd", "wkv4_bwd", "wkv4_fwd_gated", "wkv4_bwd_gated", "wkv6_fwd",
+                                         "wkv6_bwd", "wkv7_fwd", "wkv4_chunk"],
                     help="profiling mode: run only this kernel --steps times on --workload (no JSON line)")
     ap.add_argument("--workload", default=None,
                     help="with --kernel: a recipe name of synth (RWKV-4 or RWKV-6), optionally resized "
@@ -311,6 +312,22 @@ def secondary(dev, flush, peak):
         res[name] = {"B": B, "T": T, "C": C, "dtype": rec.dtype, "fwd_ms": tf, "bwd_ms": tb,
                      "fwd_GBps": gf, "bwd_GBps": gb, "fwd_frac": gf / peak, "bwd_frac": gb / peak,
                      "fwd_bwd_Gtokch_per_s": n / ((tf + tb) * 1e-3) / 1e9}
+        if name.endswith("c4096"):
+            # the time-mix gate sigmoid(r) * WKV fused in: one more input (r)
+            # forward, one more input and output (r, gr) backward
+            r = (torch.randn(B, T, C, device=dev, generator=g) * 2.0).to(dt)
+            gr = torch.empty_like(k)
+            fg = lambda: wkv.wkv4_forward_gated(w, u, k, v, r, y=y, ckpt=ck)
+            bg = lambda: wkv.wkv4_backward_gated(w, u, k, v, r, gy, ck, gk=gk, gv=gv, gr=gr, gw=gw, gu=gu,
+                                                 workspace=ws)
+            fg(); bg()
+            tfg = _events_ms(fg, 5, flush, stream)
+            tbg = _events_ms(bg, 5, flush, stream)
+            gfg, gbg = 4 * es * n / (tfg * 1e-3) / 1e9, 7 * es * n / (tbg * 1e-3) / 1e9
+            res[name + "_gated"] = {"fwd_ms": tfg, "bwd_ms": tbg, "fwd_GBps": gfg, "bwd_GBps": gbg,
+                                    "fwd_frac": gfg / peak, "bwd_frac": gbg / peak,
+                                    "fwd_bwd_Gtokch_per_s": n / ((tfg + tbg) * 1e-3) / 1e9}
+            del r, gr
         del k, v, gy, y, gk, gv, ck, ws
         torch.cuda.empty_cache()
 
@@ -703,10 +720,15 @@ def run_kernel_only(args):
         gw, gu = torch.empty(C, device=dev), torch.empty(C, device=dev)
         ck = torch.empty(wkv.ckpt_shape(B, T, C), device=dev)
         ws = torch.empty(max(16, wkv.wkv4_backward_workspace_bytes(B, T, C, True)), dtype=torch.uint8, device=dev)
+        r = (torch.randn(B, T, C, device=dev, generator=g) * 2.0).to(dt) if "gated" in args.kernel else None
         wkv.wkv4_forward(w, u, k, v, y=y, ckpt=ck)
         for _ in range(args.steps):
             if args.kernel == "wkv4_fwd":
                 wkv.wkv4_forward(w, u, k, v, y=y, ckpt=ck)
+            elif args.kernel == "wkv4_fwd_gated":
+                wkv.wkv4_forward_gated(w, u, k, v, r, y=y, ckpt=ck)
+            elif args.kernel == "wkv4_bwd_gated":
+                wkv.wkv4_backward_gated(w, u, k, v, r, gy, ck, gk=gk, gv=gv, gw=gw, gu=gu, workspace=ws)
             else:
                 wkv.wkv4_backward(w, u, k, v, gy, ck, gk=gk, gv=gv, gw=gw, gu=gu, workspace=ws)
     torch.cuda.synchronize()

@@ -151,6 +151,41 @@ wkv_status wkv4_backward(int64_t B, int64_t T, int64_t C, int dtype,
                          void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * RWKV-4 WKV forward with the time-mix gate fused into its output: the
+ * receptance gate of RWKV_TimeMix ("代码连连看——RWKV", section
+ * RWKV_TimeMix: the block output is sigmoid(r) * WKV before the output
+ * projection), y = sigmoid(r) * wkv4_forward(...), in one pass over HBM.
+ *   r           [B][T][C] of `dtype`: the gate input (receptance before the
+ *               sigmoid), read-only.
+ *   y           [B][T][C] of `dtype`, required (the gated output).
+ *   ckpt        as for wkv4_forward (optional): the checkpoints do not
+ *               depend on r.
+ * Other arguments, errors and limits are those of wkv4_forward. r and y
+ * must not overlap.
+ */
+wkv_status wkv4_forward_gated(int64_t B, int64_t T, int64_t C, int dtype,
+                              const float *w, const float *u,
+                              const void *k, const void *v, const void *r,
+                              void *y, float *ckpt, void *stream);
+
+/*
+ * Gradients of L = sum(gy * y) for y = wkv4_forward_gated(...): with
+ * s = sigmoid(r) and wkv the ungated output, the WKV sees the output
+ * gradient gy * s, and dL/dr = gy * wkv * s * (1 - s).
+ *   r           [B][T][C] of `dtype`, the gate input of the forward.
+ *   gy          [B][T][C] of `dtype`, gradient of the gated output.
+ *   gr          [B][T][C] of `dtype`, written: dL/dr.
+ *   ckpt, gk, gv, gw, gu, workspace: as for wkv4_backward (the workspace
+ *               size is wkv4_backward_workspace_bytes for the same shape).
+ */
+wkv_status wkv4_backward_gated(int64_t B, int64_t T, int64_t C, int dtype,
+                               const float *w, const float *u,
+                               const void *k, const void *v, const void *r,
+                               const void *gy, const float *ckpt,
+                               void *gk, void *gv, void *gr, float *gw, float *gu,
+                               void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Set S slot states [S][5][C] float32 to the empty past:
  * aa = bb = 0, base = -1e38, n = 0, ref = 0 (ref is set by the first token).
  */

@@ -157,8 +157,9 @@ WKV_EXPORT size_t wkv4_ckpt_floats(int64_t B, int64_t T, int64_t C) {
   return (size_t)B * (size_t)ceil_div(T, WKV4_CKPT_LEN) * 3u * (size_t)C;
 }
 
-WKV_EXPORT wkv_status wkv4_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, const float* u,
-                                   const void* k, const void* v, void* y, float* ckpt, void* stream) {
+// r: the gate input of the gated entry point, null for the plain one
+static wkv_status wkv4_forward_any(int64_t B, int64_t T, int64_t C, int dtype, const float* w, const float* u,
+                                   const void* k, const void* v, const void* r, void* y, float* ckpt, void* stream) {
   if (wkv_status s = check_act(B, T, C, dtype)) return s;
   if (B == 0 || T == 0 || C == 0) return WKV_OK;
   WKV_REQUIRE_PTR(w, "w");
@@ -172,8 +173,25 @@ WKV_EXPORT wkv_status wkv4_forward(int64_t B, int64_t T, int64_t C, int dtype, c
   if (wkv_status s = device_error_ptr(&err)) return s;
   const char* why = "";
   Wkv4FwdArgs a{B, T, C, dtype, w, u, k, v, y, ckpt};
+  a.r = y ? r : nullptr;  // without y there is nothing to gate
   wkv_status s = launch_wkv4_forward(a, static_cast<cudaStream_t>(stream), err, &why);
   return s == WKV_OK ? s : fail(s, why);
+}
+
+WKV_EXPORT wkv_status wkv4_forward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, const float* u,
+                                   const void* k, const void* v, void* y, float* ckpt, void* stream) {
+  return wkv4_forward_any(B, T, C, dtype, w, u, k, v, nullptr, y, ckpt, stream);
+}
+
+WKV_EXPORT wkv_status wkv4_forward_gated(int64_t B, int64_t T, int64_t C, int dtype, const float* w,
+                                         const float* u, const void* k, const void* v, const void* r, void* y,
+                                         float* ckpt, void* stream) {
+  if (wkv_status s = check_act(B, T, C, dtype)) return s;
+  if (B > 0 && T > 0 && C > 0) {
+    WKV_REQUIRE_PTR(r, "r");
+    WKV_REQUIRE_PTR(y, "y");
+  }
+  return wkv4_forward_any(B, T, C, dtype, w, u, k, v, r, y, ckpt, stream);
 }
 
 WKV_EXPORT size_t wkv4_backward_workspace_bytes(int64_t B, int64_t T, int64_t C, int has_ckpt) {
@@ -185,10 +203,11 @@ WKV_EXPORT size_t wkv4_backward_workspace_bytes(int64_t B, int64_t T, int64_t C,
   return bytes;
 }
 
-WKV_EXPORT wkv_status wkv4_backward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, const float* u,
-                                    const void* k, const void* v, const void* gy, const float* ckpt, void* gk,
-                                    void* gv, float* gw, float* gu, void* workspace, size_t workspace_bytes,
-                                    void* stream) {
+// r, gr: the gate input and its gradient (gated entry point), null otherwise
+static wkv_status wkv4_backward_any(int64_t B, int64_t T, int64_t C, int dtype, const float* w, const float* u,
+                                    const void* k, const void* v, const void* r, const void* gy, const float* ckpt,
+                                    void* gk, void* gv, void* gr, float* gw, float* gu, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
   if (wkv_status s = check_act(B, T, C, dtype)) return s;
   if (C == 0) return WKV_OK;
   WKV_REQUIRE_PTR(gw, "gw");
@@ -225,8 +244,32 @@ WKV_EXPORT wkv_status wkv4_backward(int64_t B, int64_t T, int64_t C, int dtype, 
     ck = regen;
   }
   Wkv4BwdArgs a{B, T, C, dtype, w, u, k, v, gy, ck, gk, gv, gw, gu, part};
+  a.r = r;
+  a.gr = gr;
   wkv_status s = launch_wkv4_backward(a, st, err, &why);
   return s == WKV_OK ? s : fail(s, why);
+}
+
+WKV_EXPORT wkv_status wkv4_backward(int64_t B, int64_t T, int64_t C, int dtype, const float* w, const float* u,
+                                    const void* k, const void* v, const void* gy, const float* ckpt, void* gk,
+                                    void* gv, float* gw, float* gu, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+  return wkv4_backward_any(B, T, C, dtype, w, u, k, v, nullptr, gy, ckpt, gk, gv, nullptr, gw, gu, workspace,
+                           workspace_bytes, stream);
+}
+
+WKV_EXPORT wkv_status wkv4_backward_gated(int64_t B, int64_t T, int64_t C, int dtype, const float* w,
+                                          const float* u, const void* k, const void* v, const void* r,
+                                          const void* gy, const float* ckpt, void* gk, void* gv, void* gr,
+                                          float* gw, float* gu, void* workspace, size_t workspace_bytes,
+                                          void* stream) {
+  if (wkv_status s = check_act(B, T, C, dtype)) return s;
+  if (B > 0 && T > 0 && C > 0) {
+    WKV_REQUIRE_PTR(r, "r");
+    WKV_REQUIRE_PTR(gr, "gr");
+  }
+  return wkv4_backward_any(B, T, C, dtype, w, u, k, v, r, gy, ckpt, gk, gv, gr, gw, gu, workspace, workspace_bytes,
+                           stream);
 }
 
 WKV_EXPORT wkv_status wkv4_state_init(int64_t S, int64_t C, float* state, void* stream) {

@@ -81,20 +81,35 @@ template <class E>
 constexpr bool bwd_smem_stash() {
   return WKV4_BWD_SMEM_STASH && (sizeof(E) == 2 || WKV4_BWD_SMEM_STASH_F32);
 }
-template <bool S>
+// GATE: the gated kernel's ring carries a fourth tile (r); its stash drops
+// v (read again from the ring) so that a warp's shared memory stays the same.
+template <bool S, bool GATE>
 struct Wkv4Stash {
   float4 ab[kBwdL][32];  // (aa.x, aa.y, bb.x, bb.y) of each step, per lane
   float4 zv[kBwdL][32];  // (z1.x, z1.y, v.x, v.y): v unpacked once
 };
 template <>
-struct Wkv4Stash<false> {};
+struct Wkv4Stash<true, true> {
+  float4 ab[kBwdL][32];
+  float2 zv[kBwdL][32];  // z1 only
+};
+template <bool GATE>
+struct Wkv4Stash<false, GATE> {};
 
+template <class E, int STAGES, bool GATE>
+struct Wkv4BwdGateRing {
+  E r[STAGES][kBwdL][kBwdCh];
+};
 template <class E, int STAGES>
+struct Wkv4BwdGateRing<E, STAGES, false> {};
+
+template <class E, int STAGES, bool GATE>
 struct alignas(128) Wkv4BwdSmem {
   E k[STAGES][kBwdL][kBwdCh];
   E v[STAGES][kBwdL][kBwdCh];
   E gy[STAGES][kBwdL][kBwdCh];
-  Wkv4Stash<bwd_smem_stash<E>()> stash;
+  Wkv4BwdGateRing<E, STAGES, GATE> g;
+  Wkv4Stash<bwd_smem_stash<E>(), GATE> stash;
   uint64_t full[STAGES];
   float2 carry[5][32];  // this segment's local carry A, B, A', B' and its product of f1
 };
@@ -111,11 +126,13 @@ __device__ __forceinline__ float2 neg2(float2 a) { return make_float2(-a.x, -a.y
 // the forward quantities of the token: the state (aa, bb) before it, its
 // absorb exponent z (z1 of the forward), v and gy. FULL: also write gk, gv
 // at gkp, gvp and add the token's gw, gu terms (gwn holds -gw); otherwise
-// only fold the token into the carries and fprod.
-template <bool FULL, class E>
+// only fold the token into the carries and fprod. GATE: gy is the gradient
+// of the gated output sigmoid(r) * y; the step writes
+// dL/dr = gy y s (1 - s) at grp (s = sigmoid(r)) and carries gy s on as y's.
+template <bool FULL, bool GATE, class E>
 __device__ __forceinline__ void wkv4_bwd_rstep(float2& A, float2& B, float2& Ap, float2& Bp, float2& fprod,
-                                               float2& gwn, float2& gu_acc, float2 vv, float2 g, float2 aa,
-                                               float2 bb, float2 z, float2 uw2, E* gkp, E* gvp) {
+                                               float2& gwn, float2& gu_acc, float2 vv, float2 g, float2 rr,
+                                               float2 aa, float2 bb, float2 z, float2 uw2, E* gkp, E* gvp, E* grp) {
   // output of the token, in units of the past's exponent P: weight
   // e = 2^{u + k - P} = 2^{z1 + u - w} of the current token (capped as in
   // the forward), D = 2^P (bb + e), y = (aa + e v) / (bb + e)
@@ -128,6 +145,11 @@ __device__ __forceinline__ void wkv4_bwd_rstep(float2& A, float2& B, float2& Ap,
   const bool kx = z.x <= 0.f, ky = z.y <= 0.f;
   const float2 f1 = make_float2(kx ? 1.f : ea.x, ky ? 1.f : ea.y);
   const float2 f2 = make_float2(kx ? ea.x : 1.f, ky ? ea.y : 1.f);
+  if constexpr (GATE) {
+    const float2 sg = sigmoid2(rr);
+    if constexpr (FULL) st_pair(grp, mul2(mul2(g, yv), mul2(sg, sub2(splat2(1.f), sg))));
+    g = mul2(g, sg);
+  }
   const float2 ag = mul2(g, rd);  // gy 2^P / D
   if constexpr (FULL) {
     const float2 rg = mul2(ag, e);  // gy rho, rho = e^{u+k} / D
@@ -155,12 +177,12 @@ __device__ __forceinline__ void wkv4_bwd_rstep(float2& A, float2& B, float2& Ap,
 // accumulates -gw. WHOLE (n == kBwdL): the reverse steps are not
 // predicated, so the compiler can overlap the independent parts of
 // consecutive steps; the recompute loop always is.
-template <bool FULL, bool WHOLE, class E, bool S>
+template <bool FULL, bool WHOLE, bool GATE, class E, bool S>
 __device__ __forceinline__ void wkv4_bwd_interval(const E (*ks)[kBwdCh], const E (*vs)[kBwdCh],
-                                                  const E (*gs)[kBwdCh], Wkv4Stash<S>& sx, int lane, int n,
-                                                  Wkv4State2 st, float2 ref, float2 uw2, float2 w2, Wkv4Carry2& cr,
-                                                  float2& fprod, float2& gwn, float2& gu_acc, E* gkl, E* gvl,
-                                                  int C) {
+                                                  const E (*gs)[kBwdCh], const E (*rs)[kBwdCh],
+                                                  Wkv4Stash<S, GATE>& sx, int lane, int n, Wkv4State2 st,
+                                                  float2 ref, float2 uw2, float2 w2, Wkv4Carry2& cr, float2& fprod,
+                                                  float2& gwn, float2& gu_acc, E* gkl, E* gvl, E* grl, int C) {
   // forward recompute over the interval: state before each token and the
   // token's absorb exponent z1 (the forward's own rounding of it)
   constexpr int kReg = S ? 1 : kBwdL;
@@ -173,7 +195,10 @@ __device__ __forceinline__ void wkv4_bwd_interval(const E (*ks)[kBwdCh], const E
       const float2 z1 = wkv4_absorb2(st, wkv4_key2(ld_pair(&ks[jj][2 * lane]), ref), vj, w2);
       if constexpr (S) {
         sx.ab[jj][lane] = make_float4(aa.x, aa.y, bb.x, bb.y);
-        sx.zv[jj][lane] = make_float4(z1.x, z1.y, vj.x, vj.y);
+        if constexpr (GATE)
+          sx.zv[jj][lane] = z1;
+        else
+          sx.zv[jj][lane] = make_float4(z1.x, z1.y, vj.x, vj.y);
       } else {
         saa[jj] = aa;
         sbb[jj] = bb;
@@ -186,22 +211,29 @@ __device__ __forceinline__ void wkv4_bwd_interval(const E (*ks)[kBwdCh], const E
   for (int jj = kBwdL - 1; jj >= 0; --jj) {
     if (WHOLE || jj < n) {
       const float2 g = ld_pair(&gs[jj][2 * lane]);
+      const float2 rr = GATE ? ld_pair(&rs[jj][2 * lane]) : splat2(0.f);
       float2 aa, bb, z, vv;
       if constexpr (S) {
         const float4 ab = sx.ab[jj][lane];
-        const float4 zv = sx.zv[jj][lane];
         aa = make_float2(ab.x, ab.y);
         bb = make_float2(ab.z, ab.w);
-        z = make_float2(zv.x, zv.y);
-        vv = make_float2(zv.z, zv.w);
+        if constexpr (GATE) {
+          z = sx.zv[jj][lane];
+          vv = ld_pair(&vs[jj][2 * lane]);
+        } else {
+          const float4 zv = sx.zv[jj][lane];
+          z = make_float2(zv.x, zv.y);
+          vv = make_float2(zv.z, zv.w);
+        }
       } else {
         aa = saa[jj];
         bb = sbb[jj];
         z = sz[jj];
         vv = ld_pair(&vs[jj][2 * lane]);
       }
-      wkv4_bwd_rstep<FULL>(A, B, Ap, Bp, fprod, gwn, gu_acc, vv, g, aa, bb, z, uw2, gkl + (int64_t)jj * C,
-                           gvl + (int64_t)jj * C);
+      wkv4_bwd_rstep<FULL, GATE>(A, B, Ap, Bp, fprod, gwn, gu_acc, vv, g, rr, aa, bb, z, uw2,
+                                 gkl + (int64_t)jj * C, gvl + (int64_t)jj * C,
+                                 GATE ? grl + (int64_t)jj * C : nullptr);
     }
   }
   cr = {A, B, Ap, Bp};
@@ -220,19 +252,22 @@ __device__ __forceinline__ void wkv4_carry_fold(float& A, float& B, float& Ap, f
   Bp = nBp;
 }
 
-template <class E, int STAGES, int NSEG, int NW>
+template <class E, int STAGES, int NSEG, int NW, bool GATE>
 __global__ void __launch_bounds__(32 * NW, NSEG == 1 ? 8 : 1) wkv4_bwd_kernel(const __grid_constant__ CUtensorMap tk,
                                                            const __grid_constant__ CUtensorMap tv,
-                                                           const __grid_constant__ CUtensorMap tg, int T, int C,
+                                                           const __grid_constant__ CUtensorMap tg,
+                                                           const __grid_constant__ CUtensorMap tr, int T, int C,
                                                            int ncb, int ngroups, const float* __restrict__ w,
                                                            const float* __restrict__ u, const E* __restrict__ kraw,
                                                            const float* __restrict__ ckpt, E* __restrict__ gk,
-                                                           E* __restrict__ gv, float* __restrict__ part_gw,
+                                                           E* __restrict__ gv, E* __restrict__ gr,
+                                                           float* __restrict__ part_gw,
                                                            float* __restrict__ part_gu, unsigned* err) {
   extern __shared__ __align__(128) unsigned char wkv4_bwd_dsmem[];
   // each warp is an independent lane group with its own ring and barriers
-  Wkv4BwdSmem<E, STAGES>& sm = reinterpret_cast<Wkv4BwdSmem<E, STAGES>*>(wkv4_bwd_dsmem)[threadIdx.x / 32];
-  constexpr uint32_t kStageBytes = 3u * kBwdL * kBwdCh * sizeof(E);
+  Wkv4BwdSmem<E, STAGES, GATE>& sm =
+      reinterpret_cast<Wkv4BwdSmem<E, STAGES, GATE>*>(wkv4_bwd_dsmem)[threadIdx.x / 32];
+  constexpr uint32_t kStageBytes = (GATE ? 4u : 3u) * kBwdL * kBwdCh * sizeof(E);
   constexpr int kPasses = NSEG > 1 ? 2 : 1;
 
   const int lane = threadIdx.x % 32;
@@ -260,11 +295,13 @@ __global__ void __launch_bounds__(32 * NW, NSEG == 1 ? 8 : 1) wkv4_bwd_kernel(co
     tma_load_3d(&sm.k[s][0][0], &tk, &sm.full[s], c0, t0, b);
     tma_load_3d(&sm.v[s][0][0], &tv, &sm.full[s], c0, t0, b);
     tma_load_3d(&sm.gy[s][0][0], &tg, &sm.full[s], c0, t0, b);
+    if constexpr (GATE) tma_load_3d(&sm.g.r[s][0][0], &tr, &sm.full[s], c0, t0, b);
   };
   if (lane == 0) {
     tma_prefetch_desc(&tk);
     tma_prefetch_desc(&tv);
     tma_prefetch_desc(&tg);
+    if constexpr (GATE) tma_prefetch_desc(&tr);
     for (int s = 0; s < STAGES; ++s) mbar_init(&sm.full[s], 1);
     mbar_init_fence();
     for (int qq = 0; qq < STAGES && qq < total; ++qq) issue(qq);
@@ -309,14 +346,17 @@ __global__ void __launch_bounds__(32 * NW, NSEG == 1 ? 8 : 1) wkv4_bwd_kernel(co
     const int64_t off = lane_off + (int64_t)i * kBwdL * C;
     E* gkp = kFull ? gk + off : nullptr;
     E* gvp = kFull ? gv + off : nullptr;
+    E* grp = kFull && GATE ? gr + off : nullptr;
+    const E (*rs)[kBwdCh] = nullptr;
+    if constexpr (GATE) rs = sm.g.r[s];
 #if WKV4_BWD_WHOLE
     if (n == kBwdL)
-      wkv4_bwd_interval<kFull, true>(sm.k[s], sm.v[s], sm.gy[s], sm.stash, lane, n, st, ref, uw2, w2, cr, fprod, gwn,
-                                        gu_acc, gkp, gvp, C);
+      wkv4_bwd_interval<kFull, true, GATE>(sm.k[s], sm.v[s], sm.gy[s], rs, sm.stash, lane, n, st, ref, uw2, w2, cr,
+                                           fprod, gwn, gu_acc, gkp, gvp, grp, C);
     else
 #endif
-      wkv4_bwd_interval<kFull, false>(sm.k[s], sm.v[s], sm.gy[s], sm.stash, lane, n, st, ref, uw2, w2, cr, fprod, gwn,
-                                         gu_acc, gkp, gvp, C);
+      wkv4_bwd_interval<kFull, false, GATE>(sm.k[s], sm.v[s], sm.gy[s], rs, sm.stash, lane, n, st, ref, uw2, w2, cr,
+                                            fprod, gwn, gu_acc, gkp, gvp, grp, C);
   };
 
   if constexpr (NSEG > 1) {
@@ -416,21 +456,25 @@ __global__ void __launch_bounds__(32 * kReduceWarps) wkv4_reduce_kernel(const fl
   }
 }
 
-template <class E, int STAGES, int NSEG, int NW>
+template <class E, int STAGES, int NSEG, int NW, bool GATE>
 static wkv_status run_bwd(const Wkv4BwdArgs& a, cudaStream_t stream, unsigned* err, const char** why) {
-  CUtensorMap tk, tv, tg;
+  CUtensorMap tk, tv, tg, tr;
   const CUtensorMapDataType ty = Elem<E>::tma_type;
   if (!encode_tmap_3d(&tk, a.k, ty, sizeof(E), a.C, a.T, a.B, kBwdCh, kBwdL, 1, why) ||
       !encode_tmap_3d(&tv, a.v, ty, sizeof(E), a.C, a.T, a.B, kBwdCh, kBwdL, 1, why) ||
       !encode_tmap_3d(&tg, a.gy, ty, sizeof(E), a.C, a.T, a.B, kBwdCh, kBwdL, 1, why))
+    return WKV_ERR_INVALID_ARG;
+  if (!GATE)
+    tr = tk;  // unused
+  else if (!encode_tmap_3d(&tr, a.r, ty, sizeof(E), a.C, a.T, a.B, kBwdCh, kBwdL, 1, why))
     return WKV_ERR_INVALID_ARG;
   const int ncb = (int)ceil_div(a.C, kBwdCh);
   const int ngroups = (int)(ncb * a.B);
   const int64_t rows = a.B * NSEG;
   float* part_gw = a.part;
   float* part_gu = a.part + rows * a.C;
-  auto kern = wkv4_bwd_kernel<E, STAGES, NSEG, NW>;
-  const size_t smem = NW * sizeof(Wkv4BwdSmem<E, STAGES>);
+  auto kern = wkv4_bwd_kernel<E, STAGES, NSEG, NW, GATE>;
+  const size_t smem = NW * sizeof(Wkv4BwdSmem<E, STAGES, GATE>);
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
     *why = "wkv4_backward: shared memory configuration failed";
@@ -455,9 +499,9 @@ static wkv_status run_bwd(const Wkv4BwdArgs& a, cudaStream_t stream, unsigned* e
     cfg.attrs = attr;
     cfg.numAttrs = 1;
   }
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tk, tv, tg, (int)a.T, (int)a.C, ncb, ngroups, a.w, a.u,
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tk, tv, tg, tr, (int)a.T, (int)a.C, ncb, ngroups, a.w, a.u,
                                      static_cast<const E*>(a.k), a.ckpt, static_cast<E*>(a.gk), static_cast<E*>(a.gv),
-                                     part_gw, part_gu, err);
+                                     static_cast<E*>(a.gr), part_gw, part_gu, err);
   if (e == cudaSuccess) {
     wkv4_reduce_kernel<<<(unsigned)ceil_div(a.C, 32), 32 * kReduceWarps, 0, stream>>>(part_gw, part_gu, (int)rows,
                                                                                      (int)a.C, a.gw, a.gu);
@@ -470,35 +514,40 @@ static wkv_status run_bwd(const Wkv4BwdArgs& a, cudaStream_t stream, unsigned* e
   return WKV_OK;
 }
 
-// Stages of the k/v/gy ring (one checkpoint interval each): four for bf16
-// (6 KB a stage), two for float32 (12 KB), so that the 7-8 one-warp CTAs an
-// SM holds still fit in shared memory.
-template <class E, int STAGES, int NSEG>
+// Stages of the k/v/gy ring (one checkpoint interval each): two for bf16
+// next to the stash (6 KB a stage, 8 KB gated), two for float32 (12 KB,
+// 16 KB gated), so that the 6-7 one-warp CTAs an SM holds still fit in
+// shared memory.
+template <class E, int STAGES, int NSEG, bool GATE>
 static wkv_status run_bwd_nw(const Wkv4BwdArgs& a, cudaStream_t stream, unsigned* err, const char** why) {
   switch (wkv4_warps_per_cta(a.B, a.C, NSEG)) {
-    case 4: return run_bwd<E, STAGES, NSEG, 4>(a, stream, err, why);
-    case 2: return run_bwd<E, STAGES, NSEG, 2>(a, stream, err, why);
-    default: return run_bwd<E, STAGES, NSEG, 1>(a, stream, err, why);
+    case 4: return run_bwd<E, STAGES, NSEG, 4, GATE>(a, stream, err, why);
+    case 2: return run_bwd<E, STAGES, NSEG, 2, GATE>(a, stream, err, why);
+    default: return run_bwd<E, STAGES, NSEG, 1, GATE>(a, stream, err, why);
   }
 }
 
-template <class E>
+template <class E, bool GATE>
 static wkv_status run_bwd_nseg(const Wkv4BwdArgs& a, cudaStream_t stream, unsigned* err, const char** why) {
   constexpr int kStages = sizeof(E) == 2 ? (bwd_smem_stash<E>() ? WKV4_BWD_STAGES_STASH : 4) : 2;
   switch (wkv4_bwd_segments(a.B, a.T, a.C)) {
 #if WKV4_MAX_SEGMENTS_ANY > 8
-    case 16: return run_bwd_nw<E, kStages, 16>(a, stream, err, why);
+    case 16: return run_bwd_nw<E, kStages, 16, GATE>(a, stream, err, why);
 #endif
-    case 8: return run_bwd_nw<E, kStages, 8>(a, stream, err, why);
-    case 4: return run_bwd_nw<E, kStages, 4>(a, stream, err, why);
-    case 2: return run_bwd_nw<E, kStages, 2>(a, stream, err, why);
-    default: return run_bwd<E, kStages, 1, 1>(a, stream, err, why);
+    case 8: return run_bwd_nw<E, kStages, 8, GATE>(a, stream, err, why);
+    case 4: return run_bwd_nw<E, kStages, 4, GATE>(a, stream, err, why);
+    case 2: return run_bwd_nw<E, kStages, 2, GATE>(a, stream, err, why);
+    default: return run_bwd<E, kStages, 1, 1, GATE>(a, stream, err, why);
   }
 }
 
 wkv_status launch_wkv4_backward(const Wkv4BwdArgs& a, cudaStream_t stream, unsigned* err, const char** why) {
-  if (a.dtype == WKV_BF16) return run_bwd_nseg<__nv_bfloat16>(a, stream, err, why);
-  return run_bwd_nseg<float>(a, stream, err, why);
+  if (a.r) {
+    if (a.dtype == WKV_BF16) return run_bwd_nseg<__nv_bfloat16, true>(a, stream, err, why);
+    return run_bwd_nseg<float, true>(a, stream, err, why);
+  }
+  if (a.dtype == WKV_BF16) return run_bwd_nseg<__nv_bfloat16, false>(a, stream, err, why);
+  return run_bwd_nseg<float, false>(a, stream, err, why);
 }
 
 }  // namespace wkv

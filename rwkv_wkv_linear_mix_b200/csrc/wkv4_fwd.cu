@@ -33,17 +33,27 @@ namespace wkv {
 // Channels one warp covers: 32 lanes x a pair each.
 constexpr int kFwdCh = WKV4_WARP_CH;
 
+// The gate input r rides in the same ring when the output is gated.
+template <class E, int LT, int STAGES, bool GATE>
+struct Wkv4GateRing {
+  E r[STAGES][LT][kFwdCh];
+};
 template <class E, int LT, int STAGES>
+struct Wkv4GateRing<E, LT, STAGES, false> {};
+
+template <class E, int LT, int STAGES, bool GATE>
 struct alignas(128) Wkv4FwdSmem {
   E k[STAGES][LT][kFwdCh];
   E v[STAGES][LT][kFwdCh];
+  Wkv4GateRing<E, LT, STAGES, GATE> g;
   uint64_t full[STAGES];
   float2 seg_aa[32], seg_bb[32], seg_P[32];  // this segment's own state (phase 1)
 };
 
-template <class E, int LT, int STAGES, int NSEG, int NW>
+template <class E, int LT, int STAGES, int NSEG, int NW, bool GATE>
 __global__ void __launch_bounds__(32 * NW) wkv4_fwd_kernel(const __grid_constant__ CUtensorMap tk,
                                                            const __grid_constant__ CUtensorMap tv,
+                                                           const __grid_constant__ CUtensorMap tr,
                                                            const E* __restrict__ kraw, int T, int C, int ncb,
                                                            int ngroups, const float* __restrict__ w,
                                                            const float* __restrict__ u, E* __restrict__ y,
@@ -51,8 +61,9 @@ __global__ void __launch_bounds__(32 * NW) wkv4_fwd_kernel(const __grid_constant
   static_assert(LT % WKV4_CKPT_LEN == 0, "a tile must hold whole checkpoint intervals");
   extern __shared__ __align__(128) unsigned char wkv4_fwd_dsmem[];
   // each warp is an independent lane group with its own ring and barriers
-  Wkv4FwdSmem<E, LT, STAGES>& sm = reinterpret_cast<Wkv4FwdSmem<E, LT, STAGES>*>(wkv4_fwd_dsmem)[threadIdx.x / 32];
-  constexpr uint32_t kStageBytes = 2u * LT * kFwdCh * sizeof(E);
+  Wkv4FwdSmem<E, LT, STAGES, GATE>& sm =
+      reinterpret_cast<Wkv4FwdSmem<E, LT, STAGES, GATE>*>(wkv4_fwd_dsmem)[threadIdx.x / 32];
+  constexpr uint32_t kStageBytes = (GATE ? 3u : 2u) * LT * kFwdCh * sizeof(E);
   constexpr int kPasses = NSEG > 1 ? 2 : 1;
 
   const int lane = threadIdx.x % 32;
@@ -78,10 +89,12 @@ __global__ void __launch_bounds__(32 * NW) wkv4_fwd_kernel(const __grid_constant
     mbar_arrive_expect_tx(&sm.full[s], kStageBytes);
     tma_load_3d(&sm.k[s][0][0], &tk, &sm.full[s], c0, t, b);
     tma_load_3d(&sm.v[s][0][0], &tv, &sm.full[s], c0, t, b);
+    if constexpr (GATE) tma_load_3d(&sm.g.r[s][0][0], &tr, &sm.full[s], c0, t, b);
   };
   if (lane == 0) {
     tma_prefetch_desc(&tk);
     tma_prefetch_desc(&tv);
+    if constexpr (GATE) tma_prefetch_desc(&tr);
     for (int s = 0; s < STAGES; ++s) mbar_init(&sm.full[s], 1);
     mbar_init_fence();
     for (int q = 0; q < STAGES && q < total; ++q) issue(q);
@@ -176,16 +189,18 @@ __global__ void __launch_bounds__(32 * NW) wkv4_fwd_kernel(const __grid_constant
 #pragma unroll 8
           for (int j2 = 0; j2 < WKV4_CKPT_LEN; ++j2) {
             const int j = jc + j2;
-            const float2 yv = wkv4_token2(st, wkv4_key2(ld_pair(&sm.k[s][j][2 * lane]), ref),
-                                          ld_pair(&sm.v[s][j][2 * lane]), u2, w2);
+            float2 yv = wkv4_token2(st, wkv4_key2(ld_pair(&sm.k[s][j][2 * lane]), ref),
+                                    ld_pair(&sm.v[s][j][2 * lane]), u2, w2);
+            if constexpr (GATE) yv = mul2(yv, sigmoid2(ld_pair(&sm.g.r[s][j][2 * lane])));
             if (yt) st_pair(yt + (int64_t)j * C, yv);
           }
         }
       } else {
         for (int j = 0; j < n; ++j) {
           if (j > 0 && j % WKV4_CKPT_LEN == 0 && ckl) write_ckpt(t0 + j);
-          const float2 yv = wkv4_token2(st, wkv4_key2(ld_pair(&sm.k[s][j][2 * lane]), ref),
-                                        ld_pair(&sm.v[s][j][2 * lane]), u2, w2);
+          float2 yv = wkv4_token2(st, wkv4_key2(ld_pair(&sm.k[s][j][2 * lane]), ref),
+                                  ld_pair(&sm.v[s][j][2 * lane]), u2, w2);
+          if constexpr (GATE) yv = mul2(yv, sigmoid2(ld_pair(&sm.g.r[s][j][2 * lane])));
           if (yt) st_pair(yt + (int64_t)j * C, yv);
         }
       }
@@ -201,17 +216,21 @@ __global__ void __launch_bounds__(32 * NW) wkv4_fwd_kernel(const __grid_constant
   if constexpr (NSEG > 1) cluster_wait_acquire();  // peers may still read this CTA's segment state
 }
 
-template <class E, int LT, int STAGES, int NSEG, int NW>
+template <class E, int LT, int STAGES, int NSEG, int NW, bool GATE>
 static wkv_status run_fwd(const Wkv4FwdArgs& a, cudaStream_t stream, unsigned* err, const char** why) {
-  CUtensorMap tk, tv;
+  CUtensorMap tk, tv, tr;
   const CUtensorMapDataType ty = Elem<E>::tma_type;
   if (!encode_tmap_3d(&tk, a.k, ty, sizeof(E), a.C, a.T, a.B, kFwdCh, LT, 1, why) ||
       !encode_tmap_3d(&tv, a.v, ty, sizeof(E), a.C, a.T, a.B, kFwdCh, LT, 1, why))
     return WKV_ERR_INVALID_ARG;
+  if (!GATE)
+    tr = tk;  // unused
+  else if (!encode_tmap_3d(&tr, a.r, ty, sizeof(E), a.C, a.T, a.B, kFwdCh, LT, 1, why))
+    return WKV_ERR_INVALID_ARG;
   const int ncb = (int)ceil_div(a.C, kFwdCh);
   const int ngroups = (int)(ncb * a.B);
-  auto kern = wkv4_fwd_kernel<E, LT, STAGES, NSEG, NW>;
-  const size_t smem = NW * sizeof(Wkv4FwdSmem<E, LT, STAGES>);
+  auto kern = wkv4_fwd_kernel<E, LT, STAGES, NSEG, NW, GATE>;
+  const size_t smem = NW * sizeof(Wkv4FwdSmem<E, LT, STAGES, GATE>);
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
     *why = "wkv4_forward: shared memory configuration failed";
@@ -236,7 +255,7 @@ static wkv_status run_fwd(const Wkv4FwdArgs& a, cudaStream_t stream, unsigned* e
     cfg.attrs = attr;
     cfg.numAttrs = 1;
   }
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tk, tv, static_cast<const E*>(a.k), (int)a.T, (int)a.C, ncb,
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tk, tv, tr, static_cast<const E*>(a.k), (int)a.T, (int)a.C, ncb,
                                            ngroups, a.w, a.u, static_cast<E*>(a.y), a.ckpt, err);
   if (e != cudaSuccess) {
     *why = "wkv4_forward kernel launch failed";
@@ -245,25 +264,25 @@ static wkv_status run_fwd(const Wkv4FwdArgs& a, cudaStream_t stream, unsigned* e
   return WKV_OK;
 }
 
-template <class E, int LT, int STAGES, int NSEG>
+template <class E, int LT, int STAGES, int NSEG, bool GATE>
 static wkv_status run_fwd_nw(const Wkv4FwdArgs& a, cudaStream_t stream, unsigned* err, const char** why) {
   switch (wkv4_warps_per_cta(a.B, a.C, NSEG)) {
-    case 4: return run_fwd<E, LT, STAGES, NSEG, 4>(a, stream, err, why);
-    case 2: return run_fwd<E, LT, STAGES, NSEG, 2>(a, stream, err, why);
-    default: return run_fwd<E, LT, STAGES, NSEG, 1>(a, stream, err, why);
+    case 4: return run_fwd<E, LT, STAGES, NSEG, 4, GATE>(a, stream, err, why);
+    case 2: return run_fwd<E, LT, STAGES, NSEG, 2, GATE>(a, stream, err, why);
+    default: return run_fwd<E, LT, STAGES, NSEG, 1, GATE>(a, stream, err, why);
   }
 }
 
-template <class E, int LT, int STAGES>
+template <class E, int LT, int STAGES, bool GATE = false>
 static wkv_status run_fwd_nseg(const Wkv4FwdArgs& a, cudaStream_t stream, unsigned* err, const char** why) {
   switch (wkv4_fwd_segments(a.B, a.T, a.C)) {
 #if WKV4_MAX_SEGMENTS_ANY > 8
-    case 16: return run_fwd_nw<E, LT, STAGES, 16>(a, stream, err, why);
+    case 16: return run_fwd_nw<E, LT, STAGES, 16, GATE>(a, stream, err, why);
 #endif
-    case 8: return run_fwd_nw<E, LT, STAGES, 8>(a, stream, err, why);
-    case 4: return run_fwd_nw<E, LT, STAGES, 4>(a, stream, err, why);
-    case 2: return run_fwd_nw<E, LT, STAGES, 2>(a, stream, err, why);
-    default: return run_fwd<E, LT, STAGES, 1, 1>(a, stream, err, why);
+    case 8: return run_fwd_nw<E, LT, STAGES, 8, GATE>(a, stream, err, why);
+    case 4: return run_fwd_nw<E, LT, STAGES, 4, GATE>(a, stream, err, why);
+    case 2: return run_fwd_nw<E, LT, STAGES, 2, GATE>(a, stream, err, why);
+    default: return run_fwd<E, LT, STAGES, 1, 1, GATE>(a, stream, err, why);
   }
 }
 
@@ -277,6 +296,11 @@ static wkv_status run_fwd_nseg(const Wkv4FwdArgs& a, cudaStream_t stream, unsign
 #endif
 
 wkv_status launch_wkv4_forward(const Wkv4FwdArgs& a, cudaStream_t stream, unsigned* err, const char** why) {
+  if (a.r) {
+    // gated: a third tile per stage, one stage fewer (same shared memory per warp)
+    if (a.dtype == WKV_BF16) return run_fwd_nseg<__nv_bfloat16, 32, 2, true>(a, stream, err, why);
+    return run_fwd_nseg<float, 16, 2, true>(a, stream, err, why);
+  }
   if (a.dtype == WKV_BF16) return run_fwd_nseg<__nv_bfloat16, 32, WKV4_FWD_STAGES_BF16>(a, stream, err, why);
   return run_fwd_nseg<float, 16, WKV4_FWD_STAGES_F32>(a, stream, err, why);
 }

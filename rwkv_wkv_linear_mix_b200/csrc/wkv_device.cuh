@@ -410,6 +410,12 @@ __device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __ffma2_rn(b
 __device__ __forceinline__ float2 ex2_2(float2 a) { return make_float2(ex2(a.x), ex2(a.y)); }
 __device__ __forceinline__ float2 rcp2(float2 a) { return make_float2(rcp(a.x), rcp(a.y)); }
 
+// sigmoid(x) = 1 / (1 + 2^{-x log2 e}) of a pair
+__device__ __forceinline__ float2 sigmoid2(float2 x) {
+  const float2 e = make_float2(ex2(__fmul_rn(-x.x, kLog2e)), ex2(__fmul_rn(-x.y, kLog2e)));
+  return rcp2(add2(e, splat2(1.f)));
+}
+
 __device__ __forceinline__ float2 ld_pair(const float* p) { return *reinterpret_cast<const float2*>(p); }
 __device__ __forceinline__ float2 ld_pair(const __nv_bfloat16* p) {
   const uint32_t x = *reinterpret_cast<const uint32_t*>(p);  // channel c in the low half

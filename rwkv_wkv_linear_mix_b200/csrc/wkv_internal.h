@@ -91,6 +91,7 @@ struct Wkv4FwdArgs {
   const void* v;
   void* y;      // may be null
   float* ckpt;  // may be null
+  const void* r = nullptr;  // gate input: y = sigmoid(r) * WKV (may be null: ungated)
 };
 
 struct Wkv4BwdArgs {
@@ -107,6 +108,8 @@ struct Wkv4BwdArgs {
   float* gw;
   float* gu;
   float* part;  // [2][B * wkv4_bwd_segments(B, T, C)][C] scratch
+  const void* r = nullptr;  // gate input (gy is then dL/d(sigmoid(r) * WKV)); null: ungated
+  void* gr = nullptr;       // dL/dr, written when r is given
 };
 
 struct Wkv4ChunkArgs {

@@ -28,6 +28,7 @@ __all__ = [
     "f32_to_bf16_bits",
     "bf16_bits_to_f32",
     "Wkv4Recipe",
+    "gate_input",
     "Wkv6Recipe",
     "wkv4_inputs",
     "wkv4_slot_inputs",
@@ -153,6 +154,17 @@ def wkv4_inputs(recipe: Wkv4Recipe, seed: int = 0) -> dict:
         gy = rng.standard_normal(size=(B, T, C), dtype=np.float32)
         out["gy"], out["gy32"] = _store(gy, recipe.dtype)
     return out
+
+
+def gate_input(shape, dtype: str, seed: int = 0, std: float = 2.0):
+    """The receptance before its sigmoid, r ~ N(0, std^2) (std 2 reaches the
+    saturated ends of the gate), as (storage array, exact float32 values).
+    Drawn from its own stream so that the other inputs of a seed stay put."""
+    rng = np.random.Generator(np.random.PCG64([seed, 0x5167]))
+    r = rng.standard_normal(size=shape, dtype=np.float32)
+    if std != 1.0:
+        r *= np.float32(std)
+    return _store(r, dtype)
 
 
 # ----------------------------------------------------------------------------

@@ -42,6 +42,8 @@ SIGNATURES = {
     "wkv_wait_selfcheck": (_int, [_i64, _vp]),
     "wkv7_forward": (_int, [_i64, _i64, _i64, _i64, _int] + [_vp] * 10),
     "wkv6_backward": (_int, [_i64, _i64, _i64, _i64, _int] + [_vp] * 7 + [_i64] + [_vp] * 9 + [_sz, _vp]),
+    "wkv4_forward_gated": (_int, [_i64, _i64, _i64, _int] + [_vp] * 8),
+    "wkv4_backward_gated": (_int, [_i64, _i64, _i64, _int] + [_vp] * 13 + [_sz, _vp]),
 }
 
 
@@ -206,6 +208,53 @@ def wkv4_backward_noalloc(w, u, k, v, gy, ckpt: Optional[torch.Tensor] = None, *
                                       _ptr(ckpt), _ptr(gk), _ptr(gv), _ptr(gw), _ptr(gu), _stream(k)),
            "wkv4_backward_noalloc")
     return gk, gv, gw, gu
+
+
+def wkv4_forward_gated(w, u, k, v, r, *, y: Optional[torch.Tensor] = None, ckpt: Optional[torch.Tensor] = None,
+                       want_ckpt: bool = False):
+    """sigmoid(r) * WKV in one kernel (the time-mix gate fused into the RWKV-4
+    forward). r: [B, T, C] like k. Returns y, or (y, ckpt)."""
+    B, T, C = k.shape
+    dev = k.device
+    for name, t in (("k", k), ("v", v), ("r", r)):
+        _want(t, name, dtype=k.dtype, shape=k.shape, device=dev)
+    _want(w, "w", dtype=torch.float32, shape=(C,), device=dev)
+    _want(u, "u", dtype=torch.float32, shape=(C,), device=dev)
+    y = torch.empty_like(k) if y is None else y
+    _want(y, "y", dtype=k.dtype, shape=k.shape, device=dev)
+    if ckpt is None and want_ckpt:
+        ckpt = torch.empty(ckpt_shape(B, T, C), dtype=torch.float32, device=dev)
+    if ckpt is not None:
+        _want(ckpt, "ckpt", dtype=torch.float32, shape=ckpt_shape(B, T, C), device=dev)
+    _check(_lib.wkv4_forward_gated(B, T, C, _dtype_code(k), _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(y),
+                                   _ptr(ckpt), _stream(k)), "wkv4_forward_gated")
+    return (y, ckpt) if (want_ckpt or ckpt is not None) else y
+
+
+def wkv4_backward_gated(w, u, k, v, r, gy, ckpt: Optional[torch.Tensor] = None, *, gk=None, gv=None, gr=None,
+                        gw=None, gu=None, workspace: Optional[torch.Tensor] = None):
+    """Gradients of the gated forward. Returns (gk, gv, gr, gw, gu)."""
+    B, T, C = k.shape
+    dev = k.device
+    for name, t in (("k", k), ("v", v), ("r", r), ("gy", gy)):
+        _want(t, name, dtype=k.dtype, shape=k.shape, device=dev)
+    _want(w, "w", dtype=torch.float32, shape=(C,), device=dev)
+    _want(u, "u", dtype=torch.float32, shape=(C,), device=dev)
+    if ckpt is not None:
+        _want(ckpt, "ckpt", dtype=torch.float32, shape=ckpt_shape(B, T, C), device=dev)
+    gk = torch.empty_like(k) if gk is None else gk
+    gv = torch.empty_like(k) if gv is None else gv
+    gr = torch.empty_like(k) if gr is None else gr
+    gw = torch.empty(C, dtype=torch.float32, device=dev) if gw is None else gw
+    gu = torch.empty(C, dtype=torch.float32, device=dev) if gu is None else gu
+    nbytes = wkv4_backward_workspace_bytes(B, T, C, ckpt is not None)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    _want(workspace, "workspace", device=dev)
+    _check(_lib.wkv4_backward_gated(B, T, C, _dtype_code(k), _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(r), _ptr(gy),
+                                    _ptr(ckpt), _ptr(gk), _ptr(gv), _ptr(gr), _ptr(gw), _ptr(gu), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(k)), "wkv4_backward_gated")
+    return gk, gv, gr, gw, gu
 
 
 STATE_ROWS = 5  # aa, bb, base, n, ref

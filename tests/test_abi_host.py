@@ -35,7 +35,8 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("wkv4_forward", "wkv4_backward", "wkv4_chunk_step", "wkv4_state_init", "wkv6_forward",
               "wkv4_backward_workspace_bytes", "wkv4_ckpt_floats", "wkv_status_string", "wkv_last_error",
-              "wkv_device_error", "wkv_abi_version", "wkv6_backward", "wkv6_backward_workspace_bytes"):
+              "wkv_device_error", "wkv_abi_version", "wkv6_backward", "wkv6_backward_workspace_bytes",
+              "wkv4_forward_gated", "wkv4_backward_gated", "wkv7_forward"):
         assert n in names
 
 
@@ -98,6 +99,22 @@ def test_backward_argument_errors(W):
     rc = L.wkv4_backward(2, 8, 8, 0, FAKE, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None)
     assert rc == W.WKV_ERR_INVALID_ARG and b"gy" in L.wkv_last_error()
     assert L.wkv4_backward(2, 8, 10, 0, *args[:10], FAKE, 1 << 30, None) == W.WKV_ERR_UNSUPPORTED
+
+
+def test_gated_argument_errors(W):
+    L = W.lib()
+    fg = lambda B=1, T=4, C=8, dt=0, r=FAKE, y=FAKE: L.wkv4_forward_gated(B, T, C, dt, FAKE, FAKE, FAKE, FAKE, r,
+                                                                          y, None, None)
+    assert fg(r=None) == W.WKV_ERR_INVALID_ARG and b"r is NULL" in L.wkv_last_error()
+    assert fg(y=None) == W.WKV_ERR_INVALID_ARG and b"y is NULL" in L.wkv_last_error()
+    assert fg(r=FAKE + 8) == W.WKV_ERR_INVALID_ARG and b"aligned" in L.wkv_last_error()
+    assert fg(C=6) == W.WKV_ERR_UNSUPPORTED
+    assert fg(B=0, r=None, y=None) == W.WKV_OK
+    bg = lambda T=8, r=FAKE, gr=FAKE, ws=1 << 30: L.wkv4_backward_gated(
+        2, T, 8, 0, FAKE, FAKE, FAKE, FAKE, r, FAKE, None, FAKE, FAKE, gr, FAKE, FAKE, FAKE, ws, None)
+    assert bg(r=None) == W.WKV_ERR_INVALID_ARG and b"r is NULL" in L.wkv_last_error()
+    assert bg(gr=None) == W.WKV_ERR_INVALID_ARG and b"gr is NULL" in L.wkv_last_error()
+    assert bg(ws=0) == W.WKV_ERR_INVALID_ARG and b"workspace" in L.wkv_last_error()
 
 
 def test_chunk_and_wkv6_argument_errors(W):
