@@ -16,6 +16,9 @@ Definitions followed:
     S_t = diag(w_t) S_{t-1} + k_t^T v_t; the op is trainable (the page's
     backend table lists its PyTorch CUDA backward), so its gradients are the
     chain rule of this recurrence.
+  * Time-shift mix: the prologue of RWKV_TimeMix.jit_func (same RWKV-4 page):
+    x_m,t = x_t mix_m + x_{t-1} (1 - mix_m), x_{-1} = 0 (time_shift pads one
+    zero row), for m in (k, v, r).
 """
 
 from __future__ import annotations
@@ -63,6 +66,10 @@ def _open(path):
     lib.oracle_wkv7_forward.argtypes = [i64, i64, i64, i64] + [dp] * 9
     lib.oracle_wkv7_forward.restype = ctypes.c_int
     lib.oracle_wkv6_backward.restype = ctypes.c_int
+    lib.oracle_time_shift_mix.argtypes = [i64, i64, i64, i64] + [dp] * 4
+    lib.oracle_time_shift_mix.restype = ctypes.c_int
+    lib.oracle_time_shift_mix_backward.argtypes = [i64, i64, i64, i64] + [dp] * 7
+    lib.oracle_time_shift_mix_backward.restype = ctypes.c_int
     return lib
 
 
@@ -289,3 +296,38 @@ def wkv7_forward(r, w, k, v, a, b, init_state=None, head_size: int = 64, _lib=No
     if rc != 0:
         raise FloatingPointError(f"oracle_wkv7_forward failed (rc={rc})")
     return o, fs
+
+
+def time_shift_mix(x, mix, x_prev=None, _lib=None):
+    """The time-shift mix in fp64 (see oracle_time_shift_mix). x: [B, T, C];
+    mix: [n_mix, C]; x_prev: [B, C] or None (zeros). Returns [n_mix, B, T, C]."""
+    lib = _lib or _load()
+    x, mix = _f64(x), _f64(mix)
+    B, T, C = x.shape
+    n = mix.shape[0]
+    assert mix.shape == (n, C)
+    xp = None if x_prev is None else _f64(x_prev)
+    assert xp is None or xp.shape == (B, C)
+    out = np.empty((n, B, T, C))
+    if lib.oracle_time_shift_mix(B, T, C, n, _ptr(x), _ptr(mix), _ptr(xp), _ptr(out)) != 0:
+        raise FloatingPointError("oracle_time_shift_mix: non-finite output")
+    return out
+
+
+def time_shift_mix_backward(x, mix, g, x_prev=None, _lib=None):
+    """Gradients of sum(g * time_shift_mix(x, mix, x_prev)) in fp64.
+    g: [n_mix, B, T, C]. Returns (gx [B, T, C], gmix [n_mix, C],
+    gx_prev [B, C] or None when x_prev is None)."""
+    lib = _lib or _load()
+    x, mix, g = _f64(x), _f64(mix), _f64(g)
+    B, T, C = x.shape
+    n = mix.shape[0]
+    assert g.shape == (n, B, T, C)
+    xp = None if x_prev is None else _f64(x_prev)
+    gx = np.empty((B, T, C))
+    gmix = np.empty((n, C))
+    gxp = None if xp is None else np.empty((B, C))
+    if lib.oracle_time_shift_mix_backward(B, T, C, n, _ptr(x), _ptr(mix), _ptr(xp), _ptr(g), _ptr(gx),
+                                          _ptr(gmix), _ptr(gxp)) != 0:
+        raise FloatingPointError("oracle_time_shift_mix_backward: non-finite output")
+    return gx, gmix, gxp

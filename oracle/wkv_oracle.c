@@ -41,6 +41,10 @@
  *
  *      S_t = (diag(e^{w_t}) + b_t a_t^T) S_{t-1} + k_t^T v_t,    o_t = r_t S_t
  *
+ *  Time-shift mix (the prologue of RWKV_TimeMix.jit_func on the same RWKV-4
+ *  page): the input shifted one token along T blended per channel with the
+ *  token itself, once for each of k, v, r, and its backward.
+ *
  * Layouts: activations [B][T][C] row-major, C fastest. All inputs are fp64
  * (the Python wrapper widens float32 / bf16 inputs exactly).
  * Parallelism: OpenMP over independent lanes / heads only; every lane's
@@ -497,5 +501,83 @@ int oracle_wkv7_forward(int64_t B, int64_t T, int64_t H, int64_t K,
         free(S);
         free(sa);
     }
+    return bad;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Time-shift mix (time-mix prologue)                                        */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * RWKV_TimeMix.jit_func ("代码连连看——RWKV", section RWKV_TimeMix): time_shift
+ * is ZeroPad2d((0, 0, 1, -1)) on [B][T][C], i.e. one row of zeros padded
+ * before T and the last row cut, so row t of the shifted input xx is row t-1
+ * of x and row 0 is zero. Each of k, v, r then takes
+ *
+ *     x_m,t = x_t * mix_m + xx_t * (1 - mix_m)        (mix_m = time_mix_{k,v,r})
+ *
+ * x_prev [B][C] (may be NULL: zeros) replaces the zero row, so that a
+ * sequence cut into pieces gives the same result as one call (the RNN form
+ * carries the last token as state).
+ * mix [n_mix][C]; out [n_mix][B][T][C]. Returns 0, or 1 if a value is not finite.
+ */
+int oracle_time_shift_mix(int64_t B, int64_t T, int64_t C, int64_t n_mix,
+                          const double *x, const double *mix, const double *x_prev,
+                          double *out)
+{
+    int bad = 0;
+    for (int64_t m = 0; m < n_mix; ++m)
+        for (int64_t bi = 0; bi < B; ++bi)
+            for (int64_t t = 0; t < T; ++t)
+                for (int64_t c = 0; c < C; ++c) {
+                    const double xt = x[(bi * T + t) * C + c];
+                    double xx = 0.0;
+                    if (t > 0)
+                        xx = x[(bi * T + t - 1) * C + c];
+                    else if (x_prev)
+                        xx = x_prev[bi * C + c];
+                    const double o = xt * mix[m * C + c] + xx * (1.0 - mix[m * C + c]);
+                    out[((m * B + bi) * T + t) * C + c] = o;
+                    if (!isfinite(o)) bad = 1;
+                }
+    return bad;
+}
+
+/*
+ * Gradients of L = sum_m sum(g_m * x_m) for the time-shift mix above, by
+ * scattering each output's two partial derivatives to their inputs:
+ *   d x_m,t / d x_t     = mix_m
+ *   d x_m,t / d xx_t    = 1 - mix_m   (xx_t = x_{t-1}, or x_prev at t = 0)
+ *   d x_m,t / d mix_m   = x_t - xx_t
+ * g [n_mix][B][T][C]; gx [B][T][C]; gmix [n_mix][C] (summed over b, t);
+ * gx_prev [B][C] (may be NULL; written only if given).
+ */
+int oracle_time_shift_mix_backward(int64_t B, int64_t T, int64_t C, int64_t n_mix,
+                                   const double *x, const double *mix, const double *x_prev,
+                                   const double *g, double *gx, double *gmix, double *gx_prev)
+{
+    memset(gx, 0, sizeof(double) * (size_t)(B * T * C));
+    memset(gmix, 0, sizeof(double) * (size_t)(n_mix * C));
+    if (gx_prev) memset(gx_prev, 0, sizeof(double) * (size_t)(B * C));
+    for (int64_t m = 0; m < n_mix; ++m)
+        for (int64_t bi = 0; bi < B; ++bi)
+            for (int64_t t = 0; t < T; ++t)
+                for (int64_t c = 0; c < C; ++c) {
+                    const double gm = g[((m * B + bi) * T + t) * C + c];
+                    const double mc = mix[m * C + c];
+                    const double xt = x[(bi * T + t) * C + c];
+                    double xx = 0.0;
+                    if (t > 0)
+                        xx = x[(bi * T + t - 1) * C + c];
+                    else if (x_prev)
+                        xx = x_prev[bi * C + c];
+                    gx[(bi * T + t) * C + c] += gm * mc;
+                    if (t > 0)
+                        gx[(bi * T + t - 1) * C + c] += gm * (1.0 - mc);
+                    else if (gx_prev)
+                        gx_prev[bi * C + c] += gm * (1.0 - mc);
+                    gmix[m * C + c] += gm * (xt - xx);
+                }
+    int bad = !all_finite(gx, B * T * C) || !all_finite(gmix, n_mix * C);
     return bad;
 }

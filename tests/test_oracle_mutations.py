@@ -49,6 +49,20 @@ MUTATIONS = {
     # RWKV-7: the read leaves out the current token's write
     "wkv7_read_without_token": ("for (int64_t j = 0; j < K; ++j) acc += r[row + j] * S[j * K + i];",
                                 "for (int64_t j = 0; j < K; ++j) acc += r[row + j] * (S[j * K + i] - k[row + j] * v[row + i]);"),
+    # time-shift mix: blend weights swapped between the token and the one before
+    "tsm_swap_weights": ("const double o = xt * mix[m * C + c] + xx * (1.0 - mix[m * C + c]);",
+                         "const double o = xx * mix[m * C + c] + xt * (1.0 - mix[m * C + c]);"),
+    # time-shift mix: the shift taken from the next token instead of the previous one
+    "tsm_shift_direction": ("                    if (t > 0)\n                        xx = x[(bi * T + t - 1) * C + c];\n"
+                            "                    else if (x_prev)\n                        xx = x_prev[bi * C + c];\n"
+                            "                    const double o",
+                            "                    if (t + 1 < T)\n                        xx = x[(bi * T + t + 1) * C + c];\n"
+                            "                    else if (x_prev)\n                        xx = x_prev[bi * C + c];\n"
+                            "                    const double o"),
+    # time-shift mix backward: the 1 - mix part scattered to the token's own row
+    "tsmb_wrong_row": ("gx[(bi * T + t - 1) * C + c] += gm * (1.0 - mc);", "gx[(bi * T + t) * C + c] += gm * (1.0 - mc);"),
+    # time-shift mix backward: flipped sign of the mix gradient
+    "tsmb_gmix_sign": ("gmix[m * C + c] += gm * (xt - xx);", "gmix[m * C + c] += gm * (xx - xt);"),
 }
 
 
@@ -115,9 +129,26 @@ def _wkv7_pins_fail(var):
     return False
 
 
+def _tsm_pins_fail(var):
+    import test_oracle_time_shift as pt
+
+    class _Adapter:
+        time_shift_mix = staticmethod(var.time_shift_mix)
+        time_shift_mix_backward = staticmethod(var.time_shift_mix_backward)
+    pins = (pt.test_hand_worked, pt.test_ends_of_the_blend, pt.test_pieces_with_x_prev_match_one_call,
+            pt.test_backward_closed_form_for_unit_gradient, lambda o: pt.test_backward_matches_finite_differences(o, True))
+    for pin in pins:
+        try:
+            pin(_Adapter)
+        except AssertionError:
+            return True
+    return False
+
+
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
 def test_mutation_is_caught(variants, name):
     check = (_wkv4_pins_fail if name.startswith("wkv4") else
+             _tsm_pins_fail if name.startswith("tsm") else
              _wkv7_pins_fail if name.startswith("wkv7") else
              _wkv6b_pins_fail if name.startswith("wkv6b") else _wkv6_pins_fail)
     assert check(variants[name]), f"planted mistake {name} passed every pin"
@@ -130,7 +161,10 @@ def test_unmutated_source_passes(oracle):
         wkv6_forward = staticmethod(oracle.wkv6_forward)
         wkv6_backward = staticmethod(oracle.wkv6_backward)
         wkv7_forward = staticmethod(oracle.wkv7_forward)
+        time_shift_mix = staticmethod(oracle.time_shift_mix)
+        time_shift_mix_backward = staticmethod(oracle.time_shift_mix_backward)
     assert not _wkv4_pins_fail(_Orig)
+    assert not _tsm_pins_fail(_Orig)
     assert not _wkv7_pins_fail(_Orig)
     assert not _wkv6_pins_fail(_Orig)
     assert not _wkv6b_pins_fail(_Orig)
