@@ -65,7 +65,7 @@ def parse():
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the secondary workloads (larger shapes, chunk step, RWKV-6)")
     ap.add_argument("--kernel", choices=["wkv4_fwd", "wkv4_bwd", "wkv4_fwd_gated", "wkv4_bwd_gated", "wkv6_fwd",
-                                         "wkv6_bwd", "wkv7_fwd", "wkv4_chunk"],
+                                         "wkv6_bwd", "wkv7_fwd", "wkv4_chunk", "time_shift_fwd", "time_shift_bwd"],
                     help="profiling mode: run only this kernel --steps times on --workload (no JSON line)")
     ap.add_argument("--workload", default=None,
                     help="with --kernel: a recipe name of synth (RWKV-4 or RWKV-6), optionally resized "
@@ -330,6 +330,28 @@ def secondary(dev, flush, peak):
             del r, gr
         del k, v, gy, y, gk, gv, ck, ws
         torch.cuda.empty_cache()
+
+    # time-mix prologue: three blends of each token with the one before
+    B, T, C, nm = 16, 4096, 4096, 3
+    g.manual_seed(0)
+    xs = torch.randn(B, T, C, device=dev, generator=g).to(torch.bfloat16)
+    mixs = torch.rand(nm, C, device=dev, generator=g)
+    outs = torch.empty(nm, B, T, C, dtype=torch.bfloat16, device=dev)
+    gs = torch.randn(nm, B, T, C, device=dev, generator=g).to(torch.bfloat16)
+    gxs, gmixs = torch.empty_like(xs), torch.empty(nm, C, device=dev)
+    wss = torch.empty(wkv.wkv4_time_shift_mix_backward_workspace_bytes(B, T, C, torch.bfloat16, nm),
+                      dtype=torch.uint8, device=dev)
+    tsf = lambda: wkv.wkv4_time_shift_mix(xs, mixs, out=outs)
+    tsb = lambda: wkv.wkv4_time_shift_mix_backward(xs, mixs, gs, gx=gxs, gmix=gmixs, workspace=wss)
+    tsf(); tsb()
+    t_f = _events_ms(tsf, 5, flush, stream)
+    t_b = _events_ms(tsb, 5, flush, stream)
+    n = B * T * C
+    gf, gb = (1 + nm) * 2 * n / (t_f * 1e-3) / 1e9, (nm + 2) * 2 * n / (t_b * 1e-3) / 1e9
+    res["time_shift_mix_bf16_c4096"] = {"B": B, "T": T, "C": C, "n_mix": nm, "fwd_ms": t_f, "bwd_ms": t_b,
+                                        "fwd_GBps": gf, "bwd_GBps": gb, "fwd_frac": gf / peak, "bwd_frac": gb / peak}
+    del xs, outs, gs, gxs, wss
+    torch.cuda.empty_cache()
 
     # batched inference slots: 32 slots, prompts ~U{1..512}, <= 32 tokens per call
     S, C = 32, 4096
@@ -674,6 +696,17 @@ def run_kernel_only(args):
             wkv.wkv4_state_init(S, C, dev, state=state)
             for kc, vc, cu in calls:
                 wkv.wkv4_chunk_step(w, u, kc, vc, cu, state)
+    elif args.kernel in ("time_shift_fwd", "time_shift_bwd"):
+        B, T, C = (int(v) for v in (resize or "16,4096,4096").split(","))
+        xs = torch.randn(B, T, C, device=dev, generator=g).to(torch.bfloat16)
+        mixs = torch.rand(3, C, device=dev, generator=g)
+        outs = torch.empty(3, B, T, C, dtype=torch.bfloat16, device=dev)
+        gs = torch.randn(3, B, T, C, device=dev, generator=g).to(torch.bfloat16)
+        for _ in range(args.steps):
+            if args.kernel == "time_shift_fwd":
+                wkv.wkv4_time_shift_mix(xs, mixs, out=outs)
+            else:
+                wkv.wkv4_time_shift_mix_backward(xs, mixs, gs)
     elif args.kernel == "wkv7_fwd":
         rec7 = synth.WKV7_RECIPES[name or "wkv7_fwd_bf16_c2048"]
         if resize:

@@ -186,6 +186,52 @@ wkv_status wkv4_backward_gated(int64_t B, int64_t T, int64_t C, int dtype,
                                void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Time-shift mix, the prologue of RWKV_TimeMix ("代码连连看——RWKV", section
+ * RWKV_TimeMix, jit_func): time_shift moves the input one token along T
+ * (a zero row padded before t = 0, the last row dropped), and each of the
+ * k, v, r inputs of the projections blends the token with the shifted one
+ * per channel:
+ *
+ *     out[m][b][t][c] = x[b][t][c] * mix[m][c] + xx[b][t][c] * (1 - mix[m][c])
+ *     xx[b][t] = x[b][t-1] for t > 0,  xx[b][0] = x_prev[b] (zeros if NULL)
+ *
+ *   n_mix       number of blends, 1..3 (3 for time_mix_k, _v, _r).
+ *   x           [B][T][C] of `dtype`.
+ *   mix         [n_mix][C] float32.
+ *   x_prev      [B][C] of `dtype` or NULL: the token before x (the last
+ *               token of the previous piece when a sequence is fed in pieces).
+ *   out         [n_mix][B][T][C] of `dtype`, written; must not overlap x.
+ * Alignment and C rules as for wkv4_forward; n_mix outside 1..3 is
+ * WKV_ERR_INVALID_ARG; empty problems are no-ops.
+ */
+wkv_status wkv4_time_shift_mix(int64_t B, int64_t T, int64_t C, int dtype, int64_t n_mix,
+                               const void *x, const float *mix, const void *x_prev,
+                               void *out, void *stream);
+
+/* Bytes of device workspace wkv4_time_shift_mix_backward needs. */
+size_t wkv4_time_shift_mix_backward_workspace_bytes(int64_t B, int64_t T, int64_t C,
+                                                    int dtype, int64_t n_mix);
+
+/*
+ * Gradients of L = sum(g * out) for out = wkv4_time_shift_mix(...):
+ *   g           [n_mix][B][T][C] of `dtype`.
+ *   gx          [B][T][C] of `dtype`, written:
+ *               sum_m g[m][t] mix[m] + sum_m g[m][t+1] (1 - mix[m]).
+ *   gmix        [n_mix][C] float32, written: sum over b, t of
+ *               g[m][b][t] (x[b][t] - xx[b][t]), added in a fixed order
+ *               (run-to-run deterministic).
+ *   gx_prev     [B][C] of `dtype` or NULL; if given, written:
+ *               sum_m g[m][b][0] (1 - mix[m]).
+ *   workspace   device scratch of at least
+ *               wkv4_time_shift_mix_backward_workspace_bytes(B, T, C, dtype, n_mix)
+ *               bytes, 16-byte aligned; contents on entry are ignored.
+ */
+wkv_status wkv4_time_shift_mix_backward(int64_t B, int64_t T, int64_t C, int dtype, int64_t n_mix,
+                                        const void *x, const float *mix, const void *x_prev,
+                                        const void *g, void *gx, float *gmix, void *gx_prev,
+                                        void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Set S slot states [S][5][C] float32 to the empty past:
  * aa = bb = 0, base = -1e38, n = 0, ref = 0 (ref is set by the first token).
  */

@@ -425,3 +425,67 @@ WKV_EXPORT wkv_status wkv6_backward(int64_t B, int64_t T, int64_t H, int64_t K, 
   wkv_status s = launch_wkv6_backward(a, static_cast<cudaStream_t>(stream), err, &why);
   return s == WKV_OK ? s : fail(s, why);
 }
+
+// ---------------------------------------------------------------------------
+// Time-shift mix (time-mix prologue)
+// ---------------------------------------------------------------------------
+
+static int ts_vec(int dtype) { return dtype == WKV_BF16 ? 8 : 4; }
+
+WKV_EXPORT wkv_status wkv4_time_shift_mix(int64_t B, int64_t T, int64_t C, int dtype, int64_t n_mix, const void* x,
+                                          const float* mix, const void* x_prev, void* out, void* stream) {
+  if (wkv_status s = check_act(B, T, C, dtype)) return s;
+  if (n_mix < 1 || n_mix > 3) return fail(WKV_ERR_INVALID_ARG, "n_mix must be 1, 2 or 3");
+  if (B == 0 || T == 0 || C == 0) return WKV_OK;
+  if (B * T * C * n_mix > ((int64_t)1 << 40)) return fail(WKV_ERR_UNSUPPORTED, "problem above 2^40 elements");
+  WKV_REQUIRE_PTR(x, "x");
+  WKV_REQUIRE_PTR(mix, "mix");
+  WKV_OPTIONAL_PTR(x_prev, "x_prev");
+  WKV_REQUIRE_PTR(out, "out");
+  TimeShiftArgs a{B, T, C, dtype, (int)n_mix, x, mix, x_prev, out, nullptr, nullptr, nullptr, nullptr, nullptr};
+  const char* why = "";
+  wkv_status s = launch_time_shift_mix(a, static_cast<cudaStream_t>(stream), &why);
+  return s == WKV_OK ? s : fail(s, why);
+}
+
+WKV_EXPORT size_t wkv4_time_shift_mix_backward_workspace_bytes(int64_t B, int64_t T, int64_t C, int dtype,
+                                                               int64_t n_mix) {
+  if (B <= 0 || T <= 0 || C <= 0 || n_mix < 1 || n_mix > 3 || (dtype != WKV_F32 && dtype != WKV_BF16)) return 0;
+  const TsShape sh = time_shift_shape(B, T, C, ts_vec(dtype));
+  return (size_t)n_mix * (size_t)B * (size_t)sh.nrun * (size_t)C * sizeof(float);
+}
+
+WKV_EXPORT wkv_status wkv4_time_shift_mix_backward(int64_t B, int64_t T, int64_t C, int dtype, int64_t n_mix,
+                                                   const void* x, const float* mix, const void* x_prev,
+                                                   const void* g, void* gx, float* gmix, void* gx_prev,
+                                                   void* workspace, size_t workspace_bytes, void* stream) {
+  if (wkv_status s = check_act(B, T, C, dtype)) return s;
+  if (n_mix < 1 || n_mix > 3) return fail(WKV_ERR_INVALID_ARG, "n_mix must be 1, 2 or 3");
+  if (C == 0) return WKV_OK;
+  WKV_REQUIRE_PTR(gmix, "gmix");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (B == 0 || T == 0) {
+    // nothing flows back: the mix gradients (and gx_prev) are zero
+    WKV_OPTIONAL_PTR(gx_prev, "gx_prev");
+    const size_t esz = dtype == WKV_BF16 ? 2 : 4;
+    if (cudaMemsetAsync(gmix, 0, (size_t)n_mix * C * sizeof(float), st) != cudaSuccess ||
+        (gx_prev && B > 0 && cudaMemsetAsync(gx_prev, 0, (size_t)B * C * esz, st) != cudaSuccess))
+      return fail(WKV_ERR_CUDA, "cudaMemsetAsync failed");
+    return WKV_OK;
+  }
+  if (B * T * C * n_mix > ((int64_t)1 << 40)) return fail(WKV_ERR_UNSUPPORTED, "problem above 2^40 elements");
+  WKV_REQUIRE_PTR(x, "x");
+  WKV_REQUIRE_PTR(mix, "mix");
+  WKV_OPTIONAL_PTR(x_prev, "x_prev");
+  WKV_REQUIRE_PTR(g, "g");
+  WKV_REQUIRE_PTR(gx, "gx");
+  WKV_OPTIONAL_PTR(gx_prev, "gx_prev");
+  WKV_REQUIRE_PTR(workspace, "workspace");
+  if (workspace_bytes < wkv4_time_shift_mix_backward_workspace_bytes(B, T, C, dtype, n_mix))
+    return fail(WKV_ERR_INVALID_ARG, "workspace_bytes below wkv4_time_shift_mix_backward_workspace_bytes()");
+  TimeShiftArgs a{B, T, C, dtype, (int)n_mix, x, mix, x_prev, nullptr, g, gx, gmix, gx_prev,
+                  static_cast<float*>(workspace)};
+  const char* why = "";
+  wkv_status s = launch_time_shift_mix_backward(a, st, &why);
+  return s == WKV_OK ? s : fail(s, why);
+}

@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <algorithm>
+
 #include "wkv.h"
 
 namespace wkv {
@@ -186,6 +188,32 @@ wkv_status launch_wkv4_chunk_step(const Wkv4ChunkArgs& a, cudaStream_t stream, u
 wkv_status launch_wkv6_forward(const Wkv6FwdArgs& a, cudaStream_t stream, unsigned* err, const char** why);
 wkv_status launch_wkv6_backward(const Wkv6BwdArgs& a, cudaStream_t stream, unsigned* err, const char** why);
 wkv_status launch_wkv7_forward(const Wkv7FwdArgs& a, cudaStream_t stream, unsigned* err, const char** why);
+
+// Time-shift mix (time-mix prologue). out / g: [n_mix][B][T][C]; mix, gmix:
+// [n_mix][C] float32; x_prev, gx_prev: [B][C] (may be null); part: the
+// backward's partial sums, [n_mix][B * nrun][C] float32.
+struct TimeShiftArgs {
+  int64_t B, T, C;
+  int dtype;
+  int n_mix;
+  const void* x;
+  const float* mix;
+  const void* x_prev;
+  void* out;
+  const void* g;
+  void* gx;
+  float* gmix;
+  void* gx_prev;
+  float* part;
+};
+// Launch shape: channel blocks of 128 threads x `vec` channels, and each
+// sequence cut into nrun runs of Lt tokens.
+struct TsShape {
+  int ncb, nrun, Lt;
+};
+TsShape time_shift_shape(int64_t B, int64_t T, int64_t C, int vec);
+wkv_status launch_time_shift_mix(const TimeShiftArgs& a, cudaStream_t stream, const char** why);
+wkv_status launch_time_shift_mix_backward(const TimeShiftArgs& a, cudaStream_t stream, const char** why);
 wkv_status launch_wait_selfcheck(int64_t limit_ns, cudaStream_t stream, unsigned* err, const char** why);
 
 }  // namespace wkv

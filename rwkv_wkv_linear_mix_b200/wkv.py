@@ -44,6 +44,9 @@ SIGNATURES = {
     "wkv6_backward": (_int, [_i64, _i64, _i64, _i64, _int] + [_vp] * 7 + [_i64] + [_vp] * 9 + [_sz, _vp]),
     "wkv4_forward_gated": (_int, [_i64, _i64, _i64, _int] + [_vp] * 8),
     "wkv4_backward_gated": (_int, [_i64, _i64, _i64, _int] + [_vp] * 13 + [_sz, _vp]),
+    "wkv4_time_shift_mix": (_int, [_i64, _i64, _i64, _int, _i64] + [_vp] * 5),
+    "wkv4_time_shift_mix_backward_workspace_bytes": (_sz, [_i64, _i64, _i64, _int, _i64]),
+    "wkv4_time_shift_mix_backward": (_int, [_i64, _i64, _i64, _int, _i64] + [_vp] * 8 + [_sz, _vp]),
 }
 
 
@@ -255,6 +258,58 @@ def wkv4_backward_gated(w, u, k, v, r, gy, ckpt: Optional[torch.Tensor] = None, 
                                     _ptr(ckpt), _ptr(gk), _ptr(gv), _ptr(gr), _ptr(gw), _ptr(gu), _ptr(workspace),
                                     workspace.numel() * workspace.element_size(), _stream(k)), "wkv4_backward_gated")
     return gk, gv, gr, gw, gu
+
+
+def wkv4_time_shift_mix(x, mix, x_prev: Optional[torch.Tensor] = None, *, out: Optional[torch.Tensor] = None):
+    """The time-mix prologue: n_mix blends of each token with the one before.
+    x: [B, T, C]; mix: [n_mix, C] float32 (n_mix 1..3); x_prev: [B, C] like x
+    or None (zeros). Returns out [n_mix, B, T, C] (out[0], out[1], out[2] are
+    the k, v, r inputs)."""
+    B, T, C = x.shape
+    dev = x.device
+    _want(x, "x")
+    n = mix.shape[0] if mix.dim() == 2 else -1
+    _want(mix, "mix", dtype=torch.float32, shape=(n, C), device=dev)
+    if x_prev is not None:
+        _want(x_prev, "x_prev", dtype=x.dtype, shape=(B, C), device=dev)
+    out = torch.empty((n, B, T, C), dtype=x.dtype, device=dev) if out is None else out
+    _want(out, "out", dtype=x.dtype, shape=(n, B, T, C), device=dev)
+    _check(_lib.wkv4_time_shift_mix(B, T, C, _dtype_code(x), n, _ptr(x), _ptr(mix), _ptr(x_prev), _ptr(out),
+                                    _stream(x)), "wkv4_time_shift_mix")
+    return out
+
+
+def wkv4_time_shift_mix_backward_workspace_bytes(B: int, T: int, C: int, dtype: torch.dtype, n_mix: int) -> int:
+    code = WKV_BF16 if dtype == torch.bfloat16 else WKV_F32
+    return int(_lib.wkv4_time_shift_mix_backward_workspace_bytes(B, T, C, code, n_mix))
+
+
+def wkv4_time_shift_mix_backward(x, mix, g, x_prev: Optional[torch.Tensor] = None, *, want_gx_prev: bool = False,
+                                 gx=None, gmix=None, gx_prev=None, workspace: Optional[torch.Tensor] = None):
+    """Gradients of sum(g * wkv4_time_shift_mix(x, mix, x_prev)). g: [n_mix, B,
+    T, C]. Returns (gx, gmix, gx_prev); gx_prev is None unless wanted (or a
+    buffer is passed)."""
+    B, T, C = x.shape
+    dev = x.device
+    _want(x, "x")
+    n = mix.shape[0] if mix.dim() == 2 else -1
+    _want(mix, "mix", dtype=torch.float32, shape=(n, C), device=dev)
+    _want(g, "g", dtype=x.dtype, shape=(n, B, T, C), device=dev)
+    if x_prev is not None:
+        _want(x_prev, "x_prev", dtype=x.dtype, shape=(B, C), device=dev)
+    gx = torch.empty_like(x) if gx is None else gx
+    gmix = torch.empty((n, C), dtype=torch.float32, device=dev) if gmix is None else gmix
+    if gx_prev is None and want_gx_prev:
+        gx_prev = torch.empty((B, C), dtype=x.dtype, device=dev)
+    nbytes = wkv4_time_shift_mix_backward_workspace_bytes(B, T, C, x.dtype, n)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    _want(workspace, "workspace", device=dev)
+    _check(_lib.wkv4_time_shift_mix_backward(B, T, C, _dtype_code(x), n, _ptr(x), _ptr(mix), _ptr(x_prev), _ptr(g),
+                                             _ptr(gx), _ptr(gmix), _ptr(gx_prev), _ptr(workspace),
+                                             workspace.numel() * workspace.element_size(), _stream(x)),
+           "wkv4_time_shift_mix_backward")
+    return gx, gmix, gx_prev
 
 
 STATE_ROWS = 5  # aa, bb, base, n, ref

@@ -36,7 +36,8 @@ def test_header_declares_the_entry_points():
     for n in ("wkv4_forward", "wkv4_backward", "wkv4_chunk_step", "wkv4_state_init", "wkv6_forward",
               "wkv4_backward_workspace_bytes", "wkv4_ckpt_floats", "wkv_status_string", "wkv_last_error",
               "wkv_device_error", "wkv_abi_version", "wkv6_backward", "wkv6_backward_workspace_bytes",
-              "wkv4_forward_gated", "wkv4_backward_gated", "wkv7_forward"):
+              "wkv4_forward_gated", "wkv4_backward_gated", "wkv7_forward", "wkv4_time_shift_mix",
+              "wkv4_time_shift_mix_backward", "wkv4_time_shift_mix_backward_workspace_bytes"):
         assert n in names
 
 
@@ -115,6 +116,27 @@ def test_gated_argument_errors(W):
     assert bg(r=None) == W.WKV_ERR_INVALID_ARG and b"r is NULL" in L.wkv_last_error()
     assert bg(gr=None) == W.WKV_ERR_INVALID_ARG and b"gr is NULL" in L.wkv_last_error()
     assert bg(ws=0) == W.WKV_ERR_INVALID_ARG and b"workspace" in L.wkv_last_error()
+
+
+def test_time_shift_argument_errors(W):
+    L = W.lib()
+    f = lambda B=2, T=4, C=8, dt=0, n=3, x=FAKE, mix=FAKE, xp=None, out=FAKE: L.wkv4_time_shift_mix(
+        B, T, C, dt, n, x, mix, xp, out, None)
+    assert f(n=0) == W.WKV_ERR_INVALID_ARG and b"n_mix" in L.wkv_last_error()
+    assert f(n=4) == W.WKV_ERR_INVALID_ARG
+    assert f(x=None) == W.WKV_ERR_INVALID_ARG and b"x is NULL" in L.wkv_last_error()
+    assert f(out=None) == W.WKV_ERR_INVALID_ARG and b"out is NULL" in L.wkv_last_error()
+    assert f(xp=FAKE + 4) == W.WKV_ERR_INVALID_ARG and b"x_prev" in L.wkv_last_error()
+    assert f(C=12, dt=1) == W.WKV_ERR_UNSUPPORTED
+    assert f(T=0, x=None, out=None) == W.WKV_OK
+    ws = L.wkv4_time_shift_mix_backward_workspace_bytes
+    assert ws(2, 64, 128, 0, 3) >= 3 * 2 * 128 * 4
+    assert ws(2, 64, 128, 0, 4) == 0 and ws(0, 64, 128, 0, 3) == 0
+    b = lambda n=3, g=FAKE, gx=FAKE, gmix=FAKE, wsb=1 << 30: L.wkv4_time_shift_mix_backward(
+        2, 64, 128, 0, n, FAKE, FAKE, None, g, gx, gmix, None, FAKE, wsb, None)
+    assert b(g=None) == W.WKV_ERR_INVALID_ARG and b"g is NULL" in L.wkv_last_error()
+    assert b(gmix=None) == W.WKV_ERR_INVALID_ARG and b"gmix" in L.wkv_last_error()
+    assert b(wsb=16) == W.WKV_ERR_INVALID_ARG and b"workspace" in L.wkv_last_error()
 
 
 def test_chunk_and_wkv6_argument_errors(W):
