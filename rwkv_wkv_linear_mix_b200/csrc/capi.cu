@@ -430,8 +430,6 @@ WKV_EXPORT wkv_status wkv6_backward(int64_t B, int64_t T, int64_t H, int64_t K, 
 // Time-shift mix (time-mix prologue)
 // ---------------------------------------------------------------------------
 
-static int ts_vec(int dtype) { return dtype == WKV_BF16 ? 8 : 4; }
-
 WKV_EXPORT wkv_status wkv4_time_shift_mix(int64_t B, int64_t T, int64_t C, int dtype, int64_t n_mix, const void* x,
                                           const float* mix, const void* x_prev, void* out, void* stream) {
   if (wkv_status s = check_act(B, T, C, dtype)) return s;
@@ -451,7 +449,7 @@ WKV_EXPORT wkv_status wkv4_time_shift_mix(int64_t B, int64_t T, int64_t C, int d
 WKV_EXPORT size_t wkv4_time_shift_mix_backward_workspace_bytes(int64_t B, int64_t T, int64_t C, int dtype,
                                                                int64_t n_mix) {
   if (B <= 0 || T <= 0 || C <= 0 || n_mix < 1 || n_mix > 3 || (dtype != WKV_F32 && dtype != WKV_BF16)) return 0;
-  const TsShape sh = time_shift_shape(B, T, C, ts_vec(dtype));
+  const TsShape sh = time_shift_shape(B, T, C, time_shift_bwd_vec(dtype));
   return (size_t)n_mix * (size_t)B * (size_t)sh.nrun * (size_t)C * sizeof(float);
 }
 

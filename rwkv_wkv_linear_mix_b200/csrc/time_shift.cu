@@ -14,10 +14,13 @@
 // Both are pure streams: one read of x gives all n_mix outputs (the three
 // blends of the page read x and its shifted copy three times each), and one
 // read of the n_mix gradients and x gives gx and the mix gradients. A thread
-// owns 16 bytes of channels (4 float32 or 8 bf16) over a run of Lt tokens of
-// one sequence and keeps the previous token in registers, so only the first
-// token of each run is read twice. The mix gradients leave as per-run
-// partial sums that a second kernel adds in a fixed order (deterministic).
+// owns a few channels (forward: 16 bytes, 4 float32 or 8 bf16; backward: 4
+// channels) over a run of Lt tokens of one sequence and keeps the previous
+// token in registers, so only the first token of each run is read twice.
+// Loads are issued a batch of tokens at a time and kept packed until used,
+// so that enough bytes are in flight per SM for the HBM rate. The mix
+// gradients leave as per-run partial sums that a second kernel adds in a
+// fixed order (deterministic).
 #include "wkv_device.cuh"
 #include "wkv_internal.h"
 
@@ -31,6 +34,12 @@ constexpr int kTsReduceWarps = 8;
 template <class E>
 struct Vec16 {
   static constexpr int N = 16 / sizeof(E);  // channels per 16-byte access
+};
+// Channels per thread of the backward (its registers hold n_mix + 1 rows of
+// them per token in flight) and tokens whose loads it issues together.
+template <class E>
+struct BwdVec {
+  static constexpr int N = sizeof(E) == 2 ? TS_BWD_BF16_VEC : 4;
 };
 
 // 16 bytes of E <-> N floats
@@ -52,6 +61,16 @@ __device__ __forceinline__ void ld_vec(const __nv_bfloat16* p, float (&f)[8]) {
   f[6] = bf16lo(q.w);
   f[7] = bf16hi(q.w);
 }
+__device__ __forceinline__ void ld_vec(const __nv_bfloat16* p, float (&f)[4]) {
+  const uint2 q = *reinterpret_cast<const uint2*>(p);
+  f[0] = bf16lo(q.x);
+  f[1] = bf16hi(q.x);
+  f[2] = bf16lo(q.y);
+  f[3] = bf16hi(q.y);
+}
+__device__ __forceinline__ void st_vec(__nv_bfloat16* p, const float (&f)[4]) {
+  *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]));
+}
 __device__ __forceinline__ void st_vec(float* p, const float (&f)[4]) {
   *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]);
 }
@@ -59,6 +78,49 @@ __device__ __forceinline__ void st_vec(__nv_bfloat16* p, const float (&f)[8]) {
   *reinterpret_cast<uint4*>(p) =
       make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]), pack_bf16x2(f[6], f[7]));
 }
+// The raw 16- or 8-byte word of N channels: the backward keeps its batch of
+// loads packed (bf16 unpacked takes twice the registers) and unpacks at use.
+template <class E, int N>
+struct Raw;
+template <>
+struct Raw<float, 4> {
+  using T = float4;
+  static __device__ __forceinline__ void unpack(const T& q, float (&f)[4]) {
+    f[0] = q.x;
+    f[1] = q.y;
+    f[2] = q.z;
+    f[3] = q.w;
+  }
+};
+template <>
+struct Raw<__nv_bfloat16, 8> {
+  using T = uint4;
+  static __device__ __forceinline__ void unpack(const T& q, float (&f)[8]) {
+    f[0] = bf16lo(q.x);
+    f[1] = bf16hi(q.x);
+    f[2] = bf16lo(q.y);
+    f[3] = bf16hi(q.y);
+    f[4] = bf16lo(q.z);
+    f[5] = bf16hi(q.z);
+    f[6] = bf16lo(q.w);
+    f[7] = bf16hi(q.w);
+  }
+};
+template <>
+struct Raw<__nv_bfloat16, 4> {
+  using T = uint2;
+  static __device__ __forceinline__ void unpack(const T& q, float (&f)[4]) {
+    f[0] = bf16lo(q.x);
+    f[1] = bf16hi(q.x);
+    f[2] = bf16lo(q.y);
+    f[3] = bf16hi(q.y);
+  }
+};
+template <class E, int N>
+__device__ __forceinline__ typename Raw<E, N>::T ld_raw(const E* p) {
+  return *reinterpret_cast<const typename Raw<E, N>::T*>(p);
+}
+
 template <int N>
 __device__ __forceinline__ void ld_mix(const float* p, float (&f)[N]) {
 #pragma unroll
@@ -98,7 +160,8 @@ __global__ void __launch_bounds__(kTsThreads) time_shift_mix_kernel(const E* __r
                                                                     E* __restrict__ out, int T, int C, int ncb,
                                                                     int nrun, int Lt, int64_t plane) {
   constexpr int N = Vec16<E>::N;
-  constexpr int U = 4;
+  constexpr int U = TS_FWD_U;
+  using R = Raw<E, N>;
   const TsRun r = ts_run(T, C, ncb, nrun, Lt, N);
   if (!r.valid) return;
   float m[NMIX][N], om[NMIX][N];
@@ -121,22 +184,24 @@ __global__ void __launch_bounds__(kTsThreads) time_shift_mix_kernel(const E* __r
   const E* xp = x + row0;
   E* op = out + row0;
   for (int t = r.t0; t < r.t1; t += U) {
-    float cur[U][N];
+    typename R::T raw[U];
 #pragma unroll
     for (int j = 0; j < U; ++j)
-      if (t + j < r.t1) ld_vec(xp + (int64_t)j * C, cur[j]);
+      if (t + j < r.t1) raw[j] = ld_raw<E, N>(xp + (int64_t)j * C);
 #pragma unroll
     for (int j = 0; j < U; ++j) {
       if (t + j < r.t1) {
+        float cur[N];
+        R::unpack(raw[j], cur);
 #pragma unroll
         for (int i = 0; i < NMIX; ++i) {
           float o[N];
 #pragma unroll
-          for (int n = 0; n < N; ++n) o[n] = __fmaf_rn(cur[j][n], m[i][n], __fmul_rn(prev[n], om[i][n]));
+          for (int n = 0; n < N; ++n) o[n] = __fmaf_rn(cur[n], m[i][n], __fmul_rn(prev[n], om[i][n]));
           st_vec(op + (int64_t)i * plane + (int64_t)j * C, o);
         }
 #pragma unroll
-        for (int n = 0; n < N; ++n) prev[n] = cur[j][n];
+        for (int n = 0; n < N; ++n) prev[n] = cur[n];
       }
     }
     xp += (int64_t)U * C;
@@ -145,14 +210,16 @@ __global__ void __launch_bounds__(kTsThreads) time_shift_mix_kernel(const E* __r
 }
 
 // Backward. Walks the run upward holding x_{t-1} and g_t; per token it
-// reads x_t and the NMIX gradients of token t+1. part: [NMIX][B*nrun][C]
-// partial mix gradients of each run.
+// reads x_t and the NMIX gradients of token t+1, the loads of U tokens
+// issued before any of them is used. part: [NMIX][B*nrun][C] partial mix
+// gradients of each run.
 template <class E, int NMIX>
 __global__ void __launch_bounds__(kTsThreads) time_shift_mix_bwd_kernel(
     const E* __restrict__ x, const float* __restrict__ mix, const E* __restrict__ x_prev, const E* __restrict__ g,
     E* __restrict__ gx, E* __restrict__ gx_prev, float* __restrict__ part, int B, int T, int C, int ncb, int nrun,
     int Lt, int64_t plane) {
-  constexpr int N = Vec16<E>::N;
+  constexpr int N = BwdVec<E>::N;
+  constexpr int U = TS_BWD_U;
   const TsRun r = ts_run(T, C, ncb, nrun, Lt, N);
   if (!r.valid) return;
   float m[NMIX][N];
@@ -189,40 +256,51 @@ __global__ void __launch_bounds__(kTsThreads) time_shift_mix_bwd_kernel(
   const E* xp = x + row0;
   const E* gp = g + row0 + C;  // token t+1
   E* gxp = gx + row0;
-  for (int t = r.t0; t < r.t1; ++t) {
-    float xt[N], gnext[NMIX][N];
-    ld_vec(xp, xt);
-    if (t + 1 < T) {
+  using R = Raw<E, N>;
+  for (int t = r.t0; t < r.t1; t += U) {
+    typename R::T xr[U], gr[U][NMIX];
 #pragma unroll
-      for (int i = 0; i < NMIX; ++i) ld_vec(gp + (int64_t)i * plane, gnext[i]);
-    } else {
+    for (int j = 0; j < U; ++j) {
+      if (t + j < r.t1) xr[j] = ld_raw<E, N>(xp + (int64_t)j * C);
+      if (t + j + 1 < T && t + j < r.t1) {
 #pragma unroll
-      for (int i = 0; i < NMIX; ++i)
+        for (int i = 0; i < NMIX; ++i) gr[j][i] = ld_raw<E, N>(gp + (int64_t)i * plane + (int64_t)j * C);
+      } else {
 #pragma unroll
-        for (int n = 0; n < N; ++n) gnext[i][n] = 0.f;
-    }
-    float o[N];
-#pragma unroll
-    for (int n = 0; n < N; ++n) {
-      float s = 0.f;
-#pragma unroll
-      for (int i = 0; i < NMIX; ++i) {
-        s = __fmaf_rn(gcur[i][n], m[i][n], s);
-        s = __fmaf_rn(gnext[i][n], 1.f - m[i][n], s);
-        acc[i][n] = __fmaf_rn(gcur[i][n], xt[n] - xprev[n], acc[i][n]);
+        for (int i = 0; i < NMIX; ++i) gr[j][i] = typename R::T{};
       }
-      o[n] = s;
     }
-    st_vec(gxp, o);
 #pragma unroll
-    for (int n = 0; n < N; ++n) {
-      xprev[n] = xt[n];
+    for (int j = 0; j < U; ++j) {
+      if (t + j < r.t1) {
+        float xt[1][N], gn[1][NMIX][N];
+        R::unpack(xr[j], xt[0]);
 #pragma unroll
-      for (int i = 0; i < NMIX; ++i) gcur[i][n] = gnext[i][n];
+        for (int i = 0; i < NMIX; ++i) R::unpack(gr[j][i], gn[0][i]);
+        float o[N];
+#pragma unroll
+        for (int n = 0; n < N; ++n) {
+          float s = 0.f;
+#pragma unroll
+          for (int i = 0; i < NMIX; ++i) {
+            s = __fmaf_rn(gcur[i][n], m[i][n], s);
+            s = __fmaf_rn(gn[0][i][n], 1.f - m[i][n], s);
+            acc[i][n] = __fmaf_rn(gcur[i][n], xt[0][n] - xprev[n], acc[i][n]);
+          }
+          o[n] = s;
+        }
+        st_vec(gxp + (int64_t)j * C, o);
+#pragma unroll
+        for (int n = 0; n < N; ++n) {
+          xprev[n] = xt[0][n];
+#pragma unroll
+          for (int i = 0; i < NMIX; ++i) gcur[i][n] = gn[0][i][n];
+        }
+      }
     }
-    xp += C;
-    gp += C;
-    gxp += C;
+    xp += (int64_t)U * C;
+    gp += (int64_t)U * C;
+    gxp += (int64_t)U * C;
   }
   const int64_t rows = (int64_t)B * nrun;
   const int64_t prow = (int64_t)r.b * nrun + r.run;
@@ -259,14 +337,10 @@ __global__ void __launch_bounds__(32 * kTsReduceWarps) time_shift_reduce_kernel(
   }
 }
 
-template <class E>
-TsShape ts_shape_of(int64_t B, int64_t T, int64_t C) {
-  return time_shift_shape(B, T, C, Vec16<E>::N);
-}
 
 template <class E, int NMIX>
 wkv_status run_ts_fwd(const TimeShiftArgs& a, cudaStream_t stream, const char** why) {
-  const TsShape s = ts_shape_of<E>(a.B, a.T, a.C);
+  const TsShape s = time_shift_shape(a.B, a.T, a.C, Vec16<E>::N);
   const int64_t plane = a.B * a.T * a.C;
   time_shift_mix_kernel<E, NMIX><<<(unsigned)(s.ncb * s.nrun * a.B), kTsThreads, 0, stream>>>(
       static_cast<const E*>(a.x), a.mix, static_cast<const E*>(a.x_prev), static_cast<E*>(a.out), (int)a.T,
@@ -280,7 +354,7 @@ wkv_status run_ts_fwd(const TimeShiftArgs& a, cudaStream_t stream, const char** 
 
 template <class E, int NMIX>
 wkv_status run_ts_bwd(const TimeShiftArgs& a, cudaStream_t stream, const char** why) {
-  const TsShape s = ts_shape_of<E>(a.B, a.T, a.C);
+  const TsShape s = time_shift_shape(a.B, a.T, a.C, BwdVec<E>::N);
   const int64_t plane = a.B * a.T * a.C;
   time_shift_mix_bwd_kernel<E, NMIX><<<(unsigned)(s.ncb * s.nrun * a.B), kTsThreads, 0, stream>>>(
       static_cast<const E*>(a.x), a.mix, static_cast<const E*>(a.x_prev), static_cast<const E*>(a.g),

@@ -212,6 +212,19 @@ struct TsShape {
   int ncb, nrun, Lt;
 };
 TsShape time_shift_shape(int64_t B, int64_t T, int64_t C, int vec);
+// Channels per thread of the backward kernel (bf16: 4 or 8; float32: 4) and
+// tokens per batch of loads of each kernel (a batch is loaded, still packed,
+// before any of it is used).
+#ifndef TS_BWD_BF16_VEC
+#define TS_BWD_BF16_VEC 4
+#endif
+#ifndef TS_BWD_U
+#define TS_BWD_U 8
+#endif
+#ifndef TS_FWD_U
+#define TS_FWD_U 4
+#endif
+inline int time_shift_bwd_vec(int dtype) { return dtype == WKV_BF16 ? TS_BWD_BF16_VEC : 4; }
 wkv_status launch_time_shift_mix(const TimeShiftArgs& a, cudaStream_t stream, const char** why);
 wkv_status launch_time_shift_mix_backward(const TimeShiftArgs& a, cudaStream_t stream, const char** why);
 wkv_status launch_wait_selfcheck(int64_t limit_ns, cudaStream_t stream, unsigned* err, const char** why);
