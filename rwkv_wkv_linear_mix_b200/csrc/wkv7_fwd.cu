@@ -16,7 +16,9 @@
 // holds values 4g .. 4g + 3 for keys 8q .. 8q + 7 (32 fp32: 4 columns x 4
 // key pairs, on packed fp32 pair instructions); the two key reductions are
 // sums over the 8 threads of a column group (lanes 8m .. 8m + 7, three
-// shuffles). Inputs arrive per 32-token chunk by TMA into two stages; the
+// shuffles; the output's reduction is transposed, so that after it each of
+// the 8 threads holds one column's total and no value is summed twice).
+// Inputs arrive per 32-token chunk by TMA into two stages; the
 // chunk's decays e^{w} are formed once into shared memory; each step reads
 // its key slices as bf16 one step ahead and widens them in registers; o
 // leaves through a shared-memory tile as coalesced 16-byte stores. Waits are
@@ -157,21 +159,28 @@ __global__ void __launch_bounds__(kT7, 3) wkv7_fwd_kernel(
       const float2 d2[4] = {make_float2(cu.d0.x, cu.d0.y), make_float2(cu.d0.z, cu.d0.w),
                             make_float2(cu.d1.x, cu.d1.y), make_float2(cu.d1.z, cu.d1.w)};
       const float vv[4] = {bf16lo(cu.v.x), bf16hi(cu.v.x), bf16lo(cu.v.y), bf16hi(cu.v.y)};
-      float oo[4];
+      float po[4];  // this thread's 8-key part of (r_t S_t)[4g + c]
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const float sa = keys_sum8(dot4(a2, S[c]));  // (a_t S_{t-1})[4g + c]
         const float2 sa2 = make_float2(sa, sa), v2 = make_float2(vv[c], vv[c]);
 #pragma unroll
         for (int m = 0; m < 4; ++m) S[c][m] = fma2(S[c][m], d2[m], fma2(b2[m], sa2, mul2(k2[m], v2)));
-        oo[c] = keys_sum8(dot4(r2, S[c]));  // (r_t S_t)[4g + c]
+        po[c] = dot4(r2, S[c]);
       }
-      if (q == 0) {
-        uint2 pk;
-        pk.x = pack_bf16x2(oo[0], oo[1]);
-        pk.y = pack_bf16x2(oo[2], oo[3]);
-        *reinterpret_cast<uint2*>(&sm.out[jt][4 * g]) = pk;
-      }
+      // transposed sum over the 8 key threads: each exchange passes on the
+      // half of the columns this thread does not keep (the same pairwise
+      // tree as a butterfly, so the same bits); thread q ends with column
+      // 2 (q & 1) + (q & 2) / 2, twice per group
+      const bool q0 = q & 1, q1 = q & 2;
+      float k0 = q0 ? po[2] : po[0], k1 = q0 ? po[3] : po[1];
+      const float s0 = q0 ? po[0] : po[2], s1 = q0 ? po[1] : po[3];
+      k0 = __fadd_rn(k0, __shfl_xor_sync(0xffffffffu, s0, 1));
+      k1 = __fadd_rn(k1, __shfl_xor_sync(0xffffffffu, s1, 1));
+      float kk = q1 ? k1 : k0;
+      kk = __fadd_rn(kk, __shfl_xor_sync(0xffffffffu, q1 ? k0 : k1, 2));
+      kk = __fadd_rn(kk, __shfl_xor_sync(0xffffffffu, kk, 4));
+      if (!(q & 4)) sm.out[jt][4 * g + (q0 ? 2 : 0) + (q1 ? 1 : 0)] = __float2bfloat16_rn(kk);
     }
     __syncthreads();
     if (tid == 0 && ch + 2 < nchunk) issue(ch + 2);  // every read of stage s is done
