@@ -426,10 +426,30 @@ def secondary(dev, flush, peak):
             decode_calls()
     torch.cuda.synchronize()
     t_dec = _events_ms(graph.replay, 5, flush, stream)
+    del graph
+
+    # the same 64 calls through the decode fast path (one streaming kernel)
+    def decode_fast():
+        wkv.wkv4_state_init(S, C, dev, state=stated)
+        for t in range(steps):
+            wkv.wkv4_decode_step(w, u, kd[t], vd[t], stated, y=yd[t])
+
+    decode_fast()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        decode_fast()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(graph, stream=side):
+            decode_fast()
+    torch.cuda.synchronize()
+    t_fast = _events_ms(graph.replay, 5, flush, stream)
     res["wkv4_decode_bf16_slots256"] = {
-        "S": S, "C": C, "calls": steps, "graph_ms": t_dec, "per_call_us_graph": 1e3 * t_dec / steps,
-        "Gtokch_per_s_graph": steps * S * C / (t_dec * 1e-3) / 1e9,
-        "GBps_graph": (6 + 40) * steps * S * C / (t_dec * 1e-3) / 1e9}
+        "S": S, "C": C, "calls": steps, "graph_ms": t_fast, "per_call_us_graph": 1e3 * t_fast / steps,
+        "Gtokch_per_s_graph": steps * S * C / (t_fast * 1e-3) / 1e9,
+        "GBps_graph": (6 + 40) * steps * S * C / (t_fast * 1e-3) / 1e9,
+        "bytes_note": "GBps counts the state (21 MB) read and written by every call; it stays in L2 "
+                      "between the calls of one replay, so this is an effective rate, not HBM traffic",
+        "via_chunk_step_per_call_us_graph": 1e3 * t_dec / steps}
     del graph, kd, vd, yd
     torch.cuda.empty_cache()
 

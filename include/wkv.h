@@ -260,6 +260,24 @@ wkv_status wkv4_chunk_step(int64_t S, int64_t C, int dtype,
                            const int32_t *cu_tokens, float *state, void *stream);
 
 /*
+ * The T = 1 fast path of wkv4_chunk_step (batched decode): every one of the S
+ * slots takes exactly one token.
+ *   k, v        [S][C] of `dtype`: slot s's token is row s.
+ *   y           [S][C] of `dtype`, written.
+ *   state       [S][5][C] float32, read and written, as for wkv4_chunk_step.
+ * y and the new state are bit-identical to wkv4_chunk_step with
+ * cu_tokens = {0, 1, ..., S} on the same inputs (the same float32 step in
+ * the same order); a slot whose state is the empty past takes its reference
+ * exponent from this token. Pointers are required (16-byte aligned); size
+ * rules as for wkv4_chunk_step; S = 0 or C = 0 is a no-op. Launches one
+ * kernel; no device error codes (there are no offsets to check).
+ */
+wkv_status wkv4_decode_step(int64_t S, int64_t C, int dtype,
+                            const float *w, const float *u,
+                            const void *k, const void *v, void *y,
+                            float *state, void *stream);
+
+/*
  * wkv4_backward without a workspace argument, for callers that cannot
  * allocate device memory per call (code behind a plain C interface that only
  * receives the tensors it reads and writes, or latency-critical loops that

@@ -305,6 +305,21 @@ WKV_EXPORT wkv_status wkv4_chunk_step(int64_t S, int64_t C, int dtype, const flo
   return s == WKV_OK ? s : fail(s, why);
 }
 
+WKV_EXPORT wkv_status wkv4_decode_step(int64_t S, int64_t C, int dtype, const float* w, const float* u,
+                                       const void* k, const void* v, void* y, float* state, void* stream) {
+  if (wkv_status s = check_act(S, 1, C, dtype)) return s;
+  if (S == 0 || C == 0) return WKV_OK;
+  WKV_REQUIRE_PTR(w, "w");
+  WKV_REQUIRE_PTR(u, "u");
+  WKV_REQUIRE_PTR(k, "k");
+  WKV_REQUIRE_PTR(v, "v");
+  WKV_REQUIRE_PTR(y, "y");
+  WKV_REQUIRE_PTR(state, "state");
+  const char* why = "";
+  wkv_status s = launch_wkv4_decode_step(S, C, dtype, w, u, k, v, y, state, static_cast<cudaStream_t>(stream), &why);
+  return s == WKV_OK ? s : fail(s, why);
+}
+
 WKV_EXPORT wkv_status wkv6_forward(int64_t B, int64_t T, int64_t H, int64_t K, int dtype, const void* r,
                                    const void* k, const void* v, const void* w, const float* u,
                                    const float* init_state, const int32_t* state_map, int64_t n_state,

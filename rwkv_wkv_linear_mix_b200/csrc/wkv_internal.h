@@ -185,6 +185,9 @@ wkv_status launch_wkv4_forward(const Wkv4FwdArgs& a, cudaStream_t stream, unsign
 wkv_status launch_wkv4_backward(const Wkv4BwdArgs& a, cudaStream_t stream, unsigned* err, const char** why);
 wkv_status launch_wkv4_state_init(int64_t S, int64_t C, float* state, cudaStream_t stream, const char** why);
 wkv_status launch_wkv4_chunk_step(const Wkv4ChunkArgs& a, cudaStream_t stream, unsigned* err, const char** why);
+// One token per slot: k, v, y [S][C], state [S][5][C].
+wkv_status launch_wkv4_decode_step(int64_t S, int64_t C, int dtype, const float* w, const float* u, const void* k,
+                                   const void* v, void* y, float* state, cudaStream_t stream, const char** why);
 wkv_status launch_wkv6_forward(const Wkv6FwdArgs& a, cudaStream_t stream, unsigned* err, const char** why);
 wkv_status launch_wkv6_backward(const Wkv6BwdArgs& a, cudaStream_t stream, unsigned* err, const char** why);
 wkv_status launch_wkv7_forward(const Wkv7FwdArgs& a, cudaStream_t stream, unsigned* err, const char** why);

@@ -45,6 +45,7 @@ SIGNATURES = {
     "wkv4_forward_gated": (_int, [_i64, _i64, _i64, _int] + [_vp] * 8),
     "wkv4_backward_gated": (_int, [_i64, _i64, _i64, _int] + [_vp] * 13 + [_sz, _vp]),
     "wkv4_time_shift_mix": (_int, [_i64, _i64, _i64, _int, _i64] + [_vp] * 5),
+    "wkv4_decode_step": (_int, [_i64, _i64, _int] + [_vp] * 7),
     "wkv4_time_shift_mix_backward_workspace_bytes": (_sz, [_i64, _i64, _i64, _int, _i64]),
     "wkv4_time_shift_mix_backward": (_int, [_i64, _i64, _i64, _int, _i64] + [_vp] * 8 + [_sz, _vp]),
 }
@@ -340,6 +341,24 @@ def wkv4_chunk_step(w, u, k, v, cu_tokens: torch.Tensor, state: torch.Tensor, *,
     _want(y, "y", dtype=k.dtype, shape=k.shape, device=dev)
     _check(_lib.wkv4_chunk_step(S, C, _dtype_code(k), _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(y), N,
                                 _ptr(cu_tokens), _ptr(state), _stream(k)), "wkv4_chunk_step")
+    return y
+
+
+def wkv4_decode_step(w, u, k, v, state: torch.Tensor, *, y=None) -> torch.Tensor:
+    """One decode call: slot s takes token k[s], v[s] (k, v: [S, C]); state
+    [S, 5, C] float32 (in/out). Same results as wkv4_chunk_step with one
+    token per slot, in one streaming kernel."""
+    S, C = k.shape
+    dev = k.device
+    _want(k, "k")
+    _want(v, "v", dtype=k.dtype, shape=k.shape, device=dev)
+    _want(w, "w", dtype=torch.float32, shape=(C,), device=dev)
+    _want(u, "u", dtype=torch.float32, shape=(C,), device=dev)
+    _want(state, "state", dtype=torch.float32, shape=(S, STATE_ROWS, C), device=dev)
+    y = torch.empty_like(k) if y is None else y
+    _want(y, "y", dtype=k.dtype, shape=k.shape, device=dev)
+    _check(_lib.wkv4_decode_step(S, C, _dtype_code(k), _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(y), _ptr(state),
+                                 _stream(k)), "wkv4_decode_step")
     return y
 
 

@@ -37,7 +37,8 @@ def test_header_declares_the_entry_points():
               "wkv4_backward_workspace_bytes", "wkv4_ckpt_floats", "wkv_status_string", "wkv_last_error",
               "wkv_device_error", "wkv_abi_version", "wkv6_backward", "wkv6_backward_workspace_bytes",
               "wkv4_forward_gated", "wkv4_backward_gated", "wkv7_forward", "wkv4_time_shift_mix",
-              "wkv4_time_shift_mix_backward", "wkv4_time_shift_mix_backward_workspace_bytes"):
+              "wkv4_time_shift_mix_backward", "wkv4_time_shift_mix_backward_workspace_bytes",
+              "wkv4_decode_step"):
         assert n in names
 
 
@@ -141,6 +142,13 @@ def test_time_shift_argument_errors(W):
 
 def test_chunk_and_wkv6_argument_errors(W):
     L = W.lib()
+    dec = lambda S=4, C=8, dt=0, k=FAKE, state=FAKE: L.wkv4_decode_step(S, C, dt, FAKE, FAKE, k, FAKE, FAKE, state,
+                                                                       None)
+    assert dec(k=None) == W.WKV_ERR_INVALID_ARG and b"k is NULL" in L.wkv_last_error()
+    assert dec(state=FAKE + 4) == W.WKV_ERR_INVALID_ARG and b"state" in L.wkv_last_error()
+    assert dec(C=6) == W.WKV_ERR_UNSUPPORTED
+    assert dec(S=-1) == W.WKV_ERR_INVALID_ARG
+    assert dec(S=0, k=None, state=None) == W.WKV_OK
     assert L.wkv4_chunk_step(4, 8, 0, FAKE, FAKE, FAKE, FAKE, FAKE, -1, FAKE, FAKE, None) == W.WKV_ERR_INVALID_ARG
     assert L.wkv4_chunk_step(4, 8, 0, FAKE, FAKE, FAKE, FAKE, FAKE, 10, None, FAKE, None) == W.WKV_ERR_INVALID_ARG
     assert L.wkv4_chunk_step(0, 8, 0, FAKE, FAKE, FAKE, FAKE, FAKE, 0, FAKE, FAKE, None) == W.WKV_OK
