@@ -66,7 +66,8 @@ def parse():
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the secondary workloads (larger shapes, chunk step, RWKV-6)")
     ap.add_argument("--kernel", choices=["wkv4_fwd", "wkv4_bwd", "wkv4_fwd_gated", "wkv4_bwd_gated", "wkv6_fwd",
-                                         "wkv6_bwd", "wkv7_fwd", "wkv4_chunk", "time_shift_fwd", "time_shift_bwd"],
+                                         "wkv6_bwd", "wkv7_fwd", "wkv4_chunk", "wkv4_decode", "time_shift_fwd",
+                                         "time_shift_bwd"],
                     help="profiling mode: run only this kernel --steps times on --workload (no JSON line)")
     ap.add_argument("--workload", default=None,
                     help="with --kernel: a recipe name of synth (RWKV-4 or RWKV-6), optionally resized "
@@ -725,6 +726,15 @@ def run_kernel_only(args):
             wkv.wkv4_state_init(S, C, dev, state=state)
             for kc, vc, cu in calls:
                 wkv.wkv4_chunk_step(w, u, kc, vc, cu, state)
+    elif args.kernel == "wkv4_decode":
+        S, C = 256, 4096
+        w = torch.exp(torch.rand(C, device=dev, generator=g) * 7.0 - 6.0)
+        u = torch.rand(C, device=dev, generator=g) * 2.0 - 1.0
+        kd = torch.randn(S, C, device=dev, generator=g).to(torch.bfloat16)
+        vd = torch.randn(S, C, device=dev, generator=g).to(torch.bfloat16)
+        state = wkv.wkv4_state_init(S, C, dev)
+        for _ in range(args.steps):
+            wkv.wkv4_decode_step(w, u, kd, vd, state)
     elif args.kernel in ("time_shift_fwd", "time_shift_bwd"):
         B, T, C = (int(v) for v in (resize or "16,4096,4096").split(","))
         xs = torch.randn(B, T, C, device=dev, generator=g).to(torch.bfloat16)
