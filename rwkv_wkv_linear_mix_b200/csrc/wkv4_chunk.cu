@@ -3,25 +3,33 @@
 // batched inference: num_batch slots, at most token_chunk_size tokens per
 // run() call, empty slots skipped, state persisting between calls).
 //
-// A thread serves 4 adjacent channels of one slot: it loads the slot's
-// (aa, bb, base, n, ref) rows for them as 16-byte words, runs the same
-// float32 step as wkv4_forward (its packed pair form, two pairs) over the
-// slot's tokens of this call, writes y and stores the state back. A call moves at
-// most a few tens of MB, so the kernel is bound by latency and by the bytes
-// it has in flight: each thread issues the loads of a whole group of tokens
-// (kept packed until used) before it starts computing, and 8- or 16-byte
-// accesses give a warp 128 channels of a token row per load.
+// A thread serves a channel pair of one slot: it loads the slot's
+// (aa, bb, base, n, ref) for them, runs the same float32 step as
+// wkv4_forward (its packed pair form) over the slot's tokens of this call,
+// writes y and stores the state back. A slot's tokens are a serial chain, so
+// the kernel is bound by latency: each thread issues the loads of a whole
+// group of tokens (kept packed until used), the first group before the
+// state, and a thread per pair gives the SMs as many warps as the batch has.
 #include "wkv_device.cuh"
 #include "wkv_internal.h"
 
 namespace wkv {
 
-constexpr int kChunkThreads = 128;
+// Channels per thread (2: one packed pair, or 4: two pairs) and threads per
+// CTA. Two channels per thread give twice the warps, which is what the
+// latency-bound token chains want; four give wider accesses.
+#ifndef WKV4_CHUNK_CH
+#define WKV4_CHUNK_CH 2
+#endif
+constexpr int kChunkCh = WKV4_CHUNK_CH;
+constexpr int kChunkThreads = kChunkCh == 2 ? 64 : 128;
+constexpr int kChunkMinBlocks = kChunkCh == 2 ? 8 : 1;  // two channels: <= 128 registers, 16 warps per SM
 
-template <class E>
-struct ChunkRaw;  // 4 channels of one token, packed
+// NCH channels of one token, packed as loaded.
+template <class E, int NCH>
+struct ChunkRaw;
 template <>
-struct ChunkRaw<float> {
+struct ChunkRaw<float, 4> {
   using T = float4;
   static constexpr int kGroup = 16;
   static __device__ __forceinline__ void unpack(const T& q, float (&f)[4]) {
@@ -35,7 +43,7 @@ struct ChunkRaw<float> {
   }
 };
 template <>
-struct ChunkRaw<__nv_bfloat16> {
+struct ChunkRaw<__nv_bfloat16, 4> {
   using T = uint2;
   static constexpr int kGroup = 32;
   static __device__ __forceinline__ void unpack(const T& q, float (&f)[4]) {
@@ -48,25 +56,46 @@ struct ChunkRaw<__nv_bfloat16> {
     *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]));
   }
 };
-
-__device__ __forceinline__ float comp4(const float4& x, int j) {
-  return j == 0 ? x.x : j == 1 ? x.y : j == 2 ? x.z : x.w;
-}
+template <>
+struct ChunkRaw<float, 2> {
+  using T = float2;
+  static constexpr int kGroup = 16;
+  static __device__ __forceinline__ void unpack(const T& q, float (&f)[2]) {
+    f[0] = q.x;
+    f[1] = q.y;
+  }
+  static __device__ __forceinline__ void store(float* p, const float (&f)[2]) {
+    *reinterpret_cast<float2*>(p) = make_float2(f[0], f[1]);
+  }
+};
+template <>
+struct ChunkRaw<__nv_bfloat16, 2> {
+  using T = uint32_t;
+  static constexpr int kGroup = 16;
+  static __device__ __forceinline__ void unpack(const T& q, float (&f)[2]) {
+    f[0] = bf16lo(q);
+    f[1] = bf16hi(q);
+  }
+  static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&f)[2]) {
+    *reinterpret_cast<uint32_t*>(p) = pack_bf16x2(f[0], f[1]);
+  }
+};
 
 template <class E>
-__global__ void __launch_bounds__(kChunkThreads) wkv4_chunk_kernel(int S, int C, const float* __restrict__ w,
+__global__ void __launch_bounds__(kChunkThreads, kChunkMinBlocks) wkv4_chunk_kernel(int S, int C, const float* __restrict__ w,
                                                                   const float* __restrict__ u,
                                                                   const E* __restrict__ k, const E* __restrict__ v,
                                                                   E* __restrict__ y, int64_t n_tokens,
                                                                   const int32_t* __restrict__ cu,
                                                                   float* __restrict__ state, unsigned* err) {
-  using R = ChunkRaw<E>;
+  constexpr int NCH = kChunkCh, NP = NCH / 2;
+  using R = ChunkRaw<E, NCH>;
   constexpr int G = R::kGroup;
-  const int nq = C / 4;
+  const int nq = C / NCH;
   const int64_t gid = (int64_t)blockIdx.x * kChunkThreads + threadIdx.x;
   if (gid >= (int64_t)S * nq) return;
   const int s = (int)(gid / nq);
-  const int c = (int)(gid - (int64_t)s * nq) * 4;
+  const int c = (int)(gid - (int64_t)s * nq) * NCH;
   const int64_t beg = cu[s];
   const int64_t end = cu[s + 1];
   if (end == beg) return;  // empty slot: skipped, state untouched
@@ -92,39 +121,35 @@ __global__ void __launch_bounds__(kChunkThreads) wkv4_chunk_kernel(int S, int C,
   };
   load_group(0);
 
-  float* sp = state + (int64_t)s * 5 * C + c;
-  const float4 aa = *reinterpret_cast<const float4*>(sp), bb = *reinterpret_cast<const float4*>(sp + C),
-               base = *reinterpret_cast<const float4*>(sp + 2 * (int64_t)C),
-               nn = *reinterpret_cast<const float4*>(sp + 3 * (int64_t)C),
-               rf = *reinterpret_cast<const float4*>(sp + 4 * (int64_t)C);
-  const float4 w4 = *reinterpret_cast<const float4*>(w + c), u4 = *reinterpret_cast<const float4*>(u + c);
-  // two channel pairs, each on the packed fp32 pair form of the step (its
+  // NP channel pairs, each on the packed fp32 pair form of the step (its
   // components round exactly as the scalar step)
-  Wkv4State2 st[2];
-  float2 ref[2], w2[2], u2[2];
-  float k0[4];
+  float* sp = state + (int64_t)s * 5 * C + c;
+  Wkv4State2 st[NP];
+  float2 ref[NP], w2[NP], u2[NP];
+  float k0[NCH];
   R::unpack(kr[0], k0);
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
+  for (int h = 0; h < NP; ++h) {
     const int j = 2 * h;
-    st[h] = {make_float2(comp4(aa, j), comp4(aa, j + 1)), make_float2(comp4(bb, j), comp4(bb, j + 1)),
-             make_float2(comp4(base, j), comp4(base, j + 1)), make_float2(comp4(nn, j), comp4(nn, j + 1))};
+    st[h] = {ld_pair(sp + j), ld_pair(sp + C + j), ld_pair(sp + 2 * (int64_t)C + j), ld_pair(sp + 3 * (int64_t)C + j)};
+    const float2 rf = ld_pair(sp + 4 * (int64_t)C + j);
     // a slot that has absorbed nothing yet takes its reference from this call's first token
-    ref[h] = make_float2(st[h].base.x == kEmptyPP ? wkv4_ref(k0[j]) : comp4(rf, j),
-                         st[h].base.y == kEmptyPP ? wkv4_ref(k0[j + 1]) : comp4(rf, j + 1));
-    w2[h] = make_float2(__fmul_rn(comp4(w4, j), kLog2e), __fmul_rn(comp4(w4, j + 1), kLog2e));
-    u2[h] = make_float2(__fmul_rn(comp4(u4, j), kLog2e), __fmul_rn(comp4(u4, j + 1), kLog2e));
+    ref[h] = make_float2(st[h].base.x == kEmptyPP ? wkv4_ref(k0[j]) : rf.x,
+                         st[h].base.y == kEmptyPP ? wkv4_ref(k0[j + 1]) : rf.y);
+    const float2 wc = ld_pair(w + c + j), uc = ld_pair(u + c + j);
+    w2[h] = make_float2(__fmul_rn(wc.x, kLog2e), __fmul_rn(wc.y, kLog2e));
+    u2[h] = make_float2(__fmul_rn(uc.x, kLog2e), __fmul_rn(uc.y, kLog2e));
   }
   for (int64_t t0 = 0; t0 < n; t0 += G) {
     if (t0 > 0) load_group(t0);
 #pragma unroll
     for (int j = 0; j < G; ++j) {
       if (t0 + j < n) {
-        float kk[4], vv[4], yy[4];
+        float kk[NCH], vv[NCH], yy[NCH];
         R::unpack(kr[j], kk);
         R::unpack(vr[j], vv);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < NP; ++h) {
           const float2 yv = wkv4_token2(st[h], wkv4_key2(make_float2(kk[2 * h], kk[2 * h + 1]), ref[h]),
                                         make_float2(vv[2 * h], vv[2 * h + 1]), u2[h], w2[h]);
           yy[2 * h] = yv.x;
@@ -134,12 +159,15 @@ __global__ void __launch_bounds__(kChunkThreads) wkv4_chunk_kernel(int S, int C,
       }
     }
   }
-  *reinterpret_cast<float4*>(sp) = make_float4(st[0].aa.x, st[0].aa.y, st[1].aa.x, st[1].aa.y);
-  *reinterpret_cast<float4*>(sp + C) = make_float4(st[0].bb.x, st[0].bb.y, st[1].bb.x, st[1].bb.y);
-  *reinterpret_cast<float4*>(sp + 2 * (int64_t)C) =
-      make_float4(st[0].base.x, st[0].base.y, st[1].base.x, st[1].base.y);
-  *reinterpret_cast<float4*>(sp + 3 * (int64_t)C) = make_float4(st[0].n.x, st[0].n.y, st[1].n.x, st[1].n.y);
-  *reinterpret_cast<float4*>(sp + 4 * (int64_t)C) = make_float4(ref[0].x, ref[0].y, ref[1].x, ref[1].y);
+#pragma unroll
+  for (int h = 0; h < NP; ++h) {
+    const int j = 2 * h;
+    st_pair(sp + j, st[h].aa);
+    st_pair(sp + C + j, st[h].bb);
+    st_pair(sp + 2 * (int64_t)C + j, st[h].base);
+    st_pair(sp + 3 * (int64_t)C + j, st[h].n);
+    st_pair(sp + 4 * (int64_t)C + j, ref[h]);
+  }
 }
 
 __global__ void wkv4_state_init_kernel(int64_t total, int C, float* __restrict__ state) {
@@ -160,7 +188,7 @@ wkv_status launch_wkv4_state_init(int64_t S, int64_t C, float* state, cudaStream
 }
 
 wkv_status launch_wkv4_chunk_step(const Wkv4ChunkArgs& a, cudaStream_t stream, unsigned* err, const char** why) {
-  const unsigned grid = (unsigned)ceil_div(a.S * (a.C / 4), kChunkThreads);
+  const unsigned grid = (unsigned)ceil_div(a.S * (a.C / kChunkCh), kChunkThreads);
   if (a.dtype == WKV_BF16)
     wkv4_chunk_kernel<__nv_bfloat16><<<grid, kChunkThreads, 0, stream>>>(
         (int)a.S, (int)a.C, a.w, a.u, static_cast<const __nv_bfloat16*>(a.k), static_cast<const __nv_bfloat16*>(a.v),
