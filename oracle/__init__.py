@@ -66,6 +66,8 @@ def _open(path):
     lib.oracle_wkv7_forward.argtypes = [i64, i64, i64, i64] + [dp] * 9
     lib.oracle_wkv7_forward.restype = ctypes.c_int
     lib.oracle_wkv6_backward.restype = ctypes.c_int
+    lib.oracle_wkv7_backward.argtypes = [i64, i64, i64, i64] + [dp] * 16
+    lib.oracle_wkv7_backward.restype = ctypes.c_int
     lib.oracle_time_shift_mix.argtypes = [i64, i64, i64, i64] + [dp] * 4
     lib.oracle_time_shift_mix.restype = ctypes.c_int
     lib.oracle_time_shift_mix_backward.argtypes = [i64, i64, i64, i64] + [dp] * 7
@@ -296,6 +298,29 @@ def wkv7_forward(r, w, k, v, a, b, init_state=None, head_size: int = 64, _lib=No
     if rc != 0:
         raise FloatingPointError(f"oracle_wkv7_forward failed (rc={rc})")
     return o, fs
+
+
+def wkv7_backward(r, w, k, v, a, b, dout, init_state=None, g_final=None, head_size: int = 64, _lib=None):
+    """Gradients of sum(dout * o) + sum(g_final * S_final) for wkv7_forward
+    (see oracle_wkv7_backward), in fp64. Returns (dr, dw, dk, dv, da, db,
+    d_init); dw is with respect to the log decay w."""
+    lib = _lib or _load()
+    r, w, k, v, a, b, dout = (_f64(x) for x in (r, w, k, v, a, b, dout))
+    B, T, HK = r.shape
+    K = head_size
+    assert HK % K == 0 and all(x.shape == r.shape for x in (w, k, v, a, b, dout))
+    H = HK // K
+    s0 = None if init_state is None else _f64(init_state)
+    gf = None if g_final is None else _f64(g_final)
+    for x in (s0, gf):
+        assert x is None or x.shape == (B, H, K, K)
+    outs = [np.empty_like(r) for _ in range(6)]
+    d_init = np.empty((B, H, K, K))
+    rc = lib.oracle_wkv7_backward(B, T, H, K, _ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(a), _ptr(b), _ptr(s0),
+                                  _ptr(dout), _ptr(gf), *[_ptr(o) for o in outs], _ptr(d_init))
+    if rc != 0:
+        raise FloatingPointError(f"oracle_wkv7_backward failed (rc={rc})")
+    return (*outs, d_init)
 
 
 def time_shift_mix(x, mix, x_prev=None, _lib=None):

@@ -41,6 +41,10 @@
  *
  *      S_t = (diag(e^{w_t}) + b_t a_t^T) S_{t-1} + k_t^T v_t,    o_t = r_t S_t
  *
+ *  and its backward (the page's generalized_delta_rule carries gradients;
+ *  its _inference twin does not): the chain rule with G_t = dL/dS_t walked
+ *  down, every S_t stored.
+ *
  *  Time-shift mix (the prologue of RWKV_TimeMix.jit_func on the same RWKV-4
  *  page): the input shifted one token along T blended per channel with the
  *  token itself, once for each of k, v, r, and its backward.
@@ -500,6 +504,126 @@ int oracle_wkv7_forward(int64_t B, int64_t T, int64_t H, int64_t K,
         }
         free(S);
         free(sa);
+    }
+    return bad;
+}
+
+/* ------------------------------------------------------------------------ */
+/* RWKV-7 generalized delta rule, backward                                   */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Gradients of L = sum_t sum_i dout_t[i] o_t[i] + sum g_final o S_{T-1} for
+ * the forward above (g_final nullable: 0). With G = dL/dS_t, per token from
+ * the last one down (j the key index, i the value index, d = e^{w_t}):
+ *
+ *   G[j][i]  += r_t[j] dout_t[i]                    (o_t reads S_t)
+ *   dr_t[j]   = sum_i S_t[j][i] dout_t[i]
+ *   dv_t[i]   = sum_j k_t[j] G[j][i]
+ *   dk_t[j]   = sum_i G[j][i] v_t[i]
+ *   db_t[j]   = sum_i G[j][i] sa[i]
+ *   dsa[i]    = sum_j b_t[j] G[j][i]
+ *   dw_t[j]   = d[j] sum_i G[j][i] S_{t-1}[j][i]     (w is the log decay)
+ *   da_t[j]   = sum_i S_{t-1}[j][i] dsa[i]           (sa = a_t S_{t-1})
+ *   G[j][i]  <- d[j] G[j][i] + a_t[j] dsa[i]         (G becomes dL/dS_{t-1})
+ *
+ * and d_init = G after token 0. Shapes as for oracle_wkv7_forward; dout,
+ * dr, dw, dk, dv, da, db [B][T][H*K]; init_state, g_final, d_init
+ * [B][H][K][K] (init_state, g_final nullable; d_init written).
+ * Returns 0 on success, 1 on a non-finite result, 2 on allocation failure.
+ */
+int oracle_wkv7_backward(int64_t B, int64_t T, int64_t H, int64_t K,
+                         const double *r, const double *w, const double *k, const double *v,
+                         const double *a, const double *b, const double *init_state,
+                         const double *dout, const double *g_final,
+                         double *dr, double *dw, double *dk, double *dv, double *da, double *db,
+                         double *d_init)
+{
+    const int64_t HK = H * K, KK = K * K;
+    int bad = 0;
+    #pragma omp parallel reduction(|:bad)
+    {
+        double *Sh = (double *)malloc(sizeof(double) * (size_t)((T + 1) * KK));  /* Sh[t] = S_{t-1} */
+        double *SA = (double *)malloc(sizeof(double) * (size_t)(T * K));         /* sa of every token */
+        double *G = (double *)malloc(sizeof(double) * (size_t)KK);
+        double *dsa = (double *)malloc(sizeof(double) * (size_t)K);
+        if (!Sh || !SA || !G || !dsa) bad = 2;
+        #pragma omp for collapse(2) schedule(static)
+        for (int64_t bi = 0; bi < B; ++bi) {
+            for (int64_t h = 0; h < H; ++h) {
+                if (!Sh || !SA || !G || !dsa) continue;
+                const double *S0 = init_state ? init_state + (bi * H + h) * KK : NULL;
+                for (int64_t e = 0; e < KK; ++e) Sh[e] = S0 ? S0[e] : 0.0;
+                /* forward, keeping every state */
+                for (int64_t t = 0; t < T; ++t) {
+                    const int64_t row = (bi * T + t) * HK + h * K;
+                    const double *S = Sh + t * KK;
+                    double *Sn = Sh + (t + 1) * KK;
+                    for (int64_t i = 0; i < K; ++i) {
+                        double proj = 0.0;
+                        for (int64_t j = 0; j < K; ++j) proj += a[row + j] * S[j * K + i];
+                        SA[t * K + i] = proj;
+                    }
+                    for (int64_t j = 0; j < K; ++j)
+                        for (int64_t i = 0; i < K; ++i)
+                            Sn[j * K + i] = exp(w[row + j]) * S[j * K + i] + b[row + j] * SA[t * K + i]
+                                            + k[row + j] * v[row + i];
+                }
+                /* reverse */
+                const double *GF = g_final ? g_final + (bi * H + h) * KK : NULL;
+                for (int64_t e = 0; e < KK; ++e) G[e] = GF ? GF[e] : 0.0;
+                for (int64_t t = T - 1; t >= 0; --t) {
+                    const int64_t row = (bi * T + t) * HK + h * K;
+                    const double *Sp = Sh + t * KK;        /* S_{t-1} */
+                    const double *St = Sh + (t + 1) * KK;  /* S_t */
+                    const double *sa = SA + t * K;
+                    for (int64_t j = 0; j < K; ++j)
+                        for (int64_t i = 0; i < K; ++i) G[j * K + i] += r[row + j] * dout[row + i];
+                    for (int64_t j = 0; j < K; ++j) {
+                        double sr = 0.0, sk = 0.0, sb = 0.0, sw = 0.0;
+                        for (int64_t i = 0; i < K; ++i) {
+                            sr += St[j * K + i] * dout[row + i];
+                            sk += G[j * K + i] * v[row + i];
+                            sb += G[j * K + i] * sa[i];
+                            sw += G[j * K + i] * Sp[j * K + i];
+                        }
+                        dr[row + j] = sr;
+                        dk[row + j] = sk;
+                        db[row + j] = sb;
+                        dw[row + j] = exp(w[row + j]) * sw;
+                    }
+                    for (int64_t i = 0; i < K; ++i) {
+                        double sv = 0.0, ss = 0.0;
+                        for (int64_t j = 0; j < K; ++j) {
+                            sv += k[row + j] * G[j * K + i];
+                            ss += b[row + j] * G[j * K + i];
+                        }
+                        dv[row + i] = sv;
+                        dsa[i] = ss;
+                    }
+                    for (int64_t j = 0; j < K; ++j) {
+                        double s = 0.0;
+                        for (int64_t i = 0; i < K; ++i) s += Sp[j * K + i] * dsa[i];
+                        da[row + j] = s;
+                    }
+                    for (int64_t j = 0; j < K; ++j)
+                        for (int64_t i = 0; i < K; ++i)
+                            G[j * K + i] = exp(w[row + j]) * G[j * K + i] + a[row + j] * dsa[i];
+                }
+                memcpy(d_init + (bi * H + h) * KK, G, sizeof(double) * (size_t)KK);
+                if (!all_finite(G, KK)) bad |= 1;
+            }
+        }
+        free(Sh);
+        free(SA);
+        free(G);
+        free(dsa);
+    }
+    if (!bad) {
+        const int64_t n = B * T * HK;
+        if (!all_finite(dr, n) || !all_finite(dw, n) || !all_finite(dk, n) || !all_finite(dv, n) ||
+            !all_finite(da, n) || !all_finite(db, n))
+            bad = 1;
     }
     return bad;
 }

@@ -49,6 +49,13 @@ MUTATIONS = {
     # RWKV-7: the read leaves out the current token's write
     "wkv7_read_without_token": ("for (int64_t j = 0; j < K; ++j) acc += r[row + j] * S[j * K + i];",
                                 "for (int64_t j = 0; j < K; ++j) acc += r[row + j] * (S[j * K + i] - k[row + j] * v[row + i]);"),
+    # RWKV-7 backward: the rank-one term dropped from the adjoint walk
+    "wkv7b_drop_rank_one": ("G[j * K + i] = exp(w[row + j]) * G[j * K + i] + a[row + j] * dsa[i];",
+                            "G[j * K + i] = exp(w[row + j]) * G[j * K + i];"),
+    # RWKV-7 backward: the decay gradient without the chain factor e^{w}
+    "wkv7b_dw_factor": ("dw[row + j] = exp(w[row + j]) * sw;", "dw[row + j] = sw;"),
+    # RWKV-7 backward: dr taken against S_{t-1} instead of S_t
+    "wkv7b_dr_state": ("sr += St[j * K + i] * dout[row + i];", "sr += Sp[j * K + i] * dout[row + i];"),
     # time-shift mix: blend weights swapped between the token and the one before
     "tsm_swap_weights": ("const double o = xt * mix[m * C + c] + xx * (1.0 - mix[m * C + c]);",
                          "const double o = xx * mix[m * C + c] + xt * (1.0 - mix[m * C + c]);"),
@@ -129,6 +136,20 @@ def _wkv7_pins_fail(var):
     return False
 
 
+def _wkv7b_pins_fail(var):
+    import test_oracle_wkv7 as p7
+
+    class _Adapter:
+        wkv7_forward = staticmethod(var.wkv7_forward)
+        wkv7_backward = staticmethod(var.wkv7_backward)
+    for pin in (lambda o: p7.test_backward_matches_finite_differences(o, True), p7.test_backward_homogeneity):
+        try:
+            pin(_Adapter)
+        except AssertionError:
+            return True
+    return False
+
+
 def _tsm_pins_fail(var):
     import test_oracle_time_shift as pt
 
@@ -148,6 +169,7 @@ def _tsm_pins_fail(var):
 @pytest.mark.parametrize("name", sorted(MUTATIONS))
 def test_mutation_is_caught(variants, name):
     check = (_wkv4_pins_fail if name.startswith("wkv4") else
+             _wkv7b_pins_fail if name.startswith("wkv7b") else
              _tsm_pins_fail if name.startswith("tsm") else
              _wkv7_pins_fail if name.startswith("wkv7") else
              _wkv6b_pins_fail if name.startswith("wkv6b") else _wkv6_pins_fail)
@@ -161,10 +183,12 @@ def test_unmutated_source_passes(oracle):
         wkv6_forward = staticmethod(oracle.wkv6_forward)
         wkv6_backward = staticmethod(oracle.wkv6_backward)
         wkv7_forward = staticmethod(oracle.wkv7_forward)
+        wkv7_backward = staticmethod(oracle.wkv7_backward)
         time_shift_mix = staticmethod(oracle.time_shift_mix)
         time_shift_mix_backward = staticmethod(oracle.time_shift_mix_backward)
     assert not _wkv4_pins_fail(_Orig)
     assert not _tsm_pins_fail(_Orig)
+    assert not _wkv7b_pins_fail(_Orig)
     assert not _wkv7_pins_fail(_Orig)
     assert not _wkv6_pins_fail(_Orig)
     assert not _wkv6b_pins_fail(_Orig)

@@ -133,3 +133,68 @@ def test_linear_in_values_and_initial_state(oracle):
     oc, fc = oracle.wkv7_forward(r, w, k, 2 * v1 - 3 * v2, a, b, init_state=2 * s1 - 3 * s2, head_size=K)
     assert rel_err(oc, 2 * oa - 3 * ob) < 1e-12
     assert rel_err(fc, 2 * fa - 3 * fb) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# backward (the page's generalized_delta_rule carries gradients)
+# ---------------------------------------------------------------------------
+
+def _wkv7_loss(oracle, args, dout, init, gfin, K):
+    o, fs = oracle.wkv7_forward(*args, init_state=init, head_size=K)
+    return float(np.sum(dout * o) + (0.0 if gfin is None else np.sum(gfin * fs)))
+
+
+def _wkv7_draw(seed, B=1, T=5, H=2, K=3):
+    rng = np.random.default_rng(seed)
+    shape = (B, T, H * K)
+    r, k, v = (rng.normal(size=shape) for _ in range(3))
+    w = -np.exp(rng.normal(-1.0, 0.5, size=shape))
+    kap = unit_rows(rng, B * T * H, K).reshape(shape)
+    a, b = -kap, kap * rng.uniform(0, 1, size=shape)
+    dout = rng.normal(size=shape)
+    init = rng.normal(size=(B, H, K, K))
+    gfin = rng.normal(size=(B, H, K, K))
+    return [r, w, k, v, a, b], dout, init, gfin
+
+
+@pytest.mark.parametrize("with_state", [False, True])
+def test_backward_matches_finite_differences(oracle, with_state):
+    """Central differences of L = sum(dout * o) (+ sum(g_final * S_final) and
+    an initial state) in every entry of r, w, k, v, a, b and the initial
+    state; the loss is a polynomial of low degree in each entry, so h = 1e-5
+    leaves only rounding."""
+    K = 3
+    args, dout, init, gfin = _wkv7_draw(5 + with_state, K=K)
+    if not with_state:
+        init = gfin = None
+    got = oracle.wkv7_backward(*args, dout, init_state=init, g_final=gfin, head_size=K)
+    h = 1e-5
+    for n in range(6):
+        num = np.zeros_like(args[n])
+        for idx in np.ndindex(args[n].shape):
+            hi = [x.copy() for x in args]
+            lo = [x.copy() for x in args]
+            hi[n][idx] += h
+            lo[n][idx] -= h
+            num[idx] = (_wkv7_loss(oracle, hi, dout, init, gfin, K) - _wkv7_loss(oracle, lo, dout, init, gfin, K)) / (2 * h)
+        assert rel_err(got[n], num) < 1e-7, "rwkabv"[n]
+    s0 = init if init is not None else np.zeros((1, 2, K, K))
+    num = np.zeros_like(s0)
+    for idx in np.ndindex(s0.shape):
+        hi, lo = s0.copy(), s0.copy()
+        hi[idx] += h
+        lo[idx] -= h
+        num[idx] = (_wkv7_loss(oracle, args, dout, hi, gfin, K) - _wkv7_loss(oracle, args, dout, lo, gfin, K)) / (2 * h)
+    assert rel_err(got[6], num) < 1e-7
+
+
+def test_backward_homogeneity(oracle):
+    """o is linear in r, and jointly linear in (v, S_init) (the state
+    transition does not depend on them): Euler's identity gives
+    sum r dr = L and sum v dv + sum S_init d_init = L for L = sum(dout * o)."""
+    K = 4
+    args, dout, init, _ = _wkv7_draw(9, T=7, K=K)
+    L = _wkv7_loss(oracle, args, dout, init, None, K)
+    dr, dw, dk, dv, da, db, di = oracle.wkv7_backward(*args, dout, init_state=init, head_size=K)
+    assert abs(np.sum(args[0] * dr) - L) < 1e-10 * max(1.0, abs(L))
+    assert abs(np.sum(args[3] * dv) + np.sum(init * di) - L) < 1e-10 * max(1.0, abs(L))
