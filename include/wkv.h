@@ -407,6 +407,36 @@ wkv_status wkv7_forward(int64_t B, int64_t T, int64_t H, int64_t K, int dtype,
                         const void *a, const void *b,
                         const float *init_state, float *final_state, void *o, void *stream);
 
+/* Bytes of device workspace wkv7_backward needs (0 for an unsupported shape). */
+size_t wkv7_backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K);
+
+/*
+ * Gradients of L = sum(dout * o) + sum(g_final * S_final) for
+ * o, S_final = wkv7_forward(...) on the same inputs (generalized_delta_rule
+ * of the rwkv-ops package page carries gradients). With G = dL/dS_t walked
+ * down from the last token (j key, i value, d = e^{w_t}, sa = a_t S_{t-1}):
+ *   G += r_t^T dout_t;  dr_t = S_t dout_t;  dk_t = G v_t;  db_t = G sa;
+ *   dw_t = d o rowsum(G o S_{t-1});  dsa = b_t G;  dv_t = k_t G;
+ *   da_t = S_{t-1} dsa;  G <- diag(d) G + a_t^T dsa;  d_init = G at the end.
+ *   r, w, k, v, a, b, dout  [B][T][H*K] bf16 (w the log decay, as for
+ *               wkv7_forward); dw is the gradient with respect to w.
+ *   init_state  [B][H][K][K] float32 or NULL (zeros), as for the forward.
+ *   g_final     [B][H][K][K] float32 or NULL (no final-state term).
+ *   dr, dw, dk, dv, da, db  [B][T][H*K] bf16, written.
+ *   d_init      [B][H][K][K] float32, written (dL/dS_init).
+ *   workspace   device scratch of at least wkv7_backward_workspace_bytes
+ *               bytes: the state before every 4th token, written by a
+ *               checkpoint sweep of the forward kernel, read back per group.
+ * bf16 and K = 64 only (WKV_ERR_UNSUPPORTED otherwise). T = 0 gives
+ * d_init = g_final (or 0). Launches two kernels on `stream`.
+ */
+wkv_status wkv7_backward(int64_t B, int64_t T, int64_t H, int64_t K, int dtype,
+                         const void *r, const void *w, const void *k, const void *v,
+                         const void *a, const void *b, const float *init_state,
+                         const void *dout, const float *g_final,
+                         void *dr, void *dw, void *dk, void *dv, void *da, void *db,
+                         float *d_init, void *workspace, size_t workspace_bytes, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

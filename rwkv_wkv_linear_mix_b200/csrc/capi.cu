@@ -382,6 +382,61 @@ WKV_EXPORT wkv_status wkv7_forward(int64_t B, int64_t T, int64_t H, int64_t K, i
   return s == WKV_OK ? s : fail(s, why);
 }
 
+WKV_EXPORT size_t wkv7_backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K) {
+  if (B <= 0 || T <= 0 || H <= 0 || K != 64) return 0;
+  return (size_t)B * (size_t)H * (size_t)ceil_div(T, WKV7_CKPT_LEN) * 64u * 64u * sizeof(float);
+}
+
+WKV_EXPORT wkv_status wkv7_backward(int64_t B, int64_t T, int64_t H, int64_t K, int dtype, const void* r,
+                                    const void* w, const void* k, const void* v, const void* a, const void* b,
+                                    const float* init_state, const void* dout, const float* g_final, void* dr,
+                                    void* dw, void* dk, void* dv, void* da, void* db, float* d_init,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+  if (B < 0 || T < 0 || H < 0 || K < 0) return fail(WKV_ERR_INVALID_ARG, "negative size");
+  if (dtype != WKV_F32 && dtype != WKV_BF16) return fail(WKV_ERR_INVALID_ARG, "unknown dtype");
+  if (dtype != WKV_BF16) return fail(WKV_ERR_UNSUPPORTED, "wkv7_backward supports bf16 only");
+  if (K != 64) return fail(WKV_ERR_UNSUPPORTED, "wkv7_backward supports head size 64 only");
+  if (B == 0 || H == 0) return WKV_OK;
+  if (T > INT32_MAX || H > 65535 || B * H > INT32_MAX) return fail(WKV_ERR_UNSUPPORTED, "size out of range");
+  WKV_OPTIONAL_PTR(init_state, "init_state");
+  WKV_OPTIONAL_PTR(g_final, "g_final");
+  WKV_REQUIRE_PTR(d_init, "d_init");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t state_bytes = (size_t)B * (size_t)H * 64u * 64u * sizeof(float);
+  if (T == 0) {
+    // nothing flows through time: d_init = g_final (or 0)
+    const cudaError_t e = g_final ? cudaMemcpyAsync(d_init, g_final, state_bytes, cudaMemcpyDeviceToDevice, st)
+                                  : cudaMemsetAsync(d_init, 0, state_bytes, st);
+    return e == cudaSuccess ? WKV_OK : fail(WKV_ERR_CUDA, "copy of g_final failed");
+  }
+  WKV_REQUIRE_PTR(r, "r");
+  WKV_REQUIRE_PTR(w, "w");
+  WKV_REQUIRE_PTR(k, "k");
+  WKV_REQUIRE_PTR(v, "v");
+  WKV_REQUIRE_PTR(a, "a");
+  WKV_REQUIRE_PTR(b, "b");
+  WKV_REQUIRE_PTR(dout, "dout");
+  WKV_REQUIRE_PTR(dr, "dr");
+  WKV_REQUIRE_PTR(dw, "dw");
+  WKV_REQUIRE_PTR(dk, "dk");
+  WKV_REQUIRE_PTR(dv, "dv");
+  WKV_REQUIRE_PTR(da, "da");
+  WKV_REQUIRE_PTR(db, "db");
+  WKV_REQUIRE_PTR(workspace, "workspace");
+  if (workspace_bytes < wkv7_backward_workspace_bytes(B, T, H, K))
+    return fail(WKV_ERR_INVALID_ARG, "workspace_bytes below wkv7_backward_workspace_bytes()");
+  unsigned* err = nullptr;
+  if (wkv_status s = device_error_ptr(&err)) return s;
+  const char* why = "";
+  float* ck = static_cast<float*>(workspace);
+  Wkv7FwdArgs fa{B, T, H, K, r, w, k, v, a, b, init_state, nullptr, nullptr};
+  fa.ckpt = ck;
+  if (wkv_status s = launch_wkv7_forward(fa, st, err, &why)) return fail(s, why);
+  Wkv7BwdArgs ba{B, T, H, r, w, k, v, a, b, dout, ck, g_final, dr, dw, dk, dv, da, db, d_init};
+  wkv_status s = launch_wkv7_backward(ba, st, &why);
+  return s == WKV_OK ? s : fail(s, why);
+}
+
 WKV_EXPORT wkv_status wkv_wait_selfcheck(int64_t limit_ns, void* stream) {
   if (limit_ns < 1000 || limit_ns > 10000000000ll) return fail(WKV_ERR_INVALID_ARG, "limit_ns outside 1 us .. 10 s");
   unsigned* err = nullptr;

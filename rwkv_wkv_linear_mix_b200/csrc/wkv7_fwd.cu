@@ -66,12 +66,15 @@ struct Wkv7Tok {
   uint2 v;
 };
 
+// CKPT: the backward's forward sweep: no output, the state before every
+// WKV7_CKPT_LEN-th token written to ckpt [B*H][ceil(T / WKV7_CKPT_LEN)][K][K].
+template <bool CKPT>
 __global__ void __launch_bounds__(kT7, 3) wkv7_fwd_kernel(
     const __grid_constant__ CUtensorMap tr, const __grid_constant__ CUtensorMap tw,
     const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
     const __grid_constant__ CUtensorMap ta, const __grid_constant__ CUtensorMap tb, int T, int H,
     const float* __restrict__ init_state, float* __restrict__ final_state, __nv_bfloat16* __restrict__ o,
-    unsigned* err) {
+    float* __restrict__ ckpt, unsigned* err) {
   extern __shared__ __align__(128) unsigned char wkv7_dsmem[];
   Wkv7Smem& sm = *reinterpret_cast<Wkv7Smem*>(wkv7_dsmem);
   const int tid = threadIdx.x, g = tid >> 3, q = tid & 7;  // values 4g .., keys 8q ..
@@ -145,6 +148,20 @@ __global__ void __launch_bounds__(kT7, 3) wkv7_fwd_kernel(
     for (int jt = 0; jt < n; ++jt) {
       const Wkv7Tok cu = nx;
       if (jt + 1 < n) nx = fetch(jt + 1);
+      if constexpr (CKPT) {
+        const int t = t0 + jt;
+        if (t % WKV7_CKPT_LEN == 0) {
+          const int nck = (T + WKV7_CKPT_LEN - 1) / WKV7_CKPT_LEN;
+          float* base = ckpt + ((int64_t)bh * nck + t / WKV7_CKPT_LEN) * kK7 * kK7 + 4 * g;
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            *reinterpret_cast<float4*>(base + (8 * q + 2 * m) * kK7) =
+                make_float4(S[0][m].x, S[1][m].x, S[2][m].x, S[3][m].x);
+            *reinterpret_cast<float4*>(base + (8 * q + 2 * m + 1) * kK7) =
+                make_float4(S[0][m].y, S[1][m].y, S[2][m].y, S[3][m].y);
+          }
+        }
+      }
       auto widen4 = [](const uint4& u, float2 (&x)[4]) {
         x[0] = make_float2(bf16lo(u.x), bf16hi(u.x));
         x[1] = make_float2(bf16lo(u.y), bf16hi(u.y));
@@ -159,36 +176,40 @@ __global__ void __launch_bounds__(kT7, 3) wkv7_fwd_kernel(
       const float2 d2[4] = {make_float2(cu.d0.x, cu.d0.y), make_float2(cu.d0.z, cu.d0.w),
                             make_float2(cu.d1.x, cu.d1.y), make_float2(cu.d1.z, cu.d1.w)};
       const float vv[4] = {bf16lo(cu.v.x), bf16hi(cu.v.x), bf16lo(cu.v.y), bf16hi(cu.v.y)};
-      float po[4];  // this thread's 8-key part of (r_t S_t)[4g + c]
+      float po[4] = {0.f, 0.f, 0.f, 0.f};  // this thread's 8-key part of (r_t S_t)[4g + c]
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         const float sa = keys_sum8(dot4(a2, S[c]));  // (a_t S_{t-1})[4g + c]
         const float2 sa2 = make_float2(sa, sa), v2 = make_float2(vv[c], vv[c]);
 #pragma unroll
         for (int m = 0; m < 4; ++m) S[c][m] = fma2(S[c][m], d2[m], fma2(b2[m], sa2, mul2(k2[m], v2)));
-        po[c] = dot4(r2, S[c]);
+        if constexpr (!CKPT) po[c] = dot4(r2, S[c]);
       }
-      // transposed sum over the 8 key threads: each exchange passes on the
-      // half of the columns this thread does not keep (the same pairwise
-      // tree as a butterfly, so the same bits); thread q ends with column
-      // 2 (q & 1) + (q & 2) / 2, twice per group
-      const bool q0 = q & 1, q1 = q & 2;
-      float k0 = q0 ? po[2] : po[0], k1 = q0 ? po[3] : po[1];
-      const float s0 = q0 ? po[0] : po[2], s1 = q0 ? po[1] : po[3];
-      k0 = __fadd_rn(k0, __shfl_xor_sync(0xffffffffu, s0, 1));
-      k1 = __fadd_rn(k1, __shfl_xor_sync(0xffffffffu, s1, 1));
-      float kk = q1 ? k1 : k0;
-      kk = __fadd_rn(kk, __shfl_xor_sync(0xffffffffu, q1 ? k0 : k1, 2));
-      kk = __fadd_rn(kk, __shfl_xor_sync(0xffffffffu, kk, 4));
-      if (!(q & 4)) sm.out[jt][4 * g + (q0 ? 2 : 0) + (q1 ? 1 : 0)] = __float2bfloat16_rn(kk);
+      if constexpr (!CKPT) {
+        // transposed sum over the 8 key threads: each exchange passes on the
+        // half of the columns this thread does not keep (the same pairwise
+        // tree as a butterfly, so the same bits); thread q ends with column
+        // 2 (q & 1) + (q & 2) / 2, twice per group
+        const bool q0 = q & 1, q1 = q & 2;
+        float k0 = q0 ? po[2] : po[0], k1 = q0 ? po[3] : po[1];
+        const float s0 = q0 ? po[0] : po[2], s1 = q0 ? po[1] : po[3];
+        k0 = __fadd_rn(k0, __shfl_xor_sync(0xffffffffu, s0, 1));
+        k1 = __fadd_rn(k1, __shfl_xor_sync(0xffffffffu, s1, 1));
+        float kk = q1 ? k1 : k0;
+        kk = __fadd_rn(kk, __shfl_xor_sync(0xffffffffu, q1 ? k0 : k1, 2));
+        kk = __fadd_rn(kk, __shfl_xor_sync(0xffffffffu, kk, 4));
+        if (!(q & 4)) sm.out[jt][4 * g + (q0 ? 2 : 0) + (q1 ? 1 : 0)] = __float2bfloat16_rn(kk);
+      }
     }
     __syncthreads();
     if (tid == 0 && ch + 2 < nchunk) issue(ch + 2);  // every read of stage s is done
-    for (int p = tid; p < kL7 * 8; p += kT7) {
-      const int row = p / 8, piece = p % 8;
-      if (row < n)
-        *reinterpret_cast<uint4*>(o + ((int64_t)b * T + t0 + row) * HK + (int64_t)h * kK7 + piece * 8) =
-            reinterpret_cast<const uint4*>(&sm.out[row][0])[piece];
+    if constexpr (!CKPT) {
+      for (int p = tid; p < kL7 * 8; p += kT7) {
+        const int row = p / 8, piece = p % 8;
+        if (row < n)
+          *reinterpret_cast<uint4*>(o + ((int64_t)b * T + t0 + row) * HK + (int64_t)h * kK7 + piece * 8) =
+              reinterpret_cast<const uint4*>(&sm.out[row][0])[piece];
+      }
     }
   }
   if (!ok) {
@@ -220,13 +241,14 @@ wkv_status launch_wkv7_forward(const Wkv7FwdArgs& a, cudaStream_t stream, unsign
         return WKV_ERR_INVALID_ARG;
   }
   const size_t smem = sizeof(Wkv7Smem);
-  if (cudaFuncSetAttribute(wkv7_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
+  auto kern = a.ckpt ? wkv7_fwd_kernel<true> : wkv7_fwd_kernel<false>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
     *why = "wkv7_forward: shared memory configuration failed";
     return WKV_ERR_CUDA;
   }
-  wkv7_fwd_kernel<<<(unsigned)(a.B * a.H), kT7, smem, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5],
-                                                               (int)a.T, (int)a.H, a.init_state, a.final_state,
-                                                               static_cast<__nv_bfloat16*>(a.o), err);
+  kern<<<(unsigned)(a.B * a.H), kT7, smem, stream>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], (int)a.T,
+                                                    (int)a.H, a.init_state, a.final_state,
+                                                    static_cast<__nv_bfloat16*>(a.o), a.ckpt, err);
   if (cudaGetLastError() != cudaSuccess) {
     *why = "wkv7_forward kernel launch failed";
     return WKV_ERR_CUDA;

@@ -174,7 +174,19 @@ struct Wkv7FwdArgs {
   const float* init_state;
   float* final_state;
   void* o;
+  float* ckpt = nullptr;  // backward sweep: write state checkpoints, no o
 };
+// Tokens per RWKV-7 state checkpoint of the backward.
+#define WKV7_CKPT_LEN 4
+struct Wkv7BwdArgs {
+  int64_t B, T, H;
+  const void *r, *w, *k, *v, *a, *b, *dout;
+  const float* ckpt;     // [B*H][ceil(T/4)][64][64], from the checkpoint sweep
+  const float* g_final;  // may be null
+  void *dr, *dw, *dk, *dv, *da, *db;
+  float* d_init;
+};
+wkv_status launch_wkv7_backward(const Wkv7BwdArgs& a, cudaStream_t stream, const char** why);
 
 // Record `why` as the calling thread's wkv_last_error() message.
 void set_last_error(const char* why);

@@ -46,6 +46,8 @@ SIGNATURES = {
     "wkv4_backward_gated": (_int, [_i64, _i64, _i64, _int] + [_vp] * 13 + [_sz, _vp]),
     "wkv4_time_shift_mix": (_int, [_i64, _i64, _i64, _int, _i64] + [_vp] * 5),
     "wkv4_decode_step": (_int, [_i64, _i64, _int] + [_vp] * 7),
+    "wkv7_backward_workspace_bytes": (_sz, [_i64, _i64, _i64, _i64]),
+    "wkv7_backward": (_int, [_i64, _i64, _i64, _i64, _int] + [_vp] * 17 + [_sz, _vp]),
     "wkv4_time_shift_mix_backward_workspace_bytes": (_sz, [_i64, _i64, _i64, _int, _i64]),
     "wkv4_time_shift_mix_backward": (_int, [_i64, _i64, _i64, _int, _i64] + [_vp] * 8 + [_sz, _vp]),
 }
@@ -478,3 +480,37 @@ def wkv7_forward(r, w, k, v, a, b, init_state: Optional[torch.Tensor] = None, *,
     _check(_lib.wkv7_forward(B, T, H, K, _dtype_code(r), _ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(a), _ptr(b),
                              _ptr(init_state), _ptr(final_state), _ptr(o), _stream(r)), "wkv7_forward")
     return o, final_state
+
+
+def wkv7_backward_workspace_bytes(B: int, T: int, H: int, head_size: int = 64) -> int:
+    return int(_lib.wkv7_backward_workspace_bytes(B, T, H, head_size))
+
+
+def wkv7_backward(r, w, k, v, a, b, dout, init_state: Optional[torch.Tensor] = None,
+                  g_final: Optional[torch.Tensor] = None, *, head_size: int = 64,
+                  workspace: Optional[torch.Tensor] = None):
+    """Gradients of sum(dout * o) (+ sum(g_final * S_final)) for wkv7_forward on
+    the same inputs. Returns (dr, dw, dk, dv, da, db, d_init); dw is with respect
+    to the log decay w, d_init (float32 [B, H, K, K]) to the initial state."""
+    B, T, HK = r.shape
+    K = head_size
+    if HK % K:
+        raise ValueError("hidden size must be a multiple of head_size")
+    H = HK // K
+    dev = r.device
+    for name, t in (("r", r), ("w", w), ("k", k), ("v", v), ("a", a), ("b", b), ("dout", dout)):
+        _want(t, name, dtype=r.dtype, shape=r.shape, device=dev)
+    for name, t in (("init_state", init_state), ("g_final", g_final)):
+        if t is not None:
+            _want(t, name, dtype=torch.float32, shape=(B, H, K, K), device=dev)
+    grads = [torch.empty_like(r) for _ in range(6)]
+    d_init = torch.empty((B, H, K, K), dtype=torch.float32, device=dev)
+    nbytes = wkv7_backward_workspace_bytes(B, T, H, K)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
+    _want(workspace, "workspace", device=dev)
+    _check(_lib.wkv7_backward(B, T, H, K, _dtype_code(r), _ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(a), _ptr(b),
+                              _ptr(init_state), _ptr(dout), _ptr(g_final), *[_ptr(x) for x in grads], _ptr(d_init),
+                              _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(r)),
+           "wkv7_backward")
+    return (*grads, d_init)

@@ -38,7 +38,7 @@ def test_header_declares_the_entry_points():
               "wkv_device_error", "wkv_abi_version", "wkv6_backward", "wkv6_backward_workspace_bytes",
               "wkv4_forward_gated", "wkv4_backward_gated", "wkv7_forward", "wkv4_time_shift_mix",
               "wkv4_time_shift_mix_backward", "wkv4_time_shift_mix_backward_workspace_bytes",
-              "wkv4_decode_step"):
+              "wkv4_decode_step", "wkv7_backward", "wkv7_backward_workspace_bytes"):
         assert n in names
 
 
@@ -47,6 +47,23 @@ def test_every_declared_symbol_is_exported(W):
     for n in declared_functions():
         assert hasattr(lib, n), f"{n} declared in wkv.h but not exported"
     assert set(declared_functions()) == set(W.SIGNATURES), "binding signatures out of sync with wkv.h"
+
+
+def declared_arity():
+    """Number of parameters of every function wkv.h declares."""
+    src = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"\b(wkv[A-Za-z0-9_]*)\s*\(([^;{]*?)\)\s*;", src, flags=re.S):
+        params = m.group(2).strip()
+        out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_signatures_match_the_header(W):
+    """Every ctypes signature has as many arguments as the C declaration."""
+    arity = declared_arity()
+    for name, (_, args) in W.SIGNATURES.items():
+        assert arity[name] == len(args), f"{name}: header {arity[name]} vs binding {len(args)}"
 
 
 def test_version_and_strings(W):
@@ -138,6 +155,20 @@ def test_time_shift_argument_errors(W):
     assert b(g=None) == W.WKV_ERR_INVALID_ARG and b"g is NULL" in L.wkv_last_error()
     assert b(gmix=None) == W.WKV_ERR_INVALID_ARG and b"gmix" in L.wkv_last_error()
     assert b(wsb=16) == W.WKV_ERR_INVALID_ARG and b"workspace" in L.wkv_last_error()
+
+
+def test_wkv7_backward_argument_errors(W):
+    L = W.lib()
+    wb = lambda K=64, dt=1, dout=FAKE, ws=1 << 30, d_init=FAKE: L.wkv7_backward(
+        1, 8, 1, K, dt, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, dout, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+        d_init, FAKE, ws, None)
+    assert wb(K=32) == W.WKV_ERR_UNSUPPORTED
+    assert wb(dt=0) == W.WKV_ERR_UNSUPPORTED
+    assert wb(dout=None) == W.WKV_ERR_INVALID_ARG and b"dout is NULL" in L.wkv_last_error()
+    assert wb(d_init=None) == W.WKV_ERR_INVALID_ARG and b"d_init" in L.wkv_last_error()
+    assert wb(ws=16) == W.WKV_ERR_INVALID_ARG and b"workspace" in L.wkv_last_error()
+    assert L.wkv7_backward_workspace_bytes(2, 9, 3, 64) == 2 * 3 * 3 * 64 * 64 * 4
+    assert L.wkv7_backward_workspace_bytes(2, 9, 3, 32) == 0
 
 
 def test_chunk_and_wkv6_argument_errors(W):
