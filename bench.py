@@ -66,7 +66,7 @@ def parse():
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the secondary workloads (larger shapes, chunk step, RWKV-6)")
     ap.add_argument("--kernel", choices=["wkv4_fwd", "wkv4_bwd", "wkv4_fwd_gated", "wkv4_bwd_gated", "wkv6_fwd",
-                                         "wkv6_bwd", "wkv7_fwd", "wkv4_chunk", "wkv4_decode", "time_shift_fwd",
+                                         "wkv6_bwd", "wkv7_fwd", "wkv7_bwd", "wkv4_chunk", "wkv4_decode", "time_shift_fwd",
                                          "time_shift_bwd"],
                     help="profiling mode: run only this kernel --steps times on --workload (no JSON line)")
     ap.add_argument("--workload", default=None,
@@ -508,7 +508,17 @@ def secondary(dev, flush, peak):
     res["wkv7_fwd_bf16_c2048"] = {"B": rec7.B, "T": rec7.T, "H": rec7.H, "K": rec7.K, "fwd_ms": t7,
                                   "GBps": 14 * n7 / (t7 * 1e-3) / 1e9, "frac": 14 * n7 / (t7 * 1e-3) / 1e9 / peak,
                                   "Gtokch_per_s": n7 / (t7 * 1e-3) / 1e9}
-    del r7, k7, v7, w7, a7, b7, o7, fs7
+    # backward: checkpoint sweep + reverse kernel; 7 bf16 tensors in (r, w, k,
+    # v, a, b, dout), 6 out (dr, dw, dk, dv, da, db)
+    do7 = mk7().to(torch.bfloat16)
+    ws7 = torch.empty(wkv.wkv7_backward_workspace_bytes(rec7.B, rec7.T, rec7.H, rec7.K), dtype=torch.uint8,
+                      device=dev)
+    b7f = lambda: wkv.wkv7_backward(r7, w7, k7, v7, a7, b7, do7, workspace=ws7)
+    b7f()
+    tb7 = _events_ms(b7f, 3, flush, stream)
+    res["wkv7_fwd_bf16_c2048"].update({"bwd_ms": tb7, "bwd_GBps": 26 * n7 / (tb7 * 1e-3) / 1e9,
+                                       "bwd_frac": 26 * n7 / (tb7 * 1e-3) / 1e9 / peak})
+    del r7, k7, v7, w7, a7, b7, o7, fs7, do7, ws7
     assert wkv.device_error(reset=True) == 0, "a kernel recorded a device-side error"
     return res
 
@@ -746,7 +756,7 @@ def run_kernel_only(args):
                 wkv.wkv4_time_shift_mix(xs, mixs, out=outs)
             else:
                 wkv.wkv4_time_shift_mix_backward(xs, mixs, gs)
-    elif args.kernel == "wkv7_fwd":
+    elif args.kernel in ("wkv7_fwd", "wkv7_bwd"):
         rec7 = synth.WKV7_RECIPES[name or "wkv7_fwd_bf16_c2048"]
         if resize:
             rec7 = rec7.with_shape(*[int(x) for x in resize.split(",")])
@@ -756,8 +766,12 @@ def run_kernel_only(args):
         kap = (kap / kap.norm(dim=-1, keepdim=True)).reshape(shape)
         a7, b7 = (-kap).to(torch.bfloat16), (kap * torch.rand(shape, device=dev, generator=g)).to(torch.bfloat16)
         r7, k7, v7 = (torch.randn(shape, device=dev, generator=g).to(torch.bfloat16) for _ in range(3))
+        do7 = torch.randn(shape, device=dev, generator=g).to(torch.bfloat16)
         for _ in range(args.steps):
-            wkv.wkv7_forward(r7, w7, k7, v7, a7, b7)
+            if args.kernel == "wkv7_fwd":
+                wkv.wkv7_forward(r7, w7, k7, v7, a7, b7)
+            else:
+                wkv.wkv7_backward(r7, w7, k7, v7, a7, b7, do7)
     elif args.kernel in ("wkv6_fwd", "wkv6_bwd"):
         rec = synth.WKV6_RECIPES[name or "wkv6_fwd_bf16_c2048"]
         if resize:
