@@ -20,10 +20,12 @@
 // memory (5 x 16 KB) with the forward's own step, and then runs the group's
 // reverse steps. Thread (g = tid / 8, q = tid % 8) holds G for values
 // 4g .. 4g + 3 and keys 8q .. 8q + 7, as the forward holds S: the sums over
-// keys (dsa, dv) are three shuffles within the 8 threads of a value group;
-// the five sums over values (dr, dk, db, dw, da) leave as per-thread partials
-// in shared memory that are added across the 16 value groups in a fixed
-// order. This is a first, exact version: one token at a time on CUDA cores.
+// keys (dsa, dv) are three shuffles within the 8 threads of a value group
+// and are all the walk itself needs; the five sums over values (dr, dk, db,
+// dw, da) leave as per-thread partials in shared memory and are added
+// across the 16 value groups in a fixed order once per group, so a group
+// costs three barriers, not one per token. A first, exact version: one
+// token at a time on CUDA cores.
 #include "wkv_device.cuh"
 #include "wkv_internal.h"
 
@@ -41,7 +43,7 @@ struct alignas(16) Wkv7BwdSmem {
   float hist[kL7b + 1][kK7b][kK7b];     // state before token jt of the group (hist[jt]) and after the last
   float in[kInputs][kL7b][kK7b];        // r, e^{w}, k, v, a, b, dout of the group
   float sa[kL7b][kK7b];                 // a_t S_{t-1} of each token
-  float part[2][16][kParts][kK7b];      // per value group: partial sums over its 4 values
+  float part[kL7b][16][kParts][kK7b];   // per token and value group: partial sums over its 4 values
 };
 
 __device__ __forceinline__ float sum8(float x) {
@@ -116,7 +118,6 @@ __global__ void __launch_bounds__(kT7b, 1) wkv7_bwd_kernel(
 #pragma unroll
       for (int m = 0; m < 4; ++m) G[c][m] = make_float2(0.f, 0.f);
   }
-  int buf = 0;
   for (int grp = nck - 1; grp >= 0; --grp) {
     const int t0 = grp * kL7b, n = min(kL7b, T - t0);
     // the group's inputs, widened (e^{w} formed as the forward forms it)
@@ -202,7 +203,7 @@ __global__ void __launch_bounds__(kT7b, 1) wkv7_bwd_kernel(
       }
 #pragma unroll
       for (int x = 0; x < kParts; ++x) {
-        float* dst = &sm.part[buf][g][x][8 * q];
+        float* dst = &sm.part[jt][g][x][8 * q];
         *reinterpret_cast<float4*>(dst) = make_float4(p[x][0].x, p[x][0].y, p[x][1].x, p[x][1].y);
         *reinterpret_cast<float4*>(dst + 4) = make_float4(p[x][2].x, p[x][2].y, p[x][3].x, p[x][3].y);
       }
@@ -217,19 +218,19 @@ __global__ void __launch_bounds__(kT7b, 1) wkv7_bwd_kernel(
       for (int c = 0; c < 4; ++c)
 #pragma unroll
         for (int m = 0; m < 4; ++m) G[c][m] = fma2(d2[m], G[c][m], mul2(a2[m], make_float2(dsa[c], dsa[c])));
-      __syncthreads();
-      // the five sums over values, added across the 16 value groups in order
-      for (int e = tid; e < kParts * kK7b; e += kT7b) {
-        const int x = e / kK7b, j = e % kK7b;
-        float s = 0.f;
-#pragma unroll
-        for (int gg = 0; gg < 16; ++gg) s += sm.part[buf][gg][x][j];
-        if (x == kPW) s = __fmul_rn(s, sm.in[kID][jt][j]);
-        outs[x][row + j] = __float2bfloat16_rn(s);
-      }
-      buf ^= 1;
     }
-    __syncthreads();  // the group's inputs and states are read; the next group may overwrite them
+    __syncthreads();
+    // the group's five sums over values (they do not feed the walk), added
+    // across the 16 value groups in order
+    for (int e = tid; e < n * kParts * kK7b; e += kT7b) {
+      const int jt = e / (kParts * kK7b), x = (e / kK7b) % kParts, j = e % kK7b;
+      float s = 0.f;
+#pragma unroll
+      for (int gg = 0; gg < 16; ++gg) s += sm.part[jt][gg][x][j];
+      if (x == kPW) s = __fmul_rn(s, sm.in[kID][jt][j]);
+      outs[x][((int64_t)bi * T + t0 + jt) * HK + (int64_t)h * kK7b + j] = __float2bfloat16_rn(s);
+    }
+    __syncthreads();  // the group's inputs, states and partials are read; the next group may overwrite them
   }
   st_state(d_init + (int64_t)bh * kK7b * kK7b, g, q, G);
 }
