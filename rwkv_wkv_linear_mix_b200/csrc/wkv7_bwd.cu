@@ -93,6 +93,32 @@ __device__ __forceinline__ void st_state(float* base, int g, int q, const float2
   }
 }
 
+// The same slices of a state kept in shared memory, with the 16-byte chunk
+// index of row j swizzled by j / 8: the 8 threads of a quarter warp (same g,
+// q = 0 .. 7) then touch 8 different bank groups instead of one.
+__device__ __forceinline__ void ld_state_sm(const float* base, int g, int q, float2 (&S)[4][4]) {
+  const int col = 4 * (g ^ q);
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const float4 lo = *reinterpret_cast<const float4*>(base + (8 * q + 2 * m) * kK7b + col);
+    const float4 hi = *reinterpret_cast<const float4*>(base + (8 * q + 2 * m + 1) * kK7b + col);
+    S[0][m] = make_float2(lo.x, hi.x);
+    S[1][m] = make_float2(lo.y, hi.y);
+    S[2][m] = make_float2(lo.z, hi.z);
+    S[3][m] = make_float2(lo.w, hi.w);
+  }
+}
+__device__ __forceinline__ void st_state_sm(float* base, int g, int q, const float2 (&S)[4][4]) {
+  const int col = 4 * (g ^ q);
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    *reinterpret_cast<float4*>(base + (8 * q + 2 * m) * kK7b + col) =
+        make_float4(S[0][m].x, S[1][m].x, S[2][m].x, S[3][m].x);
+    *reinterpret_cast<float4*>(base + (8 * q + 2 * m + 1) * kK7b + col) =
+        make_float4(S[0][m].y, S[1][m].y, S[2][m].y, S[3][m].y);
+  }
+}
+
 __global__ void __launch_bounds__(kT7b, 1) wkv7_bwd_kernel(
     int T, int H, const __nv_bfloat16* __restrict__ r, const __nv_bfloat16* __restrict__ w,
     const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v, const __nv_bfloat16* __restrict__ a,
@@ -132,7 +158,7 @@ __global__ void __launch_bounds__(kT7b, 1) wkv7_bwd_kernel(
     }
     float2 S[4][4];
     ld_state(ckpt + ((int64_t)bh * nck + grp) * kK7b * kK7b, g, q, S);
-    st_state(&sm.hist[0][0][0], g, q, S);
+    st_state_sm(&sm.hist[0][0][0], g, q, S);
     __syncthreads();
     // recompute the group's states with the forward's step
     for (int jt = 0; jt < n; ++jt) {
@@ -150,7 +176,7 @@ __global__ void __launch_bounds__(kT7b, 1) wkv7_bwd_kernel(
 #pragma unroll
         for (int m = 0; m < 4; ++m) S[c][m] = fma2(S[c][m], d2[m], fma2(b2[m], sa2, mul2(k2[m], v2)));
       }
-      st_state(&sm.hist[jt + 1][0][0], g, q, S);
+      st_state_sm(&sm.hist[jt + 1][0][0], g, q, S);
     }
     __syncthreads();
     // reverse steps of the group
@@ -162,8 +188,8 @@ __global__ void __launch_bounds__(kT7b, 1) wkv7_bwd_kernel(
       keys8(sm.in[kIK][jt], q, k2);
       keys8(sm.in[kIA][jt], q, a2);
       keys8(sm.in[kIB][jt], q, b2);
-      ld_state(&sm.hist[jt][0][0], g, q, Sp);
-      ld_state(&sm.hist[jt + 1][0][0], g, q, Sc);
+      ld_state_sm(&sm.hist[jt][0][0], g, q, Sp);
+      ld_state_sm(&sm.hist[jt + 1][0][0], g, q, Sc);
       float vv[4], dov[4], sav[4], dsa[4], dvv[4];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
