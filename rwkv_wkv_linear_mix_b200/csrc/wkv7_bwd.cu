@@ -61,10 +61,14 @@ __device__ __forceinline__ float dot4b(const float2 (&a)[4], const float2 (&s)[4
   return __fadd_rn(acc.x, acc.y);
 }
 
-// 8 keys 8q .. 8q + 7 of a row of `src` as 4 pairs
+// 8 keys 8q .. 8q + 7 of a row of `src` as 4 pairs. Threads q >= 4 read the
+// two halves in the other order, so that within each load the 8 threads of a
+// quarter warp fall in 8 different bank groups.
 __device__ __forceinline__ void keys8(const float* src, int q, float2 (&x)[4]) {
-  const float4 lo = *reinterpret_cast<const float4*>(src + 8 * q);
-  const float4 hi = *reinterpret_cast<const float4*>(src + 8 * q + 4);
+  const bool sw = q & 4;
+  const float4 f0 = *reinterpret_cast<const float4*>(src + 8 * q + (sw ? 4 : 0));
+  const float4 f1 = *reinterpret_cast<const float4*>(src + 8 * q + (sw ? 0 : 4));
+  const float4 lo = sw ? f1 : f0, hi = sw ? f0 : f1;
   x[0] = make_float2(lo.x, lo.y);
   x[1] = make_float2(lo.z, lo.w);
   x[2] = make_float2(hi.x, hi.y);
@@ -230,8 +234,11 @@ __global__ void __launch_bounds__(kT7b, 1) wkv7_bwd_kernel(
 #pragma unroll
       for (int x = 0; x < kParts; ++x) {
         float* dst = &sm.part[jt][g][x][8 * q];
-        *reinterpret_cast<float4*>(dst) = make_float4(p[x][0].x, p[x][0].y, p[x][1].x, p[x][1].y);
-        *reinterpret_cast<float4*>(dst + 4) = make_float4(p[x][2].x, p[x][2].y, p[x][3].x, p[x][3].y);
+        const float4 lo = make_float4(p[x][0].x, p[x][0].y, p[x][1].x, p[x][1].y);
+        const float4 hi = make_float4(p[x][2].x, p[x][2].y, p[x][3].x, p[x][3].y);
+        const bool sw = q & 4;  // halves in the other order, as in keys8
+        *reinterpret_cast<float4*>(dst + (sw ? 4 : 0)) = sw ? hi : lo;
+        *reinterpret_cast<float4*>(dst + (sw ? 0 : 4)) = sw ? lo : hi;
       }
       if (q == 0) {
         uint2 pk2;
