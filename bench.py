@@ -8,7 +8,8 @@ wkv4_backward over one batch of the RWKV-4 169M-width workload
 (B=8, T=1024, C=768, float32 k/v/y, fp32 state; w = exp(U(-6,1)),
 u ~ U(-1,1), k ~ N(0, 2^2), v, gy ~ N(0,1); seed 0). Inputs are resident in
 HBM; L2 is flushed (a 320 MB write) before every timed step and each step is
-timed alone with CUDA events on the launching stream. Under torchrun every
+timed with CUDA events on the launching stream, the launches queued behind a
+GPU spin so that no interval includes host launch latency. Under torchrun every
 rank runs its own replica on its own GPU (no collective on the data path) and
 the job time is the max over ranks.
 
@@ -18,9 +19,10 @@ the dominant kernel (the backward) against the measured HBM bandwidth, the
 fp64 CPU oracle timed on a bounded sample, SM clocks sampled during the timed
 region, and the number of library kernels launched. Under "workloads" the
 same line carries secondary single-kernel measurements (rank 0, N=1): the
-RWKV-4 fwd/bwd at the 3B width and at C=4096 (f32 and bf16) against the HBM
-peak, the 32-slot chunk step (eager and as one CUDA-graph replay), and the
-RWKV-6 head-state forward.
+RWKV-4 fwd/bwd at the 3B width and at C=4096 (f32 and bf16, plain and with
+the time-mix gate fused) against the HBM peak, the time-mix prologue, the
+32-slot chunk step (eager and as one CUDA-graph replay), the 256-slot decode
+step, the RWKV-6 forward and backward and the RWKV-7 forward and backward.
 
 --impl reference times the fp64 CPU oracle (the only reference this project
 has) on the same workload and metric.
