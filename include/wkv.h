@@ -281,9 +281,9 @@ wkv_status wkv4_decode_step(int64_t S, int64_t C, int dtype,
  * wkv4_backward without a workspace argument, for callers that cannot
  * allocate device memory per call (code behind a plain C interface that only
  * receives the tensors it reads and writes, or latency-critical loops that
- * must not call cudaMalloc/cudaFree). The paper (the pages this library
- * follows) has no counterpart: this is a deployment convenience of the
- * library, not part of the method.
+ * must not call cudaMalloc/cudaFree). The method's source pages have no
+ * counterpart: this is a deployment convenience of the library, not part
+ * of the method.
  *   Arguments and results are those of wkv4_backward; the workspace is a
  *   file-scope device array of 4 MiB that every GPU loading the library
  *   keeps until the process exits.
