@@ -171,6 +171,21 @@ def test_wkv7_backward_argument_errors(W):
     assert L.wkv7_backward_workspace_bytes(2, 9, 3, 32) == 0
 
 
+def test_time_shift_workspace_follows_the_run_split(W):
+    """The backward's partial mix gradients are [n_mix][B * runs][C] floats,
+    each sequence cut into runs of at least 16 tokens, about 16 CTAs of 128
+    threads per SM (4 channels each) over 148 SMs."""
+    L = W.lib()
+    cdiv = lambda a, b: -(-a // b)
+    for B, T, C, n in ((16, 4096, 4096, 3), (8, 1024, 768, 2), (1, 5, 8, 1), (2, 100000, 64, 3)):
+        ncb = cdiv(C, 128 * 4)
+        nrun = max(1, min(cdiv(148 * 16, B * ncb), max(1, cdiv(T, 16))))
+        lt = cdiv(T, nrun)
+        nrun = cdiv(T, lt)
+        for dt in (0, 1):
+            assert L.wkv4_time_shift_mix_backward_workspace_bytes(B, T, C, dt, n) == n * B * nrun * C * 4
+
+
 def test_chunk_and_wkv6_argument_errors(W):
     L = W.lib()
     dec = lambda S=4, C=8, dt=0, k=FAKE, state=FAKE: L.wkv4_decode_step(S, C, dt, FAKE, FAKE, k, FAKE, FAKE, state,
