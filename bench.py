@@ -4,25 +4,27 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 One step = wkv4_forward (writing the state checkpoints) followed by
-wkv4_backward over one batch of the RWKV-4 169M-width workload
-(B=8, T=1024, C=768, float32 k/v/y, fp32 state; w = exp(U(-6,1)),
-u ~ U(-1,1), k ~ N(0, 2^2), v, gy ~ N(0,1); seed 0). Inputs are resident in
-HBM; L2 is flushed (a 320 MB write) before every timed step and each step is
-timed with CUDA events on the launching stream, the launches queued behind a
-GPU spin so that no interval includes host launch latency. Under torchrun every
-rank runs its own replica on its own GPU (no collective on the data path) and
-the job time is the max over ranks.
+wkv4_backward over one batch of the RWKV-4 3B-width workload, the largest
+forward+backward configuration (B=16, T=4096, C=2560, bf16 k/v/y/gy/gk/gv,
+fp32 w/u and fp32 state; w = exp(U(-8,2)), u ~ U(-2,2), k ~ N(0, 1.5^2),
+v, gy ~ N(0,1); seed 0). Inputs are resident in HBM; L2 is flushed (a 320 MB
+write) before every timed step (the inputs alone, 1 GB, exceed L2 too) and
+each step is timed with CUDA events on the launching stream, the launches
+queued behind a GPU spin so that no interval includes host launch latency.
+Under torchrun every rank runs its own replica on its own GPU (no collective
+on the data path) and the job time is the max over ranks.
 
 Printed (rank 0, one JSON line): G tok*ch/s = B*T*C*N / step time, the
 end-to-end figure through the C ABI with pinned host buffers, the roofline of
 the dominant kernel (the backward) against the measured HBM bandwidth, the
-fp64 CPU oracle timed on a bounded sample, SM clocks sampled during the timed
-region, and the number of library kernels launched. Under "workloads" the
-same line carries secondary single-kernel measurements (rank 0, N=1): the
-RWKV-4 fwd/bwd at the 3B width and at C=4096 (f32 and bf16, plain and with
-the time-mix gate fused) against the HBM peak, the time-mix prologue, the
-32-slot chunk step (eager and as one CUDA-graph replay), the 256-slot decode
-step, the RWKV-6 forward and backward and the RWKV-7 forward and backward.
+fp64 CPU oracle timed on a bounded sample on one host core and on all of
+them, SM clocks sampled during the timed region, and the number of library
+kernels launched. Under "workloads" the same line carries secondary
+single-kernel measurements (rank 0, N=1): the RWKV-4 fwd/bwd at the 169M
+width (float32) and at C=4096 (f32 and bf16, plain and with the time-mix gate
+fused) against the HBM peak, the time-mix prologue, the 32-slot chunk step
+(eager and as one CUDA-graph replay), the 256-slot decode step, the RWKV-6
+forward and backward and the RWKV-7 forward and backward.
 
 --impl reference times the fp64 CPU oracle (the only reference this project
 has) on the same workload and metric.
@@ -48,7 +50,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-WORKLOAD = "wkv4_fb_f32_169m"
+WORKLOAD = "wkv4_fb_bf16_3b"
 METRIC = "WKV fwd+bwd throughput (G tok·ch/s)"
 UNIT = "G tok*ch/s"
 L2_FLUSH_BYTES = 320 << 20
@@ -56,6 +58,8 @@ HOST_LEAD_CYCLES_PER_STEP = 1_000_000  # ~0.5 ms of GPU spin per step queued ahe
 # sources that determine the backward kernel's code and launch shape
 BWD_SOURCES = ["rwkv_wkv_linear_mix_b200/csrc/wkv4_bwd.cu", "rwkv_wkv_linear_mix_b200/csrc/wkv_device.cuh",
                "rwkv_wkv_linear_mix_b200/csrc/wkv_internal.h", "include/wkv.h"]
+# oracle sample: channel slices of this width, timed on one core and on all
+CPU_SLICE_WIDTH = 16
 
 
 def parse():
@@ -114,11 +118,22 @@ def measured_peaks():
     return 6650.0, "of fallback"
 
 
+def _strip_comments(src: str) -> str:
+    """C/C++ source without // and /* */ comments and blank lines (string
+    literals of the kernel sources hold no comment markers)."""
+    import re
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+
+
 def kernel_source_hash(files):
+    """Hash of the code (comments dropped) that determines a kernel, so a
+    recorded ncu figure stays attached to the code it was taken on."""
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, f), encoding="utf-8") as fh:
+            h.update(_strip_comments(fh.read()).encode())
     return h.hexdigest()[:16]
 
 
@@ -193,30 +208,62 @@ class ClockSampler:
 # CPU oracle baseline (bounded sample)
 # ----------------------------------------------------------------------------
 
-def cpu_baseline(inp, budget_s=12.0):
-    """Time the fp64 oracle's forward+backward on channel slices of the
-    workload until about `budget_s` seconds of CPU work are done."""
+def _oracle_fb_slices(inp, width, budget_s, max_slices=4096):
+    """Time the fp64 oracle's forward+backward on successive channel slices of
+    `width` channels (all B and T) until about budget_s seconds of work are
+    done. Returns (tok*ch done, seconds, slices)."""
     import oracle
-    oracle.build()
     B, T, C = inp["k32"].shape
-    width = 96
-    done_tc = 0
-    t_total = 0.0
-    c0 = 0
-    slices = 0
-    while t_total < budget_s and slices < 4096:
+    done_tc, t_total, c0, slices = 0, 0.0, 0, 0
+    while t_total < budget_s and slices < max_slices:
         cs = slice(c0, min(C, c0 + width))
-        args = (inp["w"][cs], inp["u"][cs], inp["k32"][:, :, cs], inp["v32"][:, :, cs])
+        args = (inp["w"][cs], inp["u"][cs], np.ascontiguousarray(inp["k32"][:, :, cs]),
+                np.ascontiguousarray(inp["v32"][:, :, cs]))
+        gy = np.ascontiguousarray(inp["gy32"][:, :, cs])
         t = time.perf_counter()
         oracle.wkv4_forward(*args)
-        oracle.wkv4_backward(*args, inp["gy32"][:, :, cs])
+        oracle.wkv4_backward(*args, gy)
         t_total += time.perf_counter() - t
         done_tc += B * T * (cs.stop - cs.start)
         c0 = (c0 + width) % C
         slices += 1
-    return {"value": done_tc / t_total / 1e9, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{slices} slices of {width} channels x B={B} x T={T} (fwd+bwd, fp64), "
-                      f"{done_tc / 1e6:.1f} M tok*ch in {t_total:.1f} s"}
+    return done_tc, t_total, slices
+
+
+def cpu_baseline(inp, budget_s=8.0):
+    """The fp64 oracle on the host cores: forward+backward on channel slices
+    of the workload (CPU_SLICE_WIDTH channels x all B, T each), about budget_s
+    seconds of work on one core and again on all cores, plus the RWKV-6
+    forward on one head of its 8x4096 workload."""
+    import oracle
+    oracle.build()
+    B, T, C = inp["k32"].shape
+    cores = os.cpu_count() or 1
+    res = {}
+    for n in (1, cores):
+        oracle.set_num_threads(n)
+        tc, secs, slices = _oracle_fb_slices(inp, CPU_SLICE_WIDTH, budget_s)
+        res[n] = (tc / secs / 1e9, tc, secs, slices)
+    from rwkv_wkv_linear_mix_b200 import synth
+    r6 = synth.WKV6_RECIPES["wkv6_fwd_bf16_c2048"].with_shape(None, None, 1)
+    i6 = synth.wkv6_inputs(r6, seed=0)
+    w6 = {}
+    for n in (1, cores):
+        oracle.set_num_threads(n)
+        t = time.perf_counter()
+        oracle.wkv6_forward(i6["r32"], i6["k32"], i6["v32"], i6["w32"], i6["u"].reshape(1, 64))
+        w6[n] = r6.B * r6.T * 64 / (time.perf_counter() - t) / 1e9
+    oracle.set_num_threads(cores)
+    v_all, tc, secs, slices = res[cores]
+    v_one, tc1, secs1, slices1 = res[1]
+    return {"value": v_all, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{slices} slices of {CPU_SLICE_WIDTH} channels x B={B} x T={T} (fwd+bwd, fp64), "
+                      f"{tc / 1e6:.1f} M tok*ch in {secs:.1f} s on {cores} cores",
+            "one_core": {"value": v_one, "unit": UNIT, "cores": 1,
+                         "sample": f"{slices1} slices of {CPU_SLICE_WIDTH} channels, {tc1 / 1e6:.1f} M tok*ch "
+                                   f"in {secs1:.1f} s"},
+            "wkv6_forward": {"unit": UNIT, "one_core": w6[1], "all_cores": w6[cores], "cores": cores,
+                             "sample": f"one head of B={r6.B} x T={r6.T} x K=64 (fp64 sequential)"}}
 
 
 # ----------------------------------------------------------------------------
@@ -233,15 +280,17 @@ def run_reference(args):
     import oracle
     oracle.build()
     B, T, C = rec.B, rec.T, rec.C
-    width = 48
+    width = CPU_SLICE_WIDTH
     per_step = []
     c0 = 0
     for i in range(args.warmup + args.steps):
         cs = slice(c0, c0 + width)
-        a = (inp["w"][cs], inp["u"][cs], inp["k32"][:, :, cs], inp["v32"][:, :, cs])
+        a = (inp["w"][cs], inp["u"][cs], np.ascontiguousarray(inp["k32"][:, :, cs]),
+             np.ascontiguousarray(inp["v32"][:, :, cs]))
+        gy = np.ascontiguousarray(inp["gy32"][:, :, cs])
         t = time.perf_counter()
         oracle.wkv4_forward(*a)
-        oracle.wkv4_backward(*a, inp["gy32"][:, :, cs])
+        oracle.wkv4_backward(*a, gy)
         dt = time.perf_counter() - t
         if i >= args.warmup:
             per_step.append(dt)
@@ -295,7 +344,7 @@ def secondary(dev, flush, peak):
     stream = torch.cuda.current_stream(dev)
     g = torch.Generator(device=dev)
     res = {}
-    for name in ("wkv4_fb_bf16_3b", "wkv4_fb_f32_c4096", "wkv4_fb_bf16_c4096"):
+    for name in ("wkv4_fb_f32_169m", "wkv4_fb_f32_c4096", "wkv4_fb_bf16_c4096"):
         rec = synth.WKV4_RECIPES[name]
         g.manual_seed(0)
         B, T, C = rec.B, rec.T, rec.C
@@ -544,10 +593,16 @@ def run_ours(args):
     inp = synth.wkv4_inputs(rec, seed=0)
     tok_ch = B * T * C
 
-    def to_dev(a):
-        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+    es = 2 if rec.dtype == "bf16" else 4  # bytes per element of k, v, y, gy, gk, gv
 
-    w, u, k, v, gy = (to_dev(inp[n]) for n in ("w", "u", "k", "v", "gy"))
+    def host(a):
+        """Generator array as a CPU tensor (bf16 bit patterns as bfloat16)."""
+        a = np.ascontiguousarray(a)
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
+        return torch.from_numpy(a)
+
+    w, u, k, v, gy = (host(inp[n]).to(dev) for n in ("w", "u", "k", "v", "gy"))
     y = torch.empty_like(k)
     gk, gv = torch.empty_like(k), torch.empty_like(k)
     gw = torch.empty(C, dtype=torch.float32, device=dev)
@@ -607,7 +662,7 @@ def run_ours(args):
     # two device buffer sets on separate copy-in / compute / copy-out streams,
     # so one step's results travel back while the next step's inputs arrive
     # (PCIe moves both directions at once); events order each buffer's reuse.
-    H = {n: torch.from_numpy(np.ascontiguousarray(inp[n])).pin_memory() for n in ("k", "v", "gy", "w", "u")}
+    H = {n: host(inp[n]).pin_memory() for n in ("k", "v", "gy", "w", "u")}
     hy, hgk, hgv = (torch.empty(k.shape, dtype=k.dtype).pin_memory() for _ in range(3))
     hgw, hgu = (torch.empty(C, dtype=torch.float32).pin_memory() for _ in range(2))
     h2d = sum(t.numel() * t.element_size() for t in H.values())
@@ -673,21 +728,24 @@ def run_ours(args):
     peak, peak_kind = measured_peaks()
     bwd_ms = statistics.mean(t_bwd)
     fwd_ms = statistics.mean(t_fwd)
-    bwd_bytes = 20 * tok_ch   # k, v, gy read; gk, gv written (float32)
-    fwd_bytes = 12 * tok_ch   # k, v read; y written
+    bwd_bytes = 5 * es * tok_ch   # k, v, gy read; gk, gv written
+    fwd_bytes = 3 * es * tok_ch   # k, v read; y written
     achieved = bwd_bytes / (bwd_ms * 1e-3) / 1e9
     src_hash = kernel_source_hash(BWD_SOURCES)
-    roof = {"bound": "hbm", "kernel": "wkv4_bwd_kernel<float>", "achieved": achieved, "peak": peak,
+    kname = "wkv4_bwd_kernel<%s>" % ("bf16" if es == 2 else "float")
+    roof = {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": peak,
             "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
             "traffic": recorded_traffic("wkv4_bwd_kernel", WORKLOAD, src_hash),
             "algorithmic_bytes_per_launch": bwd_bytes, "avg_launch_ms": bwd_ms,
-            "forward": {"achieved": fwd_bytes / (fwd_ms * 1e-3) / 1e9, "avg_launch_ms": fwd_ms,
-                        "algorithmic_bytes_per_launch": fwd_bytes}}
+            "forward": {"kernel": kname.replace("bwd", "fwd"), "achieved": fwd_bytes / (fwd_ms * 1e-3) / 1e9,
+                        "frac": fwd_bytes / (fwd_ms * 1e-3) / 1e9 / peak, "avg_launch_ms": fwd_ms,
+                        "algorithmic_bytes_per_launch": fwd_bytes},
+            "bytes_per_tok_ch": {"backward": 5 * es, "forward": 3 * es}}
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms_max, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "vs_baseline": None, "dtype": rec.dtype, "data": "synthetic",
         "config": {"workload": WORKLOAD, "B": B, "T": T, "C": C, "global_batch": B * world, "seq_len": T,
                    "parallelism": f"replicas{world}", "l2": "flushed (320 MB write) before every timed step",
                    "ckpt_len": wkv.CKPT_LEN},

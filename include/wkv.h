@@ -287,14 +287,20 @@ wkv_status wkv4_decode_step(int64_t S, int64_t C, int dtype,
  *   Arguments and results are those of wkv4_backward; the workspace is a
  *   file-scope device array of 4 MiB that every GPU loading the library
  *   keeps until the process exits.
- *   Problems needing more than that (2*B*C floats of partial sums, plus the
- *   checkpoints when ckpt is NULL) return WKV_ERR_UNSUPPORTED: pass ckpt, or
- *   call wkv4_backward.
- *   The first call on a device looks up the array's device address (with that
- *   device current); make that first call before any stream capture.
+ *   Problems whose workspace, wkv4_backward_workspace_bytes(B, T, C,
+ *   ckpt != NULL), exceeds 4 MiB return WKV_ERR_UNSUPPORTED (the partial sums
+ *   take 2*B*NSEG*C floats, NSEG the sequence segments of short batches, at
+ *   most 8; a NULL ckpt adds the regenerated checkpoints): pass ckpt, or call
+ *   wkv4_backward.
+ *   The array used is the one of the current device, which must be the
+ *   device of the tensors and of the stream. The first call on a device
+ *   looks up the array's device address (with that device current); make
+ *   that first call before any stream capture.
  *   All calls share the array: calls whose kernels overlap on the GPU race on
  *   it and must be serialised by the caller. Nothing in it needs clearing:
- *   every scratch element a call reads was written earlier in that call.
+ *   every scratch element a call reads was written earlier in that call
+ *   (after a copy wait that gave up, reported as WKV_DEVERR_WAIT_TIMEOUT, the
+ *   call's results are undefined, as for wkv4_backward).
  *   Allocates nothing (no cudaMalloc, cudaFree or allocating library call).
  */
 wkv_status wkv4_backward_noalloc(int64_t B, int64_t T, int64_t C, int dtype,

@@ -56,6 +56,8 @@ def _open(path):
     lib = ctypes.CDLL(path)
     i64, dp = ctypes.c_int64, ctypes.c_void_p
     lib.oracle_num_threads.restype = ctypes.c_int
+    lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
+    lib.oracle_set_num_threads.restype = None
     lib.oracle_wkv4_forward.argtypes = [i64, i64, i64] + [dp] * 8
     lib.oracle_wkv4_forward.restype = ctypes.c_int
     lib.oracle_wkv4_backward.argtypes = [i64, i64, i64] + [dp] * 10
@@ -129,6 +131,12 @@ def _ptr(a):
 def num_threads() -> int:
     """OpenMP threads the oracle uses (OMP_NUM_THREADS, else all cores)."""
     return int(_load().oracle_num_threads())
+
+
+def set_num_threads(n: int) -> None:
+    """Use n OpenMP threads from now on (the bench times the oracle on one
+    core and on all of them; results do not depend on the count)."""
+    _load().oracle_set_num_threads(int(n))
 
 
 def wkv4_forward(w, u, k, v, return_state: bool = False, _lib=None):

@@ -71,6 +71,16 @@ int oracle_num_threads(void) {
 #endif
 }
 
+/* Threads of the parallel loops that follow (timing only: the loops are over
+ * independent lanes/heads, so the results do not depend on it). */
+void oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
 static int all_finite(const double *x, int64_t n) {
     for (int64_t i = 0; i < n; ++i)
         if (!isfinite(x[i])) return 0;

@@ -54,11 +54,6 @@ namespace wkv {
 constexpr int kBwdL = WKV4_CKPT_LEN;
 constexpr int kBwdCh = WKV4_WARP_CH;  // channels of one warp: a pair per lane
 
-template <bool V>
-struct BoolTag {
-  static constexpr bool value = V;
-};
-
 // Where the recompute leaves the per-step forward quantities (state aa, bb
 // before the step and the absorb exponent z1) for the reverse steps: in
 // registers, or (bf16) in shared memory, which frees ~100 registers per
@@ -70,6 +65,11 @@ struct BoolTag {
 #endif
 #ifndef WKV4_BWD_WHOLE_RECOMPUTE
 #define WKV4_BWD_WHOLE_RECOMPUTE 1
+#endif
+// Tokens whose exponent chain the shared-memory-stash recompute runs ahead of
+// their value updates.
+#ifndef WKV4_BWD_RECOMP_GROUP
+#define WKV4_BWD_RECOMP_GROUP 8
 #endif
 #ifndef WKV4_BWD_SMEM_STASH_F32
 #define WKV4_BWD_SMEM_STASH_F32 0
@@ -124,38 +124,55 @@ __device__ __forceinline__ float2 neg2(float2 a) { return make_float2(-a.x, -a.y
 
 // One reverse step of a lane's channel pair (token t, walking down), from
 // the forward quantities of the token: the state (aa, bb) before it, its
-// absorb exponent z (z1 of the forward), v and gy. FULL: also write gk, gv
-// at gkp, gvp and add the token's gw, gu terms (gwn holds -gw); otherwise
-// only fold the token into the carries and fprod. GATE: gy is the gradient
-// of the gated output sigmoid(r) * y; the step writes
-// dL/dr = gy y s (1 - s) at grp (s = sigmoid(r)) and carries gy s on as y's.
-template <bool FULL, bool GATE, class E>
+// absorb factors f1, f2 (and absorb exponent z, for the exact output form),
+// v and gy. The output weight e = 2^{u + k - P} = 2^{z1 + u - w} of the token
+// (in units of the past's exponent P; D = 2^P (bb + e), y = (aa + e v) /
+// (bb + e)) is formed as in the forward: SCALED from f1, f2 and the channel
+// constants E2 = 2^{u - w} (den = f1 (bb + e) = f1 bb + f2 E, so 1/(bb + e) =
+// f1 / den and e/(bb + e) = f2 E / den), otherwise from a second ex2 of
+// z + uw2, capped as in the forward. FULL: also write gk, gv at gkp, gvp and
+// add the token's gw, gu terms (gwn holds -gw); otherwise only fold the token
+// into the carries and fprod. GATE: gy is the gradient of the gated output
+// sigmoid(r) * y; the step writes dL/dr = gy y s (1 - s) at grp
+// (s = sigmoid(r)) and carries gy s on as y's.
+template <bool FULL, bool GATE, bool SCALED, class E>
 __device__ __forceinline__ void wkv4_bwd_rstep(float2& A, float2& B, float2& Ap, float2& Bp, float2& fprod,
                                                float2& gwn, float2& gu_acc, float2 vv, float2 g, float2 rr,
-                                               float2 aa, float2 bb, float2 z, float2 uw2, E* gkp, E* gvp, E* grp) {
-  // output of the token, in units of the past's exponent P: weight
-  // e = 2^{u + k - P} = 2^{z1 + u - w} of the current token (capped as in
-  // the forward), D = 2^P (bb + e), y = (aa + e v) / (bb + e)
-  const float2 zo = add2(z, uw2);
-  const float2 e = make_float2(ex2(fminf(zo.x, 64.f)), ex2(fminf(zo.y, 64.f)));
-  const float2 rd = rcp2(add2(bb, e));
-  const float2 yv = mul2(fma2(e, vv, aa), rd);
-  // absorb pair of the token: P' = max(P - w, k)
-  const float2 ea = make_float2(ex2(-fabsf(z.x)), ex2(-fabsf(z.y)));
-  const bool kx = z.x <= 0.f, ky = z.y <= 0.f;
-  const float2 f1 = make_float2(kx ? 1.f : ea.x, ky ? 1.f : ea.y);
-  const float2 f2 = make_float2(kx ? ea.x : 1.f, ky ? ea.y : 1.f);
+                                               float2 aa, float2 bb, float2 z, float2 f1, float2 f2, float2 uw2,
+                                               float2 E2, E* gkp, E* gvp, E* grp) {
+  float2 yv, rd, e, rc, g2, t1, t2;
+  if constexpr (SCALED) {
+    t1 = mul2(f1, aa);
+    t2 = mul2(f1, bb);
+    g2 = mul2(f2, E2);
+    rc = rcp2(fma2(f1, bb, g2));
+    yv = mul2(fma2(g2, vv, t1), rc);
+  } else {
+    const float2 zo = add2(z, uw2);
+    e = make_float2(ex2(fminf(zo.x, 64.f)), ex2(fminf(zo.y, 64.f)));
+    rd = rcp2(add2(bb, e));
+    yv = mul2(fma2(e, vv, aa), rd);
+  }
   if constexpr (GATE) {
     const float2 sg = sigmoid2(rr);
     if constexpr (FULL) st_pair(grp, mul2(mul2(g, yv), mul2(sg, sub2(splat2(1.f), sg))));
     g = mul2(g, sg);
   }
-  const float2 ag = mul2(g, rd);  // gy 2^P / D
-  if constexpr (FULL) {
-    const float2 rg = mul2(ag, e);  // gy rho, rho = e^{u+k} / D
+  float2 ag, rg, vmy;  // gy 2^P / D; gy rho with rho = e^{u+k} / D; v - y
+  if constexpr (SCALED) {
+    const float2 q = mul2(g, rc);
+    ag = mul2(q, f1);
+    rg = mul2(q, g2);
+    // v - y = (bb v - aa) / (bb + e) = (t2 v - t1) / den
+    vmy = mul2(fma2(t2, vv, neg2(t1)), rc);
+  } else {
+    ag = mul2(g, rd);
+    rg = mul2(ag, e);
     // v - y = (bb v - aa) / (bb + e): no cancellation against v when the
     // current token dominates (y within rounding of v)
-    const float2 vmy = mul2(fma2(bb, vv, neg2(aa)), rd);
+    vmy = mul2(fma2(bb, vv, neg2(aa)), rd);
+  }
+  if constexpr (FULL) {
     const float2 gvv = fma2(f2, A, rg);
     const float2 gkv = fma2(rg, vmy, mul2(f2, fma2(vv, A, neg2(B))));
     gu_acc = fma2(rg, vmy, gu_acc);
@@ -176,33 +193,63 @@ __device__ __forceinline__ void wkv4_bwd_rstep(float2& A, float2& B, float2& Ap,
 // fprod (fold-only pass) accumulates the product of the f1 factors; gwn
 // accumulates -gw. WHOLE (n == kBwdL): the reverse steps are not
 // predicated, so the compiler can overlap the independent parts of
-// consecutive steps; the recompute loop always is.
-template <bool FULL, bool WHOLE, bool GATE, class E, bool S>
+// consecutive steps. The recompute runs the exponent chain of the interval's
+// tokens first and their value updates after it (the split of
+// wkv4_chain2 / wkv4_factors2; the same operations as wkv4_absorb2).
+template <bool FULL, bool WHOLE, bool GATE, bool SCALED, class E, bool S>
 __device__ __forceinline__ void wkv4_bwd_interval(const E (*ks)[kBwdCh], const E (*vs)[kBwdCh],
                                                   const E (*gs)[kBwdCh], const E (*rs)[kBwdCh],
                                                   Wkv4Stash<S, GATE>& sx, int lane, int n, Wkv4State2 st,
-                                                  float2 ref, float2 uw2, float2 w2, Wkv4Carry2& cr, float2& fprod,
-                                                  float2& gwn, float2& gu_acc, E* gkl, E* gvl, E* grl, int C) {
-  // forward recompute over the interval: state before each token and the
-  // token's absorb exponent z1 (the forward's own rounding of it)
+                                                  float2 ref, float2 uw2, float2 w2, float2 E2, Wkv4Carry2& cr,
+                                                  float2& fprod, float2& gwn, float2& gu_acc, E* gkl, E* gvl, E* grl,
+                                                  int C) {
+  // the stash holds f1, f2 (scaled form, ungated, shared memory) or z1
+  constexpr bool kStashF = S && SCALED && !GATE;
   constexpr int kReg = S ? 1 : kBwdL;
   float2 saa[kReg], sbb[kReg], sz[kReg];
+  if constexpr (S) {
+    // groups of kGrp tokens: the exponent chain of the group, then its value
+    // updates and stash writes (z of one group in registers)
+    constexpr int kGrp = WKV4_BWD_RECOMP_GROUP;
 #pragma unroll
-  for (int jj = 0; jj < kBwdL; ++jj) {
-    if (WKV4_BWD_WHOLE_RECOMPUTE && WHOLE || jj < n) {
-      const float2 aa = st.aa, bb = st.bb;
-      const float2 vj = ld_pair(&vs[jj][2 * lane]);
-      const float2 z1 = wkv4_absorb2(st, wkv4_key2(ld_pair(&ks[jj][2 * lane]), ref), vj, w2);
-      if constexpr (S) {
-        sx.ab[jj][lane] = make_float4(aa.x, aa.y, bb.x, bb.y);
-        if constexpr (GATE)
-          sx.zv[jj][lane] = z1;
-        else
-          sx.zv[jj][lane] = make_float4(z1.x, z1.y, vj.x, vj.y);
-      } else {
-        saa[jj] = aa;
-        sbb[jj] = bb;
-        sz[jj] = z1;
+    for (int j0 = 0; j0 < kBwdL; j0 += kGrp) {
+      float2 z[kGrp];
+#pragma unroll
+      for (int j = 0; j < kGrp; ++j) {
+        if (WKV4_BWD_WHOLE_RECOMPUTE && WHOLE || j0 + j < n) {
+          float2 unused;
+          z[j] = wkv4_chain2<true, false>(st, wkv4_key2(ld_pair(&ks[j0 + j][2 * lane]), ref), splat2(0.f), w2, unused);
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < kGrp; ++j) {
+        const int jj = j0 + j;
+        if (WKV4_BWD_WHOLE_RECOMPUTE && WHOLE || jj < n) {
+          const float2 aa = st.aa, bb = st.bb;
+          const float2 vj = ld_pair(&vs[jj][2 * lane]);
+          float2 f1, f2;
+          wkv4_factors2<false>(z[j], f1, f2);
+          st.aa = fma2(f2, vj, mul2(f1, st.aa));
+          st.bb = fma2(f1, st.bb, f2);
+          sx.ab[jj][lane] = make_float4(aa.x, aa.y, bb.x, bb.y);
+          if constexpr (GATE)
+            sx.zv[jj][lane] = z[j];
+          else if constexpr (kStashF)
+            sx.zv[jj][lane] = make_float4(f1.x, f1.y, f2.x, f2.y);
+          else
+            sx.zv[jj][lane] = make_float4(z[j].x, z[j].y, vj.x, vj.y);
+        }
+      }
+    }
+  } else {
+    // register stash: one token at a time (the stash already holds ~100
+    // registers)
+#pragma unroll
+    for (int jj = 0; jj < kBwdL; ++jj) {
+      if (WKV4_BWD_WHOLE_RECOMPUTE && WHOLE || jj < n) {
+        saa[jj] = st.aa;
+        sbb[jj] = st.bb;
+        sz[jj] = wkv4_absorb2<false>(st, wkv4_key2(ld_pair(&ks[jj][2 * lane]), ref), ld_pair(&vs[jj][2 * lane]), w2);
       }
     }
   }
@@ -212,28 +259,36 @@ __device__ __forceinline__ void wkv4_bwd_interval(const E (*ks)[kBwdCh], const E
     if (WHOLE || jj < n) {
       const float2 g = ld_pair(&gs[jj][2 * lane]);
       const float2 rr = GATE ? ld_pair(&rs[jj][2 * lane]) : splat2(0.f);
-      float2 aa, bb, z, vv;
+      float2 aa, bb, zz = splat2(0.f), vv, f1, f2;
       if constexpr (S) {
         const float4 ab = sx.ab[jj][lane];
         aa = make_float2(ab.x, ab.y);
         bb = make_float2(ab.z, ab.w);
         if constexpr (GATE) {
-          z = sx.zv[jj][lane];
+          zz = sx.zv[jj][lane];
+          vv = ld_pair(&vs[jj][2 * lane]);
+          wkv4_factors2<false>(zz, f1, f2);
+        } else if constexpr (kStashF) {
+          const float4 ff = sx.zv[jj][lane];
+          f1 = make_float2(ff.x, ff.y);
+          f2 = make_float2(ff.z, ff.w);
           vv = ld_pair(&vs[jj][2 * lane]);
         } else {
           const float4 zv = sx.zv[jj][lane];
-          z = make_float2(zv.x, zv.y);
+          zz = make_float2(zv.x, zv.y);
           vv = make_float2(zv.z, zv.w);
+          wkv4_factors2<false>(zz, f1, f2);
         }
       } else {
         aa = saa[jj];
         bb = sbb[jj];
-        z = sz[jj];
+        zz = sz[jj];
         vv = ld_pair(&vs[jj][2 * lane]);
+        wkv4_factors2<false>(zz, f1, f2);
       }
-      wkv4_bwd_rstep<FULL, GATE>(A, B, Ap, Bp, fprod, gwn, gu_acc, vv, g, rr, aa, bb, z, uw2,
-                                 gkl + (int64_t)jj * C, gvl + (int64_t)jj * C,
-                                 GATE ? grl + (int64_t)jj * C : nullptr);
+      wkv4_bwd_rstep<FULL, GATE, SCALED>(A, B, Ap, Bp, fprod, gwn, gu_acc, vv, g, rr, aa, bb, zz, f1, f2, uw2, E2,
+                                         gkl + (int64_t)jj * C, gvl + (int64_t)jj * C,
+                                         GATE ? grl + (int64_t)jj * C : nullptr);
     }
   }
   cr = {A, B, Ap, Bp};
@@ -311,6 +366,9 @@ __global__ void __launch_bounds__(32 * NW, NSEG == 1 ? 8 : 1) wkv4_bwd_kernel(co
   const float2 w2 = valid ? mul2(ld_pair(w + c), splat2(kLog2e)) : splat2(0.f);
   const float2 u2 = valid ? mul2(ld_pair(u + c), splat2(kLog2e)) : splat2(0.f);
   const float2 uw2 = sub2(u2, w2);  // output exponent minus absorb exponent
+  // output form of the pair (wkv4_scaled_pair) and its channel constants 2^{u2 - w2}
+  const bool scaled = wkv4_scaled_pair2(u2, w2);
+  const float2 E2 = wkv4_out_scale2(u2, w2);
   const int64_t lane_off = valid ? (int64_t)b * T * C + c : 0;
   // lane reference exponents: the values the forward derived from token 0
   float2 ref = splat2(0.f);
@@ -349,14 +407,22 @@ __global__ void __launch_bounds__(32 * NW, NSEG == 1 ? 8 : 1) wkv4_bwd_kernel(co
     E* grp = kFull && GATE ? gr + off : nullptr;
     const E (*rs)[kBwdCh] = nullptr;
     if constexpr (GATE) rs = sm.g.r[s];
-#if WKV4_BWD_WHOLE
-    if (n == kBwdL)
-      wkv4_bwd_interval<kFull, true, GATE>(sm.k[s], sm.v[s], sm.gy[s], rs, sm.stash, lane, n, st, ref, uw2, w2, cr,
-                                           fprod, gwn, gu_acc, gkp, gvp, grp, C);
-    else
-#endif
-      wkv4_bwd_interval<kFull, false, GATE>(sm.k[s], sm.v[s], sm.gy[s], rs, sm.stash, lane, n, st, ref, uw2, w2, cr,
-                                            fprod, gwn, gu_acc, gkp, gvp, grp, C);
+    auto go = [&](auto whole_tag, auto scaled_tag) {
+      wkv4_bwd_interval<kFull, decltype(whole_tag)::value, GATE, decltype(scaled_tag)::value>(
+          sm.k[s], sm.v[s], sm.gy[s], rs, sm.stash, lane, n, st, ref, uw2, w2, E2, cr, fprod, gwn, gu_acc, gkp, gvp,
+          grp, C);
+    };
+    if (WKV4_BWD_WHOLE && n == kBwdL) {
+      if (scaled)
+        go(BoolConst<true>{}, BoolConst<true>{});
+      else
+        go(BoolConst<true>{}, BoolConst<false>{});
+    } else {
+      if (scaled)
+        go(BoolConst<false>{}, BoolConst<true>{});
+      else
+        go(BoolConst<false>{}, BoolConst<false>{});
+    }
   };
 
   if constexpr (NSEG > 1) {
@@ -368,7 +434,7 @@ __global__ void __launch_bounds__(32 * NW, NSEG == 1 ? 8 : 1) wkv4_bwd_kernel(co
       const Wkv4State2 st = nxt;
       if (qq + 1 < nloc) nxt = load_ckpt(interval(qq + 1));
       if (!acquire(qq)) break;
-      if (valid) run_interval(BoolTag<false>{}, qq % STAGES, i, st, fprod);
+      if (valid) run_interval(BoolConst<false>{}, qq % STAGES, i, st, fprod);
       release(qq);
     }
     sm.carry[0][lane] = cr.A;
@@ -407,17 +473,19 @@ __global__ void __launch_bounds__(32 * NW, NSEG == 1 ? 8 : 1) wkv4_bwd_kernel(co
       const Wkv4State2 st = nxt;
       if (qq + 1 < total) nxt = load_ckpt(interval(qq + 1));
       if (!acquire(qq)) break;
-      if (valid) run_interval(BoolTag<true>{}, qq % STAGES, i, st, unused);
+      if (valid) run_interval(BoolConst<true>{}, qq % STAGES, i, st, unused);
       release(qq);
     }
   }
-  if (!ok) {
-    if (lane == 0)
-      for (int x = qq; x < total && x < qq + STAGES; ++x) mbar_wait_bounded(&sm.full[x % STAGES], (x / STAGES) & 1, err);
-  } else if (valid) {
+  if (!ok && lane == 0)
+    for (int x = qq; x < total && x < qq + STAGES; ++x) mbar_wait_bounded(&sm.full[x % STAGES], (x / STAGES) & 1, err);
+  if (valid) {
+    // after a wait that gave up (recorded in the device error word) the
+    // partial sums are written as zeros, so the batch sum never reads a
+    // value left in the scratch by an earlier call
     const int64_t pi = ((int64_t)b * NSEG + seg) * C + c;
-    st_pair(part_gw + pi, neg2(gwn));
-    st_pair(part_gu + pi, gu_acc);
+    st_pair(part_gw + pi, ok ? neg2(gwn) : splat2(0.f));
+    st_pair(part_gu + pi, ok ? gu_acc : splat2(0.f));
   }
   if constexpr (NSEG > 1) cluster_wait_acquire();  // peers may still read this CTA's carry
 }

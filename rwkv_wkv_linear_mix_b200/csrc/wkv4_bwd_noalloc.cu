@@ -11,12 +11,16 @@
 // file-scope device array instead.
 //
 // The array is kNoallocScratchBytes (4 MiB) and lives on every GPU that loads
-// the library until the process exits. Its device address is looked up once per
-// device, with that device current, on the first call made on it (so make that
-// first call before any stream capture). Every call shares the array: calls
-// whose kernels overlap on the GPU (several streams, or several host threads)
-// race on it and must be serialised by the caller. Nothing in it has to start
-// at zero: each call's kernels write every scratch element before reading it.
+// the library until the process exits. The call uses the array of the current
+// device (which must own the tensors and the stream); its device address is
+// looked up once per device, with that device current, on the first call made
+// on it (so make that first call before any stream capture). Every call shares
+// the array: calls whose kernels overlap on the GPU (several streams, or
+// several host threads) race on it and must be serialised by the caller.
+// Nothing in it has to start at zero: each call's kernels write every scratch
+// element before reading it (the backward writes its partial sums even after a
+// copy wait that gave up, as zeros; such a call's results are undefined and
+// the device error word says so).
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -71,8 +75,8 @@ WKV_EXPORT wkv_status wkv4_backward_noalloc(int64_t B, int64_t T, int64_t C, int
   const size_t need = wkv4_backward_workspace_bytes(B, T, C, ckpt != nullptr);
   if (need > kNoallocScratchBytes)
     return noalloc_fail(WKV_ERR_UNSUPPORTED,
-                        "wkv4_backward_noalloc: the problem needs more scratch than the 4 MiB static array "
-                        "(2*B*C floats, plus the checkpoints when ckpt is NULL); use wkv4_backward");
+                        "wkv4_backward_noalloc: wkv4_backward_workspace_bytes() of the problem exceeds the 4 MiB "
+                        "static array; pass ckpt or use wkv4_backward");
   void* scratch = nullptr;
   if (B > 0 && T > 0 && C > 0) {
     if (wkv_status s = scratch_ptr(&scratch)) return s;

@@ -140,18 +140,55 @@ __global__ void __launch_bounds__(kChunkThreads, kChunkMinBlocks) wkv4_chunk_ker
     w2[h] = make_float2(__fmul_rn(wc.x, kLog2e), __fmul_rn(wc.y, kLog2e));
     u2[h] = make_float2(__fmul_rn(uc.x, kLog2e), __fmul_rn(uc.y, kLog2e));
   }
-  for (int64_t t0 = 0; t0 < n; t0 += G) {
-    if (t0 > 0) load_group(t0);
+  // output form of each pair (wkv4_scaled_pair: decided from u and w alone)
+  bool scaled = true;
+  float2 E2[NP];
 #pragma unroll
-    for (int j = 0; j < G; ++j) {
-      if (t0 + j < n) {
+  for (int h = 0; h < NP; ++h) {
+    scaled = scaled && wkv4_scaled_pair2(u2[h], w2[h]);
+    E2[h] = wkv4_out_scale2(u2[h], w2[h]);
+  }
+  auto run = [&](auto scaled_tag) {
+    constexpr bool kScaled = decltype(scaled_tag)::value;
+    for (int64_t t0 = 0; t0 < n; t0 += G) {
+      if (t0 > 0) load_group(t0);
+#pragma unroll
+      for (int j = 0; j < G; ++j) {
+        if (t0 + j < n) {
+          float kk[NCH], vv[NCH], yy[NCH];
+          R::unpack(kr[j], kk);
+          R::unpack(vr[j], vv);
+#pragma unroll
+          for (int h = 0; h < NP; ++h) {
+            const float2 yv = wkv4_token2<kScaled>(st[h], wkv4_key2(make_float2(kk[2 * h], kk[2 * h + 1]), ref[h]),
+                                                   make_float2(vv[2 * h], vv[2 * h + 1]), u2[h], w2[h], E2[h]);
+            yy[2 * h] = yv.x;
+            yy[2 * h + 1] = yv.y;
+          }
+          R::store(yp + (t0 + j) * C, yy);
+        }
+      }
+    }
+  };
+  // (with two pairs per thread both must take the scaled form for the fast
+  // loop; a thread whose pairs differ runs the exact loop for the one that
+  // needs it and the scaled one for the other, pair by pair below)
+  if (NP == 1 || scaled) {
+    if (scaled)
+      run(BoolConst<true>{});
+    else
+      run(BoolConst<false>{});
+  } else {
+    for (int64_t t0 = 0; t0 < n; t0 += G) {
+      if (t0 > 0) load_group(t0);
+      for (int j = 0; j < G && t0 + j < n; ++j) {
         float kk[NCH], vv[NCH], yy[NCH];
         R::unpack(kr[j], kk);
         R::unpack(vr[j], vv);
-#pragma unroll
         for (int h = 0; h < NP; ++h) {
           const float2 yv = wkv4_token2(st[h], wkv4_key2(make_float2(kk[2 * h], kk[2 * h + 1]), ref[h]),
-                                        make_float2(vv[2 * h], vv[2 * h + 1]), u2[h], w2[h]);
+                                        make_float2(vv[2 * h], vv[2 * h + 1]), u2[h], w2[h],
+                                        wkv4_scaled_pair2(u2[h], w2[h]), E2[h]);
           yy[2 * h] = yv.x;
           yy[2 * h + 1] = yv.y;
         }

@@ -64,14 +64,22 @@ __global__ void __launch_bounds__(kDecThreads) wkv4_decode_kernel(int64_t total,
   float kk[4], vv[4], yy[4], o[5][4];
   ld_tok4(k + i, kk);
   ld_tok4(v + i, vv);
+  float w2c[4], u2c[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    w2c[j] = __fmul_rn(comp(w4, j), kLog2e);
+    u2c[j] = __fmul_rn(comp(u4, j), kLog2e);
+  }
+  // output form per channel pair (c, c + 1), (c + 2, c + 3), as every kernel decides it
+  const bool sc01 = wkv4_scaled_pair(u2c[0], w2c[0], u2c[1], w2c[1]);
+  const bool sc23 = wkv4_scaled_pair(u2c[2], w2c[2], u2c[3], w2c[3]);
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     Wkv4State st = {comp(aa, j), comp(bb, j), comp(base, j), comp(nn, j)};
     // a slot that has absorbed nothing yet takes its reference from this token
     const float ref = st.base == kEmptyPP ? wkv4_ref(kk[j]) : comp(rf, j);
-    const float w2 = __fmul_rn(comp(w4, j), kLog2e);
-    const float u2 = __fmul_rn(comp(u4, j), kLog2e);
-    yy[j] = wkv4_token(st, wkv4_key(kk[j], ref), vv[j], u2, w2);
+    yy[j] = wkv4_token(st, wkv4_key(kk[j], ref), vv[j], u2c[j], w2c[j], j < 2 ? sc01 : sc23,
+                       wkv4_out_scale(u2c[j], w2c[j]));
     o[0][j] = st.aa;
     o[1][j] = st.bb;
     o[2][j] = st.base;

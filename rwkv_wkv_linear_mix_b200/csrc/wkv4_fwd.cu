@@ -50,6 +50,47 @@ struct alignas(128) Wkv4FwdSmem {
   float2 seg_aa[32], seg_bb[32], seg_P[32];  // this segment's own state (phase 1)
 };
 
+// State (aa, bb, P) before a token to its checkpoint slot p ([3][C] floats).
+__device__ __forceinline__ void wkv4_write_ckpt(float* p, const Wkv4State2& st, float2 w2, int C) {
+  st_pair(p, st.aa);
+  st_pair(p + C, st.bb);
+  st_pair(p + 2 * (int64_t)C, wkv4_exponent2(st, w2));
+}
+
+// A whole tile of N tokens (N a multiple of WKV4_CKPT_LEN) for a lane's
+// channel pair, one checkpoint interval at a time: the exponent chain of the
+// interval's tokens runs first (z1, and zo for the exact form, kept in
+// registers), then their value updates and outputs. The chain is cheap and
+// serial; the second half's ex2/rcp of different tokens are independent, so
+// the split lets them overlap instead of waiting on one token at a time.
+// ckt: the tile's first checkpoint slot (null: none written).
+// A whole tile of N tokens (N a multiple of WKV4_CKPT_LEN) for a lane's
+// channel pair, one checkpoint interval at a time: the exponent chain of the
+// interval's tokens runs first (z1, and zo for the exact form, kept in
+// registers), then their value updates and outputs. The chain is cheap and
+// serial; the second half's ex2/rcp of different tokens are independent, so
+// the split lets them overlap instead of waiting on one token at a time.
+// ckt: the tile's first checkpoint slot (null: none written).
+template <bool SCALED, bool GATE, int N, class E>
+__device__ __forceinline__ void wkv4_fwd_tile(Wkv4State2& st, const E (*ks)[kFwdCh], const E (*vs)[kFwdCh],
+                                              const E (*rs)[kFwdCh], int lane, float2 ref, float2 u2, float2 w2,
+                                              float2 E2, E* yt, float* ckt, int C) {
+  constexpr int L = WKV4_CKPT_LEN;
+#pragma unroll
+  for (int jc = 0; jc < N; jc += L) {
+    if (ckt) wkv4_write_ckpt(ckt + (int64_t)(jc / L) * 3 * C, st, w2, C);
+    float2 z[L], zo[L];
+#pragma unroll
+    for (int j = 0; j < L; ++j) z[j] = wkv4_chain2<SCALED>(st, wkv4_key2(ld_pair(&ks[jc + j][2 * lane]), ref), u2, w2, zo[j]);
+#pragma unroll
+    for (int j = 0; j < L; ++j) {
+      float2 yv = wkv4_values2<SCALED>(st, z[j], zo[j], ld_pair(&vs[jc + j][2 * lane]), E2);
+      if constexpr (GATE) yv = mul2(yv, sigmoid2(ld_pair(&rs[jc + j][2 * lane])));
+      if (yt) st_pair(yt + (int64_t)(jc + j) * C, yv);
+    }
+  }
+}
+
 template <class E, int LT, int STAGES, int NSEG, int NW, bool GATE>
 __global__ void __launch_bounds__(32 * NW) wkv4_fwd_kernel(const __grid_constant__ CUtensorMap tk,
                                                            const __grid_constant__ CUtensorMap tv,
@@ -167,40 +208,29 @@ __global__ void __launch_bounds__(32 * NW) wkv4_fwd_kernel(const __grid_constant
 
   // ---- last pass: outputs and checkpoints ----
   E* yl = y ? y + lane_off : nullptr;
-  // state before token t (t a multiple of WKV4_CKPT_LEN) to the checkpoints
-  auto write_ckpt = [&](int t) {
-    float* p = ckl + (int64_t)(t / WKV4_CKPT_LEN) * 3 * C;
-    st_pair(p, st.aa);
-    st_pair(p + C, st.bb);
-    st_pair(p + 2 * (int64_t)C, wkv4_exponent2(st, w2));
-  };
+  const bool scaled = wkv4_scaled_pair2(u2, w2);
+  const float2 E2 = wkv4_out_scale2(u2, w2);
   for (; ok && q < total; ++q) {
     const int t0 = t_beg + (q % ntile) * LT;  // a multiple of WKV4_CKPT_LEN
-    if (ckl && valid) write_ckpt(t0);
     if (!acquire(q)) break;
     const int s = q % STAGES;
     const int n = min(LT, t_end - t0);
     if (valid) {
       E* yt = yl ? yl + (int64_t)t0 * C : nullptr;
+      float* ckt = ckl ? ckl + (int64_t)(t0 / WKV4_CKPT_LEN) * 3 * C : nullptr;
+      const E(*rs)[kFwdCh] = nullptr;
+      if constexpr (GATE) rs = sm.g.r[s];
       if (n == LT) {
-#pragma unroll
-        for (int jc = 0; jc < LT; jc += WKV4_CKPT_LEN) {
-          if (jc > 0 && ckl) write_ckpt(t0 + jc);
-#pragma unroll 8
-          for (int j2 = 0; j2 < WKV4_CKPT_LEN; ++j2) {
-            const int j = jc + j2;
-            float2 yv = wkv4_token2(st, wkv4_key2(ld_pair(&sm.k[s][j][2 * lane]), ref),
-                                    ld_pair(&sm.v[s][j][2 * lane]), u2, w2);
-            if constexpr (GATE) yv = mul2(yv, sigmoid2(ld_pair(&sm.g.r[s][j][2 * lane])));
-            if (yt) st_pair(yt + (int64_t)j * C, yv);
-          }
-        }
+        if (scaled)
+          wkv4_fwd_tile<true, GATE, LT>(st, sm.k[s], sm.v[s], rs, lane, ref, u2, w2, E2, yt, ckt, C);
+        else
+          wkv4_fwd_tile<false, GATE, LT>(st, sm.k[s], sm.v[s], rs, lane, ref, u2, w2, E2, yt, ckt, C);
       } else {
         for (int j = 0; j < n; ++j) {
-          if (j > 0 && j % WKV4_CKPT_LEN == 0 && ckl) write_ckpt(t0 + j);
-          float2 yv = wkv4_token2(st, wkv4_key2(ld_pair(&sm.k[s][j][2 * lane]), ref),
-                                  ld_pair(&sm.v[s][j][2 * lane]), u2, w2);
-          if constexpr (GATE) yv = mul2(yv, sigmoid2(ld_pair(&sm.g.r[s][j][2 * lane])));
+          if (j % WKV4_CKPT_LEN == 0 && ckt) wkv4_write_ckpt(ckt + (int64_t)(j / WKV4_CKPT_LEN) * 3 * C, st, w2, C);
+          float2 yv = wkv4_token2(st, wkv4_key2(ld_pair(&sm.k[s][j][2 * lane]), ref), ld_pair(&sm.v[s][j][2 * lane]),
+                                  u2, w2, scaled, E2);
+          if constexpr (GATE) yv = mul2(yv, sigmoid2(ld_pair(&rs[j][2 * lane])));
           if (yt) st_pair(yt + (int64_t)j * C, yv);
         }
       }

@@ -314,19 +314,52 @@ __device__ __forceinline__ float bf16hi(uint32_t p) { return __uint_as_float(p &
 //    half an ulp per step, always in the same direction).
 //  * each max-pair costs one ex2 and a select (one of its exponents is 0).
 // u2 = u * log2e, w2 = w * log2e. For token t with kk:
-//   output  zo = (u2 + kk) - P;   y = (aa + 2^{min(zo,64)} v) / (bb + 2^{min(zo,64)})
-//           (bb >= 1 once a token is absorbed and bb <= number of tokens, so
-//           beyond 2^64 the past is far below float32 resolution of the sum;
-//           the empty past, aa = bb = 0, gives y = v exactly)
-//   absorb  z1 = kk - (P - w2);   aa <- 2^{min(-z1,0)} aa + 2^{min(z1,0)} v,
-//                                 bb likewise, and (base, n) <- (base, n + 1)
-//                                 if z1 <= 0 else (kk, 0).
+//   absorb  z1 = kk - (P - w2), f = 2^{-|z1|}, (f1, f2) = (1, f) if z1 <= 0
+//           else (f, 1);  aa <- f2 v + fl(f1 aa),  bb <- f1 bb + f2 (each
+//           one fused multiply-add), and
+//           (base, n) <- (base, n + 1) if z1 <= 0 else (kk, 0). The choices
+//           are made with a 0/1 float mask (keep_mask) in exact fused
+//           multiply-adds rather than selects.
+//   output  the weight of the current token against the past is
+//           e = 2^{zo}, zo = (u2 + kk) - P, and y = (aa + e v) / (bb + e).
+//           It is formed in one of two ways, chosen per channel pair from
+//           u2 - w2 alone (so every kernel makes the same choice):
+//    * scaled (|u2 - w2| <= kScaledSpan): zo = z1 + (u2 - w2), so
+//      e = 2^{z1} E with the channel constant E = 2^{u2 - w2}; numerator and
+//      denominator multiplied by f1 give
+//          y = (f1 aa + f2 E v) / (f1 bb + f2 E),
+//      which reuses f1 aa and f1 bb of the absorb and needs no second ex2.
+//      The denominator is >= bb >= 1 (z1 <= 0, a token absorbed before) or
+//      >= E >= 2^-kScaledSpan (z1 > 0), so it never vanishes; a term that
+//      underflows to zero (f below 2^-126) is below 2^-68 of the other.
+//    * exact (any u2 - w2): e = 2^{min(zo, 64)} from a second ex2 (bb >= 1
+//      once a token is absorbed and bb <= number of tokens, so beyond 2^64
+//      the past is far below float32 resolution of the sum; the empty past,
+//      aa = bb = 0, gives y = v).
 // All roundings are explicit (_rn intrinsics) so that every kernel that runs
-// this step produces bit-identical results from the same state and inputs.
+// this step produces bit-identical results from the same state and inputs;
+// a sum of a product is always written as one fused multiply-add (the packed
+// pair forms of a separate multiply and add were measured to come out fused
+// in some places and not in others).
 // ----------------------------------------------------------------------------
 struct Wkv4State {
   float aa, bb, base, n;
 };
+
+// 1.0f when z <= 0 (the decayed past keeps the maximum), else 0.0f: the PTX
+// set instruction writes the float mask directly, and the step's selects
+// become exact fused multiply-adds with it (one of the two products is an
+// exact zero, the other an exact copy), which run on the FMA pipe instead of
+// the select unit.
+__device__ __forceinline__ float keep_mask(float z) {
+  float r;
+  asm("set.le.f32.f32 %0, %1, 0f00000000;" : "=f"(r) : "f"(z));
+  return r;
+}
+
+// |u2 - w2| (base 2) up to which the scaled output form is used: E and 1/E
+// stay within 2^57, far from float32 overflow and underflow.
+constexpr float kScaledSpan = 57.f;
 
 __device__ __forceinline__ Wkv4State wkv4_empty_state() { return {0.f, 0.f, kEmptyPP, 0.f}; }
 
@@ -341,25 +374,43 @@ __device__ __forceinline__ float wkv4_exponent(const Wkv4State& s, float w2) {
   return __fmaf_rn(-s.n, w2, s.base);
 }
 
-// Output of the token, then absorb it. Returns y.
-__device__ __forceinline__ float wkv4_token(Wkv4State& s, float kk, float v, float u2, float w2) {
+// Output form of the channel pair (c, c + 1) with base-2 rates (u2, w2) of
+// each: scaled iff both channels are within kScaledSpan. Every kernel decides
+// per pair, so a channel's results do not depend on how a kernel groups them.
+__device__ __forceinline__ bool wkv4_scaled_pair(float u2a, float w2a, float u2b, float w2b) {
+  return fabsf(__fsub_rn(u2a, w2a)) <= kScaledSpan && fabsf(__fsub_rn(u2b, w2b)) <= kScaledSpan;
+}
+// The channel constant E = 2^{u2 - w2} of the scaled form.
+__device__ __forceinline__ float wkv4_out_scale(float u2, float w2) { return ex2(__fsub_rn(u2, w2)); }
+
+// Output of the token, then absorb it. Returns y. scaled: the pair's output
+// form (wkv4_scaled_pair), E its channel constant.
+__device__ __forceinline__ float wkv4_token(Wkv4State& s, float kk, float v, float u2, float w2, bool scaled,
+                                            float E) {
   const float y0 = __fsub_rn(kk, s.base);
-  // output: weight of the current token (u2 + kk) relative to the past P
-  const float zo = __fmaf_rn(s.n, w2, __fadd_rn(y0, u2));
-  const float e = ex2(fminf(zo, 64.f));
-  const float y = __fmul_rn(__fmaf_rn(e, v, s.aa), rcp(__fadd_rn(s.bb, e)));
-  // absorb pair: token kk against the decayed past P - w2
   const float n1 = __fadd_rn(s.n, 1.f);
   const float z1 = __fmaf_rn(n1, w2, y0);
   const float ea = ex2(-fabsf(z1));
-  const bool pa = z1 <= 0.f;
-  const float f1 = pa ? 1.f : ea;
-  const float f2 = pa ? ea : 1.f;
-  s.aa = __fmaf_rn(f1, s.aa, __fmul_rn(f2, v));
+  const float pk = keep_mask(z1), nk = __fmaf_rn(pk, -1.f, 1.f);
+  const float f1 = __fmaf_rn(nk, ea, pk);  // 1 if the past keeps the maximum, else ea
+  const float f2 = __fmaf_rn(pk, ea, nk);  // ea if it does, else 1
+  const float t1 = __fmul_rn(f1, s.aa);
+  float num, den;
+  if (scaled) {
+    const float g = __fmul_rn(f2, E);
+    num = __fmaf_rn(g, v, t1);
+    den = __fmaf_rn(f1, s.bb, g);
+  } else {
+    const float zo = __fmaf_rn(s.n, w2, __fadd_rn(y0, u2));
+    const float e = ex2(fminf(zo, 64.f));
+    num = __fmaf_rn(e, v, s.aa);
+    den = __fadd_rn(s.bb, e);
+  }
+  s.aa = __fmaf_rn(f2, v, t1);
   s.bb = __fmaf_rn(f1, s.bb, f2);
-  s.base = pa ? s.base : kk;
-  s.n = pa ? n1 : 0.f;
-  return y;
+  s.base = __fmaf_rn(nk, kk, __fmul_rn(pk, s.base));  // base if kept, else kk
+  s.n = __fmul_rn(pk, n1);                            // n + 1 if kept, else 0
+  return __fmul_rn(num, rcp(den));
 }
 
 // Merge two states of the same lane given in the same reference: the result
@@ -376,19 +427,19 @@ __device__ __forceinline__ Wkv4Sum wkv4_merge(const Wkv4Sum& x, const Wkv4Sum& y
   return {__fmaf_rn(fx, x.aa, __fmul_rn(fy, y.aa)), __fmaf_rn(fx, x.bb, __fmul_rn(fy, y.bb)), xm ? x.P : y.P};
 }
 
-// Absorb only (no output).
+// Absorb only (no output): the same state update as wkv4_token.
 __device__ __forceinline__ void wkv4_absorb(Wkv4State& s, float kk, float v, float w2) {
   const float y0 = __fsub_rn(kk, s.base);
   const float n1 = __fadd_rn(s.n, 1.f);
   const float z1 = __fmaf_rn(n1, w2, y0);
   const float ea = ex2(-fabsf(z1));
-  const bool pa = z1 <= 0.f;
-  const float f1 = pa ? 1.f : ea;
-  const float f2 = pa ? ea : 1.f;
-  s.aa = __fmaf_rn(f1, s.aa, __fmul_rn(f2, v));
+  const float pk = keep_mask(z1), nk = __fmaf_rn(pk, -1.f, 1.f);
+  const float f1 = __fmaf_rn(nk, ea, pk);
+  const float f2 = __fmaf_rn(pk, ea, nk);
+  s.aa = __fmaf_rn(f2, v, __fmul_rn(f1, s.aa));
   s.bb = __fmaf_rn(f1, s.bb, f2);
-  s.base = pa ? s.base : kk;
-  s.n = pa ? n1 : 0.f;
+  s.base = __fmaf_rn(nk, kk, __fmul_rn(pk, s.base));
+  s.n = __fmul_rn(pk, n1);
 }
 
 // ----------------------------------------------------------------------------
@@ -426,6 +477,13 @@ __device__ __forceinline__ void st_pair(__nv_bfloat16* p, float2 v) {
   *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(v.x, v.y);
 }
 
+// A compile-time bool as a value (for generic lambdas that instantiate a
+// loop per flag).
+template <bool V>
+struct BoolConst {
+  static constexpr bool value = V;
+};
+
 struct Wkv4State2 {
   float2 aa, bb, base, n;
 };
@@ -439,42 +497,109 @@ __device__ __forceinline__ float2 wkv4_key2(float2 k, float2 ref) {
 __device__ __forceinline__ float2 wkv4_exponent2(const Wkv4State2& s, float2 w2) {
   return fma2(make_float2(-s.n.x, -s.n.y), w2, s.base);
 }
+__device__ __forceinline__ float2 keep_mask2(float2 z) { return make_float2(keep_mask(z.x), keep_mask(z.y)); }
+__device__ __forceinline__ bool wkv4_scaled_pair2(float2 u2, float2 w2) {
+  return wkv4_scaled_pair(u2.x, w2.x, u2.y, w2.y);
+}
+__device__ __forceinline__ float2 wkv4_out_scale2(float2 u2, float2 w2) {
+  return make_float2(wkv4_out_scale(u2.x, w2.x), wkv4_out_scale(u2.y, w2.y));
+}
 
-// Pair form of wkv4_token (same operations in the same order).
-__device__ __forceinline__ float2 wkv4_token2(Wkv4State2& s, float2 kk, float2 v, float2 u2, float2 w2) {
+// The step of a pair split in two halves, so that a kernel can run the
+// exponent chain of a group of tokens ahead of their value updates (the
+// chain is the only part whose latency carries from token to token that
+// involves more than one instruction; the halves together are wkv4_token
+// on each channel, operation for operation).
+// First half: the absorb exponent z1 of the token (and, for the exact output
+// form, zo), advancing (base, n).
+// MASK: make the choices with the float mask (keep_mask) on the FMA pipe;
+// otherwise with predicates and selects. Both give the same values (the
+// masked forms are exact; at most the sign of a zero base differs, which no
+// later operation can see): the forward, bound by its select unit, takes the
+// masks, the backward's recompute, bound by the latency of this chain, the
+// two-instruction select path.
+template <bool SCALED, bool MASK = true>
+__device__ __forceinline__ float2 wkv4_chain2(Wkv4State2& s, float2 kk, float2 u2, float2 w2, float2& zo) {
   const float2 y0 = sub2(kk, s.base);
-  const float2 zo = fma2(s.n, w2, add2(y0, u2));
-  const float2 e = make_float2(ex2(fminf(zo.x, 64.f)), ex2(fminf(zo.y, 64.f)));
-  const float2 y = mul2(fma2(e, v, s.aa), rcp2(add2(s.bb, e)));
+  if constexpr (!SCALED) zo = fma2(s.n, w2, add2(y0, u2));
   const float2 n1 = add2(s.n, splat2(1.f));
   const float2 z1 = fma2(n1, w2, y0);
+  if constexpr (MASK) {
+    const float2 pk = keep_mask2(z1), nk = fma2(pk, splat2(-1.f), splat2(1.f));
+    s.base = fma2(nk, kk, mul2(pk, s.base));
+    s.n = mul2(pk, n1);
+  } else {
+    const bool px = z1.x <= 0.f, py = z1.y <= 0.f;
+    s.base = make_float2(px ? s.base.x : kk.x, py ? s.base.y : kk.y);
+    s.n = make_float2(px ? n1.x : 0.f, py ? n1.y : 0.f);
+  }
+  return z1;
+}
+// Absorb factors (f1, f2) of a token with exponent z1.
+template <bool MASK = true>
+__device__ __forceinline__ void wkv4_factors2(float2 z1, float2& f1, float2& f2) {
   const float2 ea = make_float2(ex2(-fabsf(z1.x)), ex2(-fabsf(z1.y)));
-  const bool px = z1.x <= 0.f, py = z1.y <= 0.f;
-  const float2 f1 = make_float2(px ? 1.f : ea.x, py ? 1.f : ea.y);
-  const float2 f2 = make_float2(px ? ea.x : 1.f, py ? ea.y : 1.f);
-  s.aa = fma2(f1, s.aa, mul2(f2, v));
+  if constexpr (MASK) {
+    const float2 pk = keep_mask2(z1), nk = fma2(pk, splat2(-1.f), splat2(1.f));
+    f1 = fma2(nk, ea, pk);
+    f2 = fma2(pk, ea, nk);
+  } else {
+    const bool px = z1.x <= 0.f, py = z1.y <= 0.f;
+    f1 = make_float2(px ? 1.f : ea.x, py ? 1.f : ea.y);
+    f2 = make_float2(px ? ea.x : 1.f, py ? ea.y : 1.f);
+  }
+}
+// Second half: output of the token and the update of (aa, bb). E: the
+// pair's channel constants (scaled form); zo from the first half (exact).
+template <bool SCALED>
+__device__ __forceinline__ float2 wkv4_values2(Wkv4State2& s, float2 z1, float2 zo, float2 v, float2 E) {
+  float2 f1, f2;
+  wkv4_factors2(z1, f1, f2);
+  const float2 t1 = mul2(f1, s.aa);
+  float2 num, den;
+  if constexpr (SCALED) {
+    const float2 g = mul2(f2, E);
+    num = fma2(g, v, t1);
+    den = fma2(f1, s.bb, g);
+  } else {
+    const float2 e = make_float2(ex2(fminf(zo.x, 64.f)), ex2(fminf(zo.y, 64.f)));
+    num = fma2(e, v, s.aa);
+    den = add2(s.bb, e);
+  }
+  s.aa = fma2(f2, v, t1);
   s.bb = fma2(f1, s.bb, f2);
-  s.base = make_float2(px ? s.base.x : kk.x, py ? s.base.y : kk.y);
-  s.n = make_float2(px ? n1.x : 0.f, py ? n1.y : 0.f);
-  return y;
+  return mul2(num, rcp2(den));
+}
+
+// Pair form of wkv4_token (same operations in the same order).
+template <bool SCALED>
+__device__ __forceinline__ float2 wkv4_token2(Wkv4State2& s, float2 kk, float2 v, float2 u2, float2 w2, float2 E) {
+  float2 zo = splat2(0.f);
+  const float2 z1 = wkv4_chain2<SCALED>(s, kk, u2, w2, zo);
+  return wkv4_values2<SCALED>(s, z1, zo, v, E);
+}
+__device__ __forceinline__ float2 wkv4_token2(Wkv4State2& s, float2 kk, float2 v, float2 u2, float2 w2, bool scaled,
+                                              float2 E) {
+  return scaled ? wkv4_token2<true>(s, kk, v, u2, w2, E) : wkv4_token2<false>(s, kk, v, u2, w2, E);
 }
 
 // Pair form of wkv4_absorb. Returns z1, the exponent of the token against
 // the decayed past (2^{-|z1|} is the absorb factor; z1 <= 0 keeps the past's
-// maximum).
-__device__ __forceinline__ float2 wkv4_absorb2(Wkv4State2& s, float2 kk, float2 v, float2 w2) {
-  const float2 y0 = sub2(kk, s.base);
-  const float2 n1 = add2(s.n, splat2(1.f));
-  const float2 z1 = fma2(n1, w2, y0);
-  const float2 ea = make_float2(ex2(-fabsf(z1.x)), ex2(-fabsf(z1.y)));
-  const bool px = z1.x <= 0.f, py = z1.y <= 0.f;
-  const float2 f1 = make_float2(px ? 1.f : ea.x, py ? 1.f : ea.y);
-  const float2 f2 = make_float2(px ? ea.x : 1.f, py ? ea.y : 1.f);
-  s.aa = fma2(f1, s.aa, mul2(f2, v));
+// maximum), and the factors f1, f2.
+template <bool MASK = true>
+__device__ __forceinline__ float2 wkv4_absorb2(Wkv4State2& s, float2 kk, float2 v, float2 w2, float2& f1,
+                                               float2& f2) {
+  float2 unused;
+  const float2 z1 = wkv4_chain2<true, MASK>(s, kk, splat2(0.f), w2, unused);
+  wkv4_factors2<MASK>(z1, f1, f2);
+  s.aa = fma2(f2, v, mul2(f1, s.aa));
   s.bb = fma2(f1, s.bb, f2);
-  s.base = make_float2(px ? s.base.x : kk.x, py ? s.base.y : kk.y);
-  s.n = make_float2(px ? n1.x : 0.f, py ? n1.y : 0.f);
   return z1;
+}
+template <bool MASK = true>
+__device__ __forceinline__ float2 wkv4_absorb2(Wkv4State2& s, float2 kk, float2 v, float2 w2) {
+  float2 f1, f2;
+  return wkv4_absorb2<MASK>(s, kk, v, w2, f1, f2);
 }
 
 }  // namespace wkv

@@ -118,6 +118,17 @@ def _want(t: torch.Tensor, name: str, dtype=None, shape=None, device=None):
         raise ValueError(f"{name} is on {t.device}, expected {device}")
 
 
+def _want_wkv4_grads(k, gk, gv, gw, gu):
+    """Caller-provided RWKV-4 gradient buffers must match what the kernels
+    write: gk, gv like k; gw, gu float32 [C] (a smaller or mistyped buffer
+    would be written past its end)."""
+    C = k.shape[-1]
+    _want(gk, "gk", dtype=k.dtype, shape=k.shape, device=k.device)
+    _want(gv, "gv", dtype=k.dtype, shape=k.shape, device=k.device)
+    _want(gw, "gw", dtype=torch.float32, shape=(C,), device=k.device)
+    _want(gu, "gu", dtype=torch.float32, shape=(C,), device=k.device)
+
+
 def abi_version() -> int:
     return int(_lib.wkv_abi_version())
 
@@ -183,6 +194,7 @@ def wkv4_backward(w, u, k, v, gy, ckpt: Optional[torch.Tensor] = None, *, gk=Non
     gv = torch.empty_like(k) if gv is None else gv
     gw = torch.empty(C, dtype=torch.float32, device=dev) if gw is None else gw
     gu = torch.empty(C, dtype=torch.float32, device=dev) if gu is None else gu
+    _want_wkv4_grads(k, gk, gv, gw, gu)
     nbytes = wkv4_backward_workspace_bytes(B, T, C, ckpt is not None)
     if workspace is None:
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
@@ -210,9 +222,12 @@ def wkv4_backward_noalloc(w, u, k, v, gy, ckpt: Optional[torch.Tensor] = None, *
     gv = torch.empty_like(k) if gv is None else gv
     gw = torch.empty(C, dtype=torch.float32, device=dev) if gw is None else gw
     gu = torch.empty(C, dtype=torch.float32, device=dev) if gu is None else gu
-    _check(_lib.wkv4_backward_noalloc(B, T, C, _dtype_code(k), _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(gy),
-                                      _ptr(ckpt), _ptr(gk), _ptr(gv), _ptr(gw), _ptr(gu), _stream(k)),
-           "wkv4_backward_noalloc")
+    _want_wkv4_grads(k, gk, gv, gw, gu)
+    # the library finds the static array of the current device: make it k's
+    with torch.cuda.device(dev):
+        _check(_lib.wkv4_backward_noalloc(B, T, C, _dtype_code(k), _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(gy),
+                                          _ptr(ckpt), _ptr(gk), _ptr(gv), _ptr(gw), _ptr(gu), _stream(k)),
+               "wkv4_backward_noalloc")
     return gk, gv, gw, gu
 
 
@@ -253,6 +268,8 @@ def wkv4_backward_gated(w, u, k, v, r, gy, ckpt: Optional[torch.Tensor] = None, 
     gr = torch.empty_like(k) if gr is None else gr
     gw = torch.empty(C, dtype=torch.float32, device=dev) if gw is None else gw
     gu = torch.empty(C, dtype=torch.float32, device=dev) if gu is None else gu
+    _want_wkv4_grads(k, gk, gv, gw, gu)
+    _want(gr, "gr", dtype=k.dtype, shape=k.shape, device=dev)
     nbytes = wkv4_backward_workspace_bytes(B, T, C, ckpt is not None)
     if workspace is None:
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
@@ -304,6 +321,10 @@ def wkv4_time_shift_mix_backward(x, mix, g, x_prev: Optional[torch.Tensor] = Non
     gmix = torch.empty((n, C), dtype=torch.float32, device=dev) if gmix is None else gmix
     if gx_prev is None and want_gx_prev:
         gx_prev = torch.empty((B, C), dtype=x.dtype, device=dev)
+    _want(gx, "gx", dtype=x.dtype, shape=x.shape, device=dev)
+    _want(gmix, "gmix", dtype=torch.float32, shape=(n, C), device=dev)
+    if gx_prev is not None:
+        _want(gx_prev, "gx_prev", dtype=x.dtype, shape=(B, C), device=dev)
     nbytes = wkv4_time_shift_mix_backward_workspace_bytes(B, T, C, x.dtype, n)
     if workspace is None:
         workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=dev)
@@ -393,8 +414,11 @@ def wkv6_forward(r, k, v, w, u, init_state: Optional[torch.Tensor] = None,
     if state_map is not None:
         _want(state_map, "state_map", dtype=torch.int32, shape=(B,), device=dev)
     o = torch.empty_like(r) if o is None else o
+    _want(o, "o", dtype=r.dtype, shape=r.shape, device=dev)
     if want_final_state and final_state is None:
         final_state = torch.empty((B, H, K, K), dtype=torch.float32, device=dev)
+    if final_state is not None:
+        _want(final_state, "final_state", dtype=torch.float32, shape=(B, H, K, K), device=dev)
     _check(_lib.wkv6_forward(B, T, H, K, _dtype_code(r), _ptr(r), _ptr(k), _ptr(v), _ptr(w), _ptr(u),
                              _ptr(init_state), _ptr(state_map), n_state, _ptr(final_state), _ptr(o),
                              _stream(r)), "wkv6_forward")
@@ -448,9 +472,15 @@ def wkv6_backward(r, k, v, w, u, dout, init_state: Optional[torch.Tensor] = None
     gu = torch.empty(HK, dtype=torch.float32, device=dev) if gu is None else gu
     if want_g_init and g_init is None:
         g_init = torch.empty((B, H, K, K), dtype=torch.float32, device=dev)
+    for name, t in (("gr", gr), ("gk", gk), ("gv", gv), ("glogw", glogw)):
+        _want(t, name, dtype=r.dtype, shape=r.shape, device=dev)
+    _want(gu, "gu", dtype=torch.float32, shape=(HK,), device=dev)
+    if g_init is not None:
+        _want(g_init, "g_init", dtype=torch.float32, shape=(B, H, K, K), device=dev)
     need = wkv6_backward_workspace_bytes(B, T, H, K)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _want(workspace, "workspace", device=dev)
     _check(_lib.wkv6_backward(B, T, H, K, _dtype_code(r), _ptr(r), _ptr(k), _ptr(v), _ptr(w), _ptr(u),
                               _ptr(init_state), _ptr(state_map), n_state, _ptr(dout), _ptr(g_final),
                               _ptr(gr), _ptr(gk), _ptr(gv), _ptr(glogw), _ptr(gu), _ptr(g_init),
@@ -475,8 +505,11 @@ def wkv7_forward(r, w, k, v, a, b, init_state: Optional[torch.Tensor] = None, *,
     if init_state is not None:
         _want(init_state, "init_state", dtype=torch.float32, shape=(B, H, K, K), device=dev)
     o = torch.empty_like(r) if o is None else o
+    _want(o, "o", dtype=r.dtype, shape=r.shape, device=dev)
     if want_final_state and final_state is None:
         final_state = torch.empty((B, H, K, K), dtype=torch.float32, device=dev)
+    if final_state is not None:
+        _want(final_state, "final_state", dtype=torch.float32, shape=(B, H, K, K), device=dev)
     _check(_lib.wkv7_forward(B, T, H, K, _dtype_code(r), _ptr(r), _ptr(w), _ptr(k), _ptr(v), _ptr(a), _ptr(b),
                              _ptr(init_state), _ptr(final_state), _ptr(o), _stream(r)), "wkv7_forward")
     return o, final_state

@@ -21,6 +21,6 @@ def test_reference_arm_prints_one_contract_line():
                 "config", "cpu_baseline", "e2e"):
         assert key in d, key
     assert d["steps"] == 2 and d["warmup"] == 1 and d["value"] > 0
-    assert d["config"]["workload"] == "wkv4_fb_f32_169m"
+    assert d["config"]["workload"] == "wkv4_fb_bf16_3b"
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"]["value"] == d["value"] and d["e2e"]["h2d_bytes_per_step"] == 0
