@@ -1,43 +1,49 @@
-// wkv6_bwd.cu -- RWKV-6 head-state WKV backward on sm_100a.
+// wkv6_bwd.cu -- RWKV-6 head-state WKV backward on sm_100a, chunked, with the
+// contractions on the tcgen05 tensor cores.
 //
 // Gradients of L = sum(dout * o) + sum(g_final * S_final) for the forward of
-// wkv6_fwd.cu (RWKV6_OP on the rwkv-ops package page; the operator is
-// trained, and its PyTorch CUDA implementation is listed there), per head
-// with K = 64 (S indexed [i][j], i the key index, j the value index):
+// wkv6_fwd.cu (RWKV6_OP on the rwkv-ops package page, section "rwkv6op
+// 使用方法"; the operator is trained, and its PyTorch CUDA implementation is
+// listed there), per head with K = 64 (S indexed [i][j], i the key index, j
+// the value index):
 //   S_t = diag(w_t) S_{t-1} + k_t^T v_t,   o_t = r_t (S_{t-1} + diag(u) k_t^T v_t)
-// With G_t = dL/dS_t (G_{T-1} = g_final):
-//   G_{t-1} = diag(w_t) G_t + r_t^T do_t
-//   gr_t = S_{t-1} do_t + u o k_t (v_t . do_t)
-//   gk_t = G_t v_t + u o r_t (v_t . do_t)
-//   gv_t = k_t G_t + (r_t . (u o k_t)) do_t
-//   gu   = sum_t r_t o k_t (v_t . do_t)
-// and for the decay, with P_t[i] = sum_j G_t[i][j] S_t[i][j]:
-//   w_t o gw_t = P_t - k_t o (G_t v_t)
-//   P_{t-1}    = P_t - k_t o (G_t v_t) + r_t o (S_{t-1} do_t)
-// (expand S_t and G_{t-1} by their recurrences). These give the gradient
-// with respect to log w without S_{t-1} and G_t at the same step: P starts
-// from sum_j g_final S_final and walks down on two row products the passes
-// form anyway. The kernel returns glogw = w o gw (what w = exp(-exp(d))
-// consumes: dL/dd = -exp(d) glogw); it stays accurate where w_t is tiny,
-// where gw itself would be a difference of large terms divided by w_t.
+// With G_t = dL/dS_t (G_{T-1} = g_final), G_{t-1} = diag(w_t) G_t + r_t^T do_t.
 //
-// Two passes, one CTA of 128 threads per (b, h); thread (p = tid / 4,
-// q = tid % 4) holds rows 2p and 2p + 1, columns 16q .. 16q + 15 (each slice
-// of a token's vectors it reads serves two rows):
-//   pass 1 (t up):   S; writes gr and, per token, x_t = r_t o (S_{t-1} do_t)
-//                    and (c_t = r_t . (u o k_t), v_t . do_t) to the workspace;
-//                    at the end P_{T-1} = sum_j g_final S_{T-1}.
-//   pass 2 (t down): G in two copies, by rows (G v, the P walk, g_init) and
-//                    by columns 2p, 2p + 1 (rows 16q ..: k G becomes a row
-//                    product as well, so no 64-way reduction across
-//                    threads); writes gk, gv, glogw and per-(b, h) gu
-//                    partials.
-// Inputs arrive per 32-token chunk by TMA into two stages (the next chunk
-// loads while this one runs). Each step reads its 16-wide slices as bf16 (32
-// bytes per vector) one step ahead of use and widens them in registers.
-// Outputs leave through shared-memory tiles as coalesced 16-byte stores. The
-// 16-wide row work runs on packed fp32 pairs. gu is summed over samples by a
-// fixed-order reduction.
+// Three steps.
+//  1. The forward, writing the state S_in entering every 64-token chunk.
+//  2. The gradient state G walks the sequence backwards with the same
+//     recurrence as S forwards: with the time order reversed, (k, r, do, w)
+//     in the roles of (r, k, v, w) and g_final as the initial state, the
+//     forward computes gv (its output: gv_t = k_t G_t + (r_t . (u o k_t)) do_t),
+//     g_init = G_{-1} (its final state) and G at every chunk boundary (its
+//     chunk states). It runs on time-reversed copies of the four inputs,
+//     padded at the front to whole chunks (padding: r = k = do = 0, w = 1,
+//     which leaves the state as it is), so its chunks are those of step 1.
+//  3. One CTA per chunk, independent of every other chunk, from S_in and
+//     G_out of its chunk (chunk-local notation: tokens j = 0..63,
+//     E_j = prod_{tau <= j} w_tau, R^_j = r_j o E_{j-1}, K~_s = k_s / E_s,
+//     A[j][s] = R^_j . K~_s for s < j):
+//       dA  = dO V^T                (masked: dA_s strictly below the diagonal)
+//       dR^ = dA_s K~ + dO S_in^T,   gr_j = E_{j-1} o dR^_j + dA[j][j] u o k_j
+//       dK~ = dA_s^T R^,             dK^ = V G_out^T
+//       gk_s = dK~_s / E_s + dK^_s o E_{L-1} / E_s + dA[s][s] u o r_s
+//       gu  += sum_j dA[j][j] r_j o k_j
+//     and the decay gradient, w o dL/dw (= dL/dlog w), from the products with
+//     the chunk-scaled operands:
+//       glogw_t = sum_{j > t} x_j - sum_{s >= t} y_s + sum_{s < t} z_s + c
+//     with x_j = dR^_j o R^_j (= (gr_j - bonus) o r_j), y_s = dK~_s o K~_s,
+//     z_s = dK^_s o K^_s (K^ = k_s E_{L-1} / E_s) and, from the S_out =
+//     diag(E_{L-1}) S_in + ... term, c = E_{L-1} o rowsum(G_out o S_in).
+//     The five products run as tcgen05 MMAs with accumulators in tensor
+//     memory: dO V^T in bf16; dO S_in^T and V G_out^T in bf16 with the fp32
+//     state split hi + lo (hi = bf16(x), lo = bf16(x - hi)); dA_s K~ and
+//     dA_s^T R^ in tf32. A chunk whose total decay falls below 2^-96 in some
+//     channel (K~ could overflow) forms its two intra-chunk sums on the CUDA
+//     cores instead, with the decay between each pair of tokens as a running
+//     product (never a quotient).
+//
+// gu partials per (sample, head, chunk) are added in a fixed order by a
+// small kernel: every result is deterministic.
 #include <string.h>
 
 #include "wkv_device.cuh"
@@ -45,438 +51,583 @@
 
 namespace wkv {
 
-constexpr int kK6b = 64;       // head size
-constexpr int kL6b = 32;       // tokens per chunk
-constexpr int kT6b = 128;      // threads per CTA (2 rows per thread)
-constexpr int kIn6b = 5;       // r, k, v, w, do
-enum { kR = 0, kKk = 1, kV = 2, kW = 3, kDo = 4 };
+namespace {
 
-struct alignas(128) Wkv6Bwd1Smem {
-  __nv_bfloat16 in[2][kIn6b][kL6b][kK6b];  // two TMA stages
-  float cv[2][kL6b][4];                    // per stage and token: c_t, v_t . do_t
-  float xo[kL6b][kK6b];                    // x_t rows for the workspace
-  __nv_bfloat16 gro[kL6b][kK6b];           // gr tile
-  uint64_t full[2];
+constexpr int kK6 = 64;                     // head size
+constexpr int kL6 = 64;                     // tokens per chunk
+constexpr int kThr6 = 256;                  // threads per chunk CTA
+constexpr uint32_t kTile = 8192;            // 64 x 64 bf16, or one 64 x 32 fp32 panel
+constexpr uint32_t kTmemCols = 256;         // dA, dR^, dK^, dK~
+constexpr uint32_t kColDA = 0, kColDR = 64, kColDKh = 128, kColDKt = 192;
+constexpr float kMinDecay = 1.2621774e-29f;  // 2^-96, as the forward
+
+// Shared memory of the chunk kernel (1024-byte aligned tiles).
+struct alignas(1024) Bwd6Smem {
+  // bf16 tiles [t][i] as the TMA writes them (128-byte rows, 128-byte swizzle)
+  uint8_t r[kTile], k[kTile], w[kTile];
+  uint8_t v[kTile], dout[kTile];  // after the first MMAs: E_{t-1} table, then the z table ([t][64] fp32)
+  // bf16 hi/lo tiles of S_in and G_out [i][jv] (B operands); after the first
+  // MMAs two fp32 tiles: dA_s [j][s] and its transpose [s][j] (A operands);
+  // after the second MMAs the x and g tables of the decay gradient
+  uint8_t sg[4 * kTile];
+  // fp32 tiles K~^T [i][s] and R^^T [i][j] (B operands of the second MMAs);
+  // afterwards the gr, gk, glogw output tiles (bf16 [t][64])
+  uint8_t kr[4 * kTile];
+  float wprod[8][kK6];   // products of w over each warp's 8 tokens
+  float tot[kK6];        // E_{L-1}
+  float dd[kL6];         // dA[t][t]
+  float cpart[2][kK6];   // row sums of G_out o S_in, per column half
+  float u[kK6];
+  float scan[2][4][kK6];  // per quarter of the tokens: sums of the z and g tables
+  uint64_t in_bar, mma_bar;
+  uint32_t tmem_base;
 };
 
-struct alignas(128) Wkv6Bwd2Stage {
-  __nv_bfloat16 in[kIn6b][kL6b][kK6b];
-  float x[kL6b][kK6b];   // x_t rows
-  float cv[kL6b][4];     // (c_t, v_t . do_t, -, -)
-};
-
-struct alignas(128) Wkv6Bwd2Smem {
-  Wkv6Bwd2Stage st[2];                  // two TMA stages
-  __nv_bfloat16 out[3][kL6b][kK6b];     // gk, gv, glogw tiles
-  uint64_t full[2];
-};
-
-// 16 consecutive bf16 of shared memory (two 16-byte loads), and their
-// widening to 8 fp32 pairs (element 2m in the low half of word m).
-struct Bf16x16 {
-  uint4 a, b;
-};
-__device__ __forceinline__ Bf16x16 ld16b(const __nv_bfloat16* p) {
-  const uint4* p4 = reinterpret_cast<const uint4*>(p);
-  return {p4[0], p4[1]};
+// Byte offset of element (row, col) of a swizzled bf16 tile.
+__device__ __forceinline__ int bo(int row, int col) {
+  return row * 128 + ((((col >> 3) ^ (row & 7)) & 7) << 4) + (col & 7) * 2;
 }
-__device__ __forceinline__ void widen16(const Bf16x16& x, float2 (&y)[8]) {
-  const uint32_t wds[8] = {x.a.x, x.a.y, x.a.z, x.a.w, x.b.x, x.b.y, x.b.z, x.b.w};
-#pragma unroll
-  for (int m = 0; m < 8; ++m) y[m] = make_float2(bf16lo(wds[m]), bf16hi(wds[m]));
+// Byte offset of element (row, col) of a two-panel swizzled fp32 tile.
+__device__ __forceinline__ int fo(int row, int col) {
+  return (col >> 5) * (int)kTile + row * 128 + (((((col & 31) >> 2) ^ (row & 7)) & 7) << 4) + (col & 3) * 4;
 }
-__device__ __forceinline__ float bf(const __nv_bfloat16& x) { return __bfloat162float(x); }
-
-// 16 consecutive fp32 of global memory as 8 pairs.
-__device__ __forceinline__ void ld16(const float* p, float2 (&x)[8]) {
-  const float4* p4 = reinterpret_cast<const float4*>(p);
-#pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    const float4 a = p4[m];
-    x[2 * m] = make_float2(a.x, a.y);
-    x[2 * m + 1] = make_float2(a.z, a.w);
-  }
+__device__ __forceinline__ float tb(const uint8_t* tile, int row, int col) {
+  return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(tile + bo(row, col)));
+}
+__device__ __forceinline__ float& tf(uint8_t* tile, int row, int col) {
+  return *reinterpret_cast<float*>(tile + fo(row, col));
+}
+__device__ __forceinline__ float tfc(const uint8_t* tile, int row, int col) {
+  return *reinterpret_cast<const float*>(tile + fo(row, col));
 }
 
-// Sum over the 4 threads of a row (lanes 4m .. 4m + 3).
-__device__ __forceinline__ float row_sum4(float x) {
-  x += __shfl_xor_sync(0xffffffffu, x, 1);
-  x += __shfl_xor_sync(0xffffffffu, x, 2);
-  return x;
-}
+__global__ void __launch_bounds__(kThr6, 2)
+    wkv6_bwd_chunk_kernel(const __grid_constant__ CUtensorMap tr, const __grid_constant__ CUtensorMap tk,
+                          const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tw,
+                          const __grid_constant__ CUtensorMap tdo, int T, int H, int nch, const float* __restrict__ u,
+                          const float* __restrict__ ck_s, const float* __restrict__ ck_g,
+                          __nv_bfloat16* __restrict__ gr, __nv_bfloat16* __restrict__ gk,
+                          __nv_bfloat16* __restrict__ glogw, float* __restrict__ gu_part, unsigned* err) {
+  extern __shared__ uint8_t bwd6_dsmem[];
+  Bwd6Smem& sm = *reinterpret_cast<Bwd6Smem*>((reinterpret_cast<uintptr_t>(bwd6_dsmem) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int c = blockIdx.x % nch;
+  const int bh = blockIdx.x / nch;
+  const int h = bh % H, b = bh / H;
+  const int t0 = c * kL6;
+  const int valid = min(kL6, T - t0);
+  const int64_t HK = (int64_t)H * kK6;
+  // accumulator read-back layout (16x256b): TMEM sub-partition sp, column
+  // half ch; rows r0 and r1 = r0 + 8, columns cq + 8 q + {0, 1}, q = 0..3
+  const int sp = warp & 3, ch = warp >> 2;
+  const int r0 = 16 * sp + (lane >> 2), r1 = r0 + 8;
+  const int cq = 32 * ch + 2 * (lane & 3);
 
-__device__ __forceinline__ float dot16(const float2 (&a)[8], const float2 (&b)[8]) {
-  float2 s0 = make_float2(0.f, 0.f), s1 = s0;
-#pragma unroll
-  for (int m = 0; m < 8; m += 2) {
-    s0 = fma2(a[m], b[m], s0);
-    s1 = fma2(a[m + 1], b[m + 1], s1);
-  }
-  const float2 s = add2(s0, s1);
-  return __fadd_rn(s.x, s.y);
-}
-
-// Two adjacent bf16 of shared memory as a pair.
-__device__ __forceinline__ float2 ld2b(const __nv_bfloat16* p) {
-  const uint32_t x = *reinterpret_cast<const uint32_t*>(p);
-  return make_float2(bf16lo(x), bf16hi(x));
-}
-
-// Store a [kL6b][kK6b] bf16 tile to rows t0 .. t0 + n - 1 of a [B][T][HK]
-// tensor at column h * 64 (16-byte pieces).
-__device__ __forceinline__ void wkv6_store_tile(const __nv_bfloat16 (*tile)[kK6b], __nv_bfloat16* dst, int b, int T,
-                                                int HK, int h, int t0, int n, int tid) {
-  for (int g = tid; g < kL6b * 8; g += kT6b) {
-    const int row = g / 8, piece = g % 8;
-    if (row < n) {
-      const uint4 val = reinterpret_cast<const uint4*>(&tile[row][0])[piece];
-      *reinterpret_cast<uint4*>(dst + ((int64_t)b * T + t0 + row) * HK + (int64_t)h * kK6b + piece * 8) = val;
-    }
-  }
-}
-
-__global__ void __launch_bounds__(kT6b, 2) wkv6_bwd_pass1_kernel(
-    const __grid_constant__ CUtensorMap tr, const __grid_constant__ CUtensorMap tk,
-    const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tw,
-    const __grid_constant__ CUtensorMap tdo, int T, int H, const float* __restrict__ u,
-    const float* __restrict__ init_state, const int32_t* __restrict__ state_map, int n_state,
-    const float* __restrict__ g_final, __nv_bfloat16* __restrict__ gr, float* __restrict__ xws,
-    float* __restrict__ cvws, float* __restrict__ p0, unsigned* err) {
-  extern __shared__ __align__(128) unsigned char wkv6_bwd1_dsmem[];
-  Wkv6Bwd1Smem& sm = *reinterpret_cast<Wkv6Bwd1Smem*>(wkv6_bwd1_dsmem);
-  const int tid = threadIdx.x, q = tid & 3, i0 = 2 * (tid >> 2);  // rows i0, i0 + 1
-  const int bh = (int)blockIdx.x, b = bh / H, h = bh % H;
-  const int HK = H * kK6b;
-  const int nchunk = (T + kL6b - 1) / kL6b;
-  constexpr uint32_t kStageBytes = kIn6b * kL6b * kK6b * sizeof(__nv_bfloat16);
-  const CUtensorMap* maps[kIn6b] = {&tr, &tk, &tv, &tw, &tdo};
-  auto issue = [&](int ch) {
-    const int s = ch & 1;
-    mbar_arrive_expect_tx(&sm.full[s], kStageBytes);
-    for (int m = 0; m < kIn6b; ++m) tma_load_3d(&sm.in[s][m][0][0], maps[m], &sm.full[s], h * kK6b, ch * kL6b, b);
-  };
   if (tid == 0) {
-    mbar_init(&sm.full[0], 1);
-    mbar_init(&sm.full[1], 1);
+    tma_prefetch_desc(&tr);
+    tma_prefetch_desc(&tk);
+    tma_prefetch_desc(&tv);
+    tma_prefetch_desc(&tw);
+    tma_prefetch_desc(&tdo);
+    mbar_init(&sm.in_bar, 1);
+    mbar_init(&sm.mma_bar, 1);
     mbar_init_fence();
-    if (nchunk > 0)
-      for (int m = 0; m < kIn6b; ++m) tma_prefetch_desc(maps[m]);
-    for (int ch = 0; ch < 2 && ch < nchunk; ++ch) issue(ch);
+    mbar_arrive_expect_tx(&sm.in_bar, 5 * kTile);
+    tma_load_3d(sm.r, &tr, &sm.in_bar, h * kK6, t0, b);
+    tma_load_3d(sm.k, &tk, &sm.in_bar, h * kK6, t0, b);
+    tma_load_3d(sm.w, &tw, &sm.in_bar, h * kK6, t0, b);
+    tma_load_3d(sm.v, &tv, &sm.in_bar, h * kK6, t0, b);
+    tma_load_3d(sm.dout, &tdo, &sm.in_bar, h * kK6, t0, b);
   }
-  // S_{-1}: init_state[state_map[b]] (or the n_state rule), else zero
-  float2 S0[8], S1[8];
+  if (warp == 0) tmem_alloc(&sm.tmem_base, kTmemCols);
+  if (tid < kK6) sm.u[tid] = u[h * kK6 + tid];
+
+  // S_in and G_out of the chunk: hi/lo bf16 operand tiles, and the row sums
+  // of G_out o S_in (this thread's 8 columns of rows r0, r1)
+  {
+    const float* S = ck_s + ((int64_t)bh * nch + c) * kK6 * kK6;
+    const float* G = ck_g + ((int64_t)bh * nch + (nch - 1 - c)) * kK6 * kK6;
+    float p0 = 0.f, p1 = 0.f;
 #pragma unroll
-  for (int m = 0; m < 8; ++m) S0[m] = S1[m] = make_float2(0.f, 0.f);
-  if (init_state) {
-    const int sidx = state_map ? state_map[b] : (n_state == 1 ? 0 : b);
-    if (sidx < 0 || sidx >= n_state) {
-      if (tid == 0) record_error(err, WKV_DEVERR_BAD_STATE);
-    } else {
-      const float* base = init_state + (((int64_t)sidx * H + h) * kK6b + i0) * kK6b + 16 * q;
-      ld16(base, S0);
-      ld16(base + kK6b, S1);
+    for (int q = 0; q < 4; ++q) {
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int i = hh ? r1 : r0;
+        const int jv = cq + 8 * q;
+        const float2 s2 = *reinterpret_cast<const float2*>(S + i * kK6 + jv);
+        const float2 g2 = *reinterpret_cast<const float2*>(G + i * kK6 + jv);
+        uint32_t sh, sl, gh, gl;
+        sh = pack_bf16x2(s2.x, s2.y);
+        sl = pack_bf16x2(s2.x - bf16lo(sh), s2.y - bf16hi(sh));
+        gh = pack_bf16x2(g2.x, g2.y);
+        gl = pack_bf16x2(g2.x - bf16lo(gh), g2.y - bf16hi(gh));
+        *reinterpret_cast<uint32_t*>(sm.sg + 0 * kTile + bo(i, jv)) = sh;
+        *reinterpret_cast<uint32_t*>(sm.sg + 1 * kTile + bo(i, jv)) = sl;
+        *reinterpret_cast<uint32_t*>(sm.sg + 2 * kTile + bo(i, jv)) = gh;
+        *reinterpret_cast<uint32_t*>(sm.sg + 3 * kTile + bo(i, jv)) = gl;
+        const float d = fmaf(g2.x, s2.x, g2.y * s2.y);
+        if (hh) p1 += d; else p0 += d;
+      }
+    }
+    // the 4 lanes of a row hold its 8-column groups: sum them in a fixed order
+    p0 += __shfl_xor_sync(0xffffffffu, p0, 1);
+    p0 += __shfl_xor_sync(0xffffffffu, p0, 2);
+    p1 += __shfl_xor_sync(0xffffffffu, p1, 1);
+    p1 += __shfl_xor_sync(0xffffffffu, p1, 2);
+    if ((lane & 3) == 0) {
+      sm.cpart[ch][r0] = p0;
+      sm.cpart[ch][r1] = p1;
     }
   }
-  const float2 uu = make_float2(u[h * kK6b + i0], u[h * kK6b + i0 + 1]);
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tm = sm.tmem_base;
+  const uint32_t tl = tm + ((uint32_t)(32 * sp) << 16);  // this warp's TMEM lanes
+
+  bool ok = mbar_wait_bounded(&sm.in_bar, 0, err);
+  bool mma_pending = false;  // an MMA commit not yet waited for (thread 0's view)
+  uint32_t mma_phase = 0;
+  auto wait_mma = [&]() {
+    ok = mbar_wait_bounded(&sm.mma_bar, mma_phase, err) && ok;
+    mma_phase ^= 1u;
+    if (tid == 0) mma_pending = false;
+    tc_fence_after_sync();
+  };
+
+  // ---- prep: decay products, R^ and K~ (transposed, fp32), E_{t-1} ----
+  // warp g takes tokens 8g .. 8g + 7, lane the channels 2 lane, 2 lane + 1
+  const int i0 = 2 * lane;
+  float w0[8], w1[8];
+  float Em1[8][2];  // E_{t-1} of this warp's tokens, kept until the table can be written
+  bool deep = false;
+  if (ok) {
+    float p0 = 1.f, p1 = 1.f;
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      const int j = 8 * warp + jj;
+      const uint32_t x = *reinterpret_cast<const uint32_t*>(sm.w + bo(j, i0));
+      w0[jj] = j < valid ? bf16lo(x) : 1.f;
+      w1[jj] = j < valid ? bf16hi(x) : 1.f;
+      p0 *= w0[jj];
+      p1 *= w1[jj];
+    }
+    *reinterpret_cast<float2*>(&sm.wprod[warp][i0]) = make_float2(p0, p1);
+  }
+  if (__syncthreads_or(!ok)) goto finish;
+  {
+    float pre0 = 1.f, pre1 = 1.f, tot0 = 1.f, tot1 = 1.f;
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      const float2 q = *reinterpret_cast<const float2*>(&sm.wprod[g][i0]);
+      if (g < warp) {
+        pre0 *= q.x;
+        pre1 *= q.y;
+      }
+      tot0 *= q.x;
+      tot1 *= q.y;
+    }
+    deep = __syncthreads_or(!(tot0 >= kMinDecay && tot1 >= kMinDecay));
+    if (warp == 0) *reinterpret_cast<float2*>(&sm.tot[i0]) = make_float2(tot0, tot1);
+    float e0 = pre0, e1 = pre1;
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj) {
+      const int j = 8 * warp + jj;
+      const uint32_t rx = *reinterpret_cast<const uint32_t*>(sm.r + bo(j, i0));
+      const uint32_t kx = *reinterpret_cast<const uint32_t*>(sm.k + bo(j, i0));
+      Em1[jj][0] = e0;
+      Em1[jj][1] = e1;
+      tf(sm.kr + 2 * kTile, i0, j) = bf16lo(rx) * e0;  // R^^T [i][j]
+      tf(sm.kr + 2 * kTile, i0 + 1, j) = bf16hi(rx) * e1;
+      e0 *= w0[jj];
+      e1 *= w1[jj];
+      if (!deep) {
+        tf(sm.kr, i0, j) = bf16lo(kx) * rcp(e0);  // K~^T [i][s]
+        tf(sm.kr, i0 + 1, j) = bf16hi(kx) * rcp(e1);
+      }
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+
+  // ---- first MMAs: dA = dO V^T; dR^ = dO S_in^T; dK^ = V G_out^T ----
+  if (tid == 0) {
+    constexpr uint32_t idb = umma_idesc_bf16(64, 64, 0, 0);  // both operands K-major
+    const uint64_t ddo = umma_desc_sw128(smem_u32(sm.dout), 16, 1024);
+    const uint64_t dv = umma_desc_sw128(smem_u32(sm.v), 16, 1024);
+    const uint64_t dsh = umma_desc_sw128(smem_u32(sm.sg + 0 * kTile), 16, 1024);
+    const uint64_t dsl = umma_desc_sw128(smem_u32(sm.sg + 1 * kTile), 16, 1024);
+    const uint64_t dgh = umma_desc_sw128(smem_u32(sm.sg + 2 * kTile), 16, 1024);
+    const uint64_t dgl = umma_desc_sw128(smem_u32(sm.sg + 3 * kTile), 16, 1024);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) umma_bf16(tm + kColDA, ddo + 2 * kk, dv + 2 * kk, idb, kk > 0);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) umma_bf16(tm + kColDR, ddo + 2 * kk, dsh + 2 * kk, idb, kk > 0);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) umma_bf16(tm + kColDR, ddo + 2 * kk, dsl + 2 * kk, idb, true);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) umma_bf16(tm + kColDKh, dv + 2 * kk, dgh + 2 * kk, idb, kk > 0);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) umma_bf16(tm + kColDKh, dv + 2 * kk, dgl + 2 * kk, idb, true);
+    umma_commit(&sm.mma_bar);
+    mma_pending = true;
+  }
+  wait_mma();
+  if (__syncthreads_or(!ok)) goto finish;
+
+  // ---- dA_s (fp32, [j][s] and [s][j]) and the diagonal; E_{t-1} table ----
+  {
+    float a[16];
+    tmem_ld16x256b_x4(tl + kColDA + 32 * ch, a);
+    tmem_wait_ld();
+    uint8_t* A1 = sm.sg;              // [j][s]
+    uint8_t* A2 = sm.sg + 2 * kTile;  // [s][j]
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int j = hh ? r1 : r0;
+          const int s = cq + 8 * q + e;
+          const float x = a[4 * q + 2 * hh + e];
+          const float m = s < j ? x : 0.f;
+          tf(A1, j, s) = m;
+          tf(A2, s, j) = m;
+          if (s == j) sm.dd[j] = x;
+        }
+    // E_{t-1}: a plain [t][64] fp32 table over the (consumed) v and dout tiles
+    float* Et = reinterpret_cast<float*>(sm.v);
+#pragma unroll
+    for (int jj = 0; jj < 8; ++jj)
+      *reinterpret_cast<float2*>(&Et[(8 * warp + jj) * kK6 + i0]) = make_float2(Em1[jj][0], Em1[jj][1]);
+  }
+  fence_proxy_async_smem();
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+
+  // ---- second MMAs (tf32): dR^ += dA_s K~; dK~ = dA_s^T R^ ----
+  if (!deep) {
+    if (tid == 0) {
+      constexpr uint32_t idt = umma_idesc_tf32(64, 64, 0, 0);
+      const uint64_t d1 = umma_desc_sw128(smem_u32(sm.sg), 16, 1024);
+      const uint64_t d2 = umma_desc_sw128(smem_u32(sm.sg + 2 * kTile), 16, 1024);
+      const uint64_t dkt = umma_desc_sw128(smem_u32(sm.kr), 16, 1024);
+      const uint64_t drt = umma_desc_sw128(smem_u32(sm.kr + 2 * kTile), 16, 1024);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t o = ((kk >> 2) * kTile + (kk & 3) * 32) / 16;
+        umma_tf32(tm + kColDR, d1 + o, dkt + o, idt, true);
+      }
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t o = ((kk >> 2) * kTile + (kk & 3) * 32) / 16;
+        umma_tf32(tm + kColDKt, d2 + o, drt + o, idt, kk > 0);
+      }
+      umma_commit(&sm.mma_bar);
+      mma_pending = true;
+    }
+    wait_mma();
+    if (__syncthreads_or(!ok)) goto finish;
+  }
+
+  // ---- epilogue: gr, gk and the decay-gradient tables ----
+  {
+    float dR[16], dKh[16], dKt[16];
+    tmem_ld16x256b_x4(tl + kColDR + 32 * ch, dR);
+    tmem_ld16x256b_x4(tl + kColDKh + 32 * ch, dKh);
+    if (!deep) tmem_ld16x256b_x4(tl + kColDKt + 32 * ch, dKt);
+    tmem_wait_ld();
+    const float* Et = reinterpret_cast<const float*>(sm.v);
+    // deep chunk: the intra-chunk sums of dA_s with k (for gr) and r (for gk)
+    // and E_{L-1} / E_t as running products of w on the CUDA cores
+    float gri[16], gki[16], qv[16];
+    if (deep) {
+      const uint8_t* A1 = sm.sg;
+#pragma unroll
+      for (int x = 0; x < 16; ++x) {
+        const int q = x >> 2, hh = (x >> 1) & 1, e = x & 1;
+        const int t = hh ? r1 : r0;
+        const int i = cq + 8 * q + e;
+        float acc = 0.f, rho = 1.f;  // rho = prod_{tau = s+1}^{t-1} w_tau
+        for (int s = t - 1; s >= 0; --s) {
+          acc = fmaf(tfc(A1, t, s) * rho, tb(sm.k, s, i), acc);
+          rho *= (s < valid ? tb(sm.w, s, i) : 1.f);
+        }
+        gri[x] = acc;
+        float acc2 = 0.f;
+        rho = 1.f;  // prod_{tau = t+1}^{j-1} w_tau
+        for (int j = t + 1; j < kL6; ++j) {
+          acc2 = fmaf(tfc(A1, j, t) * rho, tb(sm.r, j, i), acc2);
+          rho *= (j < valid ? tb(sm.w, j, i) : 1.f);
+        }
+        gki[x] = acc2;
+        float qq = 1.f;  // prod_{tau > t} w_tau
+        for (int j = t + 1; j < valid; ++j) qq *= tb(sm.w, j, i);
+        qv[x] = qq;
+      }
+    }
+    __syncthreads();  // the deep sums above read dA_s, which the tables below overwrite
+    float* xt = reinterpret_cast<float*>(sm.sg);              // x_t           [t][64]
+    float* gt = reinterpret_cast<float*>(sm.sg + 2 * kTile);  // z_t - x_t + y_t
+    float* zt = reinterpret_cast<float*>(sm.v);               // z_t (over E_{t-1}, in place)
+    uint8_t* gro = sm.kr;                                     // bf16 [t][64] plain rows
+    uint8_t* gko = sm.kr + kTile;
+#pragma unroll
+    for (int x = 0; x < 16; ++x) {
+      const int q = x >> 2, hh = (x >> 1) & 1, e = x & 1;
+      const int t = hh ? r1 : r0;
+      const int i = cq + 8 * q + e;
+      const float em1 = Et[t * kK6 + i];
+      const float wt = t < valid ? tb(sm.w, t, i) : 1.f;
+      const float rt = tb(sm.r, t, i), kt = tb(sm.k, t, i);
+      const float ui = sm.u[i], dt = sm.dd[t];
+      float grv, gkin, Q;
+      if (deep) {
+        grv = fmaf(em1, dR[x], gri[x]);
+        gkin = gki[x];
+        Q = qv[x];
+      } else {
+        grv = em1 * dR[x];
+        const float inv_et = rcp(em1 * wt);
+        gkin = dKt[x] * inv_et;
+        Q = sm.tot[i] * inv_et;
+      }
+      const float zv = dKh[x] * Q * kt;
+      const float xv = grv * rt;
+      const float yv = gkin * kt;
+      xt[t * kK6 + i] = xv;
+      gt[t * kK6 + i] = zv - xv + yv;
+      zt[t * kK6 + i] = zv;
+      reinterpret_cast<__nv_bfloat16*>(gro)[t * kK6 + i] = __float2bfloat16_rn(fmaf(dt * ui, kt, grv));
+      reinterpret_cast<__nv_bfloat16*>(gko)[t * kK6 + i] =
+          __float2bfloat16_rn(fmaf(dt * ui, rt, fmaf(dKh[x], Q, gkin)));
+    }
+  }
   __syncthreads();
 
-  bool ok = true;
-  int ch = 0;
-  for (; ch < nchunk; ++ch) {
-    const int s = ch & 1;
-    const int t0 = ch * kL6b, n = min(kL6b, T - t0);
-    const bool got = mbar_wait_bounded(&sm.full[s], (ch >> 1) & 1, err);
-    if (!__syncthreads_and(got)) {
-      ok = false;
-      break;
+  // ---- decay gradient: glogw_t = c + D - Gsum + sum_{s < t} g_s - x_t per
+  // channel (D, Gsum the chunk's sums of z and g); 4 threads per channel,
+  // each a quarter of the tokens ----
+  {
+    const float* xt = reinterpret_cast<const float*>(sm.sg);
+    const float* gt = reinterpret_cast<const float*>(sm.sg + 2 * kTile);
+    const float* zt = reinterpret_cast<const float*>(sm.v);
+    const int i = tid & 63, qq = tid >> 6;
+    float zs = 0.f, gs = 0.f;
+    for (int t = 16 * qq; t < 16 * qq + 16; ++t) {
+      zs += zt[t * kK6 + i];
+      gs += gt[t * kK6 + i];
     }
-    const __nv_bfloat16(*in)[kL6b][kK6b] = sm.in[s];
-    {
-      // per token: c_t = r . (u o k) and v . do, 4 threads per token
-      const int jt = tid >> 2, part = tid & 3;
-      float c = 0.f, vd = 0.f;
-#pragma unroll
-      for (int m = 0; m < 16; ++m) {
-        const int e = part * 16 + m;
-        c = __fmaf_rn(bf(in[kR][jt][e]) * u[h * kK6b + e], bf(in[kKk][jt][e]), c);
-        vd = __fmaf_rn(bf(in[kV][jt][e]), bf(in[kDo][jt][e]), vd);
-      }
-      c = row_sum4(c);
-      vd = row_sum4(vd);
-      if (part == 0) reinterpret_cast<float4*>(&sm.cv[s][jt][0])[0] = make_float4(c, vd, 0.f, 0.f);
-    }
+    sm.scan[0][qq][i] = zs;
+    sm.scan[1][qq][i] = gs;
     __syncthreads();
-    // the step's vectors are fetched one step ahead
-    Bf16x16 vn = ld16b(&in[kV][0][16 * q]), dn = ld16b(&in[kDo][0][16 * q]);
-    float2 wn = ld2b(&in[kW][0][i0]), kn = ld2b(&in[kKk][0][i0]), rn = ld2b(&in[kR][0][i0]);
-    float vdn = sm.cv[s][0][1];
-    for (int jt = 0; jt < n; ++jt) {
-      const Bf16x16 vc = vn, dc = dn;
-      const float2 w2 = wn, k2 = kn, r2 = rn;
-      const float vdo = vdn;
-      if (jt + 1 < n) {
-        vn = ld16b(&in[kV][jt + 1][16 * q]);
-        dn = ld16b(&in[kDo][jt + 1][16 * q]);
-        wn = ld2b(&in[kW][jt + 1][i0]);
-        kn = ld2b(&in[kKk][jt + 1][i0]);
-        rn = ld2b(&in[kR][jt + 1][i0]);
-        vdn = sm.cv[s][jt + 1][1];
-      }
-      float2 vv[8], dd[8];
-      widen16(vc, vv);
-      widen16(dc, dd);
-      // (S_{t-1} do_t) for both rows
-      const float a0 = row_sum4(dot16(S0, dd)), a1 = row_sum4(dot16(S1, dd));
-      if (q == 0) {
-        *reinterpret_cast<__nv_bfloat162*>(&sm.gro[jt][i0]) =
-            __floats2bfloat162_rn(__fmaf_rn(uu.x * k2.x, vdo, a0), __fmaf_rn(uu.y * k2.y, vdo, a1));
-        *reinterpret_cast<float2*>(&sm.xo[jt][i0]) = make_float2(__fmul_rn(r2.x, a0), __fmul_rn(r2.y, a1));
-      }
-      const float2 wa = make_float2(w2.x, w2.x), ka = make_float2(k2.x, k2.x);
-      const float2 wb = make_float2(w2.y, w2.y), kb = make_float2(k2.y, k2.y);
-#pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        S0[m] = fma2(S0[m], wa, mul2(ka, vv[m]));
-        S1[m] = fma2(S1[m], wb, mul2(kb, vv[m]));
-      }
-    }
-    __syncthreads();
-    if (tid == 0 && ch + 2 < nchunk) issue(ch + 2);  // every read of stage s is done
-    wkv6_store_tile(sm.gro, gr, b, T, HK, h, t0, n, tid);
-    float* xrow = xws + ((int64_t)bh * T + t0) * kK6b;
-    for (int g = tid; g < kL6b * kK6b / 4; g += kT6b) {
-      const int row = g / (kK6b / 4);
-      if (row < n) reinterpret_cast<float4*>(xrow)[g] = reinterpret_cast<const float4*>(&sm.xo[0][0])[g];
-    }
-    if (tid < n) reinterpret_cast<float4*>(cvws + ((int64_t)bh * T + t0) * 4)[tid] =
-        reinterpret_cast<const float4*>(&sm.cv[s][0][0])[tid];
-  }
-  if (!ok) {
-    // a wait gave up: let the copies in flight land before the CTA exits
-    if (tid == 0)
-      for (int x = ch; x < nchunk && x < ch + 2; ++x) mbar_wait_bounded(&sm.full[x & 1], (x >> 1) & 1, err);
-    return;
-  }
-  // P_{T-1}[i] = sum_j g_final[i][j] S_{T-1}[i][j]
-  float p0a = 0.f, p0b = 0.f;
-  if (g_final) {
-    float2 gf[8];
-    const float* base = g_final + ((int64_t)bh * kK6b + i0) * kK6b + 16 * q;
-    ld16(base, gf);
-    p0a = dot16(gf, S0);
-    ld16(base + kK6b, gf);
-    p0b = dot16(gf, S1);
-  }
-  p0a = row_sum4(p0a);
-  p0b = row_sum4(p0b);
-  if (q == 0) *reinterpret_cast<float2*>(&p0[(int64_t)bh * kK6b + i0]) = make_float2(p0a, p0b);
-}
-
-__global__ void __launch_bounds__(kT6b, 2) wkv6_bwd_pass2_kernel(
-    const __grid_constant__ CUtensorMap tr, const __grid_constant__ CUtensorMap tk,
-    const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tw,
-    const __grid_constant__ CUtensorMap tdo, const __grid_constant__ CUtensorMap tx,
-    const __grid_constant__ CUtensorMap tcv, int T, int H, const float* __restrict__ u,
-    const float* __restrict__ g_final, const float* __restrict__ p0, __nv_bfloat16* __restrict__ gk,
-    __nv_bfloat16* __restrict__ gv, __nv_bfloat16* __restrict__ glogw, float* __restrict__ g_init,
-    float* __restrict__ gu_part, unsigned* err) {
-  extern __shared__ __align__(128) unsigned char wkv6_bwd2_dsmem[];
-  Wkv6Bwd2Smem& sm = *reinterpret_cast<Wkv6Bwd2Smem*>(wkv6_bwd2_dsmem);
-  // rows i0, i0 + 1 of G and columns i0, i0 + 1 of G (rows 16q .. 16q + 15)
-  const int tid = threadIdx.x, q = tid & 3, i0 = 2 * (tid >> 2);
-  const int bh = (int)blockIdx.x, b = bh / H, h = bh % H;
-  const int HK = H * kK6b;
-  const int nchunk = (T + kL6b - 1) / kL6b;
-  constexpr uint32_t kStageBytes =
-      kIn6b * kL6b * kK6b * sizeof(__nv_bfloat16) + kL6b * kK6b * sizeof(float) + kL6b * 4 * sizeof(float);
-  const CUtensorMap* maps[kIn6b] = {&tr, &tk, &tv, &tw, &tdo};
-  auto issue = [&](int ch) {  // ch counts chunks from the end
-    const int s = ch & 1;
-    const int t0 = (nchunk - 1 - ch) * kL6b;
-    mbar_arrive_expect_tx(&sm.full[s], kStageBytes);
-    for (int m = 0; m < kIn6b; ++m) tma_load_3d(&sm.st[s].in[m][0][0], maps[m], &sm.full[s], h * kK6b, t0, b);
-    tma_load_3d(&sm.st[s].x[0][0], &tx, &sm.full[s], 0, t0, bh);
-    tma_load_3d(&sm.st[s].cv[0][0], &tcv, &sm.full[s], 0, t0, bh);
-  };
-  if (tid == 0) {
-    mbar_init(&sm.full[0], 1);
-    mbar_init(&sm.full[1], 1);
-    mbar_init_fence();
-    if (nchunk > 0) {
-      for (int m = 0; m < kIn6b; ++m) tma_prefetch_desc(maps[m]);
-      tma_prefetch_desc(&tx);
-      tma_prefetch_desc(&tcv);
-    }
-    for (int ch = 0; ch < 2 && ch < nchunk; ++ch) issue(ch);
-  }
-  // G_{T-1} = g_final, by rows (G[i][16q ..]) and by columns (G[16q ..][i])
-  float2 G0[8], G1[8], C0[8], C1[8];
-#pragma unroll
-  for (int m = 0; m < 8; ++m) G0[m] = G1[m] = C0[m] = C1[m] = make_float2(0.f, 0.f);
-  if (g_final) {
-    const float* gf = g_final + (int64_t)bh * kK6b * kK6b;
-    ld16(gf + i0 * kK6b + 16 * q, G0);
-    ld16(gf + (i0 + 1) * kK6b + 16 * q, G1);
-#pragma unroll
-    for (int m = 0; m < 8; ++m) {
-      const float2 top = *reinterpret_cast<const float2*>(gf + (16 * q + 2 * m) * kK6b + i0);
-      const float2 bot = *reinterpret_cast<const float2*>(gf + (16 * q + 2 * m + 1) * kK6b + i0);
-      C0[m] = make_float2(top.x, bot.x);
-      C1[m] = make_float2(top.y, bot.y);
-    }
-  }
-  float2 P = *reinterpret_cast<const float2*>(&p0[(int64_t)bh * kK6b + i0]);
-  const float2 uu = make_float2(u[h * kK6b + i0], u[h * kK6b + i0 + 1]);
-  float2 gu2 = make_float2(0.f, 0.f);
-  __syncthreads();
-
-  bool ok = true;
-  int ch = 0;
-  for (; ch < nchunk; ++ch) {
-    const int s = ch & 1;
-    const int t0 = (nchunk - 1 - ch) * kL6b, n = min(kL6b, T - t0);
-    const bool got = mbar_wait_bounded(&sm.full[s], (ch >> 1) & 1, err);
-    if (!__syncthreads_and(got)) {
-      ok = false;
-      break;
-    }
-    const Wkv6Bwd2Stage& st = sm.st[s];
-    struct Tok {
-      Bf16x16 v, d, r, k, w;
-      float2 w2, r2, k2, d2, cvd, x2;
-    };
-    auto fetch = [&](int jt) {
-      Tok x;
-      x.v = ld16b(&st.in[kV][jt][16 * q]);
-      x.d = ld16b(&st.in[kDo][jt][16 * q]);
-      x.r = ld16b(&st.in[kR][jt][16 * q]);
-      x.k = ld16b(&st.in[kKk][jt][16 * q]);
-      x.w = ld16b(&st.in[kW][jt][16 * q]);
-      x.w2 = ld2b(&st.in[kW][jt][i0]);
-      x.r2 = ld2b(&st.in[kR][jt][i0]);
-      x.k2 = ld2b(&st.in[kKk][jt][i0]);
-      x.d2 = ld2b(&st.in[kDo][jt][i0]);
-      x.cvd = *reinterpret_cast<const float2*>(&st.cv[jt][0]);  // (c_t, v_t . do_t)
-      x.x2 = *reinterpret_cast<const float2*>(&st.x[jt][i0]);
-      return x;
-    };
-    Tok nx = fetch(n - 1);
-    for (int jt = n - 1; jt >= 0; --jt) {
-      const Tok cu = nx;
-      if (jt > 0) nx = fetch(jt - 1);
-      float2 vv[8], dd[8], rr[8], kk[8], ww[8];
-      widen16(cu.v, vv);
-      widen16(cu.d, dd);
-      widen16(cu.r, rr);
-      widen16(cu.k, kk);
-      widen16(cu.w, ww);
-      // (G_t v_t) for rows i0, i0 + 1 and (k_t G_t) for columns i0, i0 + 1
-      const float g0 = row_sum4(dot16(G0, vv)), g1 = row_sum4(dot16(G1, vv));
-      const float h0 = row_sum4(dot16(kk, C0)), h1 = row_sum4(dot16(kk, C1));
-      const float c = cu.cvd.x, vdo = cu.cvd.y;
-      const float2 gl = make_float2(__fsub_rn(P.x, __fmul_rn(cu.k2.x, g0)), __fsub_rn(P.y, __fmul_rn(cu.k2.y, g1)));
-      P = add2(gl, cu.x2);  // P_{t-1}
-      if (q == 0) {
-        *reinterpret_cast<__nv_bfloat162*>(&sm.out[0][jt][i0]) =
-            __floats2bfloat162_rn(__fmaf_rn(uu.x * cu.r2.x, vdo, g0), __fmaf_rn(uu.y * cu.r2.y, vdo, g1));
-        *reinterpret_cast<__nv_bfloat162*>(&sm.out[1][jt][i0]) =
-            __floats2bfloat162_rn(__fmaf_rn(c, cu.d2.x, h0), __fmaf_rn(c, cu.d2.y, h1));
-        *reinterpret_cast<__nv_bfloat162*>(&sm.out[2][jt][i0]) = __floats2bfloat162_rn(gl.x, gl.y);
-      }
-      gu2 = fma2(mul2(cu.r2, cu.k2), make_float2(vdo, vdo), gu2);
-      const float2 wa = make_float2(cu.w2.x, cu.w2.x), ra = make_float2(cu.r2.x, cu.r2.x);
-      const float2 wb = make_float2(cu.w2.y, cu.w2.y), rb = make_float2(cu.r2.y, cu.r2.y);
-      const float2 da = make_float2(cu.d2.x, cu.d2.x), db = make_float2(cu.d2.y, cu.d2.y);
-#pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        G0[m] = fma2(G0[m], wa, mul2(ra, dd[m]));
-        G1[m] = fma2(G1[m], wb, mul2(rb, dd[m]));
-        C0[m] = fma2(C0[m], ww[m], mul2(rr[m], da));
-        C1[m] = fma2(C1[m], ww[m], mul2(rr[m], db));
-      }
-    }
-    __syncthreads();
-    if (tid == 0 && ch + 2 < nchunk) issue(ch + 2);  // every read of stage s is done
-    wkv6_store_tile(sm.out[0], gk, b, T, HK, h, t0, n, tid);
-    wkv6_store_tile(sm.out[1], gv, b, T, HK, h, t0, n, tid);
-    wkv6_store_tile(sm.out[2], glogw, b, T, HK, h, t0, n, tid);
-  }
-  if (!ok) {
-    if (tid == 0)
-      for (int x = ch; x < nchunk && x < ch + 2; ++x) mbar_wait_bounded(&sm.full[x & 1], (x >> 1) & 1, err);
-    return;
-  }
-  if (g_init) {
-    float* base = g_init + ((int64_t)bh * kK6b + i0) * kK6b + 16 * q;
-    float4* d0 = reinterpret_cast<float4*>(base);
-    float4* d1 = reinterpret_cast<float4*>(base + kK6b);
-#pragma unroll
+    float D = 0.f, Gsum = 0.f, pre = 0.f;
     for (int m = 0; m < 4; ++m) {
-      d0[m] = make_float4(G0[2 * m].x, G0[2 * m].y, G0[2 * m + 1].x, G0[2 * m + 1].y);
-      d1[m] = make_float4(G1[2 * m].x, G1[2 * m].y, G1[2 * m + 1].x, G1[2 * m + 1].y);
+      D += sm.scan[0][m][i];
+      Gsum += sm.scan[1][m][i];
+      if (m < qq) pre += sm.scan[1][m][i];
+    }
+    const float cc = sm.tot[i] * (sm.cpart[0][i] + sm.cpart[1][i]);
+    const float base = cc + D - Gsum;
+    __nv_bfloat16* glo = reinterpret_cast<__nv_bfloat16*>(sm.kr + 2 * kTile);
+    for (int t = 16 * qq; t < 16 * qq + 16; ++t) {
+      glo[t * kK6 + i] = __float2bfloat16_rn(base + pre - xt[t * kK6 + i]);
+      pre += gt[t * kK6 + i];
+    }
+    // gu partial of the chunk: sum_t dA[t][t] r_t o k_t (thread per channel)
+    if (qq == 0) {
+      float acc = 0.f;
+      for (int t = 0; t < valid; ++t) acc = fmaf(sm.dd[t] * tb(sm.r, t, i), tb(sm.k, t, i), acc);
+      gu_part[((int64_t)bh * nch + c) * kK6 + i] = acc;
     }
   }
-  if (q == 0) *reinterpret_cast<float2*>(&gu_part[(int64_t)bh * kK6b + i0]) = gu2;
+  __syncthreads();
+  // ---- gr, gk, glogw tiles to global memory (16-byte pieces, rows < valid) ----
+  for (int g = tid; g < 3 * kL6 * 8; g += kThr6) {
+    const int which = g / (kL6 * 8), row = (g / 8) % kL6, piece = g % 8;
+    if (row < valid) {
+      const uint4 val = reinterpret_cast<const uint4*>(sm.kr + which * kTile + row * 128)[piece];
+      __nv_bfloat16* dst = which == 0 ? gr : (which == 1 ? gk : glogw);
+      *reinterpret_cast<uint4*>(dst + ((int64_t)b * T + t0 + row) * HK + (int64_t)h * kK6 + piece * 8) = val;
+    }
+  }
+
+finish:
+  if (!ok && tid == 0) {
+    // let the copies and MMAs in flight land before the memory is released
+    mbar_wait_bounded(&sm.in_bar, 0, err);
+    if (mma_pending) mbar_wait_bounded(&sm.mma_bar, mma_phase, err);
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after_sync();
+    tmem_dealloc(tm, kTmemCols);
+  }
 }
 
-// gu[c] = sum over samples b (ascending) of gu_part[b][c]: fixed order.
-__global__ void wkv6_gu_reduce_kernel(const float* __restrict__ gu_part, int B, int HK, float* __restrict__ gu) {
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= HK) return;
+// Time reversal of a [B][T][HK] bf16 tensor into [B][Tp][HK] (Tp >= T):
+// row p of the copy is row Tp - 1 - p of the source, rows with no source row
+// (the first Tp - T) hold `pad`. Four tensors in one launch (blockIdx.y).
+struct RevJob {
+  const __nv_bfloat16* src[4];
+  __nv_bfloat16* dst[4];
+  uint32_t pad[4];  // a bf16 value twice (0 or 1.0)
+};
+__global__ void wkv6_reverse_kernel(RevJob job, int B, int T, int Tp, int64_t HK) {
+  const int which = blockIdx.y;
+  const int64_t per_row = HK / 8;  // 16-byte pieces per row
+  const int64_t n = (int64_t)B * Tp * per_row;
+  for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < n; x += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t piece = x % per_row;
+    const int64_t row = x / per_row;
+    const int p = (int)(row % Tp);
+    const int bb = (int)(row / Tp);
+    const int q = Tp - 1 - p;
+    uint4 val;
+    if (q < T) {
+      val = reinterpret_cast<const uint4*>(job.src[which] + ((int64_t)bb * T + q) * HK)[piece];
+    } else {
+      const uint32_t pv = job.pad[which];
+      val = make_uint4(pv, pv, pv, pv);
+    }
+    reinterpret_cast<uint4*>(job.dst[which] + ((int64_t)bb * Tp + p) * HK)[piece] = val;
+  }
+}
+
+// gv row t = row Tp - 1 - t of the reversed pass's output.
+__global__ void wkv6_unreverse_kernel(const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ dst, int B,
+                                      int T, int Tp, int64_t HK) {
+  const int64_t per_row = HK / 8;
+  const int64_t n = (int64_t)B * T * per_row;
+  for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < n; x += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t piece = x % per_row;
+    const int64_t row = x / per_row;
+    const int t = (int)(row % T);
+    const int bb = (int)(row / T);
+    reinterpret_cast<uint4*>(dst + ((int64_t)bb * T + t) * HK)[piece] =
+        reinterpret_cast<const uint4*>(src + ((int64_t)bb * Tp + (Tp - 1 - t)) * HK)[piece];
+  }
+}
+
+// gu[h*64 + i] = sum over samples b and chunks c (in that order) of the
+// chunk partials: fixed order, deterministic.
+__global__ void wkv6_gu_reduce_kernel(const float* __restrict__ part, int B, int H, int nch, float* __restrict__ gu) {
+  const int x = blockIdx.x * blockDim.x + threadIdx.x;  // h * 64 + i
+  if (x >= H * kK6) return;
+  const int h = x / kK6, i = x % kK6;
   float s = 0.f;
-  for (int b = 0; b < B; ++b) s += gu_part[(int64_t)b * HK + c];
-  gu[c] = s;
+  for (int bb = 0; bb < B; ++bb)
+    for (int c = 0; c < nch; ++c) s += part[(((int64_t)bb * H + h) * nch + c) * kK6 + i];
+  gu[x] = s;
 }
 
-size_t wkv6_bwd_workspace_bytes(int64_t B, int64_t T, int64_t H) {
-  const int64_t BH = B * H;
-  return sizeof(float) * (size_t)(BH * T * kK6b + BH * T * 4 + 2 * BH * kK6b);
+// Workspace pieces (each 256-byte aligned).
+struct Bwd6Ws {
+  float *ck_s, *ck_g, *gu_part;
+  __nv_bfloat16 *rev[4], *orev;
+  size_t bytes;
+};
+Bwd6Ws bwd6_ws(void* base, int64_t B, int64_t T, int64_t H) {
+  const int64_t nch = ceil_div(T, kL6), Tp = nch * kL6, BH = B * H, HK = H * kK6;
+  uintptr_t p = reinterpret_cast<uintptr_t>(base);
+  size_t off = 0;
+  auto take = [&](size_t n) {
+    const size_t o = off;
+    off = (off + n + 255) & ~(size_t)255;
+    return reinterpret_cast<void*>(p + o);
+  };
+  Bwd6Ws ws;
+  ws.ck_s = static_cast<float*>(take(sizeof(float) * BH * nch * kK6 * kK6));
+  ws.ck_g = static_cast<float*>(take(sizeof(float) * BH * nch * kK6 * kK6));
+  ws.gu_part = static_cast<float*>(take(sizeof(float) * BH * nch * kK6));
+  for (int m = 0; m < 4; ++m) ws.rev[m] = static_cast<__nv_bfloat16*>(take(2 * B * Tp * HK));
+  ws.orev = static_cast<__nv_bfloat16*>(take(2 * B * Tp * HK));
+  ws.bytes = off;
+  return ws;
 }
+
+}  // namespace
+
+size_t wkv6_bwd_workspace_bytes(int64_t B, int64_t T, int64_t H) { return bwd6_ws(nullptr, B, T, H).bytes; }
 
 wkv_status launch_wkv6_backward(const Wkv6BwdArgs& a, cudaStream_t stream, unsigned* err, const char** why) {
-  const int64_t BH = a.B * a.H, HK = a.H * kK6b;
-  float* xws = static_cast<float*>(a.workspace);
-  float* cvws = xws + BH * a.T * kK6b;
-  float* p0 = cvws + BH * a.T * 4;
-  float* gu_part = p0 + BH * kK6b;
-  CUtensorMap maps[7];
-  memset(maps, 0, sizeof(maps));
+  const int64_t nch = ceil_div(a.T, kL6), Tp = nch * kL6, BH = a.B * a.H, HK = a.H * kK6;
+  const Bwd6Ws ws = bwd6_ws(a.workspace, a.B, a.T, a.H);
+  // 1. forward: the state entering every chunk (no output)
   if (a.T > 0) {
-    const void* src[kIn6b] = {a.r, a.k, a.v, a.w, a.dout};
-    for (int m = 0; m < kIn6b; ++m)
-      if (!encode_tmap_3d(&maps[m], src[m], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)HK, (uint64_t)a.T,
-                          (uint64_t)a.B, kK6b, kL6b, 1, why))
-        return WKV_ERR_INVALID_ARG;
-    if (!encode_tmap_3d(&maps[5], xws, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kK6b, (uint64_t)a.T, (uint64_t)BH, kK6b,
-                        kL6b, 1, why) ||
-        !encode_tmap_3d(&maps[6], cvws, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, 4, (uint64_t)a.T, (uint64_t)BH, 4, kL6b, 1,
-                        why))
-      return WKV_ERR_INVALID_ARG;
+    Wkv6FwdArgs f{a.B, a.T, a.H, a.K, a.r, a.k, a.v, a.w, a.u, a.init_state, a.state_map, a.n_state, nullptr,
+                  nullptr};
+    f.ck_state = ws.ck_s;
+    if (wkv_status s = launch_wkv6_forward(f, stream, err, why)) return s;
+    // 2. the gradient state backwards: the forward on the time-reversed (k, r, do, w)
+    RevJob job;
+    const void* src[4] = {a.k, a.r, a.dout, a.w};
+    for (int m = 0; m < 4; ++m) {
+      job.src[m] = static_cast<const __nv_bfloat16*>(src[m]);
+      job.dst[m] = ws.rev[m];
+      job.pad[m] = m == 3 ? 0x3F803F80u : 0u;  // w = 1.0 in the padding, else 0
+    }
+    const int64_t pieces = a.B * Tp * (HK / 8);
+    const unsigned gx = (unsigned)std::min<int64_t>(ceil_div(pieces, 256), 148 * 16);
+    wkv6_reverse_kernel<<<dim3(gx, 4), 256, 0, stream>>>(job, (int)a.B, (int)a.T, (int)Tp, HK);
+    if (cudaGetLastError() != cudaSuccess) {
+      *why = "wkv6_backward: reversal kernel launch failed";
+      return WKV_ERR_CUDA;
+    }
   }
-  const size_t smem1 = sizeof(Wkv6Bwd1Smem), smem2 = sizeof(Wkv6Bwd2Smem);
-  if (cudaFuncSetAttribute(wkv6_bwd_pass1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1) !=
-          cudaSuccess ||
-      cudaFuncSetAttribute(wkv6_bwd_pass2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2) !=
-          cudaSuccess) {
-    *why = "wkv6_backward: shared memory configuration failed";
+  {
+    Wkv6FwdArgs g{a.B, Tp, a.H, a.K, ws.rev[0], ws.rev[1], ws.rev[2], ws.rev[3], a.u, a.g_final, nullptr,
+                  a.g_final ? a.B : 0, a.g_init, a.T > 0 ? ws.orev : nullptr};
+    g.ck_state = a.T > 0 ? ws.ck_g : nullptr;
+    if (a.T > 0 || a.g_init) {
+      if (wkv_status s = launch_wkv6_forward(g, stream, err, why)) return s;
+    }
+  }
+  if (a.T > 0) {
+    const int64_t pieces = a.B * a.T * (HK / 8);
+    const unsigned gx = (unsigned)std::min<int64_t>(ceil_div(pieces, 256), 148 * 16);
+    wkv6_unreverse_kernel<<<gx, 256, 0, stream>>>(ws.orev, static_cast<__nv_bfloat16*>(a.gv), (int)a.B, (int)a.T,
+                                                  (int)Tp, HK);
+    if (cudaGetLastError() != cudaSuccess) {
+      *why = "wkv6_backward: reversal kernel launch failed";
+      return WKV_ERR_CUDA;
+    }
+    // 3. every chunk independently: gr, gk, glogw and the gu partials
+    CUtensorMap maps[5];
+    memset(maps, 0, sizeof(maps));
+    const void* src[5] = {a.r, a.k, a.v, a.w, a.dout};
+    for (int m = 0; m < 5; ++m)
+      if (!encode_tmap_3d(&maps[m], src[m], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)HK, (uint64_t)a.T,
+                          (uint64_t)a.B, kK6, kL6, 1, why, /*swizzle128=*/true))
+        return WKV_ERR_INVALID_ARG;
+    const size_t smem = sizeof(Bwd6Smem) + 1024;
+    if (cudaFuncSetAttribute(wkv6_bwd_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess) {
+      *why = "wkv6_backward: shared memory configuration failed";
+      return WKV_ERR_CUDA;
+    }
+    wkv6_bwd_chunk_kernel<<<(unsigned)(BH * nch), kThr6, smem, stream>>>(
+        maps[0], maps[1], maps[2], maps[3], maps[4], (int)a.T, (int)a.H, (int)nch, a.u, ws.ck_s, ws.ck_g,
+        static_cast<__nv_bfloat16*>(a.gr), static_cast<__nv_bfloat16*>(a.gk), static_cast<__nv_bfloat16*>(a.glogw),
+        ws.gu_part, err);
+    if (cudaGetLastError() != cudaSuccess) {
+      *why = "wkv6_backward chunk kernel launch failed";
+      return WKV_ERR_CUDA;
+    }
+  }
+  if (a.T > 0) {
+    wkv6_gu_reduce_kernel<<<(unsigned)ceil_div(HK, 256), 256, 0, stream>>>(ws.gu_part, (int)a.B, (int)a.H, (int)nch,
+                                                                          a.gu);
+  } else if (cudaMemsetAsync(a.gu, 0, sizeof(float) * HK, stream) != cudaSuccess) {
+    *why = "cudaMemsetAsync failed";
     return WKV_ERR_CUDA;
   }
-  wkv6_bwd_pass1_kernel<<<(unsigned)BH, kT6b, smem1, stream>>>(
-      maps[0], maps[1], maps[2], maps[3], maps[4], (int)a.T, (int)a.H, a.u, a.init_state, a.state_map,
-      (int)a.n_state, a.g_final, static_cast<__nv_bfloat16*>(a.gr), xws, cvws, p0, err);
-  cudaError_t e = cudaGetLastError();
-  if (e == cudaSuccess) {
-    wkv6_bwd_pass2_kernel<<<(unsigned)BH, kT6b, smem2, stream>>>(
-        maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], (int)a.T, (int)a.H, a.u, a.g_final, p0,
-        static_cast<__nv_bfloat16*>(a.gk), static_cast<__nv_bfloat16*>(a.gv), static_cast<__nv_bfloat16*>(a.glogw),
-        a.g_init, gu_part, err);
-    e = cudaGetLastError();
-  }
-  if (e == cudaSuccess) {
-    wkv6_gu_reduce_kernel<<<(unsigned)ceil_div(HK, 256), 256, 0, stream>>>(gu_part, (int)a.B, (int)HK, a.gu);
-    e = cudaGetLastError();
-  }
-  if (e != cudaSuccess) {
+  if (cudaGetLastError() != cudaSuccess) {
     *why = "wkv6_backward kernel launch failed";
     return WKV_ERR_CUDA;
   }

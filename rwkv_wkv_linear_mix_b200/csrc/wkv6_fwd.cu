@@ -29,6 +29,9 @@
 // outside the sub-chunk masked: r = k = 0, w = 1). A single token needs no
 // K~, so every w in (0, 1] is handled.
 //
+// For the backward the kernel can also write the state entering every
+// 64-token chunk (ck_state, [B*H][chunks][64][64] fp32, [i][jv]) and skip o.
+//
 // Kernel shape: one CTA of 256 threads per (b, h), walking its chunks (and
 // sub-chunks: "units") in order; two CTAs share an SM. Per unit n:
 //   B. pass 1: product of w over each warp's 8 tokens, totals, split check
@@ -168,7 +171,7 @@ __global__ void __launch_bounds__(kThreads6, 2)
                           const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tw, int T, int H,
                           const float* __restrict__ u, const float* __restrict__ init_state,
                           const int32_t* __restrict__ state_map, int n_state, float* __restrict__ final_state,
-                          __nv_bfloat16* __restrict__ o, unsigned* err) {
+                          __nv_bfloat16* __restrict__ o, float* __restrict__ ck_state, unsigned* err) {
   extern __shared__ uint8_t wkv6_dsmem[];
   Wkv6Smem& sm = *reinterpret_cast<Wkv6Smem*>((reinterpret_cast<uintptr_t>(wkv6_dsmem) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -300,7 +303,7 @@ __global__ void __launch_bounds__(kThreads6, 2)
       float ov[16];
       tmem_ld16(tl + kColO + 32 * ch + 16 * q, ov);
       tmem_wait_ld();
-      if (ok && holder && row >= prev_off && row < prev_off + prev_len) {
+      if (o && ok && holder && row >= prev_off && row < prev_off + prev_len) {
         uint32_t p[8];
 #pragma unroll
         for (int e = 0; e < 16; e += 2) p[e / 2] = pack_bf16x2(ov[e], ov[e + 1]);
@@ -319,6 +322,15 @@ __global__ void __launch_bounds__(kThreads6, 2)
     const uint32_t vt = smem_u32(sm.v[c & 1]);
     int off = 0, size = kChunk6;
     bool first_unit = true;
+    if (ck_state) {
+      // the state entering chunk c, [i][jv] fp32, for the backward
+      float* cs = ck_state + (((int64_t)b * H + h) * nch + c) * kHead6 * kHead6;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        *reinterpret_cast<float2*>(cs + r0 * kHead6 + cq + 8 * q) = make_float2(S[4 * q], S[4 * q + 1]);
+        *reinterpret_cast<float2*>(cs + r1 * kHead6 + cq + 8 * q) = make_float2(S[4 * q + 2], S[4 * q + 3]);
+      }
+    }
     wait_bar(&sm.w_bar, (uint32_t)c & 1u, &w_done, c + 1);
     while (off < valid) {
       const int len = min(size, valid - off);
@@ -519,7 +531,7 @@ wkv_status launch_wkv6_forward(const Wkv6FwdArgs& a, cudaStream_t stream, unsign
   }
   wkv6_fwd_chunk_kernel<<<(unsigned)(a.B * a.H), kThreads6, smem, stream>>>(
       maps[0], maps[1], maps[2], maps[3], (int)a.T, (int)a.H, a.u, a.init_state, a.state_map, (int)a.n_state,
-      a.final_state, static_cast<__nv_bfloat16*>(a.o), err);
+      a.final_state, static_cast<__nv_bfloat16*>(a.o), a.ck_state, err);
   if (cudaGetLastError() != cudaSuccess) {
     *why = "wkv6_forward kernel launch failed";
     return WKV_ERR_CUDA;

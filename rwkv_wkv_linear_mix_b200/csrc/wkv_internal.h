@@ -138,7 +138,8 @@ struct Wkv6FwdArgs {
   const int32_t* state_map;
   int64_t n_state;
   float* final_state;
-  void* o;
+  void* o;                   // may be null (no output written)
+  float* ck_state = nullptr;  // [B*H][ceil(T/64)][64][64]: state entering each chunk (may be null)
 };
 
 struct Wkv6BwdArgs {
