@@ -348,13 +348,10 @@ wkv_status wkv6_forward(int64_t B, int64_t T, int64_t H, int64_t K, int dtype,
                         float *final_state, void *o, void *stream);
 
 /* Bytes of workspace wkv6_backward needs for K = 64 (0 for another K), with
- * nch = ceil(T / 64) chunks and Tp = 64 * nch, each piece rounded up to a
- * multiple of 256 bytes:
+ * nch = ceil(T / 64) chunks, each piece rounded up to a multiple of 256 bytes:
  *   2 x 4*B*H*nch*64*64   the state entering every chunk, forward (S) and
  *                         backward (G = dL/dS)
- *   4*B*H*nch*64          per-chunk partial sums of gu
- *   5 x 2*B*Tp*H*64       time-reversed bf16 copies of k, r, dout, w and of
- *                         the reversed pass's output. */
+ *   4*B*H*nch*64          per-chunk partial sums of gu. */
 size_t wkv6_backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K);
 
 /*
@@ -379,10 +376,10 @@ size_t wkv6_backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t K)
  *   workspace    device memory of workspace_bytes >= wkv6_backward_workspace_bytes,
  *                16-byte aligned; overwritten, nothing in it needs clearing.
  * Every device pointer must be 16-byte aligned. The forward kernel runs twice
- * (on the inputs, recording the state entering every 64-token chunk, and on
- * time-reversed copies of k, r, dout, w from g_final, which gives gv, g_init
- * and dL/dS at every chunk boundary); then one tensor-core CTA per chunk
- * forms gr, gk, glogw and gu partials, and a last kernel sums gu.
+ * (on the inputs, recording the state entering every 64-token chunk, and as
+ * the time-reversed recurrence of k, r, dout, w from g_final, which gives gv,
+ * g_init and dL/dS at every chunk boundary); then one tensor-core CTA per
+ * chunk forms gr, gk, glogw and gu partials, and a last kernel sums gu.
  * Returns WKV_ERR_INVALID_ARG for a missing pointer or a short workspace,
  * WKV_ERR_UNSUPPORTED for K != 64 or a dtype other than WKV_BF16.
  */

@@ -16,9 +16,8 @@
 //     in the roles of (r, k, v, w) and g_final as the initial state, the
 //     forward computes gv (its output: gv_t = k_t G_t + (r_t . (u o k_t)) do_t),
 //     g_init = G_{-1} (its final state) and G at every chunk boundary (its
-//     chunk states). It runs on time-reversed copies of the four inputs,
-//     padded at the front to whole chunks (padding: r = k = do = 0, w = 1,
-//     which leaves the state as it is), so its chunks are those of step 1.
+//     chunk states). The forward kernel runs this reversed recurrence
+//     itself, on the same chunks as step 1 taken last to first.
 //  3. One CTA per chunk, independent of every other chunk, from S_in and
 //     G_out of its chunk (chunk-local notation: tokens j = 0..63,
 //     E_j = prod_{tau <= j} w_tau, R^_j = r_j o E_{j-1}, K~_s = k_s / E_s,
@@ -104,8 +103,8 @@ __device__ __forceinline__ float tfc(const uint8_t* tile, int row, int col) {
 __global__ void __launch_bounds__(kThr6, 2)
     wkv6_bwd_chunk_kernel(const __grid_constant__ CUtensorMap tr, const __grid_constant__ CUtensorMap tk,
                           const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tw,
-                          const __grid_constant__ CUtensorMap tdo, int T, int H, int nch, const float* __restrict__ u,
-                          const float* __restrict__ ck_s, const float* __restrict__ ck_g,
+                          const __grid_constant__ CUtensorMap tdo, const __grid_constant__ CUtensorMap tcs,
+                          const __grid_constant__ CUtensorMap tcg, int T, int H, int nch, const float* __restrict__ u,
                           __nv_bfloat16* __restrict__ gr, __nv_bfloat16* __restrict__ gk,
                           __nv_bfloat16* __restrict__ glogw, float* __restrict__ gu_part, unsigned* err) {
   extern __shared__ uint8_t bwd6_dsmem[];
@@ -132,21 +131,47 @@ __global__ void __launch_bounds__(kThr6, 2)
     mbar_init(&sm.in_bar, 1);
     mbar_init(&sm.mma_bar, 1);
     mbar_init_fence();
-    mbar_arrive_expect_tx(&sm.in_bar, 5 * kTile);
+    tma_prefetch_desc(&tcs);
+    tma_prefetch_desc(&tcg);
+    mbar_arrive_expect_tx(&sm.in_bar, 9 * kTile);
     tma_load_3d(sm.r, &tr, &sm.in_bar, h * kK6, t0, b);
     tma_load_3d(sm.k, &tk, &sm.in_bar, h * kK6, t0, b);
     tma_load_3d(sm.w, &tw, &sm.in_bar, h * kK6, t0, b);
     tma_load_3d(sm.v, &tv, &sm.in_bar, h * kK6, t0, b);
     tma_load_3d(sm.dout, &tdo, &sm.in_bar, h * kK6, t0, b);
+    // S_in and G_out, plain [i][jv] fp32, into the space the second MMAs'
+    // operands take later
+    tma_load_3d(sm.kr, &tcs, &sm.in_bar, 0, 0, bh * nch + c);
+    tma_load_3d(sm.kr + 2 * kTile, &tcg, &sm.in_bar, 0, 0, bh * nch + c);
   }
   if (warp == 0) tmem_alloc(&sm.tmem_base, kTmemCols);
   if (tid < kK6) sm.u[tid] = u[h * kK6 + tid];
 
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tm = sm.tmem_base;
+  const uint32_t tl = tm + ((uint32_t)(32 * sp) << 16);  // this warp's TMEM lanes
+
+  const int i0 = 2 * lane;
+  float w0[8], w1[8];
+  float Em1[8][2];  // E_{t-1} of this warp's tokens, kept until the table can be written
+  bool deep = false;
+  bool ok = mbar_wait_bounded(&sm.in_bar, 0, err);
+  bool mma_pending = false;  // an MMA commit not yet waited for (thread 0's view)
+  uint32_t mma_phase = 0;
+  auto wait_mma = [&]() {
+    ok = mbar_wait_bounded(&sm.mma_bar, mma_phase, err) && ok;
+    mma_phase ^= 1u;
+    if (tid == 0) mma_pending = false;
+    tc_fence_after_sync();
+  };
+
   // S_in and G_out of the chunk: hi/lo bf16 operand tiles, and the row sums
   // of G_out o S_in (this thread's 8 columns of rows r0, r1)
-  {
-    const float* S = ck_s + ((int64_t)bh * nch + c) * kK6 * kK6;
-    const float* G = ck_g + ((int64_t)bh * nch + (nch - 1 - c)) * kK6 * kK6;
+  if (ok) {
+    const float* S = reinterpret_cast<const float*>(sm.kr);
+    const float* G = reinterpret_cast<const float*>(sm.kr + 2 * kTile);
     float p0 = 0.f, p1 = 0.f;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -179,28 +204,11 @@ __global__ void __launch_bounds__(kThr6, 2)
       sm.cpart[ch][r1] = p1;
     }
   }
-  tc_fence_before_sync();
-  __syncthreads();
-  tc_fence_after_sync();
-  const uint32_t tm = sm.tmem_base;
-  const uint32_t tl = tm + ((uint32_t)(32 * sp) << 16);  // this warp's TMEM lanes
-
-  bool ok = mbar_wait_bounded(&sm.in_bar, 0, err);
-  bool mma_pending = false;  // an MMA commit not yet waited for (thread 0's view)
-  uint32_t mma_phase = 0;
-  auto wait_mma = [&]() {
-    ok = mbar_wait_bounded(&sm.mma_bar, mma_phase, err) && ok;
-    mma_phase ^= 1u;
-    if (tid == 0) mma_pending = false;
-    tc_fence_after_sync();
-  };
+  // (the states in kr are read by every thread before prep overwrites kr)
+  if (__syncthreads_or(!ok)) goto finish;
 
   // ---- prep: decay products, R^ and K~ (transposed, fp32), E_{t-1} ----
   // warp g takes tokens 8g .. 8g + 7, lane the channels 2 lane, 2 lane + 1
-  const int i0 = 2 * lane;
-  float w0[8], w1[8];
-  float Em1[8][2];  // E_{t-1} of this warp's tokens, kept until the table can be written
-  bool deep = false;
   if (ok) {
     float p0 = 1.f, p1 = 1.f;
 #pragma unroll
@@ -470,70 +478,31 @@ finish:
   }
 }
 
-// Time reversal of a [B][T][HK] bf16 tensor into [B][Tp][HK] (Tp >= T):
-// row p of the copy is row Tp - 1 - p of the source, rows with no source row
-// (the first Tp - T) hold `pad`. Four tensors in one launch (blockIdx.y).
-struct RevJob {
-  const __nv_bfloat16* src[4];
-  __nv_bfloat16* dst[4];
-  uint32_t pad[4];  // a bf16 value twice (0 or 1.0)
-};
-__global__ void wkv6_reverse_kernel(RevJob job, int B, int T, int Tp, int64_t HK) {
-  const int which = blockIdx.y;
-  const int64_t per_row = HK / 8;  // 16-byte pieces per row
-  const int64_t n = (int64_t)B * Tp * per_row;
-  for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < n; x += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t piece = x % per_row;
-    const int64_t row = x / per_row;
-    const int p = (int)(row % Tp);
-    const int bb = (int)(row / Tp);
-    const int q = Tp - 1 - p;
-    uint4 val;
-    if (q < T) {
-      val = reinterpret_cast<const uint4*>(job.src[which] + ((int64_t)bb * T + q) * HK)[piece];
-    } else {
-      const uint32_t pv = job.pad[which];
-      val = make_uint4(pv, pv, pv, pv);
-    }
-    reinterpret_cast<uint4*>(job.dst[which] + ((int64_t)bb * Tp + p) * HK)[piece] = val;
-  }
-}
-
-// gv row t = row Tp - 1 - t of the reversed pass's output.
-__global__ void wkv6_unreverse_kernel(const __nv_bfloat16* __restrict__ src, __nv_bfloat16* __restrict__ dst, int B,
-                                      int T, int Tp, int64_t HK) {
-  const int64_t per_row = HK / 8;
-  const int64_t n = (int64_t)B * T * per_row;
-  for (int64_t x = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; x < n; x += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t piece = x % per_row;
-    const int64_t row = x / per_row;
-    const int t = (int)(row % T);
-    const int bb = (int)(row / T);
-    reinterpret_cast<uint4*>(dst + ((int64_t)bb * T + t) * HK)[piece] =
-        reinterpret_cast<const uint4*>(src + ((int64_t)bb * Tp + (Tp - 1 - t)) * HK)[piece];
-  }
-}
-
-// gu[h*64 + i] = sum over samples b and chunks c (in that order) of the
-// chunk partials: fixed order, deterministic.
-__global__ void wkv6_gu_reduce_kernel(const float* __restrict__ part, int B, int H, int nch, float* __restrict__ gu) {
-  const int x = blockIdx.x * blockDim.x + threadIdx.x;  // h * 64 + i
-  if (x >= H * kK6) return;
-  const int h = x / kK6, i = x % kK6;
+// gu[h*64 + i] = sum over samples b and chunks c of the chunk partials, in a
+// fixed order: one CTA per head, thread (quarter m, channel i) adds every
+// fourth (b, c) pair in order, then the four quarter sums are added 0..3.
+__global__ void __launch_bounds__(256) wkv6_gu_reduce_kernel(const float* __restrict__ part, int B, int H, int nch,
+                                                            float* __restrict__ gu) {
+  __shared__ float qs[4][kK6];
+  const int h = blockIdx.x, i = threadIdx.x & 63, m = threadIdx.x >> 6;
+  const int n = B * nch;
   float s = 0.f;
-  for (int bb = 0; bb < B; ++bb)
-    for (int c = 0; c < nch; ++c) s += part[(((int64_t)bb * H + h) * nch + c) * kK6 + i];
-  gu[x] = s;
+  for (int x = m; x < n; x += 4) {
+    const int bb = x / nch, c = x % nch;
+    s += part[(((int64_t)bb * H + h) * nch + c) * kK6 + i];
+  }
+  qs[m][i] = s;
+  __syncthreads();
+  if (m == 0) gu[h * kK6 + i] = ((qs[0][i] + qs[1][i]) + qs[2][i]) + qs[3][i];
 }
 
 // Workspace pieces (each 256-byte aligned).
 struct Bwd6Ws {
   float *ck_s, *ck_g, *gu_part;
-  __nv_bfloat16 *rev[4], *orev;
   size_t bytes;
 };
 Bwd6Ws bwd6_ws(void* base, int64_t B, int64_t T, int64_t H) {
-  const int64_t nch = ceil_div(T, kL6), Tp = nch * kL6, BH = B * H, HK = H * kK6;
+  const int64_t nch = ceil_div(T, kL6), BH = B * H;
   uintptr_t p = reinterpret_cast<uintptr_t>(base);
   size_t off = 0;
   auto take = [&](size_t n) {
@@ -545,8 +514,6 @@ Bwd6Ws bwd6_ws(void* base, int64_t B, int64_t T, int64_t H) {
   ws.ck_s = static_cast<float*>(take(sizeof(float) * BH * nch * kK6 * kK6));
   ws.ck_g = static_cast<float*>(take(sizeof(float) * BH * nch * kK6 * kK6));
   ws.gu_part = static_cast<float*>(take(sizeof(float) * BH * nch * kK6));
-  for (int m = 0; m < 4; ++m) ws.rev[m] = static_cast<__nv_bfloat16*>(take(2 * B * Tp * HK));
-  ws.orev = static_cast<__nv_bfloat16*>(take(2 * B * Tp * HK));
   ws.bytes = off;
   return ws;
 }
@@ -556,7 +523,7 @@ Bwd6Ws bwd6_ws(void* base, int64_t B, int64_t T, int64_t H) {
 size_t wkv6_bwd_workspace_bytes(int64_t B, int64_t T, int64_t H) { return bwd6_ws(nullptr, B, T, H).bytes; }
 
 wkv_status launch_wkv6_backward(const Wkv6BwdArgs& a, cudaStream_t stream, unsigned* err, const char** why) {
-  const int64_t nch = ceil_div(a.T, kL6), Tp = nch * kL6, BH = a.B * a.H, HK = a.H * kK6;
+  const int64_t nch = ceil_div(a.T, kL6), BH = a.B * a.H, HK = a.H * kK6;
   const Bwd6Ws ws = bwd6_ws(a.workspace, a.B, a.T, a.H);
   // 1. forward: the state entering every chunk (no output)
   if (a.T > 0) {
@@ -564,47 +531,31 @@ wkv_status launch_wkv6_backward(const Wkv6BwdArgs& a, cudaStream_t stream, unsig
                   nullptr};
     f.ck_state = ws.ck_s;
     if (wkv_status s = launch_wkv6_forward(f, stream, err, why)) return s;
-    // 2. the gradient state backwards: the forward on the time-reversed (k, r, do, w)
-    RevJob job;
-    const void* src[4] = {a.k, a.r, a.dout, a.w};
-    for (int m = 0; m < 4; ++m) {
-      job.src[m] = static_cast<const __nv_bfloat16*>(src[m]);
-      job.dst[m] = ws.rev[m];
-      job.pad[m] = m == 3 ? 0x3F803F80u : 0u;  // w = 1.0 in the padding, else 0
-    }
-    const int64_t pieces = a.B * Tp * (HK / 8);
-    const unsigned gx = (unsigned)std::min<int64_t>(ceil_div(pieces, 256), 148 * 16);
-    wkv6_reverse_kernel<<<dim3(gx, 4), 256, 0, stream>>>(job, (int)a.B, (int)a.T, (int)Tp, HK);
-    if (cudaGetLastError() != cudaSuccess) {
-      *why = "wkv6_backward: reversal kernel launch failed";
-      return WKV_ERR_CUDA;
-    }
   }
-  {
-    Wkv6FwdArgs g{a.B, Tp, a.H, a.K, ws.rev[0], ws.rev[1], ws.rev[2], ws.rev[3], a.u, a.g_final, nullptr,
-                  a.g_final ? a.B : 0, a.g_init, a.T > 0 ? ws.orev : nullptr};
+  // 2. the gradient state backwards: the reversed recurrence on (k, r, do, w)
+  // from g_final; its output is gv, its final state g_init
+  if (a.T > 0 || a.g_init) {
+    Wkv6FwdArgs g{a.B, a.T, a.H, a.K, a.k, a.r, a.dout, a.w, a.u, a.g_final, nullptr, a.g_final ? a.B : 0, a.g_init,
+                  a.T > 0 ? a.gv : nullptr};
     g.ck_state = a.T > 0 ? ws.ck_g : nullptr;
-    if (a.T > 0 || a.g_init) {
-      if (wkv_status s = launch_wkv6_forward(g, stream, err, why)) return s;
-    }
+    g.reverse = true;
+    if (wkv_status s = launch_wkv6_forward(g, stream, err, why)) return s;
   }
   if (a.T > 0) {
-    const int64_t pieces = a.B * a.T * (HK / 8);
-    const unsigned gx = (unsigned)std::min<int64_t>(ceil_div(pieces, 256), 148 * 16);
-    wkv6_unreverse_kernel<<<gx, 256, 0, stream>>>(ws.orev, static_cast<__nv_bfloat16*>(a.gv), (int)a.B, (int)a.T,
-                                                  (int)Tp, HK);
-    if (cudaGetLastError() != cudaSuccess) {
-      *why = "wkv6_backward: reversal kernel launch failed";
-      return WKV_ERR_CUDA;
-    }
     // 3. every chunk independently: gr, gk, glogw and the gu partials
-    CUtensorMap maps[5];
+    CUtensorMap maps[7];
     memset(maps, 0, sizeof(maps));
     const void* src[5] = {a.r, a.k, a.v, a.w, a.dout};
     for (int m = 0; m < 5; ++m)
       if (!encode_tmap_3d(&maps[m], src[m], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)HK, (uint64_t)a.T,
                           (uint64_t)a.B, kK6, kL6, 1, why, /*swizzle128=*/true))
         return WKV_ERR_INVALID_ARG;
+    // chunk states: [B*H*nch][64][64] fp32, one plain 16 KB box per chunk
+    if (!encode_tmap_3d(&maps[5], ws.ck_s, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kK6, kK6, (uint64_t)(BH * nch), kK6,
+                        kK6, 1, why) ||
+        !encode_tmap_3d(&maps[6], ws.ck_g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kK6, kK6, (uint64_t)(BH * nch), kK6,
+                        kK6, 1, why))
+      return WKV_ERR_INVALID_ARG;
     const size_t smem = sizeof(Bwd6Smem) + 1024;
     if (cudaFuncSetAttribute(wkv6_bwd_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess) {
@@ -612,7 +563,7 @@ wkv_status launch_wkv6_backward(const Wkv6BwdArgs& a, cudaStream_t stream, unsig
       return WKV_ERR_CUDA;
     }
     wkv6_bwd_chunk_kernel<<<(unsigned)(BH * nch), kThr6, smem, stream>>>(
-        maps[0], maps[1], maps[2], maps[3], maps[4], (int)a.T, (int)a.H, (int)nch, a.u, ws.ck_s, ws.ck_g,
+        maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], (int)a.T, (int)a.H, (int)nch, a.u,
         static_cast<__nv_bfloat16*>(a.gr), static_cast<__nv_bfloat16*>(a.gk), static_cast<__nv_bfloat16*>(a.glogw),
         ws.gu_part, err);
     if (cudaGetLastError() != cudaSuccess) {
@@ -621,8 +572,7 @@ wkv_status launch_wkv6_backward(const Wkv6BwdArgs& a, cudaStream_t stream, unsig
     }
   }
   if (a.T > 0) {
-    wkv6_gu_reduce_kernel<<<(unsigned)ceil_div(HK, 256), 256, 0, stream>>>(ws.gu_part, (int)a.B, (int)a.H, (int)nch,
-                                                                          a.gu);
+    wkv6_gu_reduce_kernel<<<(unsigned)a.H, 256, 0, stream>>>(ws.gu_part, (int)a.B, (int)a.H, (int)nch, a.gu);
   } else if (cudaMemsetAsync(a.gu, 0, sizeof(float) * HK, stream) != cudaSuccess) {
     *why = "cudaMemsetAsync failed";
     return WKV_ERR_CUDA;

@@ -30,7 +30,11 @@
 // K~, so every w in (0, 1] is handled.
 //
 // For the backward the kernel can also write the state entering every
-// 64-token chunk (ck_state, [B*H][chunks][64][64] fp32, [i][jv]) and skip o.
+// 64-token chunk (ck_state, [B*H][chunks][64][64] fp32, [i][jv]), skip o,
+// and run the time-reversed recurrence (REV: chunks last to first, each
+// chunk's tokens in descending order; its output row t is the reversed
+// recurrence's output for token t and ck_state[c] the state entering chunk c
+// from above).
 //
 // Kernel shape: one CTA of 256 threads per (b, h), walking its chunks (and
 // sub-chunks: "units") in order; two CTAs share an SM. Per unit n:
@@ -65,7 +69,7 @@ struct alignas(1024) Wkv6Smem {
   uint8_t r[kTile6];      // bf16 r   [j][i]   of the current chunk
   uint8_t k[kTile6];      // bf16 k   [s][i]
   uint8_t w[kTile6];      // bf16 w   [j][i]
-  uint8_t v[2][kTile6];   // bf16 v   [s][jv]  of chunk c in v[c & 1]
+  uint8_t v[2][kTile6];   // bf16 v   [s][jv]  of the p-th chunk processed in v[p & 1]
   uint8_t rf[2][kTile6];  // R^ fp32, panels [i / 32][j][i % 32]            (A of MMA12)
   uint8_t bt[2][2 * kTile6];  // B of MMA12, fp32, panels [i / 32][128 rows][i % 32]:
                               // rows 0-63 K~ [s], rows 64-127 S_in^T [jv]; after
@@ -114,17 +118,21 @@ __device__ __forceinline__ void split_bf16x2(float a, float b, uint32_t& hi, uin
 // k E_{L-1} / E_s (bf16; `tot` = E_{L-1}), and the bonus r_j . (u * k_j) of
 // each token (this lane's two channels, then summed over the warp). FULL: the
 // unit is the whole 64-token chunk (no masking).
-template <bool FULL>
-__device__ __forceinline__ void wkv6_prepare(Wkv6Smem& sm, int g, int lane, int off, int len, const float (&w0)[8],
+// REV: the tokens are taken in descending order (the time-reversed
+// recurrence): E runs over the rows after j, pre holds the product over the
+// warps after this one.
+template <bool FULL, bool REV>
+__device__ __forceinline__ void wkv6_prepare(Wkv6Smem& sm, int g, int lane, int lo, int hi, const float (&w0)[8],
                                              const float (&w1)[8], float pre0, float pre1, float tot0, float tot1,
                                              float u0, float u1) {
-  const bool need_kb = FULL || len > 1;  // one token has no s < j pair
+  const bool need_kb = FULL || hi - lo > 1;  // one token has no s < j pair
   float e0 = pre0, e1 = pre1;
   float pb[8];  // this lane's part of each token's bonus
 #pragma unroll
-  for (int jj = 0; jj < 8; ++jj) {
+  for (int step = 0; step < 8; ++step) {
+    const int jj = REV ? 7 - step : step;
     const int j = 8 * g + jj;
-    const bool in = FULL || (j >= off && j < off + len);
+    const bool in = FULL || (j >= lo && j < hi);
     const uint32_t rx = tile_ld2(sm.r, j, lane), kx = tile_ld2(sm.k, j, lane);
     pb[jj] = in ? fmaf(bf16lo(rx) * u0, bf16lo(kx), bf16hi(rx) * u1 * bf16hi(kx)) : 0.f;
     float2 rh = make_float2(bf16lo(rx) * e0, bf16hi(rx) * e1);
@@ -166,6 +174,7 @@ __device__ __forceinline__ void wkv6_prepare(Wkv6Smem& sm, int g, int lane, int 
   }
 }
 
+template <bool REV>
 __global__ void __launch_bounds__(kThreads6, 2)
     wkv6_fwd_chunk_kernel(const __grid_constant__ CUtensorMap tr, const __grid_constant__ CUtensorMap tk,
                           const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tw, int T, int H,
@@ -254,20 +263,22 @@ __global__ void __launch_bounds__(kThreads6, 2)
 
   // copies and MMA commits in flight, as seen by thread 0 (which issues them)
   int w_issued = 0, w_done = 0, rk_issued = 0, rk_done = 0, v_issued = 0, v_done = 0, mma_issued = 0, mma_done = 0;
-  auto load_w = [&](int cc) {
+  // chunks are processed in order (REV: last to first); pp counts them
+  auto chunk_of = [&](int pp) { return REV ? nch - 1 - pp : pp; };
+  auto load_w = [&](int pp) {
     mbar_arrive_expect_tx(&sm.w_bar, kTile6);
-    tma_load_3d(sm.w, &tw, &sm.w_bar, h * kHead6, cc * kChunk6, b);
+    tma_load_3d(sm.w, &tw, &sm.w_bar, h * kHead6, chunk_of(pp) * kChunk6, b);
     ++w_issued;
   };
-  auto load_rk = [&](int cc) {
+  auto load_rk = [&](int pp) {
     mbar_arrive_expect_tx(&sm.rk_bar, 2 * kTile6);
-    tma_load_3d(sm.r, &tr, &sm.rk_bar, h * kHead6, cc * kChunk6, b);
-    tma_load_3d(sm.k, &tk, &sm.rk_bar, h * kHead6, cc * kChunk6, b);
+    tma_load_3d(sm.r, &tr, &sm.rk_bar, h * kHead6, chunk_of(pp) * kChunk6, b);
+    tma_load_3d(sm.k, &tk, &sm.rk_bar, h * kHead6, chunk_of(pp) * kChunk6, b);
     ++rk_issued;
   };
-  auto load_v = [&](int cc) {
-    mbar_arrive_expect_tx(&sm.v_bar[cc & 1], kTile6);
-    tma_load_3d(sm.v[cc & 1], &tv, &sm.v_bar[cc & 1], h * kHead6, cc * kChunk6, b);
+  auto load_v = [&](int pp) {
+    mbar_arrive_expect_tx(&sm.v_bar[pp & 1], kTile6);
+    tma_load_3d(sm.v[pp & 1], &tv, &sm.v_bar[pp & 1], h * kHead6, chunk_of(pp) * kChunk6, b);
     ++v_issued;
   };
   if (tid == 0 && nch > 0) {
@@ -295,7 +306,7 @@ __global__ void __launch_bounds__(kThreads6, 2)
 
   // the previous unit, whose O is still to be written out
   bool prev = false;
-  int prev_t0 = 0, prev_off = 0, prev_len = 0;
+  int prev_t0 = 0, prev_lo = 0, prev_hi = 0;
   auto epilogue = [&]() {
     // MMA3 of the previous unit has completed (waited for by the caller)
 #pragma unroll
@@ -303,7 +314,7 @@ __global__ void __launch_bounds__(kThreads6, 2)
       float ov[16];
       tmem_ld16(tl + kColO + 32 * ch + 16 * q, ov);
       tmem_wait_ld();
-      if (o && ok && holder && row >= prev_off && row < prev_off + prev_len) {
+      if (o && ok && holder && row >= prev_lo && row < prev_hi) {
         uint32_t p[8];
 #pragma unroll
         for (int e = 0; e < 16; e += 2) p[e / 2] = pack_bf16x2(ov[e], ov[e + 1]);
@@ -316,10 +327,11 @@ __global__ void __launch_bounds__(kThreads6, 2)
   };
 
   bool failed = false;
-  for (int c = 0; c < nch && !failed; ++c) {
+  for (int p = 0; p < nch && !failed; ++p) {
+    const int c = chunk_of(p);
     const int t0 = c * kChunk6;
     const int valid = min(kChunk6, T - t0);
-    const uint32_t vt = smem_u32(sm.v[c & 1]);
+    const uint32_t vt = smem_u32(sm.v[p & 1]);
     int off = 0, size = kChunk6;
     bool first_unit = true;
     if (ck_state) {
@@ -331,10 +343,13 @@ __global__ void __launch_bounds__(kThreads6, 2)
         *reinterpret_cast<float2*>(cs + r1 * kHead6 + cq + 8 * q) = make_float2(S[4 * q + 2], S[4 * q + 3]);
       }
     }
-    wait_bar(&sm.w_bar, (uint32_t)c & 1u, &w_done, c + 1);
+    wait_bar(&sm.w_bar, (uint32_t)p & 1u, &w_done, p + 1);
     while (off < valid) {
       const int len = min(size, valid - off);
       const bool full = len == kChunk6;
+      // the unit's rows: [off, off + len) in time order, or counted from the
+      // chunk's last row for the reversed recurrence
+      const int lo = REV ? valid - off - len : off, hi = lo + len;
       // ---- B. pass 1: product of w over this warp's 8 tokens (w = 1 outside) ----
       float w0[8], w1[8];
       {
@@ -342,7 +357,7 @@ __global__ void __launch_bounds__(kThreads6, 2)
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) {
           const int j = 8 * warp + jj;
-          const bool in = full || (j >= off && j < off + len);
+          const bool in = full || (j >= lo && j < hi);
           const uint32_t x = tile_ld2(sm.w, j, lane);
           w0[jj] = in ? bf16lo(x) : 1.f;
           w1[jj] = in ? bf16hi(x) : 1.f;
@@ -362,7 +377,7 @@ __global__ void __launch_bounds__(kThreads6, 2)
 #pragma unroll
         for (int g = 0; g < 8; ++g) {
           const float2 q = *reinterpret_cast<const float2*>(wq + g * kHead6 + 2 * lane);
-          if (g < warp) {
+          if (REV ? g > warp : g < warp) {
             pre0 *= q.x;
             pre1 *= q.y;
           }
@@ -379,24 +394,24 @@ __global__ void __launch_bounds__(kThreads6, 2)
       }
       const bool last_unit = off + len == valid;
       // the w tile is consumed: bring the next chunk's
-      if (tid == 0 && last_unit && c + 1 < nch) load_w(c + 1);
+      if (tid == 0 && last_unit && p + 1 < nch) load_w(p + 1);
       if (warp == 0) *reinterpret_cast<float2*>(&sm.dec[2 * lane]) = make_float2(tot0, tot1);
       // ---- E. write out the previous unit (its MMA3 overlapped pass 1) ----
       if (prev) {
         wait_mma();
         epilogue();
       }
-      // the v buffer of chunk c - 1 is free now: bring chunk c + 1's
-      if (tid == 0 && first_unit && c + 1 < nch) load_v(c + 1);
+      // the v buffer of the chunk before is free now: bring the next chunk's
+      if (tid == 0 && first_unit && p + 1 < nch) load_v(p + 1);
       if (first_unit) {
-        wait_bar(&sm.rk_bar, (uint32_t)c & 1u, &rk_done, c + 1);
-        wait_bar(&sm.v_bar[c & 1], (uint32_t)(c >> 1) & 1u, &v_done, c + 1);
+        wait_bar(&sm.rk_bar, (uint32_t)p & 1u, &rk_done, p + 1);
+        wait_bar(&sm.v_bar[p & 1], (uint32_t)(p >> 1) & 1u, &v_done, p + 1);
       }
       // ---- C. pass 2 ----
       if (full)
-        wkv6_prepare<true>(sm, warp, lane, off, len, w0, w1, pre0, pre1, tot0, tot1, u0, u1);
+        wkv6_prepare<true, REV>(sm, warp, lane, lo, hi, w0, w1, pre0, pre1, tot0, tot1, u0, u1);
       else
-        wkv6_prepare<false>(sm, warp, lane, off, len, w0, w1, pre0, pre1, tot0, tot1, u0, u1);
+        wkv6_prepare<false, REV>(sm, warp, lane, lo, hi, w0, w1, pre0, pre1, tot0, tot1, u0, u1);
       fence_proxy_async_smem();
       if (__syncthreads_or(!ok)) {
         failed = true;
@@ -404,7 +419,7 @@ __global__ void __launch_bounds__(kThreads6, 2)
       }
       // ---- D. next chunk's r, k; MMA1 A = R^ K~^T, MMA2 O = R^ S_in, MMA4 dS = K^^T V ----
       if (tid == 0) {
-        if (last_unit && c + 1 < nch) load_rk(c + 1);
+        if (last_unit && p + 1 < nch) load_rk(p + 1);
         tc_fence_after_sync();
         // descriptors advance by whole 16-byte units in their low bits
         const uint64_t da = umma_desc_sw128(smem_u32(sm.rf[0]), 16, 1024);
@@ -434,8 +449,10 @@ __global__ void __launch_bounds__(kThreads6, 2)
           for (int hh = 0; hh < 2; ++hh) {
             const int rr = hh ? r1 : r0;
             const float bb = hh ? b1 : b0;
-            const float x0 = s0 < rr ? a[4 * q + 2 * hh] : (s0 == rr ? bb : 0.f);
-            const float x1 = s0 + 1 < rr ? a[4 * q + 2 * hh + 1] : (s0 + 1 == rr ? bb : 0.f);
+            // earlier tokens only (REV: the later ones), the bonus on the diagonal
+            const bool k0 = REV ? s0 > rr : s0 < rr, k1 = REV ? s0 + 1 > rr : s0 + 1 < rr;
+            const float x0 = k0 ? a[4 * q + 2 * hh] : (s0 == rr ? bb : 0.f);
+            const float x1 = k1 ? a[4 * q + 2 * hh + 1] : (s0 + 1 == rr ? bb : 0.f);
             uint32_t ph, pl;
             split_bf16x2(x0, x1, ph, pl);
             tile_st_pair(sm.bt[0], rr, s0, ph);
@@ -476,8 +493,8 @@ __global__ void __launch_bounds__(kThreads6, 2)
       }
       prev = true;
       prev_t0 = t0;
-      prev_off = off;
-      prev_len = len;
+      prev_lo = lo;
+      prev_hi = hi;
       first_unit = false;
       off += len;
     }
@@ -524,12 +541,12 @@ wkv_status launch_wkv6_forward(const Wkv6FwdArgs& a, cudaStream_t stream, unsign
         return WKV_ERR_INVALID_ARG;
   }
   const size_t smem = sizeof(Wkv6Smem) + 1024;  // + room to align the base to 1024 bytes
-  if (cudaFuncSetAttribute(wkv6_fwd_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-      cudaSuccess) {
+  auto kern = a.reverse ? wkv6_fwd_chunk_kernel<true> : wkv6_fwd_chunk_kernel<false>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
     *why = "wkv6_forward: shared memory configuration failed";
     return WKV_ERR_CUDA;
   }
-  wkv6_fwd_chunk_kernel<<<(unsigned)(a.B * a.H), kThreads6, smem, stream>>>(
+  kern<<<(unsigned)(a.B * a.H), kThreads6, smem, stream>>>(
       maps[0], maps[1], maps[2], maps[3], (int)a.T, (int)a.H, a.u, a.init_state, a.state_map, (int)a.n_state,
       a.final_state, static_cast<__nv_bfloat16*>(a.o), a.ck_state, err);
   if (cudaGetLastError() != cudaSuccess) {

@@ -140,6 +140,7 @@ struct Wkv6FwdArgs {
   float* final_state;
   void* o;                   // may be null (no output written)
   float* ck_state = nullptr;  // [B*H][ceil(T/64)][64][64]: state entering each chunk (may be null)
+  bool reverse = false;       // run the recurrence from the last token to the first
 };
 
 struct Wkv6BwdArgs {

@@ -208,8 +208,8 @@ def test_chunk_and_wkv6_argument_errors(W):
     assert wk6(B=0) == W.WKV_OK
     need = L.wkv6_backward_workspace_bytes(2, 40, 3, 64)
     r256 = lambda n: (n + 255) // 256 * 256
-    nch, Tp = 1, 64  # ceil(40 / 64) chunks, padded length
-    assert need == 2 * r256(4 * 2 * 3 * nch * 64 * 64) + r256(4 * 2 * 3 * nch * 64) + 5 * r256(2 * 2 * Tp * 3 * 64)
+    nch = 1  # ceil(40 / 64) chunks
+    assert need == 2 * r256(4 * 2 * 3 * nch * 64 * 64) + r256(4 * 2 * 3 * nch * 64)
     assert L.wkv6_backward_workspace_bytes(2, 40, 3, 32) == 0
     wb6 = lambda B=2, T=40, H=3, K=64, dt=1, init=None, ns=0, ws=need, wsp=FAKE: L.wkv6_backward(
         B, T, H, K, dt, FAKE, FAKE, FAKE, FAKE, FAKE, init, None, ns, FAKE, None,
