@@ -77,7 +77,7 @@ struct alignas(1024) Bwd6Smem {
   float dd[kL6];         // dA[t][t]
   float cpart[2][kK6];   // row sums of G_out o S_in, per column half
   float u[kK6];
-  float scan[2][4][kK6];  // per quarter of the tokens: sums of the z and g tables
+  float scan[3][4][kK6];  // per quarter of the tokens: sums of the z and g tables, gu parts
   uint64_t in_bar, mma_bar;
   uint32_t tmem_base;
 };
@@ -104,9 +104,9 @@ __global__ void __launch_bounds__(kThr6, 2)
     wkv6_bwd_chunk_kernel(const __grid_constant__ CUtensorMap tr, const __grid_constant__ CUtensorMap tk,
                           const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tw,
                           const __grid_constant__ CUtensorMap tdo, const __grid_constant__ CUtensorMap tcs,
-                          const __grid_constant__ CUtensorMap tcg, int T, int H, int nch, const float* __restrict__ u,
-                          __nv_bfloat16* __restrict__ gr, __nv_bfloat16* __restrict__ gk,
-                          __nv_bfloat16* __restrict__ glogw, float* __restrict__ gu_part, unsigned* err) {
+                          const __grid_constant__ CUtensorMap tcg, const __grid_constant__ CUtensorMap tgr,
+                          const __grid_constant__ CUtensorMap tgk, const __grid_constant__ CUtensorMap tgw, int T,
+                          int H, int nch, const float* __restrict__ u, float* __restrict__ gu_part, unsigned* err) {
   extern __shared__ uint8_t bwd6_dsmem[];
   Bwd6Smem& sm = *reinterpret_cast<Bwd6Smem*>((reinterpret_cast<uintptr_t>(bwd6_dsmem) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -115,7 +115,6 @@ __global__ void __launch_bounds__(kThr6, 2)
   const int h = bh % H, b = bh / H;
   const int t0 = c * kL6;
   const int valid = min(kL6, T - t0);
-  const int64_t HK = (int64_t)H * kK6;
   // accumulator read-back layout (16x256b): TMEM sub-partition sp, column
   // half ch; rows r0 and r1 = r0 + 8, columns cq + 8 q + {0, 1}, q = 0..3
   const int sp = warp & 3, ch = warp >> 2;
@@ -306,11 +305,12 @@ __global__ void __launch_bounds__(kThr6, 2)
           tf(A2, s, j) = m;
           if (s == j) sm.dd[j] = x;
         }
-    // E_{t-1}: a plain [t][64] fp32 table over the (consumed) v and dout tiles
-    float* Et = reinterpret_cast<float*>(sm.v);
+    // E_{t-1}: a [t][64] fp32 table (swizzled like the operand tiles, so the
+    // read-back layout's accesses spread over the banks) over the consumed v
+    // and dout tiles
 #pragma unroll
     for (int jj = 0; jj < 8; ++jj)
-      *reinterpret_cast<float2*>(&Et[(8 * warp + jj) * kK6 + i0]) = make_float2(Em1[jj][0], Em1[jj][1]);
+      *reinterpret_cast<float2*>(sm.v + fo(8 * warp + jj, i0)) = make_float2(Em1[jj][0], Em1[jj][1]);
   }
   fence_proxy_async_smem();
   tc_fence_before_sync();
@@ -349,7 +349,6 @@ __global__ void __launch_bounds__(kThr6, 2)
     tmem_ld16x256b_x4(tl + kColDKh + 32 * ch, dKh);
     if (!deep) tmem_ld16x256b_x4(tl + kColDKt + 32 * ch, dKt);
     tmem_wait_ld();
-    const float* Et = reinterpret_cast<const float*>(sm.v);
     // deep chunk: the intra-chunk sums of dA_s with k (for gr) and r (for gk)
     // and E_{L-1} / E_t as running products of w on the CUDA cores
     float gri[16], gki[16], qv[16];
@@ -379,17 +378,19 @@ __global__ void __launch_bounds__(kThr6, 2)
       }
     }
     __syncthreads();  // the deep sums above read dA_s, which the tables below overwrite
-    float* xt = reinterpret_cast<float*>(sm.sg);              // x_t           [t][64]
-    float* gt = reinterpret_cast<float*>(sm.sg + 2 * kTile);  // z_t - x_t + y_t
-    float* zt = reinterpret_cast<float*>(sm.v);               // z_t (over E_{t-1}, in place)
-    uint8_t* gro = sm.kr;                                     // bf16 [t][64] plain rows
+    // tables [t][64] fp32 (swizzled): x_t, g_t = z_t - x_t + y_t, and z_t
+    // (over E_{t-1}, in place); outputs bf16 [t][64] plain rows (TMA stores)
+    uint8_t* xt = sm.sg;
+    uint8_t* gt = sm.sg + 2 * kTile;
+    uint8_t* zt = sm.v;
+    uint8_t* gro = sm.kr;
     uint8_t* gko = sm.kr + kTile;
 #pragma unroll
     for (int x = 0; x < 16; ++x) {
       const int q = x >> 2, hh = (x >> 1) & 1, e = x & 1;
       const int t = hh ? r1 : r0;
       const int i = cq + 8 * q + e;
-      const float em1 = Et[t * kK6 + i];
+      const float em1 = tf(sm.v, t, i);
       const float wt = t < valid ? tb(sm.w, t, i) : 1.f;
       const float rt = tb(sm.r, t, i), kt = tb(sm.k, t, i);
       const float ui = sm.u[i], dt = sm.dd[t];
@@ -407,9 +408,9 @@ __global__ void __launch_bounds__(kThr6, 2)
       const float zv = dKh[x] * Q * kt;
       const float xv = grv * rt;
       const float yv = gkin * kt;
-      xt[t * kK6 + i] = xv;
-      gt[t * kK6 + i] = zv - xv + yv;
-      zt[t * kK6 + i] = zv;
+      tf(xt, t, i) = xv;
+      tf(gt, t, i) = zv - xv + yv;
+      tf(zt, t, i) = zv;
       reinterpret_cast<__nv_bfloat16*>(gro)[t * kK6 + i] = __float2bfloat16_rn(fmaf(dt * ui, kt, grv));
       reinterpret_cast<__nv_bfloat16*>(gko)[t * kK6 + i] =
           __float2bfloat16_rn(fmaf(dt * ui, rt, fmaf(dKh[x], Q, gkin)));
@@ -419,19 +420,19 @@ __global__ void __launch_bounds__(kThr6, 2)
 
   // ---- decay gradient: glogw_t = c + D - Gsum + sum_{s < t} g_s - x_t per
   // channel (D, Gsum the chunk's sums of z and g); 4 threads per channel,
-  // each a quarter of the tokens ----
+  // each a quarter of the tokens; the same threads form the chunk's gu
+  // partial sum_t dA[t][t] r_t o k_t ----
   {
-    const float* xt = reinterpret_cast<const float*>(sm.sg);
-    const float* gt = reinterpret_cast<const float*>(sm.sg + 2 * kTile);
-    const float* zt = reinterpret_cast<const float*>(sm.v);
     const int i = tid & 63, qq = tid >> 6;
-    float zs = 0.f, gs = 0.f;
+    float zs = 0.f, gs = 0.f, us = 0.f;
     for (int t = 16 * qq; t < 16 * qq + 16; ++t) {
-      zs += zt[t * kK6 + i];
-      gs += gt[t * kK6 + i];
+      zs += tfc(sm.v, t, i);
+      gs += tfc(sm.sg + 2 * kTile, t, i);
+      us = fmaf(sm.dd[t] * tb(sm.r, t, i), tb(sm.k, t, i), us);
     }
     sm.scan[0][qq][i] = zs;
     sm.scan[1][qq][i] = gs;
+    sm.scan[2][qq][i] = us;
     __syncthreads();
     float D = 0.f, Gsum = 0.f, pre = 0.f;
     for (int m = 0; m < 4; ++m) {
@@ -443,25 +444,22 @@ __global__ void __launch_bounds__(kThr6, 2)
     const float base = cc + D - Gsum;
     __nv_bfloat16* glo = reinterpret_cast<__nv_bfloat16*>(sm.kr + 2 * kTile);
     for (int t = 16 * qq; t < 16 * qq + 16; ++t) {
-      glo[t * kK6 + i] = __float2bfloat16_rn(base + pre - xt[t * kK6 + i]);
-      pre += gt[t * kK6 + i];
+      glo[t * kK6 + i] = __float2bfloat16_rn(base + pre - tfc(sm.sg, t, i));
+      pre += tfc(sm.sg + 2 * kTile, t, i);
     }
-    // gu partial of the chunk: sum_t dA[t][t] r_t o k_t (thread per channel)
-    if (qq == 0) {
-      float acc = 0.f;
-      for (int t = 0; t < valid; ++t) acc = fmaf(sm.dd[t] * tb(sm.r, t, i), tb(sm.k, t, i), acc);
-      gu_part[((int64_t)bh * nch + c) * kK6 + i] = acc;
-    }
+    if (qq == 0)
+      gu_part[((int64_t)bh * nch + c) * kK6 + i] =
+          ((sm.scan[2][0][i] + sm.scan[2][1][i]) + sm.scan[2][2][i]) + sm.scan[2][3][i];
   }
+  // ---- gr, gk, glogw tiles to global memory by TMA (rows past T are not written) ----
+  fence_proxy_async_smem();
   __syncthreads();
-  // ---- gr, gk, glogw tiles to global memory (16-byte pieces, rows < valid) ----
-  for (int g = tid; g < 3 * kL6 * 8; g += kThr6) {
-    const int which = g / (kL6 * 8), row = (g / 8) % kL6, piece = g % 8;
-    if (row < valid) {
-      const uint4 val = reinterpret_cast<const uint4*>(sm.kr + which * kTile + row * 128)[piece];
-      __nv_bfloat16* dst = which == 0 ? gr : (which == 1 ? gk : glogw);
-      *reinterpret_cast<uint4*>(dst + ((int64_t)b * T + t0 + row) * HK + (int64_t)h * kK6 + piece * 8) = val;
-    }
+  if (tid == 0) {
+    tma_store_3d(&tgr, sm.kr, h * kK6, t0, b);
+    tma_store_3d(&tgk, sm.kr + kTile, h * kK6, t0, b);
+    tma_store_3d(&tgw, sm.kr + 2 * kTile, h * kK6, t0, b);
+    tma_store_commit();
+    tma_store_wait_read();
   }
 
 finish:
@@ -543,7 +541,7 @@ wkv_status launch_wkv6_backward(const Wkv6BwdArgs& a, cudaStream_t stream, unsig
   }
   if (a.T > 0) {
     // 3. every chunk independently: gr, gk, glogw and the gu partials
-    CUtensorMap maps[7];
+    CUtensorMap maps[10];
     memset(maps, 0, sizeof(maps));
     const void* src[5] = {a.r, a.k, a.v, a.w, a.dout};
     for (int m = 0; m < 5; ++m)
@@ -556,6 +554,12 @@ wkv_status launch_wkv6_backward(const Wkv6BwdArgs& a, cudaStream_t stream, unsig
         !encode_tmap_3d(&maps[6], ws.ck_g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kK6, kK6, (uint64_t)(BH * nch), kK6,
                         kK6, 1, why))
       return WKV_ERR_INVALID_ARG;
+    // outputs gr, gk, glogw: plain [64 tokens][64 channels] bf16 boxes (TMA stores)
+    void* dst[3] = {a.gr, a.gk, a.glogw};
+    for (int m = 0; m < 3; ++m)
+      if (!encode_tmap_3d(&maps[7 + m], dst[m], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)HK, (uint64_t)a.T,
+                          (uint64_t)a.B, kK6, kL6, 1, why))
+        return WKV_ERR_INVALID_ARG;
     const size_t smem = sizeof(Bwd6Smem) + 1024;
     if (cudaFuncSetAttribute(wkv6_bwd_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess) {
@@ -563,9 +567,8 @@ wkv_status launch_wkv6_backward(const Wkv6BwdArgs& a, cudaStream_t stream, unsig
       return WKV_ERR_CUDA;
     }
     wkv6_bwd_chunk_kernel<<<(unsigned)(BH * nch), kThr6, smem, stream>>>(
-        maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], (int)a.T, (int)a.H, (int)nch, a.u,
-        static_cast<__nv_bfloat16*>(a.gr), static_cast<__nv_bfloat16*>(a.gk), static_cast<__nv_bfloat16*>(a.glogw),
-        ws.gu_part, err);
+        maps[0], maps[1], maps[2], maps[3], maps[4], maps[5], maps[6], maps[7], maps[8], maps[9], (int)a.T, (int)a.H,
+        (int)nch, a.u, ws.gu_part, err);
     if (cudaGetLastError() != cudaSuccess) {
       *why = "wkv6_backward chunk kernel launch failed";
       return WKV_ERR_CUDA;
