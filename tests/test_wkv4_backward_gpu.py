@@ -64,16 +64,21 @@ def test_169m_config_full(W, oracle):
     assert_no_device_error()
 
 
-def test_3b_config_sampled_channels(W, oracle):
+def test_3b_config_every_channel(W, oracle):
+    """The 3B-width workload (B=16, T=4096, C=2560, bf16): every gradient
+    element against the oracle (run on blocks of channels to bound its
+    memory; each channel's gw, gu depend on that channel only)."""
     rec = synth.WKV4_RECIPES["wkv4_fb_bf16_3b"]
     inp = synth.wkv4_inputs(rec, seed=0)
-    gk, gv, gw, gu = run_bwd(W, inp)
-    rng = np.random.default_rng(1)
-    cs = np.unique(np.concatenate([rng.choice(rec.C, size=16, replace=False), [0, rec.C - 1]]))
-    ci = torch.from_numpy(cs).cuda()
-    ref = oracle.wkv4_backward(inp["w"][cs], inp["u"][cs], inp["k32"][:, :, cs], inp["v32"][:, :, cs],
-                               inp["gy32"][:, :, cs])
-    check((gk[:, :, ci], gv[:, :, ci], gw[ci], gu[ci]), ref, "bf16")
+    got = [host64(x).astype(np.float32) for x in run_bwd(W, inp)]
+    ref = [np.empty(g.shape, np.float32) for g in got]
+    for c0 in range(0, rec.C, 512):
+        cs = slice(c0, min(rec.C, c0 + 512))
+        part = oracle.wkv4_backward(inp["w"][cs], inp["u"][cs], inp["k32"][:, :, cs], inp["v32"][:, :, cs],
+                                    inp["gy32"][:, :, cs])
+        ref[0][:, :, cs], ref[1][:, :, cs], ref[2][cs], ref[3][cs] = part
+    for name, g, r in zip(("gk", "gv", "gw", "gu"), got, ref):
+        assert rel_err(g.astype(np.float64), r.astype(np.float64)) < TOL["bf16"], name
     assert_no_device_error()
 
 

@@ -89,7 +89,7 @@ def test_equals_forward_and_oracle(W, oracle, slots):
         a, b = int(short["offsets"][s]), int(short["offsets"][s + 1])
         yf = W.wkv4_forward(w, u, ks[a:b][None].contiguous(), vs[a:b][None].contiguous())
         assert torch.equal(yf[0], ys[a:b]), f"short slot {s}"
-    for s in (0, 5, 17, 31):
+    for s in range(len(slots["lengths"])):  # every slot against the oracle
         a, b = int(offs[s]), int(offs[s + 1])
         ref, st = oracle.wkv4_forward(slots["w"], slots["u"], slots["k32"][None, a:b], slots["v32"][None, a:b],
                                       return_state=True)

@@ -63,16 +63,18 @@ def test_169m_config_full(W, oracle):
     assert_no_device_error()
 
 
-def test_3b_config_sampled_lanes(W, oracle):
+def test_3b_config_every_channel(W, oracle):
+    """The 3B-width workload (B=16, T=4096, C=2560, bf16): every output
+    element against the oracle (run on blocks of channels to bound its
+    memory). The error metric's RMS floor is taken over the whole tensor."""
     rec = synth.WKV4_RECIPES["wkv4_fb_bf16_3b"]
     inp = synth.wkv4_inputs(rec, seed=0)
-    y = run_fwd(W, inp)
-    rng = np.random.default_rng(0)
-    cs = np.sort(rng.choice(rec.C, size=24, replace=False))
-    cs = np.unique(np.concatenate([cs, [0, rec.C - 1]]))
-    yc = host64(y[:, :, torch.from_numpy(cs).cuda()])
-    ref = oracle.wkv4_forward(inp["w"][cs], inp["u"][cs], inp["k32"][:, :, cs], inp["v32"][:, :, cs])
-    assert rel_err(yc, ref) < TOL["bf16"]
+    y = host64(run_fwd(W, inp)).astype(np.float32)
+    ref = np.empty(y.shape, np.float32)
+    for c0 in range(0, rec.C, 512):
+        cs = slice(c0, min(rec.C, c0 + 512))
+        ref[:, :, cs] = oracle.wkv4_forward(inp["w"][cs], inp["u"][cs], inp["k32"][:, :, cs], inp["v32"][:, :, cs])
+    assert rel_err(y.astype(np.float64), ref.astype(np.float64)) < TOL["bf16"]
     assert_no_device_error()
 
 

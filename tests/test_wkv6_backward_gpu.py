@@ -129,30 +129,29 @@ def test_empty_sequence(W):
     assert torch.count_nonzero(gu).item() == 0
 
 
-def test_full_size_sampled_heads(W, oracle):
-    """The bench shape (B=8, T=4096, H=32): every head runs on the GPU; three
-    (sample, head) pairs are checked against the oracle run on their slices."""
+def test_full_size_32_heads(W, oracle):
+    """The bench shape (B=8, T=4096, H=32): every head runs on the GPU; 32
+    (sample, head) pairs, four of every sample, are checked against the oracle
+    run on their slices (side by side as the heads of one sample); gu, which
+    sums every sample, against the oracle on all samples of one head."""
+    from test_wkv6_forward_gpu import HEADS32, gather_heads
     rec = synth.WKV6_RECIPES["wkv6_fwd_bf16_c2048"]
     B, T, H = rec.B, rec.T, rec.H
     inp = draw(B, T, H, seed=0)
     got = run(W, inp)
     torch.cuda.synchronize()
-    gu_all = host64(got[4])
-    for b, h in ((0, 0), (3, 17), (7, 31)):
+    sub = gather_heads(inp, HEADS32, ("r32", "k32", "v32", "w32", "do32"))
+    want = ref(oracle, sub, len(HEADS32))
+    for m, (b, h) in enumerate(HEADS32):
         cols = slice(h * 64, (h + 1) * 64)
-        sl = {n: inp[n][b:b + 1, :, cols] for n in ("r32", "k32", "v32", "w32", "do32")}
-        sl["u"] = inp["u"][cols]
-        want = ref(oracle, sl, 1)
+        mc = slice(m * 64, (m + 1) * 64)
         for name, g, r in zip(NAMES[:4], got[:4], want[:4]):
-            e = rel_err(host64(g[b:b + 1, :, cols]), r)
+            e = rel_err(host64(g[b:b + 1, :, cols]), r[:, :, mc])
             assert e < TOL["bf16"], f"{name} (b={b}, h={h}): {e:.3g}"
-    # gu sums every sample: check one head's total against the oracle on that head
     h = 5
     cols = slice(h * 64, (h + 1) * 64)
-    total = np.zeros(64)
-    for b in range(B):
-        sl = {n: inp[n][b:b + 1, :, cols] for n in ("r32", "k32", "v32", "w32", "do32")}
-        sl["u"] = inp["u"][cols]
-        total += ref(oracle, sl, 1)[4]
-    assert rel_err(gu_all[cols], total) < TOL["bf16"]
+    sl = {n: inp[n][:, :, cols] for n in ("r32", "k32", "v32", "w32", "do32")}
+    sl["u"] = inp["u"][cols]
+    total = ref(oracle, sl, 1)[4]
+    assert rel_err(host64(got[4])[cols], total) < TOL["bf16"]
     assert W.device_error(reset=True) == 0

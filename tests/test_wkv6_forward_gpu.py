@@ -86,14 +86,29 @@ def test_init_state_and_map(W, oracle):
     assert rel_err(host64(ob[1:2]), rz) < TOL["bf16"]
 
 
-def test_c2048_config_sampled_heads(W, oracle):
+# 32 of the 256 (sample, head) pairs of the 8x4096x32 workload: four heads of
+# every sample, spread over the head index
+HEADS32 = [(b, (b + 8 * m + 3 * b * m) % 32) for b in range(8) for m in range(4)]
+
+
+def gather_heads(inp, pairs, names):
+    """The (b, h) slices of [B, T, H*64] arrays side by side as the heads of
+    one [1, T, len(pairs)*64] sample (the oracle runs them in parallel), and
+    their bonus vectors as u [len(pairs), 64]."""
+    out = {n: np.concatenate([inp[n][b:b + 1, :, h * 64:(h + 1) * 64] for b, h in pairs], axis=2) for n in names}
+    out["u"] = np.stack([inp["u"][h * 64:(h + 1) * 64] for _, h in pairs])
+    return out
+
+
+def test_c2048_config_32_heads(W, oracle):
     rec = synth.WKV6_RECIPES["wkv6_fwd_bf16_c2048"]
     inp = synth.wkv6_inputs(rec, seed=0)
     o, fs = run(W, inp)
-    for (b, h) in [(0, 0), (3, 17), (7, 31)]:
+    assert len(set(HEADS32)) == 32 and {b for b, _ in HEADS32} == set(range(8))
+    sub = gather_heads(inp, HEADS32, ("r32", "k32", "v32", "w32"))
+    ro, rfs = oracle.wkv6_forward(sub["r32"], sub["k32"], sub["v32"], sub["w32"], sub["u"])
+    for m, (b, h) in enumerate(HEADS32):
         sl = slice(h * 64, (h + 1) * 64)
-        sub = {n: inp[n + "32"][b:b + 1, :, sl] for n in ("r", "k", "v", "w")}
-        ro, rfs = oracle.wkv6_forward(sub["r"], sub["k"], sub["v"], sub["w"], inp["u"][sl].reshape(1, 64))
-        assert rel_err(host64(o[b:b + 1, :, sl]), ro) < TOL["bf16"], (b, h)
-        assert rel_err(host64(fs[b, h]), rfs[0, 0]) < TOL["bf16"], (b, h)
+        assert rel_err(host64(o[b:b + 1, :, sl]), ro[:, :, m * 64:(m + 1) * 64]) < TOL["bf16"], (b, h)
+        assert rel_err(host64(fs[b, h]), rfs[0, m]) < TOL["bf16"], (b, h)
     assert W.device_error(reset=True) == 0
