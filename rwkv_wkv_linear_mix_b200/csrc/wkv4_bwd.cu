@@ -445,16 +445,24 @@ __global__ void __launch_bounds__(32 * NW, NSEG == 1 ? 8 : 1) wkv4_bwd_kernel(co
     cluster_arrive_release();
     cluster_wait_acquire();
     // ---- phase 2: the exact carry entering this segment from the later ones ----
-    float in[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    for (int r = NSEG - 1; r > seg; --r) {
-      const int len = min(T, wkv4_seg_begin(r + 1, NSEG, nck) * kBwdL) - wkv4_seg_begin(r, NSEG, nck) * kBwdL;
-      const float m = (float)len;
+    // every later segment's carry is requested first (independent remote
+    // loads in flight together), then they are folded in order
+    float2 pc[NSEG][5];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        auto peer = [&](int comp) {
-          return ld_shared_cluster(map_shared_rank(reinterpret_cast<const float*>(&sm.carry[comp][lane]) + h, r));
-        };
-        wkv4_carry_fold(in[h][0], in[h][1], in[h][2], in[h][3], peer(4), m, peer(0), peer(1), peer(2), peer(3));
+    for (int r = 1; r < NSEG; ++r)
+      if (r > seg)
+#pragma unroll
+        for (int comp = 0; comp < 5; ++comp) pc[r][comp] = ld_shared_cluster_f2(map_shared_rank(&sm.carry[comp][lane], r));
+    float in[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int r = NSEG - 1; r >= 1; --r) {
+      if (r > seg) {
+        const int len = min(T, wkv4_seg_begin(r + 1, NSEG, nck) * kBwdL) - wkv4_seg_begin(r, NSEG, nck) * kBwdL;
+        const float m = (float)len;
+        wkv4_carry_fold(in[0][0], in[0][1], in[0][2], in[0][3], pc[r][4].x, m, pc[r][0].x, pc[r][1].x, pc[r][2].x,
+                        pc[r][3].x);
+        wkv4_carry_fold(in[1][0], in[1][1], in[1][2], in[1][3], pc[r][4].y, m, pc[r][0].y, pc[r][1].y, pc[r][2].y,
+                        pc[r][3].y);
       }
     }
     cluster_arrive_release();  // done reading peers; waited for before exit

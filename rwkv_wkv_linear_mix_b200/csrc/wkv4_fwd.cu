@@ -184,23 +184,29 @@ __global__ void __launch_bounds__(32 * NW) wkv4_fwd_kernel(const __grid_constant
     cluster_arrive_release();
     cluster_wait_acquire();
     // ---- phase 2: fold the segments before this one into the incoming state ----
+    // every earlier segment's state is requested first (independent remote
+    // loads in flight together), then they are merged in order
+    float2 ra[NSEG], rb[NSEG], rp[NSEG];
+#pragma unroll
+    for (int r = 0; r < NSEG - 1; ++r) {
+      if (r < seg) {
+        ra[r] = ld_shared_cluster_f2(map_shared_rank(&sm.seg_aa[lane], r));
+        rb[r] = ld_shared_cluster_f2(map_shared_rank(&sm.seg_bb[lane], r));
+        rp[r] = ld_shared_cluster_f2(map_shared_rank(&sm.seg_P[lane], r));
+      }
+    }
     Wkv4Sum inx = {0.f, 0.f, kEmptyPP}, iny = inx;
-    for (int r = 0; r < seg; ++r) {
-      const int len = min(T, wkv4_seg_begin(r + 1, NSEG, nck) * WKV4_CKPT_LEN) -
-                      wkv4_seg_begin(r, NSEG, nck) * WKV4_CKPT_LEN;
-      const float* pa = reinterpret_cast<const float*>(&sm.seg_aa[lane]);
-      const float* pb = reinterpret_cast<const float*>(&sm.seg_bb[lane]);
-      const float* pp = reinterpret_cast<const float*>(&sm.seg_P[lane]);
-      const Wkv4Sum ownx = {ld_shared_cluster(map_shared_rank(pa, r)), ld_shared_cluster(map_shared_rank(pb, r)),
-                            ld_shared_cluster(map_shared_rank(pp, r))};
-      const Wkv4Sum owny = {ld_shared_cluster(map_shared_rank(pa + 1, r)),
-                            ld_shared_cluster(map_shared_rank(pb + 1, r)),
-                            ld_shared_cluster(map_shared_rank(pp + 1, r))};
-      // decay the earlier part across segment r
-      inx.P = __fmaf_rn(-(float)len, w2.x, inx.P);
-      iny.P = __fmaf_rn(-(float)len, w2.y, iny.P);
-      inx = wkv4_merge(inx, ownx);
-      iny = wkv4_merge(iny, owny);
+#pragma unroll
+    for (int r = 0; r < NSEG - 1; ++r) {
+      if (r < seg) {
+        const int len = min(T, wkv4_seg_begin(r + 1, NSEG, nck) * WKV4_CKPT_LEN) -
+                        wkv4_seg_begin(r, NSEG, nck) * WKV4_CKPT_LEN;
+        // decay the earlier part across segment r
+        inx.P = __fmaf_rn(-(float)len, w2.x, inx.P);
+        iny.P = __fmaf_rn(-(float)len, w2.y, iny.P);
+        inx = wkv4_merge(inx, Wkv4Sum{ra[r].x, rb[r].x, rp[r].x});
+        iny = wkv4_merge(iny, Wkv4Sum{ra[r].y, rb[r].y, rp[r].y});
+      }
     }
     cluster_arrive_release();  // done reading peers; waited for before exit
     st = {make_float2(inx.aa, iny.aa), make_float2(inx.bb, iny.bb), make_float2(inx.P, iny.P), splat2(0.f)};
