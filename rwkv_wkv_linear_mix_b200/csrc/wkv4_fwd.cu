@@ -33,6 +33,16 @@ namespace wkv {
 // Channels one warp covers: 32 lanes x a pair each.
 constexpr int kFwdCh = WKV4_WARP_CH;
 
+// Output form of the tiles of each kernel (kYTest, or kYNone / kYStore
+// chosen per launch). Measured on the B200 at B = 16, T = 4096, C = 4096
+// (bf16): the general kernel 0.307 ms with the per-token test, 0.337 ms with
+// the fixed forms; gated, 0.487 against 0.448 ms the other way round; the
+// sequential kernel at the 3B width 0.274 ms with the fixed forms, 0.298 ms
+// with the test.
+#ifndef WKV4_FWD_GENERAL_YTEST
+#define WKV4_FWD_GENERAL_YTEST 1
+#endif
+
 // The gate input r rides in the same ring when the output is gated.
 template <class E, int LT, int STAGES, bool GATE>
 struct Wkv4GateRing {
@@ -63,15 +73,17 @@ __device__ __forceinline__ void wkv4_write_ckpt(float* p, const Wkv4State2& st, 
 // registers), then their value updates and outputs. The chain is cheap and
 // serial; the second half's ex2/rcp of different tokens are independent, so
 // the split lets them overlap instead of waiting on one token at a time.
-// ckt: the tile's first checkpoint slot (null: none written).
-// A whole tile of N tokens (N a multiple of WKV4_CKPT_LEN) for a lane's
-// channel pair, one checkpoint interval at a time: the exponent chain of the
-// interval's tokens runs first (z1, and zo for the exact form, kept in
-// registers), then their value updates and outputs. The chain is cheap and
-// serial; the second half's ex2/rcp of different tokens are independent, so
-// the split lets them overlap instead of waiting on one token at a time.
-// ckt: the tile's first checkpoint slot (null: none written).
-template <bool SCALED, bool GATE, int N, class E>
+// ckt: the tile's first checkpoint slot (null: none written). YM: how the
+// outputs are written: kYNone (yt null), kYStore (yt not null) or kYTest
+// (yt tested at every token). The two fixed forms and the test compile to
+// different schedules; which is faster depends on the kernel around the tile
+// (measured on the B200, see the launchers).
+constexpr int kYNone = 0, kYStore = 1, kYTest = 2;
+template <int V>
+struct IntConst {
+  static constexpr int value = V;
+};
+template <bool SCALED, bool GATE, int N, int YM, class E>
 __device__ __forceinline__ void wkv4_fwd_tile(Wkv4State2& st, const E (*ks)[kFwdCh], const E (*vs)[kFwdCh],
                                               const E (*rs)[kFwdCh], int lane, float2 ref, float2 u2, float2 w2,
                                               float2 E2, E* yt, float* ckt, int C) {
@@ -86,7 +98,10 @@ __device__ __forceinline__ void wkv4_fwd_tile(Wkv4State2& st, const E (*ks)[kFwd
     for (int j = 0; j < L; ++j) {
       float2 yv = wkv4_values2<SCALED>(st, z[j], zo[j], ld_pair(&vs[jc + j][2 * lane]), E2);
       if constexpr (GATE) yv = mul2(yv, sigmoid2(ld_pair(&rs[jc + j][2 * lane])));
-      if (yt) st_pair(yt + (int64_t)(jc + j) * C, yv);
+      if constexpr (YM == kYStore)
+        st_pair(yt + (int64_t)(jc + j) * C, yv);
+      else if constexpr (YM == kYTest)
+        if (yt) st_pair(yt + (int64_t)(jc + j) * C, yv);
     }
   }
 }
@@ -227,10 +242,22 @@ __global__ void __launch_bounds__(32 * NW) wkv4_fwd_kernel(const __grid_constant
       const E(*rs)[kFwdCh] = nullptr;
       if constexpr (GATE) rs = sm.g.r[s];
       if (n == LT) {
-        if (scaled)
-          wkv4_fwd_tile<true, GATE, LT>(st, sm.k[s], sm.v[s], rs, lane, ref, u2, w2, E2, yt, ckt, C);
-        else
-          wkv4_fwd_tile<false, GATE, LT>(st, sm.k[s], sm.v[s], rs, lane, ref, u2, w2, E2, yt, ckt, C);
+        auto tile = [&](auto sc, auto ym) {
+          wkv4_fwd_tile<decltype(sc)::value, GATE, LT, decltype(ym)::value>(st, sm.k[s], sm.v[s], rs, lane, ref, u2,
+                                                                           w2, E2, yt, ckt, C);
+        };
+        if constexpr (WKV4_FWD_GENERAL_YTEST && !GATE) {
+          if (scaled) tile(BoolConst<true>{}, IntConst<kYTest>{});
+          else tile(BoolConst<false>{}, IntConst<kYTest>{});
+        } else {
+          if (scaled) {
+            if (yt) tile(BoolConst<true>{}, IntConst<kYStore>{});
+            else tile(BoolConst<true>{}, IntConst<kYNone>{});
+          } else {
+            if (yt) tile(BoolConst<false>{}, IntConst<kYStore>{});
+            else tile(BoolConst<false>{}, IntConst<kYNone>{});
+          }
+        }
       } else {
         for (int j = 0; j < n; ++j) {
           if (j % WKV4_CKPT_LEN == 0 && ckt) wkv4_write_ckpt(ckt + (int64_t)(j / WKV4_CKPT_LEN) * 3 * C, st, w2, C);
@@ -252,6 +279,125 @@ __global__ void __launch_bounds__(32 * NW) wkv4_fwd_kernel(const __grid_constant
   if constexpr (NSEG > 1) cluster_wait_acquire();  // peers may still read this CTA's segment state
 }
 
+// The unsplit launch (every lane group runs its whole sequence): one warp
+// per CTA, its ring in statically sized shared arrays, and a plain loop of
+// wait, tile, refill. The same step as wkv4_fwd_kernel with NSEG = 1; kept
+// apart because the compiler schedules the tile's loads and arithmetic
+// further apart in this form (a probe of the same tile code on the B200: 57
+// cycles per token from static shared arrays, 87 from the dynamic array).
+template <class E, int LT, int STAGES, bool GATE>
+__global__ void __launch_bounds__(32) wkv4_fwd_seq_kernel(const __grid_constant__ CUtensorMap tk,
+                                                          const __grid_constant__ CUtensorMap tv,
+                                                          const __grid_constant__ CUtensorMap tr,
+                                                          const E* __restrict__ kraw, int T, int C, int ncb,
+                                                          const float* __restrict__ w, const float* __restrict__ u,
+                                                          E* __restrict__ y, float* __restrict__ ckpt, unsigned* err) {
+  static_assert(LT % WKV4_CKPT_LEN == 0, "a tile must hold whole checkpoint intervals");
+  constexpr int RS = GATE ? STAGES : 1;
+  __shared__ __align__(128) E ks[STAGES][LT][kFwdCh];
+  __shared__ __align__(128) E vs[STAGES][LT][kFwdCh];
+  __shared__ __align__(128) E rsm[RS][GATE ? LT : 1][kFwdCh];
+  __shared__ uint64_t full[STAGES];
+  constexpr uint32_t kStageBytes = (GATE ? 3u : 2u) * LT * kFwdCh * sizeof(E);
+
+  const int lane = threadIdx.x;
+  const int cb = blockIdx.x % ncb;
+  const int b = blockIdx.x / ncb;
+  const int c0 = cb * kFwdCh;
+  const int c = c0 + 2 * lane;  // this lane's channels c, c + 1
+  const bool valid = c < C;
+  const int nck = (T + WKV4_CKPT_LEN - 1) / WKV4_CKPT_LEN;
+  const int ntile = (T + LT - 1) / LT;
+
+  auto issue = [&](int q) {
+    const int s = q % STAGES;
+    mbar_arrive_expect_tx(&full[s], kStageBytes);
+    tma_load_3d(&ks[s][0][0], &tk, &full[s], c0, q * LT, b);
+    tma_load_3d(&vs[s][0][0], &tv, &full[s], c0, q * LT, b);
+    if constexpr (GATE) tma_load_3d(&rsm[s % RS][0][0], &tr, &full[s], c0, q * LT, b);
+  };
+  if (lane == 0) {
+    tma_prefetch_desc(&tk);
+    tma_prefetch_desc(&tv);
+    if constexpr (GATE) tma_prefetch_desc(&tr);
+    for (int s = 0; s < STAGES; ++s) mbar_init(&full[s], 1);
+    mbar_init_fence();
+    for (int q = 0; q < STAGES && q < ntile; ++q) issue(q);
+  }
+  __syncwarp();
+
+  const int64_t lane_off = valid ? (int64_t)b * T * C + c : 0;
+  const float2 w2 = valid ? mul2(ld_pair(w + c), splat2(kLog2e)) : splat2(0.f);
+  const float2 u2 = valid ? mul2(ld_pair(u + c), splat2(kLog2e)) : splat2(0.f);
+  float2 ref = splat2(0.f);
+  if (valid) {
+    const float2 kf = ld_pair(kraw + lane_off);
+    ref = make_float2(wkv4_ref(kf.x), wkv4_ref(kf.y));
+  }
+  float* ckl = (ckpt && valid) ? ckpt + (int64_t)b * nck * 3 * C + c : nullptr;
+  E* yl = (y && valid) ? y + lane_off : nullptr;
+  const bool scaled = wkv4_scaled_pair2(u2, w2);
+  const float2 E2 = wkv4_out_scale2(u2, w2);
+
+  Wkv4State2 st = wkv4_empty_state2();
+  int q = 0;
+  bool ok = true;
+  for (; q < ntile; ++q) {
+    const int s = q % STAGES;
+    ok = __all_sync(0xffffffffu, mbar_wait_bounded(&full[s], (q / STAGES) & 1, err));
+    if (!ok) break;
+    const int t0 = q * LT;
+    const int n = min(LT, T - t0);
+    if (valid) {
+      E* yt = yl ? yl + (int64_t)t0 * C : nullptr;
+      float* ckt = ckl ? ckl + (int64_t)(t0 / WKV4_CKPT_LEN) * 3 * C : nullptr;
+      const E(*rs)[kFwdCh] = nullptr;
+      if constexpr (GATE) rs = rsm[s % RS];
+      if (n == LT) {
+        auto tile = [&](auto sc, auto ym) {
+          wkv4_fwd_tile<decltype(sc)::value, GATE, LT, decltype(ym)::value>(st, ks[s], vs[s], rs, lane, ref, u2, w2,
+                                                                           E2, yt, ckt, C);
+        };
+        if (scaled) {
+          if (yt) tile(BoolConst<true>{}, IntConst<kYStore>{});
+          else tile(BoolConst<true>{}, IntConst<kYNone>{});
+        } else {
+          if (yt) tile(BoolConst<false>{}, IntConst<kYStore>{});
+          else tile(BoolConst<false>{}, IntConst<kYNone>{});
+        }
+      } else {
+        for (int j = 0; j < n; ++j) {
+          if (j % WKV4_CKPT_LEN == 0 && ckt) wkv4_write_ckpt(ckt + (int64_t)(j / WKV4_CKPT_LEN) * 3 * C, st, w2, C);
+          float2 yv = wkv4_token2(st, wkv4_key2(ld_pair(&ks[s][j][2 * lane]), ref), ld_pair(&vs[s][j][2 * lane]), u2,
+                                  w2, scaled, E2);
+          if constexpr (GATE) yv = mul2(yv, sigmoid2(ld_pair(&rs[j][2 * lane])));
+          if (yt) st_pair(yt + (int64_t)j * C, yv);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0 && q + STAGES < ntile) issue(q + STAGES);
+  }
+  if (!ok && lane == 0) {
+    // A wait gave up: let the copies still in flight land before the CTA's
+    // shared memory is released (each wait is itself bounded).
+    for (int qq = q; qq < ntile && qq < q + STAGES; ++qq) mbar_wait_bounded(&full[qq % STAGES], (qq / STAGES) & 1, err);
+  }
+}
+
+// Which unsplit launches take wkv4_fwd_seq_kernel. Measured on the B200
+// (B = 16, T = 4096): bf16 at the 3B width (640 lane groups, 4.3 warps per
+// SM) 0.274 ms against 0.307 ms for wkv4_fwd_kernel, but at C = 4096 (1,024
+// groups, 6.9 per SM) 0.356 ms against 0.309 ms; float32 at C = 4096 0.58-
+// 0.59 ms against 0.60-0.62 ms. So bf16 launches of more than
+// WKV4_FWD_SEQ_MAX_GROUPS lane groups keep the general kernel.
+#ifndef WKV4_FWD_SEQ_KERNEL
+#define WKV4_FWD_SEQ_KERNEL 1
+#endif
+#ifndef WKV4_FWD_SEQ_MAX_GROUPS
+#define WKV4_FWD_SEQ_MAX_GROUPS (148 * 5)
+#endif
+
 template <class E, int LT, int STAGES, int NSEG, int NW, bool GATE>
 static wkv_status run_fwd(const Wkv4FwdArgs& a, cudaStream_t stream, unsigned* err, const char** why) {
   CUtensorMap tk, tv, tr;
@@ -265,6 +411,24 @@ static wkv_status run_fwd(const Wkv4FwdArgs& a, cudaStream_t stream, unsigned* e
     return WKV_ERR_INVALID_ARG;
   const int ncb = (int)ceil_div(a.C, kFwdCh);
   const int ngroups = (int)(ncb * a.B);
+  if (NSEG == 1 && NW == 1 && WKV4_FWD_SEQ_KERNEL && (sizeof(E) == 4 || ngroups <= WKV4_FWD_SEQ_MAX_GROUPS)) {
+    // all static: without a preference the driver may leave part of the
+    // unified L1/shared memory to L1 and fit fewer of these CTAs on an SM
+    auto seq = wkv4_fwd_seq_kernel<E, LT, STAGES, GATE>;
+    if (cudaFuncSetAttribute(seq, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared) !=
+        cudaSuccess) {
+      *why = "wkv4_forward: shared memory configuration failed";
+      return WKV_ERR_CUDA;
+    }
+    const unsigned grid = (unsigned)ngroups;
+    seq<<<grid, 32, 0, stream>>>(
+        tk, tv, tr, static_cast<const E*>(a.k), (int)a.T, (int)a.C, ncb, a.w, a.u, static_cast<E*>(a.y), a.ckpt, err);
+    if (cudaGetLastError() != cudaSuccess) {
+      *why = "wkv4_forward kernel launch failed";
+      return WKV_ERR_CUDA;
+    }
+    return WKV_OK;
+  }
   auto kern = wkv4_fwd_kernel<E, LT, STAGES, NSEG, NW, GATE>;
   const size_t smem = NW * sizeof(Wkv4FwdSmem<E, LT, STAGES, GATE>);
   if (smem > 48 * 1024 &&

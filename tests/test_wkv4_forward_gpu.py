@@ -32,6 +32,10 @@ SHAPES = [
     (1, 300, 8200),
     # few lane groups, long ragged sequence: 8-CTA clusters, two sub-segments per CTA
     (2, 1500, 96),
+    # 780 lane groups, too short to split: bf16 takes the general one-segment
+    # kernel (above the one-warp sequential kernel's group limit), float32 the
+    # sequential kernel; the last channel block is ragged
+    (12, 100, 4104),
 ]
 
 
