@@ -17,7 +17,9 @@
 //      segments after it, into its exact incoming state;
 //   3. every CTA reruns its segment from that state, writing y and the
 //      checkpoints (the second read of k, v mostly hits L2).
-// With NSEG = 1 phases 1-2 vanish and the kernel is the plain sequential scan.
+// With NSEG = 1 phases 1-2 vanish and the kernel is the plain sequential scan
+// (most such launches run it as wkv4_fwd_seq_kernel, below: the same tile in
+// a one-warp CTA with static shared arrays).
 // k and v stream through a ring of STAGES shared-memory tiles of LT steps,
 // filled by 3-D TMA loads (box {64 ch, LT steps, 1 sample}; rows past the
 // segment are ignored) that complete on per-stage mbarriers; lane 0 refills a
